@@ -1,0 +1,166 @@
+"""fp64 CPU oracle for the Mamba-2 SSD forward scan -- TEST INFRASTRUCTURE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA library
+and the library never calls it.
+
+Python side: argument marshalling to the C implementation in ``ssd_oracle.c``
+(every function widens its inputs to fp64; bf16-valued inputs widen exactly).
+
+Method (per batch b, head h, group g = h // (H // G)):
+    h_t = exp(dt_t A_h) h_{t-1} + dt_t x_t B_t^T,   y_t = h_t C_t + D_h x_t
+-- the scalar-identity SSM recurrence (akillness.github.io "State Space Duality
+and Mamba-2", "Mathematical Foundations" and "The Scalar-Identity Structural
+Constraint"; aifetchly blog "Mamba-2 Architecture: State Space Duality
+Explained", section 1 "The Core Duality", the sum form of y_t), with the step
+size dt on the decay and on the input.
+
+Shapes: x, y [B,T,H,P]; dt [B,T,H]; A, D [H]; B, C [B,T,G,N];
+init/final state [B,H,P,N].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "default_threads"]
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups")]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_ssd_recurrent.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 9 + [
+            ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, ctypes.c_int]
+        lib.oracle_ssd_recurrent.restype = ctypes.c_int
+        lib.oracle_ssd_quadratic.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 9
+        lib.oracle_ssd_quadratic.restype = ctypes.c_int
+        lib.oracle_ssd_chunked.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int64] + [dp] * 14
+        lib.oracle_ssd_chunked.restype = ctypes.c_int
+        lib.oracle_default_threads.argtypes = []
+        lib.oracle_default_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    """Number of host cores in this process's affinity mask."""
+    return int(_load().oracle_default_threads())
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _dims(x, B):
+    bsz, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    return _Dims(bsz, T, H, P, N, G)
+
+
+def _prep(x, dt, A, B, C, D, h0):
+    x, dt, A, B, C = (_f64(v) for v in (x, dt, A, B, C))
+    D, h0 = _f64(D), _f64(h0)
+    bsz, T, H, P = x.shape
+    if dt.shape != (bsz, T, H) or A.shape != (H,):
+        raise ValueError("dt must be [B,T,H] and A [H]")
+    if B.shape != C.shape or B.shape[:2] != (bsz, T):
+        raise ValueError("B and C must be [B,T,G,N]")
+    if D is not None and D.shape != (H,):
+        raise ValueError("D must be [H]")
+    if h0 is not None and h0.shape != (bsz, H, P, B.shape[3]):
+        raise ValueError("init state must be [B,H,P,N]")
+    return x, dt, A, B, C, D, h0
+
+
+def ssd_recurrent(x, dt, A, B, C, D=None, h0=None, units=None, nthreads=0):
+    """Token-by-token recurrence in fp64 (the oracle).
+
+    ``units``: optional iterable of (b, h) pairs; only those heads are evaluated
+    and the other entries of the returned arrays are NaN.
+    Returns (y [B,T,H,P], final_state [B,H,P,N]) as float64 arrays.
+    """
+    x, dt, A, B, C, D, h0 = _prep(x, dt, A, B, C, D, h0)
+    d = _dims(x, B)
+    y = np.full(x.shape, np.nan)
+    fin = np.full((d.batch, d.nheads, d.headdim, d.dstate), np.nan)
+    if units is None:
+        uarr, nu = None, 0
+    else:
+        ul = np.ascontiguousarray([b * d.nheads + h for (b, h) in units], dtype=np.int64)
+        uarr, nu = ul.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), len(ul)
+    rc = _load().oracle_ssd_recurrent(ctypes.byref(d), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                      _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(fin),
+                                      uarr, nu, int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle_ssd_recurrent failed ({rc})")
+    return y, fin
+
+
+def ssd_quadratic(x, dt, A, B, C, D=None, h0=None):
+    """Dual form with the explicit T x T semiseparable matrix (small T only)."""
+    x, dt, A, B, C, D, h0 = _prep(x, dt, A, B, C, D, h0)
+    d = _dims(x, B)
+    y = np.zeros(x.shape)
+    fin = np.zeros((d.batch, d.nheads, d.headdim, d.dstate))
+    rc = _load().oracle_ssd_quadratic(ctypes.byref(d), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                      _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(fin))
+    if rc != 0:
+        raise ValueError(f"oracle_ssd_quadratic failed ({rc})")
+    return y, fin
+
+
+def ssd_chunked(x, dt, A, B, C, chunk_len, D=None, h0=None, intermediates=False):
+    """Chunked algorithm in fp64.
+
+    Returns (y, final_state) or, with ``intermediates=True``,
+    (y, final_state, dict(l, w, alpha, S, s_in)) where
+    l, w [B,H,nc,Q]; alpha [B,H,nc]; S [B,nc,H,P,N]; s_in [B,nc,H,P,N]
+    (the state entering each chunk).
+    """
+    x, dt, A, B, C, D, h0 = _prep(x, dt, A, B, C, D, h0)
+    d = _dims(x, B)
+    Q = int(chunk_len)
+    if Q <= 0 or d.seqlen % Q:
+        raise ValueError("chunk_len must divide T")
+    nc = d.seqlen // Q
+    y = np.zeros(x.shape)
+    fin = np.zeros((d.batch, d.nheads, d.headdim, d.dstate))
+    if intermediates:
+        l = np.zeros((d.batch, d.nheads, nc, Q))
+        w = np.zeros_like(l)
+        alpha = np.zeros((d.batch, d.nheads, nc))
+        S = np.zeros((d.batch, nc, d.nheads, d.headdim, d.dstate))
+        s_in = np.zeros((d.batch, nc + 1, d.nheads, d.headdim, d.dstate))
+    else:
+        l = w = alpha = S = s_in = None
+    rc = _load().oracle_ssd_chunked(ctypes.byref(d), Q, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                    _ptr(C), _ptr(D), _ptr(h0), _ptr(y), _ptr(fin),
+                                    _ptr(l), _ptr(w), _ptr(alpha), _ptr(S), _ptr(s_in))
+    if rc != 0:
+        raise ValueError(f"oracle_ssd_chunked failed ({rc})")
+    if intermediates:
+        return y, fin, dict(l=l, w=w, alpha=alpha, S=S, s_in=s_in[:, :nc])
+    return y, fin
