@@ -1,0 +1,398 @@
+"""Benchmark of the SSD forward scan on B200: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one ssd_forward call -- the whole hot path (ssd_chunk_cumsum,
+ssd_chunk_state, ssd_state_passing, ssd_chunk_scan) -- over one batch of the
+Mamba-2-2.7B-shaped layer (B=4, T=4096, H=80, P=64, N=128, G=1, chunk 256,
+bf16 x/B/C, fp32 dt/A/D, final state returned), seeded synthetic inputs resident
+in HBM.  Every step's inputs and outputs exceed L2 (x and y are 168 MB each,
+L2 is 126 MB), so steps run back to back without a flush.
+
+Multi-GPU (torchrun, one process per GPU): the path is not sharded; every rank
+runs an independent replica of the same workload ("weak" scaling) and the
+time is the max over ranks.  --impl reference times the fp64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from structured_state_space_mamba_b200.inputs import WORKLOADS, make_workload  # noqa: E402
+
+METRIC = "SSD scan tokens/sec on 1 B200 and % of bf16 tensor-core roofline"
+UNIT = "tokens/s"
+SPEC_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                 0x100: "display_clock_setting"}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (chunked algorithm; compulsory bytes only)
+# ---------------------------------------------------------------------------
+def work_model(cfg, final_state=True):
+    B, T, H, P, N, G, Q = (cfg[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
+                                            "ngroups", "chunk_len"))
+    nc = T // Q
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    flops_bch = Q * (Q + 1) * P + 4 * Q * N * P          # masked product + state + C.s_in
+    flops_bcg = Q * (Q + 1) * N                          # causal C B^T, shared by H/G heads
+    flops = B * nc * (H * flops_bch + G * flops_bcg)
+    x_bytes = B * T * H * P * esz
+    bc_bytes = 2 * B * T * G * N * esz
+    dt_bytes = B * T * H * 4
+    state_bytes = B * H * P * N * 4
+    comp = (2 * x_bytes + bc_bytes + dt_bytes + 2 * H * 4
+            + (state_bytes if cfg.get("init_state") else 0)
+            + (state_bytes if final_state else 0))
+    # per-kernel algorithmic bytes (what each kernel must read and write)
+    st_elems = B * nc * H * P * N
+    per_kernel = {
+        "ssd_chunk_cumsum": dt_bytes + H * 4 + 2 * B * H * nc * Q * 4 + B * H * nc * 4,
+        "ssd_chunk_state": x_bytes + bc_bytes // 2 + B * H * nc * Q * 4 + st_elems * 4,
+        "ssd_state_passing": st_elems * 4 + B * H * nc * 4 + st_elems * 2
+                             + (state_bytes if final_state else 0),
+        "ssd_chunk_scan": 2 * x_bytes + bc_bytes + dt_bytes + B * H * nc * Q * 4 + st_elems * 2
+                          + H * 4,
+    }
+    per_kernel_flops = {
+        "ssd_chunk_state": 2 * B * nc * H * Q * N * P,
+        "ssd_chunk_scan": B * nc * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * flops_bcg),
+    }
+    return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
+                per_kernel_flops=per_kernel_flops)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(SPEC_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, index=0):
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        if self.proc is None or not getattr(self, "out", None):
+            return None
+        sm, mx, reasons = [], [], set()
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                s, m = float(parts[0]), float(parts[1])
+                bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
+            except ValueError:
+                continue
+            if bits & 0x1:  # idle samples say nothing about the load
+                continue
+            sm.append(s)
+            mx.append(m)
+            for bit, name in THROTTLE_BITS.items():
+                if bits & bit:
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# oracle leg (CPU)
+# ---------------------------------------------------------------------------
+def oracle_sample(inp, tokens, batches=1):
+    """Run the oracle over the first `tokens` tokens of `batches` batch rows
+    (all heads); returns (seconds, tokens processed, threads)."""
+    import oracle
+    sl = slice(0, tokens)
+    bs = slice(0, batches)
+    args = [inp.x[bs, sl], inp.dt[bs, sl], inp.A, inp.B[bs, sl], inp.C[bs, sl]]
+    h0 = None if inp.h0 is None else inp.h0[bs]
+    t0 = time.perf_counter()
+    oracle.ssd_recurrent(*args, D=inp.D, h0=h0)
+    return time.perf_counter() - t0, tokens * batches, oracle.default_threads()
+
+
+def cpu_baseline(inp, budget_s=12.0):
+    import oracle  # noqa: F401  (builds the C oracle if needed)
+    T = inp.x.shape[1]
+    tokens = min(T, 512)
+    sec, tok, th = oracle_sample(inp, tokens)
+    # grow the sample to roughly budget_s of CPU work
+    scale = max(1, int(budget_s / max(sec, 1e-3)))
+    bmax = inp.x.shape[0]
+    tokens2 = min(T, tokens * scale)
+    batches = min(bmax, max(1, (tokens * scale) // T)) if tokens2 == T else 1
+    sec, tok, th = oracle_sample(inp, tokens2, batches)
+    return {"value": tok / sec, "unit": UNIT, "cores": th, "kind": "oracle",
+            "sample": f"fp64 recurrence over the first {tokens2} tokens x {batches} batch row(s), "
+                      f"all {inp.x.shape[2]} heads ({tok} tokens, {sec:.1f} s on {th} threads)"}
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    inp = make_workload(args.workload)
+    T = inp.x.shape[1]
+    tokens = min(T, args.ref_tokens)
+    for _ in range(args.warmup):
+        oracle_sample(inp, tokens)
+    secs = []
+    th = 1
+    for _ in range(args.steps):
+        s, _, th = oracle_sample(inp, tokens)
+        secs.append(s)
+    total = sum(secs)
+    value = tokens * args.steps / total
+    sample = (f"each step: fp64 recurrence over the first {tokens} of {T} tokens of batch row 0, "
+              f"all {inp.x.shape[2]} heads")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference", "config": config_block(cfg, args.workload),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": th, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_block(cfg, name):
+    return {"workload": (f"{name}: B={cfg['batch']} T={cfg['seqlen']} H={cfg['nheads']} "
+                         f"P={cfg['headdim']} N={cfg['dstate']} G={cfg['ngroups']} "
+                         f"chunk={cfg['chunk_len']} {cfg['dtype']}"),
+            "batch": cfg["batch"], "seqlen": cfg["seqlen"], "nheads": cfg["nheads"],
+            "headdim": cfg["headdim"], "dstate": cfg["dstate"], "ngroups": cfg["ngroups"],
+            "chunk_len": cfg["chunk_len"], "init_state": bool(cfg.get("init_state")),
+            "final_state": bool(cfg.get("final_state", True)),
+            "l2": "no flush: inputs larger than L2 (x and y exceed 126 MB each)",
+            "parallelism": "replicas"}
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+def run_gpu(args, cfg, rank, world, local_rank):
+    import torch
+
+    from structured_state_space_mamba_b200 import binding
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = make_workload(args.workload)
+    tt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    host = dict(x=(inp.x, tt), dt=(inp.dt, torch.float32), A=(inp.A, torch.float32),
+                B=(inp.B, tt), C=(inp.C, tt), D=(inp.D, torch.float32))
+    if inp.h0 is not None:
+        host["init_state"] = (inp.h0, torch.float32)
+    # pinned host copies (storage dtype) for the end-to-end leg
+    pinned = {k: torch.from_numpy(v).to(t).pin_memory() for k, (v, t) in host.items()}
+    d = {k: v.to(dev, non_blocking=False) for k, v in pinned.items()}
+    want_final = bool(cfg.get("final_state", True))
+    y = torch.empty_like(d["x"])
+    fin = (torch.empty((inp.x.shape[0], inp.x.shape[2], inp.x.shape[3], inp.B.shape[3]),
+                       dtype=torch.float32, device=dev) if want_final else None)
+    dims = binding.make_dims(*inp.x.shape[:2], inp.x.shape[2], inp.x.shape[3], inp.B.shape[3],
+                             inp.B.shape[2], inp.dtype)
+    lay = binding.workspace_layout(dims, inp.chunk_len)
+    ws = torch.empty(lay.total_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(stage=None):
+        binding.forward(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                        chunk_len=inp.chunk_len, init_state=d.get("init_state"), out=y,
+                        final_out=fin, workspace=ws, stage=stage)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K back-to-back steps -------------------------------
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    clocks = clk.summary()
+
+    # ---- per-kernel durations: the same steps, one stage per launch ---------
+    nst = len(binding.STAGES)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        for s in range(nst):
+            step(stage=s)
+            ev[k][s + 1].record(stream)
+    torch.cuda.synchronize()
+    kern_ms = {binding.STAGES[s]: statistics.mean(ev[k][s].elapsed_time(ev[k][s + 1])
+                                                  for k in range(args.steps))
+               for s in range(nst)}
+    barrier()
+
+    # ---- end to end through the public call, host buffers ------------------
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    fin_host = torch.empty(fin.shape, dtype=fin.dtype).pin_memory() if fin is not None else None
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * y_host.element_size() + (
+        fin_host.numel() * fin_host.element_size() if fin_host is not None else 0)
+
+    def e2e_step():
+        for k, v in pinned.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        if fin_host is not None:
+            fin_host.copy_(fin, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    barrier()
+
+    if rank != 0:
+        return
+    tokens_step = inp.x.shape[0] * inp.x.shape[1]
+    value = world * tokens_step * args.steps / (ms_total * 1e-3)
+    wm = work_model(cfg, final_state=want_final)
+    peaks, peak_src = load_peaks()
+    top = max(kern_ms, key=kern_ms.get)
+    bound = "hbm"
+    achieved = wm["per_kernel_bytes"][top] / (kern_ms[top] * 1e-3) / 1e9
+    peak = peaks["hbm_gbs"]
+    t_step = ms_total / args.steps * 1e-3
+    t_roof = max(wm["flops"] / (peaks["bf16_tflops"] * 1e12), wm["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
+        "config": config_block(cfg, args.workload),
+        "roofline": {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"},
+        "path_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": t_step * 1e6,
+                          "frac": t_roof / t_step, "flops": wm["flops"],
+                          "compulsory_bytes": wm["bytes"],
+                          "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, "
+                                   f"bf16 {peaks['bf16_tflops']} TF/s"},
+        "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "gpu_launches": args.steps * lay.launches,
+        "tensor_core": bool(lay.tensor_core),
+        "e2e": {"value": world * tokens_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mamba2_2p7b", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = dict(WORKLOADS[args.workload])
+    cfg.setdefault("final_state", True)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+/*
+ * ssd.h -- C ABI of libssd.so, the B200 (sm_100a) Mamba-2 SSD forward scan.
+ *
+ * The operation (per batch b, head h; group g = h / (H / G)):
+ *
+ *     h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T      (state, P x N)
+ *     y_t = h_t C_t + D_h * x_t
+ *
+ * the selective SSM with a scalar-times-identity transition ("Transformers are
+ * SSMs", Dao & Gu 2024; akillness.github.io "State Space Duality and Mamba-2",
+ * sections "Mathematical Foundations" and "The Scalar-Identity Structural
+ * Constraint"), evaluated blockwise as the chunked SSD algorithm (aifetchly
+ * blog "Mamba-2 Architecture: State Space Duality Explained", section "The
+ * Chunked SSD Algorithm"): the masked product (L o C B^T) X inside each chunk of
+ * chunk_len tokens, and the state recurrence between chunks.  The kernels are
+ * ssd_chunk_cumsum, ssd_chunk_state, ssd_state_passing and ssd_chunk_scan.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers to contiguous row-major memory,
+ *    16-byte aligned.  The caller owns every buffer; the library keeps no
+ *    pointer after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the host.  Argument errors are detected and
+ *    returned BEFORE anything is launched; launch errors come back as
+ *    SSD_ERR_CUDA.  Errors of kernels that already ran surface, as usual in
+ *    CUDA, on the next synchronising call.
+ *  - Re-entrant: no global mutable state except a per-device cache of device
+ *    properties.
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_NULL_ARG = 1,       /* a required pointer is NULL                    */
+    SSD_ERR_INVALID_DIM = 2,    /* a size is <= 0, H % G != 0, T % chunk_len != 0 */
+    SSD_ERR_UNSUPPORTED = 3,    /* sizes outside the supported set (see below)   */
+    SSD_ERR_MISALIGNED = 4,     /* a pointer is not 16-byte aligned              */
+    SSD_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed          */
+    SSD_ERR_DEVICE_TIMEOUT = 6, /* reserved: a bounded device-side wait expired  */
+    SSD_ERR_WORKSPACE = 7       /* workspace NULL/too small, or allocation failed */
+} ssd_status_t;
+
+/* Storage dtype of x, B, C and y.  dt, A, D and the states are always fp32. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
+
+typedef struct {
+    int64_t batch;   /* B */
+    int64_t seqlen;  /* T */
+    int64_t nheads;  /* H */
+    int64_t headdim; /* P */
+    int64_t dstate;  /* N */
+    int64_t ngroups; /* G: B and C are shared by H/G consecutive heads */
+    int32_t dtype;   /* ssd_dtype_t */
+    int32_t reserved; /* must be 0 */
+} ssd_dims_t;
+
+/*
+ * Supported sizes (anything else returns SSD_ERR_UNSUPPORTED):
+ *   chunk_len in {32, 64, 128, 256}, seqlen % chunk_len == 0 (else INVALID_DIM);
+ *   1 <= headdim <= 256, 1 <= dstate <= 256; nheads % ngroups == 0;
+ *   SSD_BF16 additionally: headdim % 8 == 0 and dstate % 8 == 0.
+ * The tensor-core path runs for SSD_BF16 with headdim == 64,
+ * dstate in {16, 32, 64, 128, 256} and chunk_len in {64, 128, 256}; other
+ * supported shapes run on the CUDA-core kernels of the same library.
+ */
+
+/*
+ * ssd_forward -- one forward scan.
+ *
+ *   x          [B, T, H, P]  dtype
+ *   dt         [B, T, H]     fp32, the step sizes as used (positive; any
+ *                            softplus/bias is applied by the caller)
+ *   A          [H]           fp32, the per-head decay rate (negative for decay)
+ *   Bm, Cm     [B, T, G, N]  dtype (input and output projections)
+ *   D          [H]           fp32 skip weights, or NULL for no skip term
+ *   chunk_len                tokens per chunk
+ *   init_state [B, H, P, N]  fp32 initial state, or NULL for zeros
+ *   y_out      [B, T, H, P]  dtype, written; must not alias any input
+ *   final_state_out [B,H,P,N] fp32 final state, or NULL; it may alias
+ *                            init_state (it is written after every read)
+ *   stream                   cudaStream_t
+ *
+ * Intermediates (ssd_workspace_bytes) are allocated stream-ordered on
+ * `stream` and released before return (cudaMallocAsync / cudaFreeAsync).
+ * Accuracy against the fp64 recurrence: max|y - y_ref| / max|y_ref| <= 1e-4
+ * for SSD_F32 and <= 2e-2 for SSD_BF16 when every dt_t * A_h <= 0; the same
+ * bound holds for the final state.
+ */
+SSD_API ssd_status_t ssd_forward(const ssd_dims_t *dims, const void *x, const float *dt,
+                         const float *A, const void *Bm, const void *Cm, const float *D,
+                         int chunk_len, const float *init_state, void *y_out,
+                         float *final_state_out, void *stream);
+
+/*
+ * ssd_forward_ws -- ssd_forward with caller-provided workspace.
+ * `workspace` is a device buffer of at least ssd_workspace_bytes(dims,
+ * chunk_len) bytes, 256-byte aligned; otherwise SSD_ERR_WORKSPACE.  After the
+ * call the workspace holds the intermediates described by
+ * ssd_workspace_layout (valid once the stream reaches that point).
+ */
+SSD_API ssd_status_t ssd_forward_ws(const ssd_dims_t *dims, const void *x, const float *dt,
+                            const float *A, const void *Bm, const void *Cm, const float *D,
+                            int chunk_len, const float *init_state, void *y_out,
+                            float *final_state_out, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/*
+ * ssd_forward_stage -- run ONE of the four kernels of ssd_forward_ws, with the
+ * same arguments and the same launch configuration, reading the earlier
+ * stages' results from `workspace` and writing its own there (or to y_out /
+ * final_state_out).  Calling the stages 0, 1, 2, 3 in order on one stream is
+ * equivalent to one ssd_forward_ws call; this exists to time and test each
+ * kernel on its own.
+ *   stage 0  ssd_chunk_cumsum   dt, A          -> l, w, alpha
+ *   stage 1  ssd_chunk_state    x, B, w        -> states
+ *   stage 2  ssd_state_passing  states, alpha, init_state -> s_in, final_state_out
+ *   stage 3  ssd_chunk_scan     x, dt, B, C, D, l, s_in   -> y_out
+ * Any other stage value returns SSD_ERR_INVALID_DIM.
+ */
+typedef enum {
+    SSD_STAGE_CHUNK_CUMSUM = 0,
+    SSD_STAGE_CHUNK_STATE = 1,
+    SSD_STAGE_STATE_PASSING = 2,
+    SSD_STAGE_CHUNK_SCAN = 3
+} ssd_stage_t;
+
+SSD_API ssd_status_t ssd_forward_stage(int stage, const ssd_dims_t *dims, const void *x,
+                                       const float *dt, const float *A, const void *Bm,
+                                       const void *Cm, const float *D, int chunk_len,
+                                       const float *init_state, void *y_out,
+                                       float *final_state_out, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace one call needs (0 if the arguments are invalid). */
+SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
+
+/*
+ * Where each intermediate sits inside the workspace (byte offsets; nc = T/Q):
+ *   l      fp32 [B, H, nc, Q]  chunk-local inclusive cumsum of dt*A
+ *   w      fp32 [B, H, nc, Q]  exp(l_last - l_s) * dt_s (chunk-state weights)
+ *   alpha  fp32 [B, H, nc]     exp(l_last), the decay across a whole chunk
+ *   states fp32 [B, nc, H, P, N]  per-chunk states S_c = sum_s w_s x_s B_s^T
+ *   s_in   [B, nc, H, P, N]    state entering each chunk; element type given
+ *                              by s_in_dtype (SSD_F32 or SSD_BF16)
+ * `tensor_core` is 1 when the call runs the tcgen05 kernels, 0 otherwise;
+ * `launches` is the number of kernels one call launches.
+ */
+typedef struct {
+    size_t total_bytes;
+    size_t l_offset, w_offset, alpha_offset, states_offset, s_in_offset;
+    int32_t s_in_dtype;
+    int32_t tensor_core;
+    int32_t launches;
+    int32_t reserved;
+} ssd_workspace_layout_t;
+
+SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,
+                                  ssd_workspace_layout_t *out);
+
+/* Static description of a status code (never NULL). */
+SSD_API const char *ssd_status_string(ssd_status_t status);
+
+/* Library version, e.g. "ssd-b200 0.1.0 sm_100a". */
+SSD_API const char *ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H_ */

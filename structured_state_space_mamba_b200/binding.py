@@ -1,0 +1,189 @@
+"""ctypes binding of ``libssd.so`` (the C ABI in ``include/ssd.h``).
+
+Argument marshalling only: shapes, dtypes and devices of torch tensors are
+checked, their device pointers and the current CUDA stream are passed to the C
+call, and a non-zero status is raised as :class:`SSDError`.  Every step of the
+computation runs in the library's CUDA kernels; there is no other code path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(HERE, "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_ERR_UNSUPPORTED",
+          4: "SSD_ERR_MISALIGNED", 5: "SSD_ERR_CUDA", 6: "SSD_ERR_DEVICE_TIMEOUT",
+          7: "SSD_ERR_WORKSPACE"}
+
+EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
+           "ssd_workspace_layout", "ssd_status_string", "ssd_version")
+STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("l_offset", ctypes.c_size_t),
+                ("w_offset", ctypes.c_size_t), ("alpha_offset", ctypes.c_size_t),
+                ("states_offset", ctypes.c_size_t), ("s_in_offset", ctypes.c_size_t),
+                ("s_in_dtype", ctypes.c_int32), ("tensor_core", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libssd.so (raises if it has not been built; there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m structured_state_space_mamba_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, fp = ctypes.c_void_p, ctypes.c_void_p
+    dims_p = ctypes.POINTER(Dims)
+    lib.ssd_forward.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp, vp, fp, vp]
+    lib.ssd_forward.restype = ctypes.c_int
+    lib.ssd_forward_ws.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp, vp, fp,
+                                   vp, ctypes.c_size_t, vp]
+    lib.ssd_forward_ws.restype = ctypes.c_int
+    lib.ssd_forward_stage.argtypes = [ctypes.c_int] + lib.ssd_forward_ws.argtypes
+    lib.ssd_forward_stage.restype = ctypes.c_int
+    lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
+    lib.ssd_workspace_bytes.restype = ctypes.c_size_t
+    lib.ssd_workspace_layout.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]
+    lib.ssd_workspace_layout.restype = ctypes.c_int
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_version.argtypes = []
+    lib.ssd_version.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def make_dims(batch, seqlen, nheads, headdim, dstate, ngroups, dtype) -> Dims:
+    code = {"f32": SSD_F32, "bf16": SSD_BF16, torch.float32: SSD_F32,
+            torch.bfloat16: SSD_BF16}[dtype]
+    return Dims(batch, seqlen, nheads, headdim, dstate, ngroups, code, 0)
+
+
+def _check(status: int):
+    if status != 0:
+        raise SSDError(status, load().ssd_status_string(status).decode())
+
+
+def workspace_bytes(dims: Dims, chunk_len: int) -> int:
+    return int(load().ssd_workspace_bytes(ctypes.byref(dims), int(chunk_len)))
+
+
+def workspace_layout(dims: Dims, chunk_len: int) -> WorkspaceLayout:
+    out = WorkspaceLayout()
+    _check(load().ssd_workspace_layout(ctypes.byref(dims), int(chunk_len), ctypes.byref(out)))
+    return out
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _validate(x, dt, A, B, C, D, init_state):
+    if not x.is_cuda:
+        raise ValueError("ssd.forward runs on CUDA tensors only")
+    dev = x.device
+    for name, t in (("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D),
+                    ("init_state", init_state)):
+        if t is None:
+            continue
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, x on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if x.dtype not in (torch.float32, torch.bfloat16) or B.dtype != x.dtype or C.dtype != x.dtype:
+        raise ValueError("x, B and C must share a dtype: float32 or bfloat16")
+    for name, t in (("dt", dt), ("A", A), ("D", D), ("init_state", init_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32")
+    bsz, T, H, P = x.shape
+    if B.dim() != 4 or B.shape[:2] != (bsz, T) or C.shape != B.shape:
+        raise ValueError("B and C must be [batch, seqlen, ngroups, dstate]")
+    G, N = B.shape[2], B.shape[3]
+    if dt.shape != (bsz, T, H) or A.shape != (H,):
+        raise ValueError("dt must be [batch, seqlen, nheads] and A [nheads]")
+    if D is not None and D.shape != (H,):
+        raise ValueError("D must be [nheads]")
+    if init_state is not None and init_state.shape != (bsz, H, P, N):
+        raise ValueError("init_state must be [batch, nheads, headdim, dstate]")
+    return make_dims(bsz, T, H, P, N, G, x.dtype)
+
+
+def forward(x, dt, A, B, C, D=None, chunk_len=256, init_state=None, return_final_state=False,
+            out=None, final_out=None, workspace=None, stream=None, stage=None):
+    """y (and optionally the final state) of the SSD forward scan.
+
+    x [B,T,H,P], B/C [B,T,G,N] (float32 or bfloat16); dt [B,T,H], A [H], D [H],
+    init_state [B,H,P,N] float32.  Returns ``y`` or ``(y, final_state)``.
+    ``workspace``: optional uint8 CUDA tensor of at least ``workspace_bytes``
+    bytes (otherwise the library allocates it stream-ordered).
+    """
+    dims = _validate(x, dt, A, B, C, D, init_state)
+    y = out if out is not None else torch.empty_like(x)
+    fin = final_out
+    if fin is None and return_final_state:
+        fin = torch.empty((dims.batch, dims.nheads, dims.headdim, dims.dstate),
+                          dtype=torch.float32, device=x.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device).cuda_stream
+    lib = load()
+    args = [ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+            int(chunk_len), _ptr(init_state), _ptr(y), _ptr(fin)]
+    with torch.cuda.device(x.device):
+        if stage is not None:
+            if workspace is None:
+                raise ValueError("a single stage needs workspace=")
+            st = lib.ssd_forward_stage(int(stage), *args, _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(),
+                                       ctypes.c_void_p(stream))
+        elif workspace is None:
+            st = lib.ssd_forward(*args, ctypes.c_void_p(stream))
+        else:
+            st = lib.ssd_forward_ws(*args, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    ctypes.c_void_p(stream))
+    _check(st)
+    if return_final_state or final_out is not None:
+        return y, fin
+    return y
+
+
+def forward_ws(*args, **kwargs):
+    """``forward`` with a required ``workspace`` keyword."""
+    if kwargs.get("workspace") is None:
+        raise ValueError("forward_ws needs workspace=")
+    return forward(*args, **kwargs)
+
+
+def version() -> str:
+    return load().ssd_version().decode()

@@ -1,0 +1,38 @@
+// kernels.h -- host-side launchers of the SSD kernels (internal to libssd.so).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace ssd {
+
+// ssd_chunk_cumsum: dt, A -> l, w [B,H,nc,Q], alpha [B,H,nc]
+cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
+                                float *w, float *alpha, cudaStream_t stream);
+
+// ssd_state_passing: states [B,nc,H,P,N] fp32, alpha -> s_in [B,nc,H,P,N]
+// (fp32 or bf16 per s_in_bf16), final state [B,H,P,N] fp32 (may be NULL)
+cudaError_t launch_state_passing(const Dims &d, const float *states, const float *alpha,
+                                 const float *init_state, void *s_in, bool s_in_bf16,
+                                 float *final_state, cudaStream_t stream);
+
+// CUDA-core (SIMT) chunk state and chunk scan, any supported shape.
+// bf16 selects the storage type of x/B/C/y.  s_in is fp32 here.
+cudaError_t launch_chunk_state_simt(const Dims &d, bool bf16, const void *x, const void *Bm,
+                                    const float *w, float *states, cudaStream_t stream);
+cudaError_t launch_chunk_scan_simt(const Dims &d, bool bf16, const void *x, const float *dt,
+                                   const void *Bm, const void *Cm, const float *D,
+                                   const float *l, const float *s_in, void *y,
+                                   cudaStream_t stream);
+
+// Tensor-core (tcgen05) kernels, bf16 storage, P == 64.
+bool tc_chunk_state_supported(const Dims &d);
+bool tc_chunk_scan_supported(const Dims &d);
+cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, const float *w,
+                                  float *states, cudaStream_t stream);
+cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
+                                 const void *Cm, const float *D, const float *l,
+                                 const void *s_in_bf16, void *y, cudaStream_t stream);
+
+}  // namespace ssd

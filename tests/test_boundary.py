@@ -1,0 +1,141 @@
+"""The C ABI boundary on the CPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything.
+
+Every call here that passes pointers returns an error from the host-side
+checks (nothing is launched), so the fake addresses are never dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from structured_state_space_mamba_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from structured_state_space_mamba_b200 import build
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"SSD_API\s+[\w\s\*]+?\b(ssd_\w+)\s*\(", src)
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for n in ("ssd_forward", "ssd_forward_ws", "ssd_workspace_bytes", "ssd_workspace_layout",
+              "ssd_status_string", "ssd_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(binding.EXPORTS) <= set(declared_functions())
+
+
+def test_struct_sizes_match_header(lib):
+    assert ctypes.sizeof(binding.Dims) == 6 * 8 + 2 * 4
+    assert ctypes.sizeof(binding.WorkspaceLayout) == 6 * 8 + 4 * 4
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS.items():
+        s = lib.ssd_status_string(code).decode()
+        assert s.startswith(name)
+    assert lib.ssd_status_string(99).decode().startswith("SSD_ERR_UNKNOWN")
+    assert "sm_100a" in lib.ssd_version().decode()
+
+
+def dims(**kw):
+    base = dict(batch=2, seqlen=512, nheads=8, headdim=64, dstate=128, ngroups=2, dtype="bf16")
+    base.update(kw)
+    return binding.make_dims(**base)
+
+
+def test_workspace_layout(lib):
+    d = dims()
+    lay = binding.workspace_layout(d, 128)
+    nc = 512 // 128
+    assert lay.l_offset == 0
+    assert lay.w_offset >= 2 * 8 * nc * 128 * 4
+    assert lay.states_offset % 256 == 0 and lay.s_in_offset % 256 == 0
+    state_elems = 2 * nc * 8 * 64 * 128
+    assert lay.s_in_offset >= lay.states_offset + state_elems * 4
+    sz = 2 if lay.s_in_dtype == binding.SSD_BF16 else 4
+    assert lay.total_bytes >= lay.s_in_offset + state_elems * sz
+    assert lay.launches == 4
+    assert binding.workspace_bytes(d, 128) == lay.total_bytes
+    # fp32 storage never uses the tensor-core kernels
+    lay32 = binding.workspace_layout(dims(dtype="f32"), 128)
+    assert lay32.tensor_core == 0 and lay32.s_in_dtype == binding.SSD_F32
+
+
+@pytest.mark.parametrize("kw,chunk,code", [
+    (dict(seqlen=500), 128, 2),          # T % chunk_len != 0
+    (dict(nheads=6, ngroups=4), 128, 2),  # H % G != 0
+    (dict(batch=0), 128, 2),
+    (dict(dstate=-1), 128, 2),
+    ({}, 96, 3),                          # chunk_len not supported
+    (dict(headdim=512), 128, 3),
+    (dict(dstate=300), 128, 3),
+    (dict(headdim=60), 128, 3),           # bf16 needs P % 8 == 0
+    (dict(dtype="f32", headdim=60), 128, 0),  # fp32 accepts any P <= 256
+])
+def test_dims_validation(lib, kw, chunk, code):
+    d = dims(**kw)
+    lay = binding.WorkspaceLayout()
+    assert lib.ssd_workspace_layout(ctypes.byref(d), chunk, ctypes.byref(lay)) == code
+    assert (lib.ssd_workspace_bytes(ctypes.byref(d), chunk) > 0) == (code == 0)
+
+
+FAKE = 0x10000  # never dereferenced: each call below fails its host checks
+
+
+def call_forward(lib, d, chunk=128, **ptrs):
+    p = dict(x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, h0=None, y=FAKE, fin=None)
+    p.update(ptrs)
+    v = {k: (None if val is None else ctypes.c_void_p(val)) for k, val in p.items()}
+    return lib.ssd_forward(ctypes.byref(d), v["x"], v["dt"], v["A"], v["B"], v["C"], v["D"],
+                           chunk, v["h0"], v["y"], v["fin"], None)
+
+
+@pytest.mark.parametrize("name", ["x", "dt", "A", "B", "C", "y"])
+def test_null_required_pointer(lib, name):
+    assert call_forward(lib, dims(), **{name: None}) == 1
+
+
+@pytest.mark.parametrize("name", ["x", "dt", "A", "B", "C", "D", "h0", "y", "fin"])
+def test_misaligned_pointer(lib, name):
+    assert call_forward(lib, dims(), **{name: FAKE + 4}) == 4
+
+
+def test_bad_dims_before_pointers(lib):
+    assert call_forward(lib, dims(seqlen=100)) == 2
+    assert lib.ssd_forward(None, None, None, None, None, None, None, 128, None, None, None,
+                           None) == 1
+
+
+def test_workspace_too_small(lib):
+    d = dims()
+    need = binding.workspace_bytes(d, 128)
+    f = ctypes.c_void_p(FAKE)
+    args = [ctypes.byref(d), f, f, f, f, f, None, 128, None, f, None]
+    assert lib.ssd_forward_ws(*args, None, need, None) == 7
+    assert lib.ssd_forward_ws(*args, ctypes.c_void_p(1 << 20), need - 1, None) == 7
+    assert lib.ssd_forward_ws(*args, ctypes.c_void_p((1 << 20) + 16), need, None) == 7
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 2, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.forward(x, torch.zeros(1, 64, 2), torch.zeros(2), torch.zeros(1, 64, 1, 16),
+                        torch.zeros(1, 64, 1, 16), chunk_len=64)

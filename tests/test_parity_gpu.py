@@ -1,0 +1,204 @@
+"""GPU parity: libssd.so against the fp64 oracle, element by element.
+
+Tolerance (max |y_gpu - y_oracle| / max |y_oracle|, and the same for the final
+state): 1e-4 for fp32 storage, 2e-2 for bf16 storage.  Small cases are
+compared in full; the full-size workloads are compared on sampled heads, which
+the oracle evaluates one (batch, head) unit at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+from structured_state_space_mamba_b200 import binding
+from structured_state_space_mamba_b200.inputs import WORKLOADS, make_inputs, make_workload
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def to_dev(inp):
+    dt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    dev = torch.device("cuda:0")
+    t = lambda a, ty=torch.float32: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(ty)  # noqa: E731
+    return dict(x=t(inp.x, dt), dt=t(inp.dt), A=t(inp.A), B=t(inp.B, dt), C=t(inp.C, dt),
+                D=t(inp.D), init_state=t(inp.h0))
+
+
+def run_gpu(inp, final=True, **kw):
+    a = to_dev(inp)
+    out = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"],
+                          chunk_len=inp.chunk_len, init_state=a["init_state"],
+                          return_final_state=final, **kw)
+    torch.cuda.synchronize()
+    if final:
+        y, f = out
+        return y.double().cpu().numpy(), f.double().cpu().numpy()
+    return out.double().cpu().numpy(), None
+
+
+def rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
+
+
+def check_full(inp, oracle, final=True):
+    y, f = run_gpu(inp, final=final)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    tol = TOL[inp.dtype]
+    assert np.isfinite(y).all()
+    assert rel(y, yr) <= tol, rel(y, yr)
+    if final:
+        assert rel(f, fr) <= tol, rel(f, fr)
+    return rel(y, yr), (rel(f, fr) if final else None)
+
+
+def check_sampled(inp, oracle, units, final=True):
+    y, f = run_gpu(inp, final=final)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0,
+                                  units=units)
+    tol = TOL[inp.dtype]
+    assert np.isfinite(y).all()
+    ys = np.stack([y[b, :, h] for b, h in units])
+    yrs = np.stack([yr[b, :, h] for b, h in units])
+    assert rel(ys, yrs) <= tol, rel(ys, yrs)
+    if final:
+        fs = np.stack([f[b, h] for b, h in units])
+        frs = np.stack([fr[b, h] for b, h in units])
+        assert rel(fs, frs) <= tol, rel(fs, frs)
+
+
+# ---------------------------------------------------------------------------
+# small shapes, compared in full
+# ---------------------------------------------------------------------------
+def test_tiny_f32_workload(oracle):
+    check_full(make_workload("tiny_f32"), oracle)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=1, seqlen=64, nheads=1, headdim=16, dstate=16, ngroups=1, chunk_len=64),
+    dict(batch=2, seqlen=96, nheads=3, headdim=5, dstate=7, ngroups=1, chunk_len=32),
+    dict(batch=1, seqlen=256, nheads=4, headdim=64, dstate=128, ngroups=2, chunk_len=128),
+    dict(batch=1, seqlen=512, nheads=2, headdim=256, dstate=256, ngroups=2, chunk_len=256),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_f32_shapes(oracle, shape, h0):
+    inp = make_inputs(**shape, dtype="f32", seed=7, init_state=h0)
+    check_full(inp, oracle)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=1, seqlen=256, nheads=2, headdim=64, dstate=128, ngroups=1, chunk_len=256),
+    dict(batch=2, seqlen=512, nheads=4, headdim=64, dstate=128, ngroups=1, chunk_len=128),
+    dict(batch=1, seqlen=512, nheads=8, headdim=64, dstate=64, ngroups=2, chunk_len=64),
+    dict(batch=1, seqlen=768, nheads=4, headdim=64, dstate=16, ngroups=4, chunk_len=256),
+    dict(batch=1, seqlen=512, nheads=2, headdim=64, dstate=256, ngroups=1, chunk_len=256),
+    dict(batch=1, seqlen=256, nheads=2, headdim=32, dstate=32, ngroups=1, chunk_len=64),
+    dict(batch=3, seqlen=1024, nheads=6, headdim=64, dstate=128, ngroups=3, chunk_len=256),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_bf16_shapes(oracle, shape, h0):
+    inp = make_inputs(**shape, dtype="bf16", seed=11, init_state=h0)
+    check_full(inp, oracle)
+
+
+def test_no_skip_term(oracle):
+    inp = make_inputs(1, 256, 2, 64, 128, 1, 128, dtype="bf16", seed=3)
+    inp.D = None
+    check_full(inp, oracle)
+
+
+def test_final_state_may_alias_init_state(oracle):
+    inp = make_inputs(1, 512, 4, 64, 128, 2, 256, dtype="bf16", seed=5, init_state=True)
+    a = to_dev(inp)
+    h = a["init_state"].clone()
+    y, f = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=256,
+                           init_state=h, final_out=h)
+    torch.cuda.synchronize()
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    assert rel(y.double().cpu().numpy(), yr) <= 2e-2
+    assert rel(h.double().cpu().numpy(), fr) <= 2e-2
+
+
+def test_strong_decay_stays_finite(oracle):
+    """dt*|A| up to ~16 per token: the decays underflow to zero, never overflow."""
+    inp = make_inputs(1, 512, 4, 64, 128, 1, 256, dtype="bf16", seed=9, init_state=True)
+    inp.dt = (inp.dt * 10.0).astype(np.float32)
+    check_full(inp, oracle)
+
+
+def test_chunk_len_invariance_on_gpu(oracle):
+    ys = []
+    for q in (64, 128, 256):
+        inp = make_inputs(1, 1024, 4, 64, 128, 1, q, dtype="bf16", seed=21)
+        y, f = run_gpu(inp)
+        ys.append(y)
+    yr, _ = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D)
+    for y in ys:
+        assert rel(y, yr) <= 2e-2
+
+
+def test_repeated_calls_deterministic():
+    inp = make_inputs(2, 1024, 8, 64, 128, 1, 256, dtype="bf16", seed=2)
+    y1, f1 = run_gpu(inp)
+    y2, f2 = run_gpu(inp)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(f1, f2)
+
+
+def test_workspace_entry_point_and_intermediates(oracle):
+    """ssd_forward_ws gives the same output, and the workspace afterwards
+    holds each stage's intermediates, checked against the fp64 chunked form so
+    a failure names its kernel."""
+    inp = make_inputs(1, 512, 4, 64, 128, 2, 128, dtype="bf16", seed=4, init_state=True)
+    a = to_dev(inp)
+    d = binding.make_dims(1, 512, 4, 64, 128, 2, "bf16")
+    lay = binding.workspace_layout(d, 128)
+    ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device="cuda:0")
+    y, f = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=128,
+                           init_state=a["init_state"], return_final_state=True, workspace=ws)
+    y0, f0 = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=128,
+                             init_state=a["init_state"], return_final_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0) and torch.equal(f, f0)
+    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, 128, D=inp.D, h0=inp.h0,
+                                  intermediates=True)
+    nc = 4
+
+    def view(off, count, dtype):
+        return ws[off: off + count * torch.tensor([], dtype=dtype).element_size()].view(dtype)
+
+    l = view(lay.l_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
+    w = view(lay.w_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
+    al = view(lay.alpha_offset, 4 * nc, torch.float32).double().cpu().numpy().reshape(1, 4, nc)
+    S = view(lay.states_offset, nc * 4 * 64 * 128, torch.float32).double().cpu().numpy()
+    sdt = torch.bfloat16 if lay.s_in_dtype == binding.SSD_BF16 else torch.float32
+    s_in = view(lay.s_in_offset, nc * 4 * 64 * 128, sdt).double().cpu().numpy()
+    assert rel(l, it["l"]) < 1e-5          # ssd_chunk_cumsum
+    assert rel(al, it["alpha"]) < 1e-5
+    assert rel(w, it["w"]) < 1e-5
+    assert rel(S.reshape(it["S"].shape), it["S"]) < 2e-2          # ssd_chunk_state
+    assert rel(s_in.reshape(it["s_in"].shape), it["s_in"]) < 2e-2  # ssd_state_passing
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads (sampled heads), in the bench's launch configuration
+# ---------------------------------------------------------------------------
+def test_mamba2_130m_layer(oracle):
+    inp = make_workload("mamba2_130m")
+    check_sampled(inp, oracle, [(0, 0), (3, 11), (7, 23)], final=False)
+
+
+def test_mamba2_2p7b_layer(oracle):
+    inp = make_workload("mamba2_2p7b")
+    check_sampled(inp, oracle, [(0, 0), (1, 37), (3, 79)])
+
+
+def test_long_context_grouped_layer(oracle):
+    inp = make_workload("long_g8")
+    check_sampled(inp, oracle, [(0, 0), (0, 13), (0, 31)])
+
+
+@pytest.mark.parametrize("name", [n for n in WORKLOADS if n.startswith("sweep_")])
+def test_state_chunk_sweep(oracle, name):
+    inp = make_workload(name)
+    check_sampled(inp, oracle, [(0, 0), (1, 31)], final=True)
