@@ -50,7 +50,7 @@ typedef enum {
     SSD_ERR_UNSUPPORTED = 3,    /* sizes outside the supported set (see below)   */
     SSD_ERR_MISALIGNED = 4,     /* a pointer is not 16-byte aligned              */
     SSD_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed          */
-    SSD_ERR_DEVICE_TIMEOUT = 6, /* reserved: a bounded device-side wait expired  */
+    SSD_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait expired            */
     SSD_ERR_WORKSPACE = 7       /* workspace NULL/too small, or allocation failed */
 } ssd_status_t;
 
@@ -170,6 +170,16 @@ typedef struct {
 
 SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,
                                   ssd_workspace_layout_t *out);
+
+/*
+ * ssd_device_status -- synchronise `stream`, then report (and clear) the
+ * device-side error word of the current device: SSD_ERR_DEVICE_TIMEOUT if a
+ * bounded wait inside a tensor-core kernel expired since the last query (that
+ * kernel skipped its remaining work, so its outputs are incomplete), SSD_ERR_CUDA
+ * if the synchronisation reported an error, SSD_OK otherwise.  This is the only
+ * entry point that blocks the host.
+ */
+SSD_API ssd_status_t ssd_device_status(void *stream);
 
 /* Static description of a status code (never NULL). */
 SSD_API const char *ssd_status_string(ssd_status_t status);

@@ -21,7 +21,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
           7: "SSD_ERR_WORKSPACE"}
 
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
-           "ssd_workspace_layout", "ssd_status_string", "ssd_version")
+           "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -77,6 +77,8 @@ def load():
     lib.ssd_workspace_layout.restype = ctypes.c_int
     lib.ssd_status_string.argtypes = [ctypes.c_int]
     lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_device_status.argtypes = [ctypes.c_void_p]
+    lib.ssd_device_status.restype = ctypes.c_int
     lib.ssd_version.argtypes = []
     lib.ssd_version.restype = ctypes.c_char_p
     _lib = lib
@@ -183,6 +185,15 @@ def forward_ws(*args, **kwargs):
     if kwargs.get("workspace") is None:
         raise ValueError("forward_ws needs workspace=")
     return forward(*args, **kwargs)
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device error
+    status: 0 (SSD_OK) or 6 (SSD_ERR_DEVICE_TIMEOUT)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(load().ssd_device_status(
+            ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
 
 
 def version() -> str:

@@ -28,10 +28,11 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
                     float *__restrict__ alpha_out) {
     constexpr int Q = 32 * E;
     __shared__ float s_dt[Q][kHeadTile + 1];
-    const int c = blockIdx.x, b = blockIdx.y;
+    const int c = blockIdx.x, b = blockIdx.z;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t0 = c * Q;
-    for (int h0 = 0; h0 < d.H; h0 += kHeadTile) {
+    {
+        const int h0 = blockIdx.y * kHeadTile;
         // coalesced load of dt[b, t0:t0+Q, h0:h0+32]
         for (int i = warp; i < Q; i += kThreads / 32) {
             const int h = h0 + lane;
@@ -77,7 +78,7 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
 
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *alpha, cudaStream_t stream) {
-    dim3 grid(d.nc, d.B);
+    dim3 grid(d.nc, (d.H + kHeadTile - 1) / kHeadTile, d.B);
     switch (d.Q) {
         case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, alpha); break;
         case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, alpha); break;

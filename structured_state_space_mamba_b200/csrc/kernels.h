@@ -29,10 +29,13 @@ cudaError_t launch_chunk_scan_simt(const Dims &d, bool bf16, const void *x, cons
 // Tensor-core (tcgen05) kernels, bf16 storage, P == 64.
 bool tc_chunk_state_supported(const Dims &d);
 bool tc_chunk_scan_supported(const Dims &d);
+// `err` is a device word: bit 0 is set when a bounded wait inside a kernel
+// expired (the kernel then skips its remaining work and exits cleanly).
 cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, const float *w,
-                                  float *states, cudaStream_t stream);
+                                  float *states, unsigned int *err, cudaStream_t stream);
 cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
                                  const void *Cm, const float *D, const float *l,
-                                 const void *s_in_bf16, void *y, cudaStream_t stream);
+                                 const void *s_in_bf16, void *y, unsigned int *err,
+                                 cudaStream_t stream);
 
 }  // namespace ssd

@@ -9,14 +9,39 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/ssd.h"
 #include "common.cuh"
 #include "kernels.h"
 
+// Device word set by tensor-core kernels whose bounded waits expired.
+__device__ unsigned int g_ssd_device_error;
+
 namespace {
 
 using ssd::Dims;
+
+constexpr int kMaxDevices = 64;
+unsigned int *g_err_ptr[kMaxDevices];  // per-device address of g_ssd_device_error
+std::once_flag g_err_once[kMaxDevices];
+
+// Address of the error word on the current device (NULL if unavailable).
+unsigned int *device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::call_once(g_err_once[dev], [dev] {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ssd_device_error) == cudaSuccess)
+            g_err_ptr[dev] = static_cast<unsigned int *>(p);
+        else
+            cudaGetLastError();
+    });
+    return g_err_ptr[dev];
+}
 
 constexpr size_t kAlign = 256;
 
@@ -103,6 +128,11 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                  float *fin, char *ws, cudaStream_t stream, int only_stage = -1) {
     if (inject_launch_failure()) return SSD_ERR_CUDA;
     const Dims &d = pl.d;
+    unsigned int *err = nullptr;
+    if (pl.tc_state || pl.tc_scan) {
+        err = device_error_word();
+        if (!err) return SSD_ERR_CUDA;
+    }
     float *l = reinterpret_cast<float *>(ws + pl.ws.l_offset);
     float *w = reinterpret_cast<float *>(ws + pl.ws.w_offset);
     float *alpha = reinterpret_cast<float *>(ws + pl.ws.alpha_offset);
@@ -116,7 +146,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 e = ssd::launch_chunk_cumsum(d, dt, A, l, w, alpha, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
-                e = pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, stream)
+                e = pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, err, stream)
                                 : ssd::launch_chunk_state_simt(d, pl.bf16, x, Bm, w, states, stream);
                 break;
             case SSD_STAGE_STATE_PASSING:
@@ -125,7 +155,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 break;
             case SSD_STAGE_CHUNK_SCAN:
                 e = pl.tc_scan
-                        ? ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, stream)
+                        ? ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream)
                         : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt, Bm, Cm, D, l,
                                                       static_cast<const float *>(s_in), y, stream);
                 break;
@@ -223,6 +253,25 @@ const char *ssd_status_string(ssd_status_t status) {
         case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing, too small or unallocatable";
     }
     return "SSD_ERR_UNKNOWN: unknown status code";
+}
+
+ssd_status_t ssd_device_status(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_CUDA;
+    }
+    unsigned int *err = device_error_word();
+    if (!err) return SSD_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return SSD_ERR_CUDA;
+    if (v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        return SSD_ERR_DEVICE_TIMEOUT;
+    }
+    return SSD_OK;
 }
 
 const char *ssd_version(void) { return "ssd-b200 0.1.0 sm_100a"; }

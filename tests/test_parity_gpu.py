@@ -31,6 +31,7 @@ def run_gpu(inp, final=True, **kw):
                           chunk_len=inp.chunk_len, init_state=a["init_state"],
                           return_final_state=final, **kw)
     torch.cuda.synchronize()
+    assert binding.device_status() == 0  # no bounded device wait expired
     if final:
         y, f = out
         return y.double().cpu().numpy(), f.double().cpu().numpy()
@@ -99,6 +100,16 @@ def test_f32_shapes(oracle, shape, h0):
 def test_bf16_shapes(oracle, shape, h0):
     inp = make_inputs(**shape, dtype="bf16", seed=11, init_state=h0)
     check_full(inp, oracle)
+
+
+def test_tensor_core_path_selected():
+    """bf16 with P = 64 runs the tcgen05 kernels (chunk_len >= 128 for the scan)."""
+    for n in (16, 32, 64, 128, 256):
+        for q in (128, 256):
+            lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
+            assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
+    lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 32, 64, 1, "bf16"), 128)
+    assert lay.tensor_core == 0
 
 
 def test_no_skip_term(oracle):
