@@ -264,26 +264,53 @@ def run_gpu(args, cfg, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
 
-    # ---- timed region: K back-to-back steps -------------------------------
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    # ---- the step as a CUDA graph (one ssd_forward_ws call, captured) -------
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(graph, stream=cap):
+                step()
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+
+    def timed(run_step):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(args.steps):
-            step()
+            run_step()
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    # ---- timed region: K back-to-back steps -------------------------------
+    with ClockSampler(local_rank) as clk:
+        ms_direct = timed(step)
+        ms_graph = timed(graph.replay) if graph is not None else None
     clocks = clk.summary()
+    if ms_graph is not None and ms_graph < ms_direct:
+        ms_total, launch_mode = ms_graph, "cuda-graph replay of one ssd_forward_ws call per step"
+    else:
+        ms_total, launch_mode = ms_direct, "one ssd_forward_ws call per step"
+    del graph
 
     # ---- per-kernel durations: the same steps, one stage per launch ---------
+    # A GPU-side sleep before each step lets the host enqueue all four stages
+    # (and the events between them) first, so no host launch gap lands inside
+    # an event pair.
     nst = len(binding.STAGES)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     for k in range(args.steps):
+        torch.cuda._sleep(3_000_000)
         ev[k][0].record(stream)
         for s in range(nst):
             step(stage=s)
@@ -348,6 +375,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
                           "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, "
                                    f"bf16 {peaks['bf16_tflops']} TF/s"},
         "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
+        "launch": launch_mode,
+        "ms_per_step_direct_calls": ms_direct / args.steps,
         "gpu_launches": args.steps * lay.launches,
         "tensor_core": bool(lay.tensor_core),
         "e2e": {"value": world * tokens_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
@@ -368,6 +397,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -153,7 +153,8 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  *   l      fp32 [B, H, nc, Q]  chunk-local inclusive cumsum of dt*A
  *   w      fp32 [B, H, nc, Q]  exp(l_last - l_s) * dt_s (chunk-state weights)
  *   alpha  fp32 [B, H, nc]     exp(l_last), the decay across a whole chunk
- *   states fp32 [B, nc, H, P, N]  per-chunk states S_c = sum_s w_s x_s B_s^T
+ *   states [B, nc, H, P, N]    per-chunk states S_c = sum_s w_s x_s B_s^T;
+ *                              element type given by states_dtype
  *   s_in   [B, nc, H, P, N]    state entering each chunk; element type given
  *                              by s_in_dtype (SSD_F32 or SSD_BF16)
  * `tensor_core` is 1 when the call runs the tcgen05 kernels, 0 otherwise;
@@ -165,7 +166,7 @@ typedef struct {
     int32_t s_in_dtype;
     int32_t tensor_core;
     int32_t launches;
-    int32_t reserved;
+    int32_t states_dtype; /* element type of states: SSD_F32 or SSD_BF16 */
 } ssd_workspace_layout_t;
 
 SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,

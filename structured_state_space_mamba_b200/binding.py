@@ -37,7 +37,7 @@ class WorkspaceLayout(ctypes.Structure):
                 ("w_offset", ctypes.c_size_t), ("alpha_offset", ctypes.c_size_t),
                 ("states_offset", ctypes.c_size_t), ("s_in_offset", ctypes.c_size_t),
                 ("s_in_dtype", ctypes.c_int32), ("tensor_core", ctypes.c_int32),
-                ("launches", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("launches", ctypes.c_int32), ("states_dtype", ctypes.c_int32)]
 
 
 class SSDError(RuntimeError):

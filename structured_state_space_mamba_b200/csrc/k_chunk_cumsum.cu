@@ -33,10 +33,19 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
     const int t0 = c * Q;
     {
         const int h0 = blockIdx.y * kHeadTile;
-        // coalesced load of dt[b, t0:t0+Q, h0:h0+32]
-        for (int i = warp; i < Q; i += kThreads / 32) {
+        // coalesced load of dt[b, t0:t0+Q, h0:h0+32]; all loads issued before
+        // the first store so that they are in flight together
+        {
+            constexpr int kIters = Q / (kThreads / 32);
             const int h = h0 + lane;
-            s_dt[i][lane] = h < d.H ? __ldg(dt + off_dt(d, b, t0 + i) + h) : 0.f;
+            float v[kIters];
+#pragma unroll
+            for (int k = 0; k < kIters; ++k) {
+                const int i = warp + k * (kThreads / 32);
+                v[k] = h < d.H ? __ldg(dt + off_dt(d, b, t0 + i) + h) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < kIters; ++k) s_dt[warp + k * (kThreads / 32)][lane] = v[k];
         }
         __syncthreads();
         for (int j = warp; j < kHeadTile; j += kThreads / 32) {

@@ -24,98 +24,134 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kPrefetch = 8;
+constexpr int kVec = 8;  // state elements per thread
 
-template <int VEC> struct VecF;
-template <> struct VecF<4> { using T = float4; };
-template <> struct VecF<1> { using T = float; };
+// kVec consecutive fp32 values in registers
+struct V8 {
+    float v[kVec];
+};
 
-__device__ __forceinline__ void fma_vec(float4 &s, float a, const float4 &v) {
-    s.x = fmaf(a, s.x, v.x); s.y = fmaf(a, s.y, v.y);
-    s.z = fmaf(a, s.z, v.z); s.w = fmaf(a, s.w, v.w);
+__device__ __forceinline__ void load8(const float *p, V8 &o) {
+    const float4 a = __ldcs(reinterpret_cast<const float4 *>(p));
+    const float4 b = __ldcs(reinterpret_cast<const float4 *>(p) + 1);
+    o.v[0] = a.x; o.v[1] = a.y; o.v[2] = a.z; o.v[3] = a.w;
+    o.v[4] = b.x; o.v[5] = b.y; o.v[6] = b.z; o.v[7] = b.w;
 }
-__device__ __forceinline__ void fma_vec(float &s, float a, const float &v) { s = fmaf(a, s, v); }
-
-__device__ __forceinline__ void store_vec(float *p, const float4 &v) {
-    *reinterpret_cast<float4 *>(p) = v;
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, V8 &o) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        o.v[2 * i] = __uint_as_float(w[i] << 16);
+        o.v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
 }
-__device__ __forceinline__ void store_vec(float *p, const float &v) { *p = v; }
-__device__ __forceinline__ void store_vec(__nv_bfloat16 *p, const float4 &v) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t *>(&lo);
-    u.y = *reinterpret_cast<uint32_t *>(&hi);
-    *reinterpret_cast<uint2 *>(p) = u;
+__device__ __forceinline__ void store8(float *p, const V8 &s) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(s.v[0], s.v[1], s.v[2], s.v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(s.v[4], s.v[5], s.v[6], s.v[7]);
 }
-__device__ __forceinline__ void store_vec(__nv_bfloat16 *p, const float &v) {
-    *p = __float2bfloat16_rn(v);
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&t);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const V8 &s) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(pack2(s.v[0], s.v[1]), pack2(s.v[2], s.v[3]),
+                                               pack2(s.v[4], s.v[5]), pack2(s.v[6], s.v[7]));
 }
 
-__device__ __forceinline__ float4 load_vec(const float4 *p) { return __ldcs(p); }
-__device__ __forceinline__ float load_vec(const float *p) { return __ldcs(p); }
-__device__ __forceinline__ void zero(float4 &v) { v = make_float4(0.f, 0.f, 0.f, 0.f); }
-__device__ __forceinline__ void zero(float &v) { v = 0.f; }
-
-template <int VEC, typename SinT>
+// Scalar fallback for state sizes that are not a multiple of kVec.
+template <typename ST, typename SinT>
 __global__ void __launch_bounds__(kThreads)
-state_passing_kernel(Dims d, const float *__restrict__ states, const float *__restrict__ alpha,
-                     const float *__restrict__ h0, SinT *__restrict__ s_in,
-                     float *__restrict__ final_state) {
-    using V = typename VecF<VEC>::T;
+state_passing_scalar_kernel(Dims d, const ST *__restrict__ states, const float *__restrict__ alpha,
+                            const float *__restrict__ h0, SinT *__restrict__ s_in,
+                            float *__restrict__ final_state) {
     const int64_t PN = int64_t(d.P) * d.N;
-    const int64_t e = (int64_t(blockIdx.x) * kThreads + threadIdx.x) * VEC;
+    const int64_t e = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     const int bh = blockIdx.y;
     const int b = bh / d.H, h = bh % d.H;
     if (e >= PN) return;
-    V cur;
-    if (h0) cur = *reinterpret_cast<const V *>(h0 + int64_t(bh) * PN + e);
-    else zero(cur);
+    float cur = h0 ? h0[int64_t(bh) * PN + e] : 0.f;
+    const float *al = alpha + off_alpha(d, b, h, 0);
+    for (int c = 0; c < d.nc; ++c) {
+        const float sc = to_f32(states[off_state(d, b, c, h) + e]);
+        s_in[off_state(d, b, c, h) + e] = from_f32<SinT>(cur);
+        cur = fmaf(__ldg(al + c), cur, sc);
+    }
+    if (final_state) final_state[int64_t(bh) * PN + e] = cur;
+}
+
+template <typename ST, typename SinT>
+__global__ void __launch_bounds__(kThreads)
+state_passing_kernel(Dims d, const ST *__restrict__ states, const float *__restrict__ alpha,
+                     const float *__restrict__ h0, SinT *__restrict__ s_in,
+                     float *__restrict__ final_state) {
+    const int64_t PN = int64_t(d.P) * d.N;
+    const int64_t e = (int64_t(blockIdx.x) * kThreads + threadIdx.x) * kVec;
+    const int bh = blockIdx.y;
+    const int b = bh / d.H, h = bh % d.H;
+    if (e >= PN) return;
+    V8 cur;
+    if (h0) load8(h0 + int64_t(bh) * PN + e, cur);
+    else
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) cur.v[i] = 0.f;
     const float *al = alpha + off_alpha(d, b, h, 0);
     for (int c0 = 0; c0 < d.nc; c0 += kPrefetch) {
-        V buf[kPrefetch];
+        V8 buf[kPrefetch];
         float a[kPrefetch];
 #pragma unroll
         for (int k = 0; k < kPrefetch; ++k) {
             if (c0 + k < d.nc) {
-                buf[k] = load_vec(reinterpret_cast<const V *>(states + off_state(d, b, c0 + k, h) + e));
+                load8(states + off_state(d, b, c0 + k, h) + e, buf[k]);
                 a[k] = __ldg(al + c0 + k);
             }
         }
 #pragma unroll
         for (int k = 0; k < kPrefetch; ++k) {
             if (c0 + k < d.nc) {
-                store_vec(s_in + off_state(d, b, c0 + k, h) + e, cur);
-                fma_vec(cur, a[k], buf[k]);
+                store8(s_in + off_state(d, b, c0 + k, h) + e, cur);
+#pragma unroll
+                for (int i = 0; i < kVec; ++i) cur.v[i] = fmaf(a[k], cur.v[i], buf[k].v[i]);
             }
         }
     }
-    if (final_state) store_vec(final_state + int64_t(bh) * PN + e, cur);
+    if (final_state) store8(final_state + int64_t(bh) * PN + e, cur);
 }
 
-template <int VEC, typename SinT>
-cudaError_t launch_sp(const Dims &d, const float *states, const float *alpha, const float *h0,
+template <typename ST, typename SinT>
+cudaError_t launch_sp(const Dims &d, const ST *states, const float *alpha, const float *h0,
                       SinT *s_in, float *final_state, cudaStream_t stream) {
     const int64_t PN = int64_t(d.P) * d.N;
-    dim3 grid(unsigned((PN / VEC + kThreads - 1) / kThreads), unsigned(d.B * d.H));
-    state_passing_kernel<VEC, SinT><<<grid, kThreads, 0, stream>>>(d, states, alpha, h0, s_in,
-                                                                  final_state);
+    if (PN % kVec == 0) {
+        dim3 grid(unsigned((PN / kVec + kThreads - 1) / kThreads), unsigned(d.B * d.H));
+        state_passing_kernel<ST, SinT><<<grid, kThreads, 0, stream>>>(d, states, alpha, h0, s_in,
+                                                                      final_state);
+    } else {
+        dim3 grid(unsigned((PN + kThreads - 1) / kThreads), unsigned(d.B * d.H));
+        state_passing_scalar_kernel<ST, SinT><<<grid, kThreads, 0, stream>>>(d, states, alpha, h0,
+                                                                             s_in, final_state);
+    }
     return cudaGetLastError();
+}
+
+template <typename ST>
+cudaError_t dispatch_out(const Dims &d, const ST *states, const float *alpha, const float *h0,
+                         void *s_in, bool s_in_bf16, float *final_state, cudaStream_t stream) {
+    if (s_in_bf16)
+        return launch_sp(d, states, alpha, h0, static_cast<__nv_bfloat16 *>(s_in), final_state, stream);
+    return launch_sp(d, states, alpha, h0, static_cast<float *>(s_in), final_state, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_state_passing(const Dims &d, const float *states, const float *alpha,
-                                 const float *init_state, void *s_in, bool s_in_bf16,
-                                 float *final_state, cudaStream_t stream) {
-    const bool vec4 = ((int64_t(d.P) * d.N) % 4) == 0;
-    if (s_in_bf16) {
-        auto *p = static_cast<__nv_bfloat16 *>(s_in);
-        return vec4 ? launch_sp<4>(d, states, alpha, init_state, p, final_state, stream)
-                    : launch_sp<1>(d, states, alpha, init_state, p, final_state, stream);
-    }
-    auto *p = static_cast<float *>(s_in);
-    return vec4 ? launch_sp<4>(d, states, alpha, init_state, p, final_state, stream)
-                : launch_sp<1>(d, states, alpha, init_state, p, final_state, stream);
+cudaError_t launch_state_passing(const Dims &d, const void *states, bool states_bf16,
+                                 const float *alpha, const float *init_state, void *s_in,
+                                 bool s_in_bf16, float *final_state, cudaStream_t stream) {
+    if (states_bf16)
+        return dispatch_out(d, static_cast<const __nv_bfloat16 *>(states), alpha, init_state, s_in,
+                            s_in_bf16, final_state, stream);
+    return dispatch_out(d, static_cast<const float *>(states), alpha, init_state, s_in, s_in_bf16,
+                        final_state, stream);
 }
 
 }  // namespace ssd

@@ -279,9 +279,8 @@ cudaError_t launch_n(const Dims &d, const CUtensorMap *maps, int hpc, const floa
     const ScanSmem L = scan_smem(d.Q, N);
     // at least 116 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
     const int smem = int(L.total < 116 * 1024 ? 116 * 1024 : L.total);
-    if (cudaFuncSetAttribute(chunk_scan_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
-        return cudaGetLastError();
+    if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan_tc_kernel<N>), smem))
+        return cudaErrorInvalidValue;
     dim3 grid(d.Q / kRows, d.nc, d.B * (d.H / hpc));
     chunk_scan_tc_kernel<N><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3],
                                                                 d, hpc, dt, D, l, y, err);

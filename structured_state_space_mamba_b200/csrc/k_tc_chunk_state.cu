@@ -7,13 +7,17 @@
 // B_chunk^T X_chunk; the decay weights w and the step dt follow from the
 // recurrence h_t = exp(dt_t A) h_{t-1} + dt_t x_t B_t^T unrolled over the chunk).
 //
-// As one UMMA per CTA: D[m, n] = sum_s A[m, s] Bop[s, n] with
-//   m = (head j, p): two heads of the same group stacked -> M = 128,
-//   A   = (w o X)^T  read MN-major from the x tile [s][p] (TMA, 128B swizzle),
-//   Bop = B          read MN-major from the B tile [s][n] (TMA),
-//   K   = Q tokens, D (fp32) in tensor memory, N = dstate columns.
-// The weights are applied in shared memory (bf16 round trip) between the TMA
-// load and the MMA.  One thread issues the MMAs; four warps drain TMEM.
+// One work unit = (b, c, a pair of heads of one group): one UMMA
+//     D[m, n] = sum_s A[m, s] Bop[s, n],   m = (head j, p) -> M = 128,
+//     A = (w o X)^T read MN-major from the x tile [s][p], Bop = B read MN-major
+//     from the B tile [s][n], K = Q tokens, D in tensor memory (fp32).
+// The kernel is persistent (one CTA per SM walks the units) and warp
+// specialised around a ring of 64-token stages:
+//     warp 0      TMA producer: x rows of both heads + B rows -> stage
+//     warps 2..5  scale each x row by its weight w_s in place (bf16 -> bf16)
+//     warp 1      MMA issuer: 4 UMMAs (K = 16 each) per stage into one of two
+//                 TMEM accumulators; the commit frees the stage
+//     warps 6..9  epilogue: TMEM -> bf16 S_c -> global (overlaps the next unit)
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -25,148 +29,217 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kKS = 64;        // tokens per stage
+constexpr int kStages = 4;
 
-__host__ __device__ constexpr int tmem_cols_for(int n) { return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : 256)); }
+__host__ __device__ constexpr int acc_cols(int ns) { return ns < 16 ? 16 : ns; }
+__host__ __device__ constexpr int tmem_alloc_cols(int ns) {
+    return 2 * acc_cols(ns) <= 32 ? 32 : (2 * acc_cols(ns) <= 64 ? 64 : (2 * acc_cols(ns) <= 128 ? 128 : (2 * acc_cols(ns) <= 256 ? 256 : 512)));
+}
 __host__ __device__ constexpr int brow_bytes(int ns) { return ns >= 64 ? 128 : ns * 2; }
 __host__ __device__ constexpr uint32_t bswz(int ns) { return ns >= 64 ? kSw128 : (ns == 32 ? kSw64 : kSw32); }
+__host__ __device__ constexpr uint32_t x_stage_bytes() { return 2 * kKS * 128; }
+__host__ __device__ constexpr uint32_t b_stage_bytes(int ns) { return kKS * ns * 2; }
+__host__ __device__ constexpr uint32_t stage_bytes(int ns) { return x_stage_bytes() + b_stage_bytes(ns); }
 
-size_t state_smem_bytes(int Q, int NS) {
-    return 1024 /*align slack*/ + size_t(2) * Q * 128 + size_t(Q) * NS * 2 + size_t(2) * Q * 4 + 64;
-}
+size_t state_smem_bytes(int NS) { return 1024 + size_t(kStages) * stage_bytes(NS) + 256; }
 
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                      Dims d, int nh, const float *__restrict__ w, float *__restrict__ states,
-                      unsigned int *err) {
-    constexpr int kCols = tmem_cols_for(NS);
+                      Dims d, int nh, int units, const float *__restrict__ w,
+                      __nv_bfloat16 *__restrict__ states, unsigned int *err) {
+    constexpr int kAcc = acc_cols(NS);
+    constexpr int kCols = tmem_alloc_cols(NS);
     constexpr int kRowB = brow_bytes(NS);
+    if (device_failed(err)) return;  // an earlier wait expired: skip all work
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int Q = d.Q;
-    uint8_t *sX = smem;                           // [2][Q][64] bf16, 128B rows, swizzled
-    uint8_t *sB = smem + 2 * Q * 128;             // [NS/64][Q][64] (or [Q][NS]) bf16, swizzled
-    float *sW = reinterpret_cast<float *>(sB + Q * NS * 2);  // [2][Q]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sW + 2 * Q);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2);
-    __shared__ int s_abort;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * stage_bytes(NS));
+    uint64_t *full = bars, *scaled = bars + kStages, *empty = bars + 2 * kStages;
+    uint64_t *accf = bars + 3 * kStages, *acce = accf + 2, *done = acce + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
 
-    const int c = blockIdx.x, b = blockIdx.z;
-    const int h0 = blockIdx.y * nh;
-    const int g = h0 / d.r;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int trow = b * d.T + c * Q;  // first token row in the [B*T] view
+    const int nhp = d.H / nh;
+    const int ksteps = d.Q / kKS;
 
-    if (device_failed(err)) return;  // an earlier wait expired: skip all work
     if (tid == 0) {
-        s_abort = 0;
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&scaled[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accf[a], 1);
+            mbar_init(&acce[a], 128);
+        }
+        mbar_init(done, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_b);
     }
-    if (warp == 0) tmem_alloc(tmem_holder, kCols);
+    if (warp == 1) tmem_alloc(tmem_holder, kCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (tid == 0) {
-        const uint32_t bytes = uint32_t(nh) * Q * 128 + uint32_t(Q) * NS * 2;
-        mbar_expect_tx(&bars[0], bytes);
-        for (int j = 0; j < nh; ++j) tma_load_3d(sX + j * Q * 128, &tm_x, &bars[0], 0, h0 + j, trow);
-        if (NS >= 64) {
-            for (int s = 0; s < NS / 64; ++s) tma_load_3d(sB + s * Q * 128, &tm_b, &bars[0], s * 64, g, trow);
-        } else {
-            tma_load_3d(sB, &tm_b, &bars[0], 0, g, trow);
-        }
-    }
-    for (int i = tid; i < nh * Q; i += kThreads) sW[i] = __ldg(w + off_lq(d, b, h0 + i / Q, c) + i % Q);
-    if (nh == 1)
-        for (int i = tid; i < Q * 8; i += kThreads)
-            reinterpret_cast<uint4 *>(sX + Q * 128)[i] = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
-
-    if (!mbar_wait(&bars[0], 0, err)) s_abort = 1;
-    // x <- bf16(w_s * x_s): the swizzle permutes 16-byte chunks within a
-    // 128-byte row, so every chunk of row (j, s) takes the same weight.
-    for (int i = tid; i < nh * Q * 8; i += kThreads) {
-        uint4 *p = reinterpret_cast<uint4 *>(sX) + i;
-        const float wv = sW[i >> 3];
-        uint4 v = *p;
-        v.x = pack_bf16x2(bf16lo(v.x) * wv, bf16hi(v.x) * wv);
-        v.y = pack_bf16x2(bf16lo(v.y) * wv, bf16hi(v.y) * wv);
-        v.z = pack_bf16x2(bf16lo(v.z) * wv, bf16hi(v.z) * wv);
-        v.w = pack_bf16x2(bf16lo(v.w) * wv, bf16hi(v.w) * wv);
-        *p = v;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    const bool go = s_abort == 0;
-
-    if (tid == 0 && go) {
-        tc_fence_after();
-        constexpr uint32_t idesc = idesc_bf16_f32(128, NS, 1, 1);
-        const uint32_t xa = smem_u32(sX), ba = smem_u32(sB);
-        for (int k = 0; k < Q / 16; ++k) {
-            const uint64_t ad = smem_desc(xa + k * 16 * 128, Q * 128, 1024, kSw128);
-            const uint64_t bd = smem_desc(ba + k * 16 * kRowB, Q * 128, 8 * kRowB, bswz(NS));
-            mma_bf16_ss(tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars[1]);
-    }
-    __syncthreads();
-    if (go && !mbar_wait(&bars[1], 0, err)) s_abort = 1;
-    tc_fence_after();
-    __syncthreads();
-
-    // epilogue: TMEM lane m = 32*warp + lane holds row (head m/64, p = m%64)
-    const int m = warp * 32 + lane;
-    const int j = m >> 6, p = m & 63;
-    if (s_abort == 0) {
-        const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-        float *dst = states + off_state(d, b, c, h0 + (j < nh ? j : 0)) + int64_t(p) * NS;
-        if (NS >= 32) {
-#pragma unroll 1
-            for (int n0 = 0; n0 < NS; n0 += 32) {
-                float v[32];
-                tmem_ld32(taddr + n0, v);
-                if (j < nh) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        reinterpret_cast<float4 *>(dst + n0)[q] =
-                            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int hp = u % nhp, bc = u / nhp;
+                const int c = bc % d.nc, b = bc / d.nc;
+                const int h0 = hp * nh, g = h0 / d.r;
+                const int trow = b * d.T + c * d.Q;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, err)) { ok = false; break; }
+                    uint8_t *sx = smem + s * stage_bytes(NS);
+                    uint8_t *sb = sx + x_stage_bytes();
+                    mbar_expect_tx(&full[s], uint32_t(nh) * kKS * 128 + b_stage_bytes(NS));
+                    for (int j = 0; j < nh; ++j)
+                        tma_load_3d(sx + j * kKS * 128, &tm_x, &full[s], 0, h0 + j, trow + ks * kKS);
+                    if (NS >= 64) {
+                        for (int sl = 0; sl < NS / 64; ++sl)
+                            tma_load_3d(sb + sl * kKS * 128, &tm_b, &full[s], sl * 64, g, trow + ks * kKS);
+                    } else {
+                        tma_load_3d(sb, &tm_b, &full[s], 0, g, trow + ks * kKS);
+                    }
+                    ++it;
                 }
             }
-        } else {
-            float v[16];
-            tmem_ld16(taddr, v);
-            if (j < nh) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    reinterpret_cast<float4 *>(dst)[q] =
-                        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            // drain: every stage issued must have landed before the CTA exits
+            for (int k = 0; k < kStages && it > 0; ++k, --it) {
+                const uint32_t i = it - 1;
+                mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr);
             }
         }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer --------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, kAcc, 1, 1);
+            uint32_t it = 0, ui = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
+                const int a = ui & 1;
+                if (!mbar_wait(&acce[a], ((ui >> 1) & 1) ^ 1, err)) break;
+                tc_fence_after();
+                const uint32_t dacc = tmem + a * kAcc;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&scaled[s], (it / kStages) & 1, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t xa = smem_u32(smem + s * stage_bytes(NS));
+                    const uint32_t ba = xa + x_stage_bytes();
+#pragma unroll
+                    for (int k = 0; k < kKS / 16; ++k) {
+                        const uint64_t ad = smem_desc(xa + k * 16 * 128, kKS * 128, 1024, kSw128);
+                        const uint64_t bd = smem_desc(ba + k * 16 * kRowB, kKS * 128, 8 * kRowB, bswz(NS));
+                        mma_bf16_ss(dacc, ad, bd, idesc, (ks > 0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&empty[s]);
+                    ++it;
+                }
+                if (ok) mma_commit(&accf[a]);
+            }
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);
+        }
+    } else if (warp < 6) {
+        // ------------------------------ scale x by w -------------------------------
+        const int r = tid - 64;  // row of the stage's x tile: head j = r / 64, token r % 64
+        const int j = r >> 6, sr = r & 63;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int hp = u % nhp, bc = u / nhp;
+            const int c = bc % d.nc, b = bc / d.nc;
+            const int h = hp * nh + (j < nh ? j : 0);
+            const float *wp = w + off_lq(d, b, h, c) + sr;
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int s = it % kStages;
+                const float wv = __ldg(wp + ks * kKS);
+                if (!mbar_wait(&full[s], (it / kStages) & 1, err)) { ok = false; break; }
+                if (j < nh) {
+                    uint8_t *row = smem + s * stage_bytes(NS) + r * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 *p = reinterpret_cast<uint4 *>(row + ((q ^ (r & 7)) << 4));
+                        uint4 v = *p;
+                        v.x = pack_bf16x2(bf16lo(v.x) * wv, bf16hi(v.x) * wv);
+                        v.y = pack_bf16x2(bf16lo(v.y) * wv, bf16hi(v.y) * wv);
+                        v.z = pack_bf16x2(bf16lo(v.z) * wv, bf16hi(v.z) * wv);
+                        v.w = pack_bf16x2(bf16lo(v.w) * wv, bf16hi(v.w) * wv);
+                        *p = v;
+                    }
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(&scaled[s]);
+                ++it;
+            }
+        }
+    } else {
+        // ------------------------------ epilogue ----------------------------------
+        const int qd = warp & 3;
+        const int m = qd * 32 + lane;
+        const int j = m >> 6, p = m & 63;
+        uint32_t ui = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++ui) {
+            const int a = ui & 1;
+            if (!mbar_wait(&accf[a], (ui >> 1) & 1, err)) break;
+            tc_fence_after();
+            const int hp = u % nhp, bc = u / nhp;
+            const int c = bc % d.nc, b = bc / d.nc;
+            const int h = hp * nh + (j < nh ? j : 0);
+            __nv_bfloat16 *dst = states + off_state(d, b, c, h) + int64_t(p) * NS;
+            const uint32_t taddr = tmem + (uint32_t(qd * 32) << 16) + a * kAcc;
+            if (NS >= 32) {
+#pragma unroll 1
+                for (int n0 = 0; n0 < NS; n0 += 32) {
+                    float v[32];
+                    tmem_ld32(taddr + n0, v);
+                    if (j < nh) {
+                        uint4 *o = reinterpret_cast<uint4 *>(dst + n0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                              pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                    }
+                }
+            } else {
+                float v[16];
+                tmem_ld16(taddr, v);
+                if (j < nh) {
+                    uint4 *o = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q)
+                        o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[a]);
+        }
     }
-    // on an abandoned wait, give the copies in flight a bounded chance to land
-    if (tid == 0 && s_abort) mbar_wait(&bars[0], 0, nullptr);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, kCols);
+    if (warp == 1) tmem_dealloc(tmem, kCols);
 }
 
 template <int NS>
 cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb, int nh,
-                      const float *w, float *states, unsigned int *err, cudaStream_t stream) {
-    const size_t smem = state_smem_bytes(d.Q, NS);
-    if (cudaFuncSetAttribute(chunk_state_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem)) != cudaSuccess)
-        return cudaGetLastError();
-    dim3 grid(d.nc, d.H / nh, d.B);
-    chunk_state_tc_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, d, nh, w, states, err);
+                      const float *w, __nv_bfloat16 *states, unsigned int *err, cudaStream_t stream) {
+    const size_t smem = state_smem_bytes(NS);
+    if (!smem_attr_once(reinterpret_cast<const void *>(chunk_state_tc_kernel<NS>), int(smem)))
+        return cudaErrorInvalidValue;
+    const int units = d.B * d.nc * (d.H / nh);
+    const int grid = units < device_sm_count() ? units : device_sm_count();
+    chunk_state_tc_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, d, nh, units, w, states, err);
     return cudaGetLastError();
 }
 
@@ -175,30 +248,31 @@ cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &t
 bool tc_chunk_state_supported(const Dims &d) {
     const bool ns_ok = d.N == 16 || d.N == 32 || d.N == 64 || d.N == 128 || d.N == 256;
     return d.P == 64 && ns_ok && (d.Q == 64 || d.Q == 128 || d.Q == 256) &&
-           state_smem_bytes(d.Q, d.N) <= 227 * 1024;
+           state_smem_bytes(d.N) <= 227 * 1024 && int64_t(d.B) * d.nc * d.H < (int64_t(1) << 31);
 }
 
 cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, const float *w,
-                                  float *states, unsigned int *err, cudaStream_t stream) {
-    // x viewed as [B*T rows][H][P]; box = one head, Q tokens
+                                  void *states_bf16, unsigned int *err, cudaStream_t stream) {
+    // x viewed as [B*T rows][H][P]; box = one head, 64 tokens
     const uint64_t xdims[3] = {uint64_t(d.P), uint64_t(d.H), uint64_t(d.B) * d.T};
     const uint64_t xstr[2] = {uint64_t(d.P) * 2, uint64_t(d.H) * d.P * 2};
-    const uint32_t xbox[3] = {64, 1, uint32_t(d.Q)};
-    // B viewed as [B*T rows][G][N]; box = one group, Q tokens, a 64-wide slab of N
+    const uint32_t xbox[3] = {64, 1, uint32_t(kKS)};
+    // B viewed as [B*T rows][G][N]; box = one group, 64 tokens, a 64-wide slab of N
     const uint64_t bdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
     const uint64_t bstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
-    const uint32_t bbox[3] = {uint32_t(d.N >= 64 ? 64 : d.N), 1, uint32_t(d.Q)};
+    const uint32_t bbox[3] = {uint32_t(d.N >= 64 ? 64 : d.N), 1, uint32_t(kKS)};
     CUtensorMap tx, tb;
     if (!make_tmap_bf16(&tx, 3, x, xdims, xstr, xbox, 128) ||
         !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)))
         return cudaErrorInvalidValue;
     const int nh = (d.r % 2 == 0) ? 2 : 1;
+    auto *st = static_cast<__nv_bfloat16 *>(states_bf16);
     switch (d.N) {
-        case 16: return launch_ns<16>(d, tx, tb, nh, w, states, err, stream);
-        case 32: return launch_ns<32>(d, tx, tb, nh, w, states, err, stream);
-        case 64: return launch_ns<64>(d, tx, tb, nh, w, states, err, stream);
-        case 128: return launch_ns<128>(d, tx, tb, nh, w, states, err, stream);
-        case 256: return launch_ns<256>(d, tx, tb, nh, w, states, err, stream);
+        case 16: return launch_ns<16>(d, tx, tb, nh, w, st, err, stream);
+        case 32: return launch_ns<32>(d, tx, tb, nh, w, st, err, stream);
+        case 64: return launch_ns<64>(d, tx, tb, nh, w, st, err, stream);
+        case 128: return launch_ns<128>(d, tx, tb, nh, w, st, err, stream);
+        case 256: return launch_ns<256>(d, tx, tb, nh, w, st, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -11,11 +11,12 @@ namespace ssd {
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *alpha, cudaStream_t stream);
 
-// ssd_state_passing: states [B,nc,H,P,N] fp32, alpha -> s_in [B,nc,H,P,N]
-// (fp32 or bf16 per s_in_bf16), final state [B,H,P,N] fp32 (may be NULL)
-cudaError_t launch_state_passing(const Dims &d, const float *states, const float *alpha,
-                                 const float *init_state, void *s_in, bool s_in_bf16,
-                                 float *final_state, cudaStream_t stream);
+// ssd_state_passing: states [B,nc,H,P,N] (fp32 or bf16 per states_bf16), alpha
+// -> s_in [B,nc,H,P,N] (fp32 or bf16 per s_in_bf16), final state [B,H,P,N] fp32
+// (may be NULL)
+cudaError_t launch_state_passing(const Dims &d, const void *states, bool states_bf16,
+                                 const float *alpha, const float *init_state, void *s_in,
+                                 bool s_in_bf16, float *final_state, cudaStream_t stream);
 
 // CUDA-core (SIMT) chunk state and chunk scan, any supported shape.
 // bf16 selects the storage type of x/B/C/y.  s_in is fp32 here.
@@ -32,7 +33,7 @@ bool tc_chunk_scan_supported(const Dims &d);
 // `err` is a device word: bit 0 is set when a bounded wait inside a kernel
 // expired (the kernel then skips its remaining work and exits cleanly).
 cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, const float *w,
-                                  float *states, unsigned int *err, cudaStream_t stream);
+                                  void *states_bf16, unsigned int *err, cudaStream_t stream);
 cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
                                  const void *Cm, const float *D, const float *l,
                                  const void *s_in_bf16, void *y, unsigned int *err,

@@ -94,7 +94,9 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.l_offset = off; off = align_up(off + lq);
     w.w_offset = off; off = align_up(off + lq);
     w.alpha_offset = off; off = align_up(off + al);
-    w.states_offset = off; off = align_up(off + st * sizeof(float));
+    w.states_offset = off;
+    w.states_dtype = plan->tc_state ? SSD_BF16 : SSD_F32;
+    off = align_up(off + st * (plan->tc_state ? 2 : 4));
     w.s_in_offset = off;
     w.s_in_dtype = plan->tc_scan ? SSD_BF16 : SSD_F32;
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
@@ -136,7 +138,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     float *l = reinterpret_cast<float *>(ws + pl.ws.l_offset);
     float *w = reinterpret_cast<float *>(ws + pl.ws.w_offset);
     float *alpha = reinterpret_cast<float *>(ws + pl.ws.alpha_offset);
-    float *states = reinterpret_cast<float *>(ws + pl.ws.states_offset);
+    void *states = ws + pl.ws.states_offset;
     void *s_in = ws + pl.ws.s_in_offset;
     for (int stage = 0; stage < 4; ++stage) {
         if (only_stage >= 0 && stage != only_stage) continue;
@@ -147,11 +149,12 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, err, stream)
-                                : ssd::launch_chunk_state_simt(d, pl.bf16, x, Bm, w, states, stream);
+                                : ssd::launch_chunk_state_simt(d, pl.bf16, x, Bm, w,
+                                                               static_cast<float *>(states), stream);
                 break;
             case SSD_STAGE_STATE_PASSING:
-                e = ssd::launch_state_passing(d, states, alpha, init_state, s_in, pl.tc_scan, fin,
-                                              stream);
+                e = ssd::launch_state_passing(d, states, pl.tc_state, alpha, init_state, s_in,
+                                              pl.tc_scan, fin, stream);
                 break;
             case SSD_STAGE_CHUNK_SCAN:
                 e = pl.tc_scan

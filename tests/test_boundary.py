@@ -68,7 +68,8 @@ def test_workspace_layout(lib):
     assert lay.w_offset >= 2 * 8 * nc * 128 * 4
     assert lay.states_offset % 256 == 0 and lay.s_in_offset % 256 == 0
     state_elems = 2 * nc * 8 * 64 * 128
-    assert lay.s_in_offset >= lay.states_offset + state_elems * 4
+    ssz = 2 if lay.states_dtype == binding.SSD_BF16 else 4
+    assert lay.s_in_offset >= lay.states_offset + state_elems * ssz
     sz = 2 if lay.s_in_dtype == binding.SSD_BF16 else 4
     assert lay.total_bytes >= lay.s_in_offset + state_elems * sz
     assert lay.launches == 4

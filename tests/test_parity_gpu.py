@@ -181,7 +181,8 @@ def test_workspace_entry_point_and_intermediates(oracle):
     l = view(lay.l_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
     w = view(lay.w_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
     al = view(lay.alpha_offset, 4 * nc, torch.float32).double().cpu().numpy().reshape(1, 4, nc)
-    S = view(lay.states_offset, nc * 4 * 64 * 128, torch.float32).double().cpu().numpy()
+    stdt = torch.bfloat16 if lay.states_dtype == binding.SSD_BF16 else torch.float32
+    S = view(lay.states_offset, nc * 4 * 64 * 128, stdt).double().cpu().numpy()
     sdt = torch.bfloat16 if lay.s_in_dtype == binding.SSD_BF16 else torch.float32
     s_in = view(lay.s_in_offset, nc * 4 * 64 * 128, sdt).double().cpu().numpy()
     assert rel(l, it["l"]) < 1e-5          # ssd_chunk_cumsum
