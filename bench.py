@@ -225,7 +225,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    inp = make_workload(args.workload)
+    inp = make_workload(args.workload, **({"batch": cfg["batch"]} if args.batch else {}))
     tt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
     host = dict(x=(inp.x, tt), dt=(inp.dt, torch.float32), A=(inp.A, torch.float32),
                 B=(inp.B, tt), C=(inp.C, tt), D=(inp.D, torch.float32))
@@ -398,11 +398,15 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = dict(WORKLOADS[args.workload])
     cfg.setdefault("final_state", True)
+    if args.batch is not None:
+        cfg["batch"] = args.batch
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -152,6 +152,9 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * Where each intermediate sits inside the workspace (byte offsets; nc = T/Q):
  *   l      fp32 [B, H, nc, Q]  chunk-local inclusive cumsum of dt*A
  *   w      fp32 [B, H, nc, Q]  exp(l_last - l_s) * dt_s (chunk-state weights)
+ *   dtq    fp32 [B, H, nc, Q]  dt regrouped per chunk and head
+ *   beta   fp32 [B, H, nc, Q]  exp(l_{32k+31} - l_s) * dt_s, k = s / 32 (source
+ *                              factors of the factored in-chunk decay)
  *   alpha  fp32 [B, H, nc]     exp(l_last), the decay across a whole chunk
  *   states [B, nc, H, P, N]    per-chunk states S_c = sum_s w_s x_s B_s^T;
  *                              element type given by states_dtype
@@ -162,7 +165,7 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  */
 typedef struct {
     size_t total_bytes;
-    size_t l_offset, w_offset, alpha_offset, states_offset, s_in_offset;
+    size_t l_offset, w_offset, dtq_offset, beta_offset, alpha_offset, states_offset, s_in_offset;
     int32_t s_in_dtype;
     int32_t tensor_core;
     int32_t launches;

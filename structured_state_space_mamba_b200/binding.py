@@ -34,7 +34,9 @@ class Dims(ctypes.Structure):
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("l_offset", ctypes.c_size_t),
-                ("w_offset", ctypes.c_size_t), ("alpha_offset", ctypes.c_size_t),
+                ("w_offset", ctypes.c_size_t), ("dtq_offset", ctypes.c_size_t),
+                ("beta_offset", ctypes.c_size_t),
+                ("alpha_offset", ctypes.c_size_t),
                 ("states_offset", ctypes.c_size_t), ("s_in_offset", ctypes.c_size_t),
                 ("s_in_dtype", ctypes.c_int32), ("tensor_core", ctypes.c_int32),
                 ("launches", ctypes.c_int32), ("states_dtype", ctypes.c_int32)]

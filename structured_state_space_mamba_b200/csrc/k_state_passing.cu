@@ -10,21 +10,21 @@
 //
 // Every element of the P x N state is an independent scalar recurrence, so the
 // kernel is parallel over (b, h, element) and sequential only over chunks.
-// Each thread owns VEC consecutive elements; the loads of S_c do not depend on
-// the running state, so they are issued kPrefetch chunks ahead and the loop is
+// Each thread owns 8 consecutive elements; the loads of S_c do not depend on
+// the running state, so they are issued several chunks ahead and the loop is
 // bound by HBM bandwidth rather than by latency.  The running sum stays fp32
 // in registers; s_in is stored as fp32 or bf16 (the tensor-core scan consumes
 // bf16).
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace ssd {
 
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kPrefetch = 8;
-constexpr int kVec = 8;  // state elements per thread
+constexpr int kVec = 8;  // state elements per thread (one 16-byte bf16 load)
 
 // kVec consecutive fp32 values in registers
 struct V8 {
@@ -80,8 +80,11 @@ state_passing_scalar_kernel(Dims d, const ST *__restrict__ states, const float *
     if (final_state) final_state[int64_t(bh) * PN + e] = cur;
 }
 
-template <typename ST, typename SinT>
-__global__ void __launch_bounds__(kThreads)
+// kPrefetch chunks are loaded ahead: 4 with three CTAs per SM when the grid
+// fills the GPU, 16 with one CTA per SM when it does not (few (b, h) chains,
+// long sequences), so that enough bytes are in flight either way.
+template <typename ST, typename SinT, int kPrefetch, int kMinBlocks>
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 state_passing_kernel(Dims d, const ST *__restrict__ states, const float *__restrict__ alpha,
                      const float *__restrict__ h0, SinT *__restrict__ s_in,
                      float *__restrict__ final_state) {
@@ -96,24 +99,29 @@ state_passing_kernel(Dims d, const ST *__restrict__ states, const float *__restr
 #pragma unroll
         for (int i = 0; i < kVec; ++i) cur.v[i] = 0.f;
     const float *al = alpha + off_alpha(d, b, h, 0);
+    const int64_t cstride = int64_t(d.H) * PN;  // elements between consecutive chunks
+    const ST *sp = states + off_state(d, b, 0, h) + e;
+    SinT *op = s_in + off_state(d, b, 0, h) + e;
     for (int c0 = 0; c0 < d.nc; c0 += kPrefetch) {
         V8 buf[kPrefetch];
         float a[kPrefetch];
 #pragma unroll
         for (int k = 0; k < kPrefetch; ++k) {
             if (c0 + k < d.nc) {
-                load8(states + off_state(d, b, c0 + k, h) + e, buf[k]);
+                load8(sp + k * cstride, buf[k]);
                 a[k] = __ldg(al + c0 + k);
             }
         }
 #pragma unroll
         for (int k = 0; k < kPrefetch; ++k) {
             if (c0 + k < d.nc) {
-                store8(s_in + off_state(d, b, c0 + k, h) + e, cur);
+                store8(op + k * cstride, cur);
 #pragma unroll
                 for (int i = 0; i < kVec; ++i) cur.v[i] = fmaf(a[k], cur.v[i], buf[k].v[i]);
             }
         }
+        sp += kPrefetch * cstride;
+        op += kPrefetch * cstride;
     }
     if (final_state) store8(final_state + int64_t(bh) * PN + e, cur);
 }
@@ -124,8 +132,13 @@ cudaError_t launch_sp(const Dims &d, const ST *states, const float *alpha, const
     const int64_t PN = int64_t(d.P) * d.N;
     if (PN % kVec == 0) {
         dim3 grid(unsigned((PN / kVec + kThreads - 1) / kThreads), unsigned(d.B * d.H));
-        state_passing_kernel<ST, SinT><<<grid, kThreads, 0, stream>>>(d, states, alpha, h0, s_in,
-                                                                      final_state);
+        const int64_t threads = int64_t(grid.x) * grid.y * kThreads;
+        if (threads >= int64_t(device_sm_count()) * 3 * kThreads)
+            state_passing_kernel<ST, SinT, 4, 3><<<grid, kThreads, 0, stream>>>(
+                d, states, alpha, h0, s_in, final_state);
+        else
+            state_passing_kernel<ST, SinT, 16, 1><<<grid, kThreads, 0, stream>>>(
+                d, states, alpha, h0, s_in, final_state);
     } else {
         dim3 grid(unsigned((PN + kThreads - 1) / kThreads), unsigned(d.B * d.H));
         state_passing_scalar_kernel<ST, SinT><<<grid, kThreads, 0, stream>>>(d, states, alpha, h0,

@@ -1,0 +1,548 @@
+// k_tc_chunk_scan4.cu -- ssd_chunk_scan on the tensor cores: persistent, warp
+// specialised, double-buffered scores and accumulators (dstate <= 128).
+//
+// Output, for the rows t of the 128-token tile [t0, t0 + 128) of chunk c:
+//     y_t = exp(l_t) C_t s_in^T + sum_{s <= t} exp(l_t - l_s) dt_s (C_t . B_s) x_s + D_h x_t
+// (the intra-chunk masked product (L o C B^T)(dt o X) of the chunked SSD
+// algorithm -- aifetchly blog "Mamba-2 Architecture", "The Chunked SSD
+// Algorithm", step 1; akillness.github.io "State Space Duality and Mamba-2",
+// "The Scalar-Identity Structural Constraint" -- plus the state carried in from
+// earlier chunks and the skip term).
+//
+// Split of the source tokens s at the tile start t0, with r = l_{t0-1} (r = 0
+// for the first tile) and u_t = exp(l_t - r) <= 1:
+//   * s < t0:  exp(l_t - l_s) = u_t exp(r - l_s), both factors <= 1, so
+//         sum_{s<t0} = u_t (C B^T)[t, s<t0] (g o X)[s<t0],  g_s = exp(r - l_s) dt_s;
+//     the block CBoff = (C B^T)[tile, s<t0] needs no mask and serves every head.
+//   * state term:  exp(l_t) C_t s_in = u_t C_t (exp(r) s_in).
+//   * t0 <= s <= t:  the 128 x 128 diagonal tile keeps its mask, built per head.
+// So  y = Yd + u_t Yoz,  Yd = P Xd,  Yoz = CBoff X' + C S'^T,  with
+//   P  = masked diagonal scores in bf16 (+ D_h on the diagonal: the skip term),
+//   X' = g o X[s < t0],  S' = exp(r) s_in.
+//
+// Decay factors inside the diagonal tile, per 32 x 32 block:
+//   * blocks entirely below the diagonal: exp(l_t - l_s) = exp(l_t - l_k) beta_s,
+//     l_k the last l of the source block, beta_s = exp(l_k - l_s) dt_s (both <= 1);
+//   * blocks on the diagonal: exp(l_t - l_s) = exp(l_t - l_f) exp(l_f - l_s),
+//     l_f the first l of the block, when the block's decay range l_f - l_last is
+//     below 80 (the second factor then stays below e^80); otherwise the exact
+//     exp(l_t - l_s) per element.
+//
+// Tensor memory: [0,128) CB diagonal tile (fp32); [128,256) two score buffers
+// (bf16; at the start of a unit this range holds CBoff in fp32); [256,512) two
+// accumulators {Yd, Yoz}.  Shared memory: C and CBoff (bf16, A operands of the
+// Yoz MMAs), the per-head stages {x rows, s_in, l, dt, beta}, and a staging
+// tile for y, written back with a TMA store.
+//
+// Roles (14 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 scores,
+// warps 10..13 epilogue.
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "tma_host.h"
+
+namespace ssd {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 448;
+constexpr int kRows = 128;
+constexpr int kScoreThreads = 256;
+constexpr int kEpiThreads = 128;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kColCBd = 0, kColP = 128, kColTmp = 128, kColAcc = 256;
+
+__host__ __device__ constexpr int row_bytes(int n) { return n >= 64 ? 128 : n * 2; }
+__host__ __device__ constexpr uint32_t kmajor_swz(int n) { return n >= 64 ? kSw128 : (n == 32 ? kSw64 : kSw32); }
+__host__ __device__ constexpr uint32_t up1k(uint32_t v) { return (v + 1023u) & ~1023u; }
+__host__ __device__ constexpr uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
+
+struct Smem4 {
+    uint32_t c_off, b_off, stage_off, stage_bytes, x_rel, s_rel, l_rel, dt_rel, beta_rel;
+    uint32_t y_off, e_off, bar_off, total;
+};
+
+__host__ __device__ inline Smem4 scan4_smem(int Q, int N) {
+    Smem4 s;
+    s.c_off = 0;
+    s.b_off = up1k(kRows * N * 2);
+    // B rows for the CB MMAs; afterwards CBoff (128 x 128 bf16) in the same place
+    s.stage_off = s.b_off + up1k(umax(Q * N * 2, Q > kRows ? kRows * kRows * 2 : 0));
+    s.x_rel = 0;
+    s.s_rel = Q * 128;
+    s.l_rel = s.s_rel + up1k(64 * N * 2);
+    s.dt_rel = s.l_rel + Q * 4;
+    s.beta_rel = s.dt_rel + Q * 4;
+    s.stage_bytes = up1k(s.beta_rel + Q * 4);
+    s.y_off = s.stage_off + 2 * s.stage_bytes;
+    s.e_off = s.y_off + kRows * 128;
+    s.bar_off = s.e_off + 2 * kRows * 4;
+    s.total = s.bar_off + 256 + 1024;
+    return s;
+}
+
+// K-major operand descriptor for K step k of a tile split into 64-column slabs
+// of `rows` rows (N >= 64) or a single slab of narrower rows (N = 16, 32).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int k, int rows, int n) {
+    if (n >= 64) return smem_desc(base + (k >> 2) * rows * 128 + (k & 3) * 32, 16, 1024, kSw128);
+    return smem_desc(base + k * 32, 16, 8 * row_bytes(n), kmajor_swz(n));
+}
+
+// Scale every bf16 of `n16` 16-byte chunks starting at `p` by f(chunk index);
+// thread i handles chunks i, i + nthr, ...
+template <typename F>
+__device__ __forceinline__ void scale_chunks(uint8_t *p, int n16, int i, int nthr, F f) {
+    for (int k = i; k < n16; k += nthr) {
+        const float sc = f(k);
+        uint4 *q = reinterpret_cast<uint4 *>(p) + k;
+        uint4 v = *q;
+        v.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
+        v.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
+        v.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
+        v.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
+        *q = v;
+    }
+}
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_s,
+                   const __grid_constant__ CUtensorMap tm_y, Dims d, int hpc, int units,
+                   const float *__restrict__ dtq, const float *__restrict__ betaq,
+                   const float *__restrict__ Dskip, const float *__restrict__ lcum,
+                   unsigned int *err) {
+    if (device_failed(err)) return;  // an earlier wait expired: skip all work
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int Q = d.Q;
+    const Smem4 L = scan4_smem(Q, N);
+    uint8_t *sC = smem + L.c_off;
+    uint8_t *sB = smem + L.b_off;  // B rows, then CBoff
+    uint8_t *sY = smem + L.y_off;
+    float *sE = reinterpret_cast<float *>(smem + L.e_off);  // [2][128] row factors u_t
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
+    uint64_t *ld_cb = bars + 0, *cb_full = bars + 1, *cb_smem_free = bars + 2, *cvt_done = bars + 3;
+    uint64_t *head_full = bars + 4, *head_free = bars + 6;      // [2]
+    uint64_t *scores_ready = bars + 8, *p_free = bars + 10;     // [2]
+    uint64_t *acc_full = bars + 12, *acc_free = bars + 14;      // [2]
+    uint64_t *y_ready = bars + 16, *y_free = bars + 17, *done = bars + 18;
+    uint64_t *scaled_ready = bars + 19;                         // [2]
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 21);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ntiles = Q / kRows;
+    const int nhb = d.H / hpc;
+    constexpr int kSlabs = N >= 64 ? N / 64 : 1;
+    constexpr int kRB = row_bytes(N);
+
+    if (tid == 0) {
+        mbar_init(ld_cb, 1);
+        mbar_init(cb_full, 1);
+        mbar_init(cb_smem_free, 1);
+        mbar_init(cvt_done, kScoreThreads);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&head_full[i], 1);
+            mbar_init(&head_free[i], 1);
+            mbar_init(&scores_ready[i], kScoreThreads);
+            mbar_init(&p_free[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_free[i], kEpiThreads);
+            mbar_init(&scaled_ready[i], kScoreThreads);
+        }
+        mbar_init(y_ready, kEpiThreads);
+        mbar_init(y_free, 1);
+        mbar_init(done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_c);
+        tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_s);
+        tma_prefetch_desc(&tm_y);
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 0) {
+        // =============================== producer ===============================
+        if (lane == 0) {
+            uint32_t ui = 0, hit = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
+                const int hb = u % nhb;
+                const int rest = u / nhb;
+                const int mt = rest % ntiles;
+                const int bc = rest / ntiles;
+                const int c = bc % d.nc, b = bc / d.nc;
+                const int h0 = hb * hpc, g = h0 / d.r;
+                const int s_len = (mt + 1) * kRows;
+                const int trow0 = b * d.T + c * Q;
+                // C and B of this unit, once the previous unit's MMAs are done
+                if (!mbar_wait(cb_smem_free, (ui & 1) ^ 1, err)) break;
+                mbar_expect_tx(ld_cb, uint32_t(kRows) * N * 2 + uint32_t(s_len) * N * 2);
+                for (int sl = 0; sl < kSlabs; ++sl) {
+                    tma_load_3d(sC + sl * kRows * 128, &tm_c, ld_cb, sl * 64, g, trow0 + mt * kRows);
+                    for (int i = 0; i <= mt; ++i)
+                        tma_load_3d(sB + sl * s_len * 128 + i * kRows * kRB, &tm_b, ld_cb, sl * 64, g,
+                                    trow0 + i * kRows);
+                }
+                for (int hi = 0; hi < hpc; ++hi, ++hit) {
+                    const int st = hit & 1;
+                    const int h = h0 + hi;
+                    if (!mbar_wait(&head_free[st], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
+                    uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
+                    mbar_expect_tx(&head_full[st], uint32_t(s_len) * 128 + 64u * N * 2 + 3u * s_len * 4);
+                    for (int i = 0; i <= mt; ++i)
+                        tma_load_3d(stage + L.x_rel + i * kRows * 128, &tm_x, &head_full[st], 0, h,
+                                    trow0 + i * kRows);
+                    const int srow = ((b * d.nc + c) * d.H + h) * 64;
+                    for (int sl = 0; sl < kSlabs; ++sl)
+                        tma_load_2d(stage + L.s_rel + sl * 64 * 128, &tm_s, &head_full[st], sl * 64, srow);
+                    const int64_t lo = off_lq(d, b, h, c);
+                    bulk_load(stage + L.l_rel, lcum + lo, s_len * 4, &head_full[st]);
+                    bulk_load(stage + L.dt_rel, dtq + lo, s_len * 4, &head_full[st]);
+                    bulk_load(stage + L.beta_rel, betaq + lo, s_len * 4, &head_full[st]);
+                }
+            }
+            // drain: the last loads issued must have landed before the CTA exits
+            if (ui > 0) mbar_wait(ld_cb, (ui - 1) & 1, nullptr);
+            for (uint32_t k = 0; k < 2 && k < hit; ++k) {
+                const uint32_t i = hit - 1 - k;
+                mbar_wait(&head_full[i & 1], (i >> 1) & 1, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer =============================
+        if (lane == 0) {
+            uint32_t ui = 0, hit = 0;
+            bool ok = true;
+            const uint32_t ca = smem_u32(sC), ba = smem_u32(sB);
+            const uint32_t idCB = idesc_bf16_f32(kRows, kRows, 0, 0);
+            const uint32_t idX = idesc_bf16_f32(kRows, 64, 0, 1);
+            const uint32_t idS = idesc_bf16_f32(kRows, 64, 0, 0);
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
+                const int mt = (u / nhb) % ntiles;
+                const int s_len = (mt + 1) * kRows;
+                if (!mbar_wait(ld_cb, ui & 1, err)) break;
+                tc_fence_after();
+                // CB on the diagonal tile (B rows [t0, t0 + 128)) and, for t0 > 0,
+                // CB of the sources before the tile (B rows [0, 128)) into the score range
+                const uint32_t bdiag = ba + mt * kRows * kRB;
+                for (int k = 0; k < N / 16; ++k)
+                    mma_bf16_ss(tmem + kColCBd, kmajor_desc(ca, k, kRows, N),
+                                kmajor_desc(bdiag, k, s_len, N), idCB, k > 0 ? 1u : 0u);
+                if (mt > 0)
+                    for (int k = 0; k < N / 16; ++k)
+                        mma_bf16_ss(tmem + kColTmp, kmajor_desc(ca, k, kRows, N),
+                                    kmajor_desc(ba, k, s_len, N), idCB, k > 0 ? 1u : 0u);
+                mma_commit(cb_full);
+                for (int hi = 0; hi < hpc; ++hi, ++hit) {
+                    const int st = hit & 1, pb = hit & 1, ab = hit & 1;
+                    // Yoz first: it needs only the scaled operands, so it runs on the
+                    // tensor cores while the score warps still build P
+                    if (!mbar_wait(&head_full[st], (hit >> 1) & 1, err) ||
+                        !mbar_wait(&scaled_ready[st], (hit >> 1) & 1, err) ||
+                        !mbar_wait(&acc_free[ab], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
+                    const uint32_t xa = smem_u32(stage + L.x_rel);
+                    const uint32_t sa = smem_u32(stage + L.s_rel);
+                    const uint32_t dYd = tmem + kColAcc + ab * 128, dYo = dYd + 64;
+                    // Yoz = CBoff X' + C S'^T
+                    if (mt > 0)
+                        for (int k = 0; k < kRows / 16; ++k)
+                            mma_bf16_ss(dYo, kmajor_desc(ba, k, kRows, kRows),
+                                        smem_desc(xa + k * 2048, 16, 1024, kSw128), idX, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < N / 16; ++k)
+                        mma_bf16_ss(dYo, kmajor_desc(ca, k, kRows, N), kmajor_desc(sa, k, 64, N), idS,
+                                    (mt > 0 || k > 0) ? 1u : 0u);
+                    // Yd = P Xd
+                    if (!mbar_wait(&scores_ready[pb], (hit >> 1) & 1, err)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int k = 0; k < kRows / 16; ++k)
+                        mma_bf16_ts(dYd, tmem + kColP + pb * 64 + k * 8,
+                                    smem_desc(xa + mt * kRows * 128 + k * 2048, 16, 1024, kSw128), idX,
+                                    k > 0 ? 1u : 0u);
+                    mma_commit(&p_free[pb]);
+                    mma_commit(&acc_full[ab]);
+                    mma_commit(&head_free[st]);
+                }
+                if (ok) mma_commit(cb_smem_free);
+            }
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);
+        }
+    } else if (warp < 10) {
+        // ================================ scores ================================
+        const int sid = tid - 64;            // 0..255
+        const int qd = warp & 3;             // TMEM lane quarter of this warp
+        const int half = (warp - 2) >> 2;    // which half of the tile's columns
+        const int t_local = qd * 32 + lane;  // row of the tile
+        const uint32_t lane_base = uint32_t(qd * 32) << 16;
+        uint32_t ui = 0, hit = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
+            const int hb = u % nhb;
+            const int mt = (u / nhb) % ntiles;
+            const int t0 = mt * kRows;
+            if (!mbar_wait(cb_full, ui & 1, err)) break;
+            tc_fence_after();
+            if (mt > 0) {
+                // CBoff fp32 -> bf16, into shared memory as a K-major, 128B-swizzled
+                // A operand: this thread packs row t_local, columns [64 half, 64 half + 64)
+                uint8_t *slab = sB + half * (kRows * 128);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + kColTmp + half * 64 + q * 32, v);
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4)
+                        *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, q * 4 + c4)) =
+                            make_uint4(pack_bf16x2(v[8 * c4], v[8 * c4 + 1]),
+                                       pack_bf16x2(v[8 * c4 + 2], v[8 * c4 + 3]),
+                                       pack_bf16x2(v[8 * c4 + 4], v[8 * c4 + 5]),
+                                       pack_bf16x2(v[8 * c4 + 6], v[8 * c4 + 7]));
+                }
+                fence_proxy_async_smem();
+            }
+            // every score thread is done with the CBoff range before any score
+            // buffer (same tensor-memory columns) is written
+            tc_fence_before();
+            mbar_arrive(cvt_done);
+            if (!mbar_wait(cvt_done, ui & 1, err)) break;
+            tc_fence_after();
+            for (int hi = 0; hi < hpc; ++hi, ++hit) {
+                const int st = hit & 1, pb = hit & 1, ab = hit & 1;
+                const int h = hb * hpc + hi;
+                const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
+                uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
+                const float *sl_ = reinterpret_cast<const float *>(stage + L.l_rel);
+                const float *sdt = reinterpret_cast<const float *>(stage + L.dt_rel);
+                const float *beta = reinterpret_cast<const float *>(stage + L.beta_rel);
+                if (!mbar_wait(&head_full[st], (hit >> 1) & 1, err)) { ok = false; break; }
+                const float r = t0 > 0 ? sl_[t0 - 1] : 0.f;
+                if (t0 > 0) {
+                    // X' = g o X for sources before the tile, S' = exp(r) s_in
+                    scale_chunks(stage + L.x_rel, t0 * 8, sid, kScoreThreads, [&](int k) {
+                        const int s = k >> 3;
+                        return __expf(r - sl_[s]) * sdt[s];
+                    });
+                    const float er = __expf(r);
+                    scale_chunks(stage + L.s_rel, 64 * N * 2 / 16, sid, kScoreThreads,
+                                 [&](int) { return er; });
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(&scaled_ready[st]);
+                // row factors for the epilogue (its previous use of sE[ab] has ended
+                // once accumulator ab is free)
+                if (!mbar_wait(&acc_free[ab], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
+                if (sid < kRows) sE[ab * kRows + sid] = __expf(sl_[t0 + sid] - r);
+                if (!mbar_wait(&p_free[pb], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
+                tc_fence_after();
+                const float lt = sl_[t0 + t_local];
+                // both 32-column blocks of this thread's half-row: issue the TMEM
+                // loads together (one wait), skipping blocks above the diagonal
+                uint32_t raw[2][32];
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk)
+                    if (half * 64 + blk * 32 <= qd * 32)
+                        tmem_ld32_nowait(tmem + lane_base + kColCBd + half * 64 + blk * 32, raw[blk]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int j0 = half * 64 + blk * 32;  // first column within the tile
+                    uint32_t pk[16];
+                    const uint32_t *v = raw[blk];
+                    if (j0 > qd * 32) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else if (j0 == qd * 32) {
+                        // block on the diagonal (warp-uniform branch)
+                        const float lf = sl_[t0 + j0], ll = sl_[t0 + j0 + 31];
+                        if (lf - ll < 80.f) {
+                            const float at = __expf(lt - lf);
+                            const float bl = __expf(lf - sl_[t0 + j0 + lane]) * sdt[t0 + j0 + lane];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = j0 + 2 * e;
+                                const float b0 = __shfl_sync(0xffffffffu, bl, 2 * e);
+                                const float b1 = __shfl_sync(0xffffffffu, bl, 2 * e + 1);
+                                float p0 = j <= t_local ? __uint_as_float(v[2 * e]) * at * b0 : 0.f;
+                                float p1 = j + 1 <= t_local ? __uint_as_float(v[2 * e + 1]) * at * b1 : 0.f;
+                                if (j == t_local) p0 += Dh;
+                                if (j + 1 == t_local) p1 += Dh;
+                                pk[e] = pack_bf16x2(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int j = j0 + 2 * e;
+                                float p0 = j <= t_local ? __uint_as_float(v[2 * e]) * __expf(lt - sl_[t0 + j]) * sdt[t0 + j] : 0.f;
+                                float p1 = j + 1 <= t_local ? __uint_as_float(v[2 * e + 1]) * __expf(lt - sl_[t0 + j + 1]) * sdt[t0 + j + 1] : 0.f;
+                                if (j == t_local) p0 += Dh;
+                                if (j + 1 == t_local) p1 += Dh;
+                                pk[e] = pack_bf16x2(p0, p1);
+                            }
+                        }
+                    } else {
+                        // block entirely below the diagonal
+                        const float at = __expf(lt - sl_[t0 + j0 + 31]);
+                        const float4 *b4 = reinterpret_cast<const float4 *>(beta + t0 + j0);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 bb = b4[e];
+                            pk[2 * e] = pack_bf16x2(__uint_as_float(v[4 * e]) * at * bb.x,
+                                                    __uint_as_float(v[4 * e + 1]) * at * bb.y);
+                            pk[2 * e + 1] = pack_bf16x2(__uint_as_float(v[4 * e + 2]) * at * bb.z,
+                                                        __uint_as_float(v[4 * e + 3]) * at * bb.w);
+                        }
+                    }
+                    tmem_st16(tmem + lane_base + kColP + pb * 64 + (j0 >> 1), pk);
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&scores_ready[pb]);
+            }
+        }
+    } else {
+        // =============================== epilogue ===============================
+        const int qd = warp & 3;
+        const int t_local = qd * 32 + lane;
+        const uint32_t lane_base = uint32_t(qd * 32) << 16;
+        const bool issuer = (warp == 10 && lane == 0);
+        uint32_t hit = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int hb = u % nhb;
+            const int rest = u / nhb;
+            const int mt = rest % ntiles;
+            const int bc = rest / ntiles;
+            const int c = bc % d.nc, b = bc / d.nc;
+            for (int hi = 0; hi < hpc; ++hi, ++hit) {
+                const int ab = hit & 1;
+                const int h = hb * hpc + hi;
+                if (!mbar_wait(&acc_full[ab], (hit >> 1) & 1, err)) { ok = false; break; }
+                tc_fence_after();
+                const float ut = sE[ab * kRows + t_local];
+                uint32_t out[32];
+#pragma unroll
+                for (int p0 = 0; p0 < 64; p0 += 32) {
+                    uint32_t yd[32], yo[32];
+                    tmem_ld32_nowait(tmem + lane_base + kColAcc + ab * 128 + p0, yd);
+                    tmem_ld32_nowait(tmem + lane_base + kColAcc + ab * 128 + 64 + p0, yo);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        out[p0 / 2 + e] = pack_bf16x2(fmaf(ut, __uint_as_float(yo[2 * e]), __uint_as_float(yd[2 * e])),
+                                                      fmaf(ut, __uint_as_float(yo[2 * e + 1]), __uint_as_float(yd[2 * e + 1])));
+                }
+                tc_fence_before();
+                mbar_arrive(&acc_free[ab]);
+                // stage the row in shared memory (128B swizzle) and store the tile with TMA
+                if (!mbar_wait(y_free, (hit & 1) ^ 1, err)) { ok = false; break; }
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<uint4 *>(sY + sw128_off(t_local, q)) =
+                        make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+                fence_proxy_async_smem();
+                mbar_arrive(y_ready);
+                if (issuer) {
+                    if (!mbar_wait(y_ready, hit & 1, err)) { ok = false; break; }
+                    tma_store_3d(&tm_y, sY, 0, h, b * d.T + c * Q + mt * kRows);
+                    bulk_commit();
+                    bulk_wait_read();
+                    mbar_arrive(y_free);
+                }
+            }
+        }
+        if (issuer) bulk_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Heads per work unit: a divisor of the heads per group, at most 16, chosen so
+// that the persistent grid's last round of units is as full as possible.
+int heads_per_cta4(const Dims &d, int sms) {
+    int best = 1;
+    double best_eff = -1.0;
+    for (int k = 1; k <= 16; ++k) {
+        if (d.r % k) continue;
+        const double units = double(d.B) * d.nc * (d.Q / kRows) * (d.H / k);
+        const double rounds = std::ceil(units / sms);
+        const double eff = units / (rounds * sms);
+        if (eff > best_eff + 0.02 || (eff > best_eff - 0.02 && k > best)) {
+            if (eff > best_eff) best_eff = eff;
+            best = k;
+        }
+    }
+    return best;
+}
+
+template <int N>
+cudaError_t launch4(const Dims &d, const CUtensorMap *maps, int hpc, const float *dtq,
+                    const float *beta, const float *D, const float *l, unsigned int *err,
+                    cudaStream_t stream) {
+    const Smem4 L = scan4_smem(d.Q, N);
+    const int smem = int(L.total < 116 * 1024 ? 116 * 1024 : L.total);
+    if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan4_kernel<N>), smem))
+        return cudaErrorInvalidValue;
+    const int units = d.B * d.nc * (d.Q / kRows) * (d.H / hpc);
+    const int sms = device_sm_count();
+    const int grid = units < sms ? units : sms;
+    chunk_scan4_kernel<N><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                          d, hpc, units, dtq, beta, D, l, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_chunk_scan4_supported(const Dims &d) {
+    const bool n_ok = d.N == 16 || d.N == 128;
+    return d.P == 64 && n_ok && (d.Q == 128 || d.Q == 256) &&
+           scan4_smem(d.Q, d.N).total <= 227 * 1024 &&
+           int64_t(d.B) * d.nc * (d.Q / kRows) * d.H < (int64_t(1) << 31);
+}
+
+cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq,
+                                  const float *beta, const void *Bm, const void *Cm,
+                                  const float *D, const float *l, const void *s_in_bf16, void *y,
+                                  unsigned int *err, cudaStream_t stream) {
+    const uint32_t nbox = uint32_t(d.N >= 64 ? 64 : d.N);
+    const int rb = row_bytes(d.N);
+    const uint64_t bcdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
+    const uint64_t bcstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
+    const uint32_t bcbox[3] = {nbox, 1, uint32_t(kRows)};
+    const uint64_t xdims[3] = {uint64_t(d.P), uint64_t(d.H), uint64_t(d.B) * d.T};
+    const uint64_t xstr[2] = {uint64_t(d.P) * 2, uint64_t(d.H) * d.P * 2};
+    const uint32_t xbox[3] = {64, 1, uint32_t(kRows)};
+    const uint64_t sdims[2] = {uint64_t(d.N), uint64_t(d.B) * d.nc * d.H * d.P};
+    const uint64_t sstr[1] = {uint64_t(d.N) * 2};
+    const uint32_t sbox[2] = {nbox, 64};
+    CUtensorMap maps[5];
+    if (!make_tmap_bf16(&maps[0], 3, Cm, bcdims, bcstr, bcbox, rb) ||
+        !make_tmap_bf16(&maps[1], 3, Bm, bcdims, bcstr, bcbox, rb) ||
+        !make_tmap_bf16(&maps[2], 3, x, xdims, xstr, xbox, 128) ||
+        !make_tmap_bf16(&maps[3], 2, s_in_bf16, sdims, sstr, sbox, rb) ||
+        !make_tmap_bf16(&maps[4], 3, y, xdims, xstr, xbox, 128))
+        return cudaErrorInvalidValue;
+    const int hpc = heads_per_cta4(d, device_sm_count());
+    switch (d.N) {
+        case 16: return launch4<16>(d, maps, hpc, dtq, beta, D, l, err, stream);
+        case 32: return launch4<32>(d, maps, hpc, dtq, beta, D, l, err, stream);
+        case 64: return launch4<64>(d, maps, hpc, dtq, beta, D, l, err, stream);
+        case 128: return launch4<128>(d, maps, hpc, dtq, beta, D, l, err, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ssd

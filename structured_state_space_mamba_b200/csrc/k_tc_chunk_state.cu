@@ -41,7 +41,10 @@ __host__ __device__ constexpr int brow_bytes(int ns) { return ns >= 64 ? 128 : n
 __host__ __device__ constexpr uint32_t bswz(int ns) { return ns >= 64 ? kSw128 : (ns == 32 ? kSw64 : kSw32); }
 __host__ __device__ constexpr uint32_t x_stage_bytes() { return 2 * kKS * 128; }
 __host__ __device__ constexpr uint32_t b_stage_bytes(int ns) { return kKS * ns * 2; }
-__host__ __device__ constexpr uint32_t stage_bytes(int ns) { return x_stage_bytes() + b_stage_bytes(ns); }
+__host__ __device__ constexpr uint32_t w_stage_bytes() { return 2 * kKS * 4; }
+__host__ __device__ constexpr uint32_t stage_bytes(int ns) {
+    return ((x_stage_bytes() + b_stage_bytes(ns) + w_stage_bytes()) + 1023u) & ~1023u;
+}
 
 size_t state_smem_bytes(int NS) { return 1024 + size_t(kStages) * stage_bytes(NS) + 256; }
 
@@ -101,7 +104,10 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                     if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, err)) { ok = false; break; }
                     uint8_t *sx = smem + s * stage_bytes(NS);
                     uint8_t *sb = sx + x_stage_bytes();
-                    mbar_expect_tx(&full[s], uint32_t(nh) * kKS * 128 + b_stage_bytes(NS));
+                    mbar_expect_tx(&full[s], uint32_t(nh) * (kKS * 128 + kKS * 4) + b_stage_bytes(NS));
+                    float *sw = reinterpret_cast<float *>(sb + b_stage_bytes(NS));
+                    for (int j = 0; j < nh; ++j)
+                        bulk_load(sw + j * kKS, w + off_lq(d, b, h0 + j, c) + ks * kKS, kKS * 4, &full[s]);
                     for (int j = 0; j < nh; ++j)
                         tma_load_3d(sx + j * kKS * 128, &tm_x, &full[s], 0, h0 + j, trow + ks * kKS);
                     if (NS >= 64) {
@@ -152,24 +158,27 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         }
     } else if (warp < 6) {
         // ------------------------------ scale x by w -------------------------------
-        const int r = tid - 64;  // row of the stage's x tile: head j = r / 64, token r % 64
-        const int j = r >> 6, sr = r & 63;
+        // 16-byte chunk i of the stage's x tile belongs to row i / 8 (head
+        // j = row / 64, token row % 64); eight consecutive threads share a row,
+        // so a warp touches four whole 128-byte rows (no bank conflicts).  The
+        // swizzle only permutes chunks within a row, so each chunk takes its
+        // row's weight.
+        const int st = tid - 64;  // 0..127
         uint32_t it = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            const int hp = u % nhp, bc = u / nhp;
-            const int c = bc % d.nc, b = bc / d.nc;
-            const int h = hp * nh + (j < nh ? j : 0);
-            const float *wp = w + off_lq(d, b, h, c) + sr;
             for (int ks = 0; ks < ksteps; ++ks) {
                 const int s = it % kStages;
-                const float wv = __ldg(wp + ks * kKS);
                 if (!mbar_wait(&full[s], (it / kStages) & 1, err)) { ok = false; break; }
-                if (j < nh) {
-                    uint8_t *row = smem + s * stage_bytes(NS) + r * 128;
+                uint8_t *sx = smem + s * stage_bytes(NS);
+                const float *sw = reinterpret_cast<const float *>(sx + x_stage_bytes() + b_stage_bytes(NS));
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint4 *p = reinterpret_cast<uint4 *>(row + ((q ^ (r & 7)) << 4));
+                for (int k = 0; k < (2 * kKS * 8) / 128; ++k) {
+                    const int i = st + k * 128;
+                    const int row = i >> 3;
+                    if ((row >> 6) < nh) {
+                        const float wv = sw[row];
+                        uint4 *p = reinterpret_cast<uint4 *>(sx) + i;
                         uint4 v = *p;
                         v.x = pack_bf16x2(bf16lo(v.x) * wv, bf16hi(v.x) * wv);
                         v.y = pack_bf16x2(bf16lo(v.y) * wv, bf16hi(v.y) * wv);
@@ -177,8 +186,8 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                         v.w = pack_bf16x2(bf16lo(v.w) * wv, bf16hi(v.w) * wv);
                         *p = v;
                     }
-                    fence_proxy_async_smem();
                 }
+                fence_proxy_async_smem();
                 mbar_arrive(&scaled[s]);
                 ++it;
             }

@@ -7,9 +7,10 @@
 
 namespace ssd {
 
-// ssd_chunk_cumsum: dt, A -> l, w [B,H,nc,Q], alpha [B,H,nc]
+// ssd_chunk_cumsum: dt, A -> l, w, dtq, beta [B,H,nc,Q], alpha [B,H,nc]
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
-                                float *w, float *alpha, cudaStream_t stream);
+                                float *w, float *dtq, float *beta, float *alpha,
+                                cudaStream_t stream);
 
 // ssd_state_passing: states [B,nc,H,P,N] (fp32 or bf16 per states_bf16), alpha
 // -> s_in [B,nc,H,P,N] (fp32 or bf16 per s_in_bf16), final state [B,H,P,N] fp32
@@ -38,5 +39,12 @@ cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, 
                                  const void *Cm, const float *D, const float *l,
                                  const void *s_in_bf16, void *y, unsigned int *err,
                                  cudaStream_t stream);
+// Persistent warp-specialised variant (dstate <= 128); dtq and beta come from
+// ssd_chunk_cumsum.  Writes y with TMA stores.
+bool tc_chunk_scan4_supported(const Dims &d);
+cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq,
+                                  const float *beta, const void *Bm, const void *Cm,
+                                  const float *D, const float *l, const void *s_in_bf16, void *y,
+                                  unsigned int *err, cudaStream_t stream);
 
 }  // namespace ssd

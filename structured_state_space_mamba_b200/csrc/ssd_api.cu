@@ -93,6 +93,8 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     size_t off = 0;
     w.l_offset = off; off = align_up(off + lq);
     w.w_offset = off; off = align_up(off + lq);
+    w.dtq_offset = off; off = align_up(off + lq);
+    w.beta_offset = off; off = align_up(off + lq);
     w.alpha_offset = off; off = align_up(off + al);
     w.states_offset = off;
     w.states_dtype = plan->tc_state ? SSD_BF16 : SSD_F32;
@@ -137,6 +139,8 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     }
     float *l = reinterpret_cast<float *>(ws + pl.ws.l_offset);
     float *w = reinterpret_cast<float *>(ws + pl.ws.w_offset);
+    float *dtq = reinterpret_cast<float *>(ws + pl.ws.dtq_offset);
+    float *beta = reinterpret_cast<float *>(ws + pl.ws.beta_offset);
     float *alpha = reinterpret_cast<float *>(ws + pl.ws.alpha_offset);
     void *states = ws + pl.ws.states_offset;
     void *s_in = ws + pl.ws.s_in_offset;
@@ -145,7 +149,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
         cudaError_t e = cudaSuccess;
         switch (stage) {
             case SSD_STAGE_CHUNK_CUMSUM:
-                e = ssd::launch_chunk_cumsum(d, dt, A, l, w, alpha, stream);
+                e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, err, stream)
@@ -158,7 +162,9 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 break;
             case SSD_STAGE_CHUNK_SCAN:
                 e = pl.tc_scan
-                        ? ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream)
+                        ? (ssd::tc_chunk_scan4_supported(d)
+                               ? ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, err, stream)
+                               : ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream))
                         : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt, Bm, Cm, D, l,
                                                       static_cast<const float *>(s_in), y, stream);
                 break;

@@ -2,7 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
-#include <set>
+#include <map>
 #include <utility>
 
 #include "tma_host.h"
@@ -56,18 +56,19 @@ bool make_tmap_bf16(CUtensorMap *out, int rank, const void *base, const uint64_t
 
 bool smem_attr_once(const void *kernel, int bytes) {
     static std::mutex mu;
-    static std::set<std::pair<int, const void *>> done;
+    static std::map<std::pair<int, const void *>, int> done;  // largest limit set so far
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     std::lock_guard<std::mutex> lock(mu);
     const auto key = std::make_pair(dev, kernel);
-    if (done.count(key)) return true;
+    auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
         cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    done.insert(key);
+    done[key] = bytes;
     return true;
 }
 

@@ -20,8 +20,9 @@ namespace ssd {
 bool make_tmap_bf16(CUtensorMap *out, int rank, const void *base, const uint64_t *dims,
                     const uint64_t *stride_bytes, const uint32_t *box, int swizzle_bytes);
 
-// Raise a kernel's dynamic shared memory limit to `bytes`, once per device
-// and kernel (later calls are a lookup).  Returns false on failure.
+// Make sure a kernel's dynamic shared memory limit on the current device is at
+// least `bytes` (the attribute is set only when it must grow; otherwise this
+// is a lookup).  Returns false on failure.
 bool smem_attr_once(const void *kernel, int bytes);
 
 // Number of SMs of the current device (cached per device).

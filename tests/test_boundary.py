@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_struct_sizes_match_header(lib):
     assert ctypes.sizeof(binding.Dims) == 6 * 8 + 2 * 4
-    assert ctypes.sizeof(binding.WorkspaceLayout) == 6 * 8 + 4 * 4
+    assert ctypes.sizeof(binding.WorkspaceLayout) == 8 * 8 + 4 * 4
 
 
 def test_status_strings(lib):

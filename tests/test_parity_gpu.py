@@ -95,6 +95,10 @@ def test_f32_shapes(oracle, shape, h0):
     dict(batch=1, seqlen=512, nheads=2, headdim=64, dstate=256, ngroups=1, chunk_len=256),
     dict(batch=1, seqlen=256, nheads=2, headdim=32, dstate=32, ngroups=1, chunk_len=64),
     dict(batch=3, seqlen=1024, nheads=6, headdim=64, dstate=128, ngroups=3, chunk_len=256),
+    dict(batch=1, seqlen=512, nheads=2, headdim=64, dstate=32, ngroups=1, chunk_len=256),
+    dict(batch=1, seqlen=1024, nheads=24, headdim=64, dstate=32, ngroups=2, chunk_len=256),
+    dict(batch=1, seqlen=1024, nheads=12, headdim=64, dstate=64, ngroups=2, chunk_len=256),
+    dict(batch=2, seqlen=1024, nheads=10, headdim=64, dstate=16, ngroups=5, chunk_len=128),
 ])
 @pytest.mark.parametrize("h0", [False, True])
 def test_bf16_shapes(oracle, shape, h0):
