@@ -20,12 +20,13 @@
 //   P  = masked diagonal scores in bf16 (+ D_h on the diagonal: the skip term),
 //   X' = g o X[s < t0],  S' = exp(r) s_in.
 //
-// Decay factors inside the diagonal tile, per 32 x 32 block:
-//   * blocks entirely below the diagonal: exp(l_t - l_s) = exp(l_t - l_k) beta_s,
-//     l_k the last l of the source block, beta_s = exp(l_k - l_s) dt_s (both <= 1);
-//   * blocks on the diagonal: exp(l_t - l_s) = exp(l_t - l_f) exp(l_f - l_s),
-//     l_f the first l of the block, when the block's decay range l_f - l_last is
-//     below 80 (the second factor then stays below e^80); otherwise the exact
+// Decay factors inside the diagonal tile, per 32 x 32 block with source block
+// k (last token k_e): exp(l_t - l_s) dt_s = exp(l_t - l_{k_e}) beta_s, where
+// beta_s = exp(l_{k_e} - l_s) dt_s <= dt_s comes precomputed from the cumsum.
+//   * blocks entirely below the diagonal: both factors are <= 1;
+//   * blocks on the diagonal: the row factor exp(l_t - l_{k_e}) is >= 1 but at
+//     most exp(l_{k_s} - l_{k_e}), so the same factorisation holds when the
+//     block's decay range l_{k_s} - l_{k_e} is below 80; otherwise the exact
 //     exp(l_t - l_s) per element.
 //
 // Tensor memory: [0,128) CB diagonal tile (fp32); [128,256) two score buffers
@@ -34,8 +35,9 @@
 // Yoz MMAs), the per-head stages {x rows, s_in, l, dt, beta}, and a staging
 // tile for y, written back with a TMA store.
 //
-// Roles (14 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 scores,
-// warps 10..13 epilogue.
+// Roles (22 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..17 scores
+// (one 32 x 32 block of the tile each: TMEM lane quarter warp % 4, column block
+// (warp - 2) / 4), warps 18..21 epilogue.
 #include <cmath>
 
 #include "common.cuh"
@@ -49,9 +51,11 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 704;
 constexpr int kRows = 128;
-constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = 16;
+constexpr int kScoreThreads = 32 * kScoreWarps;
+constexpr int kEpiWarp0 = 2 + kScoreWarps;
 constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColCBd = 0, kColP = 128, kColTmp = 128, kColAcc = 256;
@@ -279,12 +283,13 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             mma_commit(done);
             mbar_wait(done, 0, nullptr);
         }
-    } else if (warp < 10) {
+    } else if (warp < kEpiWarp0) {
         // ================================ scores ================================
-        const int sid = tid - 64;            // 0..255
+        const int sid = tid - 64;            // 0..511
         const int qd = warp & 3;             // TMEM lane quarter of this warp
-        const int half = (warp - 2) >> 2;    // which half of the tile's columns
+        const int cb = (warp - 2) >> 2;      // 32-column block of the tile
         const int t_local = qd * 32 + lane;  // row of the tile
+        const int j0 = cb * 32;              // first column of the block
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
         uint32_t ui = 0, hit = 0;
         bool ok = true;
@@ -296,20 +301,17 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             tc_fence_after();
             if (mt > 0) {
                 // CBoff fp32 -> bf16, into shared memory as a K-major, 128B-swizzled
-                // A operand: this thread packs row t_local, columns [64 half, 64 half + 64)
-                uint8_t *slab = sB + half * (kRows * 128);
+                // A operand: this thread packs row t_local, columns [j0, j0 + 32)
+                uint8_t *slab = sB + (cb >> 1) * (kRows * 128);
+                float v[32];
+                tmem_ld32(tmem + lane_base + kColTmp + j0, v);
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + kColTmp + half * 64 + q * 32, v);
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4)
-                        *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, q * 4 + c4)) =
-                            make_uint4(pack_bf16x2(v[8 * c4], v[8 * c4 + 1]),
-                                       pack_bf16x2(v[8 * c4 + 2], v[8 * c4 + 3]),
-                                       pack_bf16x2(v[8 * c4 + 4], v[8 * c4 + 5]),
-                                       pack_bf16x2(v[8 * c4 + 6], v[8 * c4 + 7]));
-                }
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, (cb & 1) * 4 + c4)) =
+                        make_uint4(pack_bf16x2(v[8 * c4], v[8 * c4 + 1]),
+                                   pack_bf16x2(v[8 * c4 + 2], v[8 * c4 + 3]),
+                                   pack_bf16x2(v[8 * c4 + 4], v[8 * c4 + 5]),
+                                   pack_bf16x2(v[8 * c4 + 6], v[8 * c4 + 7]));
                 fence_proxy_async_smem();
             }
             // every score thread is done with the CBoff range before any score
@@ -321,7 +323,6 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             for (int hi = 0; hi < hpc; ++hi, ++hit) {
                 const int st = hit & 1, pb = hit & 1, ab = hit & 1;
                 const int h = hb * hpc + hi;
-                const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
                 uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
                 const float *sl_ = reinterpret_cast<const float *>(stage + L.l_rel);
                 const float *sdt = reinterpret_cast<const float *>(stage + L.dt_rel);
@@ -342,69 +343,75 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 mbar_arrive(&scaled_ready[st]);
                 // row factors for the epilogue (its previous use of sE[ab] has ended
                 // once accumulator ab is free)
-                if (!mbar_wait(&acc_free[ab], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
-                if (sid < kRows) sE[ab * kRows + sid] = __expf(sl_[t0 + sid] - r);
+                if (sid < kRows) {
+                    if (!mbar_wait(&acc_free[ab], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
+                    sE[ab * kRows + sid] = __expf(sl_[t0 + sid] - r);
+                }
                 if (!mbar_wait(&p_free[pb], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
                 tc_fence_after();
-                const float lt = sl_[t0 + t_local];
-                // both 32-column blocks of this thread's half-row: issue the TMEM
-                // loads together (one wait), skipping blocks above the diagonal
-                uint32_t raw[2][32];
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk)
-                    if (half * 64 + blk * 32 <= qd * 32)
-                        tmem_ld32_nowait(tmem + lane_base + kColCBd + half * 64 + blk * 32, raw[blk]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const int j0 = half * 64 + blk * 32;  // first column within the tile
+                const uint32_t pcol = tmem + lane_base + kColP + pb * 64 + (j0 >> 1);
+                if (j0 > qd * 32) {
+                    // block above the diagonal
                     uint32_t pk[16];
-                    const uint32_t *v = raw[blk];
-                    if (j0 > qd * 32) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    } else if (j0 == qd * 32) {
-                        // block on the diagonal (warp-uniform branch)
-                        const float lf = sl_[t0 + j0], ll = sl_[t0 + j0 + 31];
-                        if (lf - ll < 80.f) {
-                            const float at = __expf(lt - lf);
-                            const float bl = __expf(lf - sl_[t0 + j0 + lane]) * sdt[t0 + j0 + lane];
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    tmem_st16(pcol, pk);
+                } else if (j0 < qd * 32) {
+                    // block entirely below the diagonal
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + kColCBd + j0, v);
+                    const float at = __expf(sl_[t0 + t_local] - sl_[t0 + j0 + 31]);
+                    const float4 *b4 = reinterpret_cast<const float4 *>(beta + t0 + j0);
+                    uint32_t pk[16];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const int j = j0 + 2 * e;
-                                const float b0 = __shfl_sync(0xffffffffu, bl, 2 * e);
-                                const float b1 = __shfl_sync(0xffffffffu, bl, 2 * e + 1);
-                                float p0 = j <= t_local ? __uint_as_float(v[2 * e]) * at * b0 : 0.f;
-                                float p1 = j + 1 <= t_local ? __uint_as_float(v[2 * e + 1]) * at * b1 : 0.f;
-                                if (j == t_local) p0 += Dh;
-                                if (j + 1 == t_local) p1 += Dh;
-                                pk[e] = pack_bf16x2(p0, p1);
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 bb = b4[e];
+                        pk[2 * e] = pack_bf16x2(v[4 * e] * at * bb.x, v[4 * e + 1] * at * bb.y);
+                        pk[2 * e + 1] = pack_bf16x2(v[4 * e + 2] * at * bb.z, v[4 * e + 3] * at * bb.w);
+                    }
+                    tmem_st16(pcol, pk);
+                } else {
+                    // block on the diagonal (warp-uniform branch), in two 16-column
+                    // halves: row lane of the block sees sources 0..lane, and D_h
+                    // sits on the diagonal
+                    const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
+                    const float lt = sl_[t0 + t_local];
+                    const float lke = sl_[t0 + j0 + 31];
+                    const bool factored = sl_[t0 + j0] - lke < 80.f;
+                    const float at = __expf(lt - lke);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float v[16];
+                        tmem_ld16(tmem + lane_base + kColCBd + j0 + 16 * hf, v);
+                        if (factored) {
+                            const float4 *b4 = reinterpret_cast<const float4 *>(beta + t0 + j0 + 16 * hf);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float4 bb = b4[e];
+                                v[4 * e] *= at * bb.x;
+                                v[4 * e + 1] *= at * bb.y;
+                                v[4 * e + 2] *= at * bb.z;
+                                v[4 * e + 3] *= at * bb.w;
                             }
                         } else {
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                const int j = j0 + 2 * e;
-                                float p0 = j <= t_local ? __uint_as_float(v[2 * e]) * __expf(lt - sl_[t0 + j]) * sdt[t0 + j] : 0.f;
-                                float p1 = j + 1 <= t_local ? __uint_as_float(v[2 * e + 1]) * __expf(lt - sl_[t0 + j + 1]) * sdt[t0 + j + 1] : 0.f;
-                                if (j == t_local) p0 += Dh;
-                                if (j + 1 == t_local) p1 += Dh;
-                                pk[e] = pack_bf16x2(p0, p1);
+                                const int sidx = t0 + j0 + 16 * hf + e;
+                                v[e] *= __expf(fminf(lt - sl_[sidx], 0.f)) * sdt[sidx];
                             }
                         }
-                    } else {
-                        // block entirely below the diagonal
-                        const float at = __expf(lt - sl_[t0 + j0 + 31]);
-                        const float4 *b4 = reinterpret_cast<const float4 *>(beta + t0 + j0);
+                        uint32_t pk[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float4 bb = b4[e];
-                            pk[2 * e] = pack_bf16x2(__uint_as_float(v[4 * e]) * at * bb.x,
-                                                    __uint_as_float(v[4 * e + 1]) * at * bb.y);
-                            pk[2 * e + 1] = pack_bf16x2(__uint_as_float(v[4 * e + 2]) * at * bb.z,
-                                                        __uint_as_float(v[4 * e + 3]) * at * bb.w);
+                        for (int e = 0; e < 16; e += 2) {
+                            const int c0 = 16 * hf + e;  // column within the block
+                            float p0 = c0 <= lane ? v[e] : 0.f;
+                            float p1 = c0 + 1 <= lane ? v[e + 1] : 0.f;
+                            if (c0 == lane) p0 += Dh;
+                            if (c0 + 1 == lane) p1 += Dh;
+                            pk[e >> 1] = pack_bf16x2(p0, p1);
                         }
+                        tmem_st8(pcol + 8 * hf, pk);
                     }
-                    tmem_st16(tmem + lane_base + kColP + pb * 64 + (j0 >> 1), pk);
                 }
                 tmem_wait_st();
                 fence_proxy_async_smem();
@@ -417,7 +424,7 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         const int qd = warp & 3;
         const int t_local = qd * 32 + lane;
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
-        const bool issuer = (warp == 10 && lane == 0);
+        const bool issuer = (warp == kEpiWarp0 && lane == 0);
         uint32_t hit = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -430,28 +437,33 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 const int ab = hit & 1;
                 const int h = hb * hpc + hi;
                 if (!mbar_wait(&acc_full[ab], (hit >> 1) & 1, err)) { ok = false; break; }
+                // the staging tile is free once the previous TMA store has read it
+                if (!mbar_wait(y_free, (hit & 1) ^ 1, err)) { ok = false; break; }
                 tc_fence_after();
                 const float ut = sE[ab * kRows + t_local];
-                uint32_t out[32];
+                // y = Yd + u_t Yoz, 16 columns at a time, staged in shared memory
+                // (128B swizzle) for one TMA store of the tile
 #pragma unroll
-                for (int p0 = 0; p0 < 64; p0 += 32) {
-                    uint32_t yd[32], yo[32];
-                    tmem_ld32_nowait(tmem + lane_base + kColAcc + ab * 128 + p0, yd);
-                    tmem_ld32_nowait(tmem + lane_base + kColAcc + ab * 128 + 64 + p0, yo);
+                for (int p0 = 0; p0 < 64; p0 += 16) {
+                    uint32_t yd[16], yo[16];
+                    tmem_ld16_nowait(tmem + lane_base + kColAcc + ab * 128 + p0, yd);
+                    tmem_ld16_nowait(tmem + lane_base + kColAcc + ab * 128 + 64 + p0, yo);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        out[p0 / 2 + e] = pack_bf16x2(fmaf(ut, __uint_as_float(yo[2 * e]), __uint_as_float(yd[2 * e])),
-                                                      fmaf(ut, __uint_as_float(yo[2 * e + 1]), __uint_as_float(yd[2 * e + 1])));
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 8 * q + 2 * e;
+                            o[e] = pack_bf16x2(fmaf(ut, __uint_as_float(yo[i]), __uint_as_float(yd[i])),
+                                               fmaf(ut, __uint_as_float(yo[i + 1]), __uint_as_float(yd[i + 1])));
+                        }
+                        *reinterpret_cast<uint4 *>(sY + sw128_off(t_local, p0 / 8 + q)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_free[ab]);
-                // stage the row in shared memory (128B swizzle) and store the tile with TMA
-                if (!mbar_wait(y_free, (hit & 1) ^ 1, err)) { ok = false; break; }
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<uint4 *>(sY + sw128_off(t_local, q)) =
-                        make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
                 fence_proxy_async_smem();
                 mbar_arrive(y_ready);
                 if (issuer) {
