@@ -44,7 +44,7 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # ---------------------------------------------------------------------------
 # algorithmic work (chunked algorithm; compulsory bytes only)
 # ---------------------------------------------------------------------------
-def work_model(cfg, final_state=True):
+def work_model(cfg, final_state=True, lay=None):
     B, T, H, P, N, G, Q = (cfg[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
                                             "ngroups", "chunk_len"))
     nc = T // Q
@@ -59,15 +59,26 @@ def work_model(cfg, final_state=True):
     comp = (2 * x_bytes + bc_bytes + dt_bytes + 2 * H * 4
             + (state_bytes if cfg.get("init_state") else 0)
             + (state_bytes if final_state else 0))
-    # per-kernel algorithmic bytes (what each kernel must read and write)
+    # per-kernel algorithmic bytes (what each kernel must read and write, with the
+    # element sizes of this call's workspace layout)
     st_elems = B * nc * H * P * N
+    lq = B * H * nc * Q * 4                               # one fp32 [B,H,nc,Q] array
+    s_sz = 2 if (lay is None or lay.states_dtype == 1) else 4
+    sin_sz = 2 if (lay is None or lay.s_in_dtype == 1) else 4
+    fused = bool(lay is not None and lay.fused_state)
+    h0_bytes = state_bytes if cfg.get("init_state") else 0
+    fin_bytes = state_bytes if final_state else 0
     per_kernel = {
-        "ssd_chunk_cumsum": dt_bytes + H * 4 + 2 * B * H * nc * Q * 4 + B * H * nc * 4,
-        "ssd_chunk_state": x_bytes + bc_bytes // 2 + B * H * nc * Q * 4 + st_elems * 4,
-        "ssd_state_passing": st_elems * 4 + B * H * nc * 4 + st_elems * 2
-                             + (state_bytes if final_state else 0),
-        "ssd_chunk_scan": 2 * x_bytes + bc_bytes + dt_bytes + B * H * nc * Q * 4 + st_elems * 2
-                          + H * 4,
+        # dt, A -> l, w, dtq, beta, alpha
+        "ssd_chunk_cumsum": dt_bytes + H * 4 + 4 * lq + B * H * nc * 4,
+        # x, B, w -> S  (fused: x, B, w, alpha, h0 -> s_in, final)
+        "ssd_chunk_state": (x_bytes + bc_bytes // 2 + lq + B * H * nc * 4 + h0_bytes
+                            + st_elems * sin_sz + fin_bytes) if fused
+                           else (x_bytes + bc_bytes // 2 + lq + st_elems * s_sz),
+        "ssd_state_passing": 0 if fused else (st_elems * s_sz + B * H * nc * 4 + h0_bytes
+                                              + st_elems * sin_sz + fin_bytes),
+        # x, B, C, l, dtq, beta, s_in, D -> y
+        "ssd_chunk_scan": 2 * x_bytes + bc_bytes + 3 * lq + st_elems * sin_sz + H * 4,
     }
     per_kernel_flops = {
         "ssd_chunk_state": 2 * B * nc * H * Q * N * P,
@@ -353,7 +364,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         return
     tokens_step = inp.x.shape[0] * inp.x.shape[1]
     value = world * tokens_step * args.steps / (ms_total * 1e-3)
-    wm = work_model(cfg, final_state=want_final)
+    wm = work_model(cfg, final_state=want_final, lay=lay)
     peaks, peak_src = load_peaks()
     top = max(kern_ms, key=kern_ms.get)
     bound = "hbm"
@@ -379,6 +390,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "ms_per_step_direct_calls": ms_direct / args.steps,
         "gpu_launches": args.steps * lay.launches,
         "tensor_core": bool(lay.tensor_core),
+        "fused_state": bool(lay.fused_state),
         "e2e": {"value": world * tokens_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,

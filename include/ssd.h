@@ -127,7 +127,10 @@ SSD_API ssd_status_t ssd_forward_ws(const ssd_dims_t *dims, const void *x, const
  * kernel on its own.
  *   stage 0  ssd_chunk_cumsum   dt, A          -> l, w, alpha
  *   stage 1  ssd_chunk_state    x, B, w        -> states
+ *            (fused_state layouts: x, B, w, alpha, init_state -> s_in,
+ *            final_state_out)
  *   stage 2  ssd_state_passing  states, alpha, init_state -> s_in, final_state_out
+ *            (fused_state layouts: nothing)
  *   stage 3  ssd_chunk_scan     x, dt, B, C, D, l, s_in   -> y_out
  * Any other stage value returns SSD_ERR_INVALID_DIM.
  */
@@ -161,7 +164,12 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  *   s_in   [B, nc, H, P, N]    state entering each chunk; element type given
  *                              by s_in_dtype (SSD_F32 or SSD_BF16)
  * `tensor_core` is 1 when the call runs the tcgen05 kernels, 0 otherwise;
- * `launches` is the number of kernels one call launches.
+ * `launches` is the number of kernels one call launches.  `fused_state` is 1
+ * when ssd_chunk_state and ssd_state_passing run as one kernel (the
+ * (batch, head pair) units fill 60-100% of the GPU's SMs in one wave): the
+ * per-chunk states then never
+ * reach memory, the states region is empty (states_offset == s_in_offset) and
+ * stage 2 of ssd_forward_stage does nothing.
  */
 typedef struct {
     size_t total_bytes;
@@ -170,6 +178,7 @@ typedef struct {
     int32_t tensor_core;
     int32_t launches;
     int32_t states_dtype; /* element type of states: SSD_F32 or SSD_BF16 */
+    int32_t fused_state;
 } ssd_workspace_layout_t;
 
 SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,

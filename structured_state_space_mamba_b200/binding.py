@@ -39,7 +39,8 @@ class WorkspaceLayout(ctypes.Structure):
                 ("alpha_offset", ctypes.c_size_t),
                 ("states_offset", ctypes.c_size_t), ("s_in_offset", ctypes.c_size_t),
                 ("s_in_dtype", ctypes.c_int32), ("tensor_core", ctypes.c_int32),
-                ("launches", ctypes.c_int32), ("states_dtype", ctypes.c_int32)]
+                ("launches", ctypes.c_int32), ("states_dtype", ctypes.c_int32),
+                ("fused_state", ctypes.c_int32)]
 
 
 class SSDError(RuntimeError):

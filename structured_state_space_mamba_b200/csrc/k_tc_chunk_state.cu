@@ -31,7 +31,9 @@ using namespace tc;
 
 constexpr int kThreads = 320;  // 10 warps
 constexpr int kKS = 64;        // tokens per stage
-constexpr int kStages = 4;
+// stages in flight: as many 64-token stages as shared memory holds (each TMA
+// stage takes ~3 us to land when every SM streams, so a deep ring matters)
+__host__ __device__ constexpr int num_stages(int ns) { return ns <= 128 ? 6 : 4; }
 
 __host__ __device__ constexpr int acc_cols(int ns) { return ns < 16 ? 16 : ns; }
 __host__ __device__ constexpr int tmem_alloc_cols(int ns) {
@@ -46,7 +48,7 @@ __host__ __device__ constexpr uint32_t stage_bytes(int ns) {
     return ((x_stage_bytes() + b_stage_bytes(ns) + w_stage_bytes()) + 1023u) & ~1023u;
 }
 
-size_t state_smem_bytes(int NS) { return 1024 + size_t(kStages) * stage_bytes(NS) + 256; }
+size_t state_smem_bytes(int NS) { return 1024 + size_t(num_stages(NS)) * stage_bytes(NS) + 256; }
 
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -54,6 +56,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                       Dims d, int nh, int units, const float *__restrict__ w,
                       __nv_bfloat16 *__restrict__ states, unsigned int *err) {
     constexpr int kAcc = acc_cols(NS);
+    constexpr int kStages = num_stages(NS);
     constexpr int kCols = tmem_alloc_cols(NS);
     constexpr int kRowB = brow_bytes(NS);
     if (device_failed(err)) return;  // an earlier wait expired: skip all work

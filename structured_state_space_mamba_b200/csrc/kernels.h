@@ -30,11 +30,18 @@ cudaError_t launch_chunk_scan_simt(const Dims &d, bool bf16, const void *x, cons
 
 // Tensor-core (tcgen05) kernels, bf16 storage, P == 64.
 bool tc_chunk_state_supported(const Dims &d);
+// chunk_state + state_passing as one kernel (units of (b, head pair) walked over
+// all chunks); `sms` is the SM count the launch will fill
+bool tc_state_fused_supported(const Dims &d, int sms);
 bool tc_chunk_scan_supported(const Dims &d);
 // `err` is a device word: bit 0 is set when a bounded wait inside a kernel
 // expired (the kernel then skips its remaining work and exits cleanly).
 cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, const float *w,
                                   void *states_bf16, unsigned int *err, cudaStream_t stream);
+// writes s_in (bf16, [B, nc, H, P, N]) and, if fin != nullptr, the final state
+cudaError_t launch_state_fused(const Dims &d, const void *x, const void *Bm, const float *w,
+                               const float *alpha, const float *h0, void *s_in_bf16, float *fin,
+                               unsigned int *err, cudaStream_t stream);
 cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
                                  const void *Cm, const float *D, const float *l,
                                  const void *s_in_bf16, void *y, unsigned int *err,

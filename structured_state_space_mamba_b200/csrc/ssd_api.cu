@@ -49,11 +49,14 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 bool misaligned(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u); }
 
+constexpr int kB200Sms = 148;
+
 struct Plan {
     Dims d;
     bool bf16;
     bool tc_state;  // tcgen05 chunk state
     bool tc_scan;   // tcgen05 chunk scan (consumes bf16 s_in)
+    bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
     ssd_workspace_layout_t ws;
 };
 
@@ -84,6 +87,9 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     plan->bf16 = a.dtype == SSD_BF16;
     plan->tc_state = plan->bf16 && ssd::tc_chunk_state_supported(d);
     plan->tc_scan = plan->bf16 && ssd::tc_chunk_scan_supported(d);
+    // the fused state kernel walks each (b, head pair) over all chunks: used when
+    // those units fill most of the GPU's 148 SMs in one wave
+    plan->fused = plan->tc_state && plan->tc_scan && ssd::tc_state_fused_supported(d, kB200Sms);
 
     ssd_workspace_layout_t &w = plan->ws;
     std::memset(&w, 0, sizeof(w));
@@ -98,13 +104,14 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.alpha_offset = off; off = align_up(off + al);
     w.states_offset = off;
     w.states_dtype = plan->tc_state ? SSD_BF16 : SSD_F32;
-    off = align_up(off + st * (plan->tc_state ? 2 : 4));
+    if (!plan->fused) off = align_up(off + st * (plan->tc_state ? 2 : 4));
     w.s_in_offset = off;
     w.s_in_dtype = plan->tc_scan ? SSD_BF16 : SSD_F32;
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
-    w.launches = 4;
+    w.launches = plan->fused ? 3 : 4;
+    w.fused_state = plan->fused ? 1 : 0;
     return SSD_OK;
 }
 
@@ -152,11 +159,13 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
-                e = pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, err, stream)
+                e = pl.fused ? ssd::launch_state_fused(d, x, Bm, w, alpha, init_state, s_in, fin, err, stream)
+                    : pl.tc_state ? ssd::launch_chunk_state_tc(d, x, Bm, w, states, err, stream)
                                 : ssd::launch_chunk_state_simt(d, pl.bf16, x, Bm, w,
                                                                static_cast<float *>(states), stream);
                 break;
             case SSD_STAGE_STATE_PASSING:
+                if (pl.fused) break;  // done by the fused chunk_state kernel
                 e = ssd::launch_state_passing(d, states, pl.tc_state, alpha, init_state, s_in,
                                               pl.tc_scan, fin, stream);
                 break;

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_struct_sizes_match_header(lib):
     assert ctypes.sizeof(binding.Dims) == 6 * 8 + 2 * 4
-    assert ctypes.sizeof(binding.WorkspaceLayout) == 8 * 8 + 4 * 4
+    assert ctypes.sizeof(binding.WorkspaceLayout) == 8 * 8 + 6 * 4  # 5 int32 + padding
 
 
 def test_status_strings(lib):
@@ -72,11 +72,29 @@ def test_workspace_layout(lib):
     assert lay.s_in_offset >= lay.states_offset + state_elems * ssz
     sz = 2 if lay.s_in_dtype == binding.SSD_BF16 else 4
     assert lay.total_bytes >= lay.s_in_offset + state_elems * sz
-    assert lay.launches == 4
+    assert lay.launches == 4 and lay.fused_state == 0
     assert binding.workspace_bytes(d, 128) == lay.total_bytes
     # fp32 storage never uses the tensor-core kernels
     lay32 = binding.workspace_layout(dims(dtype="f32"), 128)
     assert lay32.tensor_core == 0 and lay32.s_in_dtype == binding.SSD_F32
+
+
+def test_fused_state_layout_for_many_head_pairs(lib):
+    """0.6 x 148 <= (batch x head pairs) <= 148 SMs: chunk_state and state_passing
+    run as one kernel, so no states region is reserved and one launch fewer is
+    made; with more units than SMs, or far fewer, they stay separate."""
+    d = binding.make_dims(batch=8, seqlen=2048, nheads=24, headdim=64, dstate=128, ngroups=1,
+                          dtype="bf16")
+    lay = binding.workspace_layout(d, 256)
+    assert lay.fused_state == 1 and lay.launches == 3 and lay.tensor_core == 1
+    assert lay.states_offset == lay.s_in_offset
+    few = binding.workspace_layout(binding.make_dims(batch=1, seqlen=65536, nheads=32, headdim=64,
+                                                     dstate=128, ngroups=8, dtype="bf16"), 256)
+    assert few.fused_state == 0 and few.launches == 4
+    assert few.s_in_offset > few.states_offset
+    many = binding.workspace_layout(binding.make_dims(batch=4, seqlen=4096, nheads=80, headdim=64,
+                                                      dstate=128, ngroups=1, dtype="bf16"), 256)
+    assert many.fused_state == 0 and many.launches == 4
 
 
 @pytest.mark.parametrize("kw,chunk,code", [

@@ -141,6 +141,22 @@ def test_strong_decay_stays_finite(oracle):
     check_full(inp, oracle)
 
 
+def test_steep_decay_inside_32_token_blocks(oracle):
+    """A_h = -16 and dt in [0.2, 1]: the decay across any 32 tokens exceeds e^-80,
+    so the chunk scan's diagonal blocks take the per-element exact path; one head
+    keeps a gentle decay so both paths meet in the same launch."""
+    inp = make_inputs(1, 1024, 4, 64, 128, 1, 256, dtype="bf16", seed=13, init_state=True)
+    rng = np.random.default_rng(13)
+    inp.dt = rng.uniform(0.2, 1.0, size=inp.dt.shape).astype(np.float32)
+    inp.A = np.array([-16.0, -16.0, -12.0, -0.01], dtype=np.float32)
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    assert np.isfinite(y).all() and np.isfinite(f).all()
+    for h in range(4):  # per head: the gentle head's scale must not hide the others
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
+
+
 def test_chunk_len_invariance_on_gpu(oracle):
     ys = []
     for q in (64, 128, 256):
@@ -194,6 +210,43 @@ def test_workspace_entry_point_and_intermediates(oracle):
     assert rel(w, it["w"]) < 1e-5
     assert rel(S.reshape(it["S"].shape), it["S"]) < 2e-2          # ssd_chunk_state
     assert rel(s_in.reshape(it["s_in"].shape), it["s_in"]) < 2e-2  # ssd_state_passing
+
+
+# ---------------------------------------------------------------------------
+# fused chunk_state + state_passing (enough (batch, head pair) units)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [
+    dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=128, ngroups=1, chunk_len=128),
+    dict(batch=2, seqlen=256, nheads=96, headdim=64, dstate=64, ngroups=2, chunk_len=128),
+    dict(batch=2, seqlen=512, nheads=90, headdim=64, dstate=16, ngroups=1, chunk_len=256),
+    dict(batch=1, seqlen=256, nheads=93, headdim=64, dstate=32, ngroups=3, chunk_len=128),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_fused_state_path(oracle, shape, h0):
+    inp = make_inputs(**shape, dtype="bf16", seed=17, init_state=h0)
+    d = binding.make_dims(**{k: shape[k] for k in ("batch", "seqlen", "nheads", "headdim",
+                                                     "dstate", "ngroups")}, dtype="bf16")
+    assert binding.workspace_layout(d, shape["chunk_len"]).fused_state == 1
+    check_full(inp, oracle)
+
+
+def test_fused_state_intermediates(oracle):
+    """s_in written by the fused kernel, against the fp64 chunked form."""
+    shape = dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=128, ngroups=1)
+    inp = make_inputs(**shape, chunk_len=128, dtype="bf16", seed=18, init_state=True)
+    a = to_dev(inp)
+    lay = binding.workspace_layout(binding.make_dims(**shape, dtype="bf16"), 128)
+    assert lay.fused_state == 1
+    ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device="cuda:0")
+    binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=128,
+                    init_state=a["init_state"], return_final_state=True, workspace=ws)
+    torch.cuda.synchronize()
+    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, 128, D=inp.D, h0=inp.h0,
+                                  intermediates=True)
+    n = it["s_in"].size
+    s_in = ws[lay.s_in_offset: lay.s_in_offset + 2 * n].view(torch.bfloat16)
+    s_in = s_in.double().cpu().numpy().reshape(it["s_in"].shape)
+    assert rel(s_in, it["s_in"]) < 2e-2
 
 
 # ---------------------------------------------------------------------------
