@@ -119,6 +119,30 @@ SSD_API ssd_status_t ssd_forward_ws(const ssd_dims_t *dims, const void *x, const
                             void *stream);
 
 /*
+ * ssd_forward_static -- ssd_forward without any allocation.  The pages have no
+ * counterpart: this is a library-level convenience for callers that cannot
+ * hand in a workspace and must not allocate (their device memory is held by
+ * another allocator, or a cudaMalloc's device-wide synchronisation is not
+ * acceptable where they run).
+ *
+ * Arguments, layouts, ownership and accuracy are those of ssd_forward.  The
+ * intermediates live in one statically sized device array of
+ * SSD_STATIC_SCRATCH_BYTES per device (64 MiB; e.g. the 8 x 2048-token,
+ * 24-head, P = 64, N = 128 layer at chunk_len 256 needs 54 MiB).  A call whose
+ * ssd_workspace_bytes exceeds that returns SSD_ERR_WORKSPACE before any CUDA
+ * call.  The array's address is looked up once per device on the first call
+ * there (set-up), so make that first call before any stream capture.  Nothing
+ * in the array needs to start at zero.  All calls on a device share it: calls
+ * that overlap in time (different streams, unordered host threads) race; calls
+ * in order on one stream do not.
+ */
+#define SSD_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+SSD_API ssd_status_t ssd_forward_static(const ssd_dims_t *dims, const void *x, const float *dt,
+                                const float *A, const void *Bm, const void *Cm, const float *D,
+                                int chunk_len, const float *init_state, void *y_out,
+                                float *final_state_out, void *stream);
+
+/*
  * ssd_forward_stage -- run ONE of the four kernels of ssd_forward_ws, with the
  * same arguments and the same launch configuration, reading the earlier
  * stages' results from `workspace` and writing its own there (or to y_out /

@@ -21,7 +21,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
           7: "SSD_ERR_WORKSPACE"}
 
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
-           "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version")
+           "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
+           "ssd_forward_static")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -72,6 +73,8 @@ def load():
     lib.ssd_forward_ws.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp, vp, fp,
                                    vp, ctypes.c_size_t, vp]
     lib.ssd_forward_ws.restype = ctypes.c_int
+    lib.ssd_forward_static.argtypes = lib.ssd_forward.argtypes
+    lib.ssd_forward_static.restype = ctypes.c_int
     lib.ssd_forward_stage.argtypes = [ctypes.c_int] + lib.ssd_forward_ws.argtypes
     lib.ssd_forward_stage.restype = ctypes.c_int
     lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
@@ -188,6 +191,34 @@ def forward_ws(*args, **kwargs):
     if kwargs.get("workspace") is None:
         raise ValueError("forward_ws needs workspace=")
     return forward(*args, **kwargs)
+
+
+def forward_static(x, dt, A, B, C, D=None, chunk_len=256, init_state=None,
+                   return_final_state=False, out=None, final_out=None, stream=None):
+    """``forward`` through ``ssd_forward_static``: the intermediates live in the
+    library's fixed per-device scratch array, and nothing is allocated.  A
+    workload whose workspace exceeds ``STATIC_SCRATCH_BYTES`` raises (status
+    SSD_ERR_WORKSPACE); calls that overlap in time on one device race on the
+    shared scratch."""
+    dims = _validate(x, dt, A, B, C, D, init_state)
+    y = out if out is not None else torch.empty_like(x)
+    fin = final_out
+    if fin is None and return_final_state:
+        fin = torch.empty((dims.batch, dims.nheads, dims.headdim, dims.dstate),
+                          dtype=torch.float32, device=x.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device).cuda_stream
+    with torch.cuda.device(x.device):
+        st = load().ssd_forward_static(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                       _ptr(C), _ptr(D), int(chunk_len), _ptr(init_state),
+                                       _ptr(y), _ptr(fin), ctypes.c_void_p(stream))
+    _check(st)
+    if return_final_state or final_out is not None:
+        return y, fin
+    return y
+
+
+STATIC_SCRATCH_BYTES = 64 << 20  # SSD_STATIC_SCRATCH_BYTES in include/ssd.h
 
 
 def device_status(device=None) -> int:
