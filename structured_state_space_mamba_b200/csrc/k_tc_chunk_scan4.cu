@@ -43,6 +43,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
+#include "tc_scan_common.cuh"
 #include "tma_host.h"
 
 namespace ssd {
@@ -60,10 +61,6 @@ constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kColCBd = 0, kColP = 128, kColTmp = 128, kColAcc = 256;
 
-__host__ __device__ constexpr int row_bytes(int n) { return n >= 64 ? 128 : n * 2; }
-__host__ __device__ constexpr uint32_t kmajor_swz(int n) { return n >= 64 ? kSw128 : (n == 32 ? kSw64 : kSw32); }
-__host__ __device__ constexpr uint32_t up1k(uint32_t v) { return (v + 1023u) & ~1023u; }
-__host__ __device__ constexpr uint32_t umax(uint32_t a, uint32_t b) { return a > b ? a : b; }
 
 struct Smem4 {
     uint32_t c_off, b_off, stage_off, stage_bytes, x_rel, s_rel, l_rel, dt_rel, beta_rel;
@@ -89,27 +86,31 @@ __host__ __device__ inline Smem4 scan4_smem(int Q, int N) {
     return s;
 }
 
-// K-major operand descriptor for K step k of a tile split into 64-column slabs
-// of `rows` rows (N >= 64) or a single slab of narrower rows (N = 16, 32).
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int k, int rows, int n) {
-    if (n >= 64) return smem_desc(base + (k >> 2) * rows * 128 + (k & 3) * 32, 16, 1024, kSw128);
-    return smem_desc(base + k * 32, 16, 8 * row_bytes(n), kmajor_swz(n));
-}
 
-// Scale every bf16 of `n16` 16-byte chunks starting at `p` by f(chunk index);
-// thread i handles chunks i, i + nthr, ...
-template <typename F>
-__device__ __forceinline__ void scale_chunks(uint8_t *p, int n16, int i, int nthr, F f) {
-    for (int k = i; k < n16; k += nthr) {
-        const float sc = f(k);
-        uint4 *q = reinterpret_cast<uint4 *>(p) + k;
-        uint4 v = *q;
-        v.x = pack_bf16x2(bf16lo(v.x) * sc, bf16hi(v.x) * sc);
-        v.y = pack_bf16x2(bf16lo(v.y) * sc, bf16hi(v.y) * sc);
-        v.z = pack_bf16x2(bf16lo(v.z) * sc, bf16hi(v.z) * sc);
-        v.w = pack_bf16x2(bf16lo(v.w) * sc, bf16hi(v.w) * sc);
-        *q = v;
+// Work unit u: (b, c, tile mt, first head h0).  Normally units enumerate
+// (b, c, mt, head block of hpc heads); in list mode (items != nullptr, hpc = 1)
+// unit u is the packed item items[u] = b << 40 | c << 24 | mt << 16 | h.
+struct Unit4 {
+    int b, c, mt, h0;
+};
+__device__ __forceinline__ Unit4 unit_at(int u, const Dims &d, int hpc, int ntiles,
+                                         const long long *items) {
+    Unit4 x;
+    if (items) {
+        const long long v = items[u];
+        x.b = int(v >> 40);
+        x.c = int((v >> 24) & 0xFFFF);
+        x.mt = int((v >> 16) & 0xFF);
+        x.h0 = int(v & 0xFFFF);
+    } else {
+        const int nhb = d.H / hpc;
+        const int rest = u / nhb;
+        x.h0 = (u % nhb) * hpc;
+        x.mt = rest % ntiles;
+        x.c = (rest / ntiles) % d.nc;
+        x.b = (rest / ntiles) / d.nc;
     }
+    return x;
 }
 
 template <int N>
@@ -119,8 +120,10 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_y, Dims d, int hpc, int units,
                    const float *__restrict__ dtq, const float *__restrict__ betaq,
                    const float *__restrict__ Dskip, const float *__restrict__ lcum,
+                   const long long *__restrict__ items, const int *__restrict__ nitems,
                    unsigned int *err) {
     if (device_failed(err)) return;  // an earlier wait expired: skip all work
+    if (items) units = min(*nitems, units);  // list mode: the listed (b, c, tile, head) items
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int Q = d.Q;
@@ -140,7 +143,6 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntiles = Q / kRows;
-    const int nhb = d.H / hpc;
     constexpr int kSlabs = N >= 64 ? N / 64 : 1;
     constexpr int kRB = row_bytes(N);
 
@@ -180,12 +182,9 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             uint32_t ui = 0, hit = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
-                const int hb = u % nhb;
-                const int rest = u / nhb;
-                const int mt = rest % ntiles;
-                const int bc = rest / ntiles;
-                const int c = bc % d.nc, b = bc / d.nc;
-                const int h0 = hb * hpc, g = h0 / d.r;
+                const Unit4 U = unit_at(u, d, hpc, ntiles, items);
+                const int mt = U.mt, c = U.c, b = U.b;
+                const int h0 = U.h0, g = h0 / d.r;
                 const int s_len = (mt + 1) * kRows;
                 const int trow0 = b * d.T + c * Q;
                 // C and B of this unit, once the previous unit's MMAs are done
@@ -232,7 +231,7 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             const uint32_t idX = idesc_bf16_f32(kRows, 64, 0, 1);
             const uint32_t idS = idesc_bf16_f32(kRows, 64, 0, 0);
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
-                const int mt = (u / nhb) % ntiles;
+                const int mt = unit_at(u, d, hpc, ntiles, items).mt;
                 const int s_len = (mt + 1) * kRows;
                 if (!mbar_wait(ld_cb, ui & 1, err)) break;
                 tc_fence_after();
@@ -294,8 +293,8 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         uint32_t ui = 0, hit = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
-            const int hb = u % nhb;
-            const int mt = (u / nhb) % ntiles;
+            const Unit4 U = unit_at(u, d, hpc, ntiles, items);
+            const int mt = U.mt;
             const int t0 = mt * kRows;
             if (!mbar_wait(cb_full, ui & 1, err)) break;
             tc_fence_after();
@@ -322,7 +321,7 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             tc_fence_after();
             for (int hi = 0; hi < hpc; ++hi, ++hit) {
                 const int st = hit & 1, pb = hit & 1, ab = hit & 1;
-                const int h = hb * hpc + hi;
+                const int h = U.h0 + hi;
                 uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
                 const float *sl_ = reinterpret_cast<const float *>(stage + L.l_rel);
                 const float *sdt = reinterpret_cast<const float *>(stage + L.dt_rel);
@@ -428,14 +427,11 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         uint32_t hit = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            const int hb = u % nhb;
-            const int rest = u / nhb;
-            const int mt = rest % ntiles;
-            const int bc = rest / ntiles;
-            const int c = bc % d.nc, b = bc / d.nc;
+            const Unit4 U = unit_at(u, d, hpc, ntiles, items);
+            const int mt = U.mt, c = U.c, b = U.b;
             for (int hi = 0; hi < hpc; ++hi, ++hit) {
                 const int ab = hit & 1;
-                const int h = hb * hpc + hi;
+                const int h = U.h0 + hi;
                 if (!mbar_wait(&acc_full[ab], (hit >> 1) & 1, err)) { ok = false; break; }
                 // the staging tile is free once the previous TMA store has read it
                 if (!mbar_wait(y_free, (hit & 1) ^ 1, err)) { ok = false; break; }
@@ -502,17 +498,19 @@ int heads_per_cta4(const Dims &d, int sms) {
 
 template <int N>
 cudaError_t launch4(const Dims &d, const CUtensorMap *maps, int hpc, const float *dtq,
-                    const float *beta, const float *D, const float *l, unsigned int *err,
-                    cudaStream_t stream) {
+                    const float *beta, const float *D, const float *l, const long long *items,
+                    const int *nitems, int max_items, unsigned int *err, cudaStream_t stream) {
     const Smem4 L = scan4_smem(d.Q, N);
     const int smem = int(L.total < 116 * 1024 ? 116 * 1024 : L.total);
     if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan4_kernel<N>), smem))
         return cudaErrorInvalidValue;
-    const int units = d.B * d.nc * (d.Q / kRows) * (d.H / hpc);
+    const int units = items ? max_items : d.B * d.nc * (d.Q / kRows) * (d.H / hpc);
     const int sms = device_sm_count();
     const int grid = units < sms ? units : sms;
+    if (grid == 0) return cudaSuccess;
     chunk_scan4_kernel<N><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
-                                                          d, hpc, units, dtq, beta, D, l, err);
+                                                          d, hpc, units, dtq, beta, D, l, items,
+                                                          nitems, err);
     return cudaGetLastError();
 }
 
@@ -528,6 +526,7 @@ bool tc_chunk_scan4_supported(const Dims &d) {
 cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq,
                                   const float *beta, const void *Bm, const void *Cm,
                                   const float *D, const float *l, const void *s_in_bf16, void *y,
+                                  const long long *items, const int *nitems, int max_items,
                                   unsigned int *err, cudaStream_t stream) {
     const uint32_t nbox = uint32_t(d.N >= 64 ? 64 : d.N);
     const int rb = row_bytes(d.N);
@@ -547,12 +546,12 @@ cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq
         !make_tmap_bf16(&maps[3], 2, s_in_bf16, sdims, sstr, sbox, rb) ||
         !make_tmap_bf16(&maps[4], 3, y, xdims, xstr, xbox, 128))
         return cudaErrorInvalidValue;
-    const int hpc = heads_per_cta4(d, device_sm_count());
+    const int hpc = items ? 1 : heads_per_cta4(d, device_sm_count());
     switch (d.N) {
-        case 16: return launch4<16>(d, maps, hpc, dtq, beta, D, l, err, stream);
-        case 32: return launch4<32>(d, maps, hpc, dtq, beta, D, l, err, stream);
-        case 64: return launch4<64>(d, maps, hpc, dtq, beta, D, l, err, stream);
-        case 128: return launch4<128>(d, maps, hpc, dtq, beta, D, l, err, stream);
+        case 16: return launch4<16>(d, maps, hpc, dtq, beta, D, l, items, nitems, max_items, err, stream);
+        case 32: return launch4<32>(d, maps, hpc, dtq, beta, D, l, items, nitems, max_items, err, stream);
+        case 64: return launch4<64>(d, maps, hpc, dtq, beta, D, l, items, nitems, max_items, err, stream);
+        case 128: return launch4<128>(d, maps, hpc, dtq, beta, D, l, items, nitems, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -49,9 +49,21 @@ cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, 
 // Persistent warp-specialised variant (dstate <= 128); dtq and beta come from
 // ssd_chunk_cumsum.  Writes y with TMA stores.
 bool tc_chunk_scan4_supported(const Dims &d);
+// items == nullptr: every (b, c, tile, head); otherwise list mode: the *nitems
+// packed (b, c, tile, head) items (at most max_items) that the chunk-wide scan
+// left to this kernel
 cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq,
                                   const float *beta, const void *Bm, const void *Cm,
                                   const float *D, const float *l, const void *s_in_bf16, void *y,
+                                  const long long *items, const int *nitems, int max_items,
+                                  unsigned int *err, cudaStream_t stream);
+// chunk-wide tensor-core scan: one accumulator per 128-row tile; tiles with a
+// decay range >= 64 are appended to (nsteep, items) for the kernel above
+bool tc_chunk_scan5_supported(const Dims &d);
+int chunk_scan5_max_steep(const Dims &d);
+cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *dtq, const void *Bm,
+                                  const void *Cm, const float *D, const float *l,
+                                  const void *s_in_bf16, void *y, int *nsteep, long long *items,
                                   unsigned int *err, cudaStream_t stream);
 
 }  // namespace ssd

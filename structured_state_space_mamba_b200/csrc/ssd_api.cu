@@ -57,6 +57,8 @@ struct Plan {
     bool tc_state;  // tcgen05 chunk state
     bool tc_scan;   // tcgen05 chunk scan (consumes bf16 s_in)
     bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
+    bool scan5;     // chunk-wide scan, steep tiles finished by the block-factored scan
+    size_t steep_offset;  // scan5: item counter (256 bytes) + packed steep items
     ssd_workspace_layout_t ws;
 };
 
@@ -90,6 +92,7 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     // the fused state kernel walks each (b, head pair) over all chunks: used when
     // those units fill most of the GPU's 148 SMs in one wave
     plan->fused = plan->tc_state && plan->tc_scan && ssd::tc_state_fused_supported(d, kB200Sms);
+    plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d) && ssd::tc_chunk_scan4_supported(d);
 
     ssd_workspace_layout_t &w = plan->ws;
     std::memset(&w, 0, sizeof(w));
@@ -108,9 +111,11 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.s_in_offset = off;
     w.s_in_dtype = plan->tc_scan ? SSD_BF16 : SSD_F32;
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
+    plan->steep_offset = off;
+    if (plan->scan5) off = align_up(off + kAlign + sizeof(long long) * size_t(ssd::chunk_scan5_max_steep(d)));
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
-    w.launches = plan->fused ? 3 : 4;
+    w.launches = (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
     w.fused_state = plan->fused ? 1 : 0;
     return SSD_OK;
 }
@@ -151,12 +156,17 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     float *alpha = reinterpret_cast<float *>(ws + pl.ws.alpha_offset);
     void *states = ws + pl.ws.states_offset;
     void *s_in = ws + pl.ws.s_in_offset;
+    int *nsteep = reinterpret_cast<int *>(ws + pl.steep_offset);
+    long long *steep_items = reinterpret_cast<long long *>(ws + pl.steep_offset + kAlign);
     for (int stage = 0; stage < 4; ++stage) {
         if (only_stage >= 0 && stage != only_stage) continue;
         cudaError_t e = cudaSuccess;
         switch (stage) {
             case SSD_STAGE_CHUNK_CUMSUM:
-                e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, stream);
+                // the steep-tile list of the chunk-wide scan starts empty each call
+                if (pl.scan5) e = cudaMemsetAsync(nsteep, 0, sizeof(int), stream);
+                if (e == cudaSuccess)
+                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.fused ? ssd::launch_state_fused(d, x, Bm, w, alpha, init_state, s_in, fin, err, stream)
@@ -170,12 +180,24 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                                               pl.tc_scan, fin, stream);
                 break;
             case SSD_STAGE_CHUNK_SCAN:
-                e = pl.tc_scan
-                        ? (ssd::tc_chunk_scan4_supported(d)
-                               ? ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, err, stream)
-                               : ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream))
-                        : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt, Bm, Cm, D, l,
-                                                      static_cast<const float *>(s_in), y, stream);
+                if (pl.scan5) {
+                    // chunk-wide scan, then the block-factored scan over the tiles
+                    // it listed as steep (an empty list costs one short launch)
+                    e = ssd::launch_chunk_scan_tc5(d, x, dtq, Bm, Cm, D, l, s_in, y, nsteep,
+                                                   steep_items, err, stream);
+                    if (e == cudaSuccess)
+                        e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
+                                                       steep_items, nsteep,
+                                                       ssd::chunk_scan5_max_steep(d), err, stream);
+                } else {
+                    e = pl.tc_scan
+                            ? (ssd::tc_chunk_scan4_supported(d)
+                                   ? ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
+                                                                nullptr, nullptr, 0, err, stream)
+                                   : ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream))
+                            : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt, Bm, Cm, D, l,
+                                                          static_cast<const float *>(s_in), y, stream);
+                }
                 break;
         }
         if (e != cudaSuccess) return SSD_ERR_CUDA;
