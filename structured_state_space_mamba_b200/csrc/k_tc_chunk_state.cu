@@ -48,13 +48,18 @@ __host__ __device__ constexpr uint32_t stage_bytes(int ns) {
     return ((x_stage_bytes() + b_stage_bytes(ns) + w_stage_bytes()) + 1023u) & ~1023u;
 }
 
-size_t state_smem_bytes(int NS) { return 1024 + size_t(num_stages(NS)) * stage_bytes(NS) + 256; }
+// Per epilogue warp, two 32 x 32 bf16 staging blocks (64-byte rows) for the
+// TMA stores of the chunk states.
+constexpr uint32_t kStgWarpBytes = 2 * 32 * 64;
+__host__ __device__ constexpr uint32_t stg_off(int ns) { return uint32_t(num_stages(ns)) * stage_bytes(ns) + 1024; }
+size_t state_smem_bytes(int NS) { return 1024 + stg_off(NS) + 4 * kStgWarpBytes; }
 
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                      Dims d, int nh, int units, const float *__restrict__ w,
-                      __nv_bfloat16 *__restrict__ states, unsigned int *err) {
+                      const __grid_constant__ CUtensorMap tm_st, Dims d, int nh, int units,
+                      const float *__restrict__ w, __nv_bfloat16 *__restrict__ states,
+                      unsigned int *err) {
     constexpr int kAcc = acc_cols(NS);
     constexpr int kStages = num_stages(NS);
     constexpr int kCols = tmem_alloc_cols(NS);
@@ -175,19 +180,27 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
                 if (!mbar_wait(&full[s], (it / kStages) & 1, err)) { ok = false; break; }
                 uint8_t *sx = smem + s * stage_bytes(NS);
                 const float *sw = reinterpret_cast<const float *>(sx + x_stage_bytes() + b_stage_bytes(NS));
+                // every load first, then the stores: the shared-memory stores may
+                // alias the loads, so a fused loop would run at load latency
+                constexpr int kPer = (2 * kKS * 8) / 128;
+                uint4 v[kPer];
+                float wv[kPer];
 #pragma unroll
-                for (int k = 0; k < (2 * kKS * 8) / 128; ++k) {
+                for (int k = 0; k < kPer; ++k) {
                     const int i = st + k * 128;
-                    const int row = i >> 3;
-                    if ((row >> 6) < nh) {
-                        const float wv = sw[row];
-                        uint4 *p = reinterpret_cast<uint4 *>(sx) + i;
-                        uint4 v = *p;
-                        v.x = pack_bf16x2(bf16lo(v.x) * wv, bf16hi(v.x) * wv);
-                        v.y = pack_bf16x2(bf16lo(v.y) * wv, bf16hi(v.y) * wv);
-                        v.z = pack_bf16x2(bf16lo(v.z) * wv, bf16hi(v.z) * wv);
-                        v.w = pack_bf16x2(bf16lo(v.w) * wv, bf16hi(v.w) * wv);
-                        *p = v;
+                    v[k] = reinterpret_cast<const uint4 *>(sx)[i];
+                    wv[k] = sw[i >> 3];
+                }
+#pragma unroll
+                for (int k = 0; k < kPer; ++k) {
+                    const int i = st + k * 128;
+                    if (((i >> 3) >> 6) < nh) {
+                        uint4 o;
+                        o.x = pack_bf16x2(bf16lo(v[k].x) * wv[k], bf16hi(v[k].x) * wv[k]);
+                        o.y = pack_bf16x2(bf16lo(v[k].y) * wv[k], bf16hi(v[k].y) * wv[k]);
+                        o.z = pack_bf16x2(bf16lo(v[k].z) * wv[k], bf16hi(v[k].z) * wv[k]);
+                        o.w = pack_bf16x2(bf16lo(v[k].w) * wv[k], bf16hi(v[k].w) * wv[k]);
+                        reinterpret_cast<uint4 *>(sx)[i] = o;
                     }
                 }
                 fence_proxy_async_smem();
@@ -197,37 +210,53 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         }
     } else {
         // ------------------------------ epilogue ----------------------------------
+        // Warp qd owns TMEM rows m = 32 qd + lane = (head j = qd / 2, p).  For
+        // N >= 32 each 32 x 32 block goes out as bf16 through a swizzled staging
+        // block and one 2-D TMA store (coalesced, and off the load/store unit
+        // that the scale warps use); N = 16 rows are stored directly.
         const int qd = warp & 3;
         const int m = qd * 32 + lane;
         const int j = m >> 6, p = m & 63;
-        uint32_t ui = 0;
+        const bool valid = j < nh;  // warp-uniform
+        uint8_t *stg = smem + stg_off(NS) + qd * kStgWarpBytes;
+        uint32_t ui = 0, nst = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++ui) {
             const int a = ui & 1;
             if (!mbar_wait(&accf[a], (ui >> 1) & 1, err)) break;
             tc_fence_after();
             const int hp = u % nhp, bc = u / nhp;
             const int c = bc % d.nc, b = bc / d.nc;
-            const int h = hp * nh + (j < nh ? j : 0);
-            __nv_bfloat16 *dst = states + off_state(d, b, c, h) + int64_t(p) * NS;
+            const int h = hp * nh + (valid ? j : 0);
             const uint32_t taddr = tmem + (uint32_t(qd * 32) << 16) + a * kAcc;
             if (NS >= 32) {
+                const int row0 = ((b * d.nc + c) * d.H + h) * 64 + (qd & 1) * 32;
 #pragma unroll 1
-                for (int n0 = 0; n0 < NS; n0 += 32) {
+                for (int n0 = 0; n0 < NS; n0 += 32, ++nst) {
                     float v[32];
                     tmem_ld32(taddr + n0, v);
-                    if (j < nh) {
-                        uint4 *o = reinterpret_cast<uint4 *>(dst + n0);
+                    if (valid) {
+                        uint8_t *blk = stg + (nst & 1) * (32 * 64);
+                        // the store that used this block two stores ago has read it
+                        if (lane == 0) bulk_wait_read_1();
+                        __syncwarp();
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                              pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                            *reinterpret_cast<uint4 *>(blk + sw64_off(lane, q)) =
+                                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_st, blk, n0, row0);
+                            bulk_commit();
+                        }
                     }
                 }
             } else {
                 float v[16];
                 tmem_ld16(taddr, v);
-                if (j < nh) {
-                    uint4 *o = reinterpret_cast<uint4 *>(dst);
+                if (valid) {
+                    uint4 *o = reinterpret_cast<uint4 *>(states + off_state(d, b, c, h) + int64_t(p) * NS);
 #pragma unroll
                     for (int q = 0; q < 2; ++q)
                         o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
@@ -237,6 +266,7 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
             tc_fence_before();
             mbar_arrive(&acce[a]);
         }
+        if (lane == 0) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -244,14 +274,15 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
 }
 
 template <int NS>
-cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb, int nh,
+cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb,
+                      const CUtensorMap &tst, int nh,
                       const float *w, __nv_bfloat16 *states, unsigned int *err, cudaStream_t stream) {
     const size_t smem = state_smem_bytes(NS);
     if (!smem_attr_once(reinterpret_cast<const void *>(chunk_state_tc_kernel<NS>), int(smem)))
         return cudaErrorInvalidValue;
     const int units = d.B * d.nc * (d.H / nh);
     const int grid = units < device_sm_count() ? units : device_sm_count();
-    chunk_state_tc_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, d, nh, units, w, states, err);
+    chunk_state_tc_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, tst, d, nh, units, w, states, err);
     return cudaGetLastError();
 }
 
@@ -273,18 +304,23 @@ cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, 
     const uint64_t bdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
     const uint64_t bstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
     const uint32_t bbox[3] = {uint32_t(d.N >= 64 ? 64 : d.N), 1, uint32_t(kKS)};
-    CUtensorMap tx, tb;
+    // states viewed as [B*nc*H*P rows][N]; box = 32 columns x 32 rows
+    const uint64_t sdims[2] = {uint64_t(d.N), uint64_t(d.B) * d.nc * d.H * d.P};
+    const uint64_t sstr[1] = {uint64_t(d.N) * 2};
+    const uint32_t sbox[2] = {32, 32};
+    CUtensorMap tx, tb, tst{};
     if (!make_tmap_bf16(&tx, 3, x, xdims, xstr, xbox, 128) ||
-        !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)))
+        !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)) ||
+        (d.N >= 32 && !make_tmap_bf16(&tst, 2, states_bf16, sdims, sstr, sbox, 64)))
         return cudaErrorInvalidValue;
     const int nh = (d.r % 2 == 0) ? 2 : 1;
     auto *st = static_cast<__nv_bfloat16 *>(states_bf16);
     switch (d.N) {
-        case 16: return launch_ns<16>(d, tx, tb, nh, w, st, err, stream);
-        case 32: return launch_ns<32>(d, tx, tb, nh, w, st, err, stream);
-        case 64: return launch_ns<64>(d, tx, tb, nh, w, st, err, stream);
-        case 128: return launch_ns<128>(d, tx, tb, nh, w, st, err, stream);
-        case 256: return launch_ns<256>(d, tx, tb, nh, w, st, err, stream);
+        case 16: return launch_ns<16>(d, tx, tb, tst, nh, w, st, err, stream);
+        case 32: return launch_ns<32>(d, tx, tb, tst, nh, w, st, err, stream);
+        case 64: return launch_ns<64>(d, tx, tb, tst, nh, w, st, err, stream);
+        case 128: return launch_ns<128>(d, tx, tb, tst, nh, w, st, err, stream);
+        case 256: return launch_ns<256>(d, tx, tb, tst, nh, w, st, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -58,7 +58,11 @@ __host__ __device__ constexpr uint32_t w_bytes() { return 2 * kKS * 4; }
 __host__ __device__ constexpr uint32_t stage_bytes(int ns) {
     return ((x_bytes() + b_bytes(ns) + w_bytes()) + 1023u) & ~1023u;
 }
-size_t fused_smem_bytes(int ns) { return 1024 + size_t(num_stages(ns)) * stage_bytes(ns) + 256; }
+// Per update warp, two 32 x 32 bf16 staging blocks (64-byte rows) for the TMA
+// stores of s_in.
+constexpr uint32_t kStgWarpBytes = 2 * 32 * 64;
+__host__ __device__ constexpr uint32_t stg_off(int ns) { return uint32_t(num_stages(ns)) * stage_bytes(ns) + 1024; }
+size_t fused_smem_bytes(int ns) { return 1024 + stg_off(ns) + 4 * kStgWarpBytes; }
 
 __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *v, int n) {
     uint4 *o = reinterpret_cast<uint4 *>(dst);
@@ -70,7 +74,8 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                   Dims d, int nh, int units, const float *__restrict__ w,
+                   const __grid_constant__ CUtensorMap tm_s, Dims d, int nh, int units,
+                   const float *__restrict__ w,
                    const float *__restrict__ alpha, const float *__restrict__ h0,
                    __nv_bfloat16 *__restrict__ s_in, float *__restrict__ fin, unsigned int *err) {
     constexpr int kAcc = acc_cols(NS);
@@ -198,19 +203,27 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     if (!mbar_wait(&full[s], (it / kStages) & 1, err)) { ok = false; break; }
                     uint8_t *sx = smem + s * stage_bytes(NS);
                     const float *sw = reinterpret_cast<const float *>(sx + x_bytes() + b_bytes(NS));
+                    // every load first, then the stores: the shared-memory stores may
+                    // alias the loads, so a fused loop would run at load latency
+                    constexpr int kPer = (2 * kKS * 8) / 128;
+                    uint4 v[kPer];
+                    float wv[kPer];
 #pragma unroll
-                    for (int k = 0; k < (2 * kKS * 8) / 128; ++k) {
+                    for (int k = 0; k < kPer; ++k) {
                         const int i = st + k * 128;
-                        const int row = i >> 3;
-                        if ((row >> 6) < nh) {
-                            const float wv = sw[row];
-                            uint4 *p = reinterpret_cast<uint4 *>(sx) + i;
-                            uint4 v = *p;
-                            v.x = pack_bf16x2(bf16lo(v.x) * wv, bf16hi(v.x) * wv);
-                            v.y = pack_bf16x2(bf16lo(v.y) * wv, bf16hi(v.y) * wv);
-                            v.z = pack_bf16x2(bf16lo(v.z) * wv, bf16hi(v.z) * wv);
-                            v.w = pack_bf16x2(bf16lo(v.w) * wv, bf16hi(v.w) * wv);
-                            *p = v;
+                        v[k] = reinterpret_cast<const uint4 *>(sx)[i];
+                        wv[k] = sw[i >> 3];
+                    }
+#pragma unroll
+                    for (int k = 0; k < kPer; ++k) {
+                        const int i = st + k * 128;
+                        if (((i >> 3) >> 6) < nh) {
+                            uint4 o;
+                            o.x = pack_bf16x2(bf16lo(v[k].x) * wv[k], bf16hi(v[k].x) * wv[k]);
+                            o.y = pack_bf16x2(bf16lo(v[k].y) * wv[k], bf16hi(v[k].y) * wv[k]);
+                            o.z = pack_bf16x2(bf16lo(v[k].z) * wv[k], bf16hi(v[k].z) * wv[k]);
+                            o.w = pack_bf16x2(bf16lo(v[k].w) * wv[k], bf16hi(v[k].w) * wv[k]);
+                            reinterpret_cast<uint4 *>(sx)[i] = o;
                         }
                     }
                     fence_proxy_async_smem();
@@ -221,19 +234,47 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         }
     } else {
         // --------------------------- state update + stores --------------------------
-        // Thread (lane quarter qd, lane) owns TMEM row m = (head j, p).
+        // Thread (lane quarter qd, lane) owns TMEM row m = (head j, p).  For
+        // N >= 32 each 32 x 32 block of s_in goes out as bf16 through a swizzled
+        // staging block and one 2-D TMA store (coalesced, and off the load/store
+        // unit that the scale warps use); N = 16 rows are stored directly.
         const int qd = warp & 3;
         const int m = qd * 32 + lane;
         const int j = m >> 6, p = m & 63;
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
         const uint32_t tR = tmem + lane_base + 2 * kAcc;  // running state
-        uint32_t ci = 0;
+        const bool valid = j < nh;  // warp-uniform
+        uint8_t *stg = smem + stg_off(NS) + qd * kStgWarpBytes;
+        uint32_t ci = 0, nst = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int hp = u % nhp, b = u / nhp;
-            const bool valid = j < nh;
             const int h = hp * nh + (valid ? j : 0);
             const int64_t row = (int64_t(b) * d.H + h) * d.P + p;  // row of [B, H, P, N]
+            // s_in[b, cc, h, p, n0 .. n0 + kSeg) = bf16(v)
+            auto emit = [&](const float *v, int cc, int n0) {
+                if (NS >= 32) {
+                    if (!valid) return;
+                    uint8_t *blk = stg + (nst & 1) * (32 * 64);
+                    // the store that used this block two stores ago has read it
+                    if (lane == 0) bulk_wait_read_1();
+                    __syncwarp();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        *reinterpret_cast<uint4 *>(blk + sw64_off(lane, q)) =
+                            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_s, blk, n0, ((b * d.nc + cc) * d.H + h) * 64 + (qd & 1) * 32);
+                        bulk_commit();
+                    }
+                    ++nst;
+                } else if (valid) {
+                    store_bf16_row(s_in + off_state(d, b, cc, h) + int64_t(p) * NS + n0, v, kSeg);
+                }
+            };
             // R = h0 (or 0); s_in[0] = R
 #pragma unroll 1
             for (int n0 = 0; n0 < NS; n0 += kSeg) {
@@ -251,7 +292,7 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 #pragma unroll
                 for (int q = 0; q < kSeg / 16; ++q)
                     tmem_st16(tR + n0 + 16 * q, reinterpret_cast<const uint32_t *>(v + 16 * q));
-                if (valid) store_bf16_row(s_in + off_state(d, b, 0, h) + int64_t(p) * NS + n0, v, kSeg);
+                emit(v, 0, n0);
             }
             tmem_wait_st();
             for (int c = 0; c < d.nc; ++c, ++ci) {
@@ -279,7 +320,7 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 #pragma unroll
                         for (int q = 0; q < kSeg / 16; ++q)
                             tmem_st16(tR + n0 + 16 * q, reinterpret_cast<const uint32_t *>(v + 16 * q));
-                        if (valid) store_bf16_row(s_in + off_state(d, b, c + 1, h) + int64_t(p) * NS + n0, v, kSeg);
+                        emit(v, c + 1, n0);
                     } else if (fin && valid) {
                         float4 *o = reinterpret_cast<float4 *>(fin + row * NS + n0);
 #pragma unroll
@@ -292,6 +333,7 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 mbar_arrive(&acce[a]);
             }
         }
+        if (lane == 0) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -299,16 +341,17 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 }
 
 template <int NS>
-cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb, int nh,
-                      const float *w, const float *alpha, const float *h0, __nv_bfloat16 *s_in,
-                      float *fin, unsigned int *err, cudaStream_t stream) {
+cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb,
+                      const CUtensorMap &ts, int nh, const float *w, const float *alpha,
+                      const float *h0, __nv_bfloat16 *s_in, float *fin, unsigned int *err,
+                      cudaStream_t stream) {
     const size_t smem = fused_smem_bytes(NS);
     if (!smem_attr_once(reinterpret_cast<const void *>(state_fused_kernel<NS>), int(smem)))
         return cudaErrorInvalidValue;
     const int units = d.B * (d.H / nh);
     const int grid = units < device_sm_count() ? units : device_sm_count();
-    state_fused_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, d, nh, units, w, alpha, h0,
-                                                             s_in, fin, err);
+    state_fused_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, ts, d, nh, units, w, alpha,
+                                                             h0, s_in, fin, err);
     return cudaGetLastError();
 }
 
@@ -337,17 +380,22 @@ cudaError_t launch_state_fused(const Dims &d, const void *x, const void *Bm, con
     const uint64_t bdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
     const uint64_t bstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
     const uint32_t bbox[3] = {nbox, 1, uint32_t(kKS)};
-    CUtensorMap tx, tb;
+    // s_in viewed as [B*nc*H*P rows][N]; box = 32 columns x 32 rows
+    const uint64_t sdims[2] = {uint64_t(d.N), uint64_t(d.B) * d.nc * d.H * d.P};
+    const uint64_t sstr[1] = {uint64_t(d.N) * 2};
+    const uint32_t sbox[2] = {32, 32};
+    CUtensorMap tx, tb, ts{};
     if (!make_tmap_bf16(&tx, 3, x, xdims, xstr, xbox, 128) ||
-        !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)))
+        !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)) ||
+        (d.N >= 32 && !make_tmap_bf16(&ts, 2, s_in_bf16, sdims, sstr, sbox, 64)))
         return cudaErrorInvalidValue;
     const int nh = fused_heads_per_unit(d);
     __nv_bfloat16 *s = static_cast<__nv_bfloat16 *>(s_in_bf16);
     switch (d.N) {
-        case 16: return launch_ns<16>(d, tx, tb, nh, w, alpha, h0, s, fin, err, stream);
-        case 32: return launch_ns<32>(d, tx, tb, nh, w, alpha, h0, s, fin, err, stream);
-        case 64: return launch_ns<64>(d, tx, tb, nh, w, alpha, h0, s, fin, err, stream);
-        case 128: return launch_ns<128>(d, tx, tb, nh, w, alpha, h0, s, fin, err, stream);
+        case 16: return launch_ns<16>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
+        case 32: return launch_ns<32>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
+        case 64: return launch_ns<64>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
+        case 128: return launch_ns<128>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
     }
     return cudaErrorInvalidValue;
 }
