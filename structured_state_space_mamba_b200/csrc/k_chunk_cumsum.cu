@@ -7,7 +7,14 @@
 //   dtq[i]  = dt_{cQ+i}                         (dt regrouped per chunk and head)
 //   beta[i] = exp(l[32k+31] - l[i]) * dt_{cQ+i}, k = i / 32
 //                                               (source factor of the factored decay
-//                                                used by the tensor-core chunk scan)
+//                                                used by the block-factored scan)
+//   gq      = the chunk-wide scan's token factors (chunk_len 128 or 256 only):
+//             gq[i] = exp(r - l[i]) dt_i (exponent clamped at 80), then one flag
+//             per 128-token tile k (1 when r - l[128k+127] >= kScanSteep or a dt
+//             of the tile is 0, below 1e-30: such tiles are computed by the
+//             block-factored scan), then r.  The reference r is 0, or l[127]
+//             when -l[Q-1] reaches kScanSteep but neither tile's own decay
+//             range does
 // The decay between tokens s <= t of one chunk is exp(l[t] - l[s]): the
 // segment-sum mask L of akillness.github.io "State Space Duality and Mamba-2",
 // "The Scalar-Identity Structural Constraint" (the product of the a_k is
@@ -33,7 +40,7 @@ __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
                     float *__restrict__ l_out, float *__restrict__ w_out,
                     float *__restrict__ dtq_out, float *__restrict__ beta_out,
-                    float *__restrict__ alpha_out) {
+                    float *__restrict__ alpha_out, float *__restrict__ gq_out) {
     constexpr int Q = 32 * E;
     __shared__ float s_dt[Q][kHeads + 1];
     const int c = blockIdx.x, b = blockIdx.z;
@@ -82,19 +89,42 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
 #pragma unroll
     for (int k = 0; k < E; ++k) w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
     if (lane == 0) alpha_out[off_alpha(d, b, h, c)] = __expf(last);
+    if (gq_out && E >= 4) {
+        float *g = gq_out + ((int64_t(b) * d.H + h) * d.nc + c) * chunk_gq(Q);
+        // reference r of the chunk-wide factors: 0, or l[127] when the decay over
+        // the whole chunk reaches kScanSteep but neither 128-token tile's does
+        const float l127 = __shfl_sync(0xffffffffu, lv[3], 31);
+        const bool shift = E == 8 && -last >= kScanSteep && -l127 < kScanSteep && l127 - last < kScanSteep;
+        const float r = shift ? l127 : 0.f;
+        bool zero = false;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            g[32 * k + lane] = __expf(fminf(r - lv[k], 80.f)) * dts[k];
+            zero |= dts[k] < 1e-30f;
+            if ((k & 3) == 3) {  // last 32 tokens of a 128-token tile
+                const bool any0 = __any_sync(0xffffffffu, zero);
+                const float lend = __shfl_sync(0xffffffffu, lv[k], 31);
+                if (lane == 0) g[Q + (k >> 2)] = (r - lend >= kScanSteep || any0) ? 1.f : 0.f;
+                zero = false;
+            }
+        }
+        if (lane == 0) g[Q + 2] = r;
+        if (lane == 0 && E == 4) g[Q + 1] = 0.f;
+        if (lane == 0) g[Q + 3] = 0.f;
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
-                                float *w, float *dtq, float *beta, float *alpha,
+                                float *w, float *dtq, float *beta, float *alpha, float *gq,
                                 cudaStream_t stream) {
     dim3 grid(d.nc, (d.H + kHeads - 1) / kHeads, d.B);
     switch (d.Q) {
-        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha); break;
-        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha); break;
-        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha); break;
-        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha); break;
+        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
+        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
+        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
+        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -9,35 +9,42 @@
 // Space Duality and Mamba-2", "The Scalar-Identity Structural Constraint" --
 // plus the state carried in from earlier chunks and the skip term).
 //
-// The chunk is split into 128-row tiles k (one or two).  With the reference
-// r_k = l_{128k-1} (r_0 = 0), u_t = exp(l_t - r_k) <= 1 and
-// g_s = exp(r_k - l_s) dt_s, every decay factorises exactly as
-// exp(l_t - l_s) dt_s = u_t g_s, so each tile needs ONE accumulator:
-//     y_t = u_t Y_k[t],
-//     Y_0 = P'_0 X_0 + C_0 s_in^T
-//     Y_1 = P'_1 X_1 + CBoff X' + C_1 S'^T,
-//     P'_k[t, s] = (C_t . B_s) g_s [s <= t] + [s = t] D_h / u_t   (t, s in tile k),
-//     X'_s = exp(l_127 - l_s) dt_s x_s (s in tile 0),   S' = exp(l_127) s_in,
-// with CBoff = C_1 B_0^T.  g_s and D_h/u_t grow like exp(decay range of the
-// tile); a tile whose range r_k - l_{128k+127} reaches kSteep is therefore not
-// computed here: its (b, c, k, h) is appended to a list that the block-factored
-// kernel of k_tc_chunk_scan4.cu finishes in a second launch.
+// With a reference r per (chunk, head), u_t = exp(l_t - r) and
+// g_s = exp(r - l_s) dt_s, every decay factorises exactly as
+// exp(l_t - l_s) dt_s = u_t g_s, so the masked scores do not depend on the head:
+//     y_t = u_t Y[t] + D_h x_t,   Y = (C B^T o M) X'' + C S'^T,
+//     X''_s = g_s x_s,  S' = e^r s_in   (scaled per head, in shared memory),
+// with M the causal mask (diagonal included); the epilogue adds the skip term
+// D_h x_t = (D_h / g_t) X''_t from the scaled rows.  The chunk is split into
+// 128-row tiles k; tile 1 also takes the sources of tile 0 through
+// CBoff = C_1 B_0^T:
+//     Y_0 = P_0 X''_0 + C_0 S'^T,   Y_1 = P_1 X''_1 + CBoff X''_0 + C_1 S'^T.
+// The masked scores P_k = C_k B_k^T o M are built once per run of heads of one
+// group in one chunk and shared by all of them; per head only x (and s_in when
+// r != 0) is scaled.
+// r is 0 (u_t <= 1), or l_127 when the chunk's decay range reaches kScanSteep
+// but neither tile's does.  g_s reaches exp(r - l_s): a tile whose
+// r - l_{128k+127} reaches kScanSteep, or with a zero dt, is flagged by the
+// cumsum kernel; it is not stored here but appended to a list that the
+// block-factored kernel of k_tc_chunk_scan4.cu finishes in a second launch.
 //
 // Work: the (b, c, h) items are split into one contiguous range per CTA
-// (persistent grid), walked in order; C and B are loaded, and C B^T computed
-// on the tensor cores, once per run of heads of one group in one chunk.  Per
-// head the x rows, s_in, l and dt of the chunk are loaded once (double
-// buffered) and both tiles are computed from them.
+// (persistent grid), walked in order.  Per head the chunk's x rows, s_in, l and
+// the factors g are loaded once (double buffered); a stage is released when
+// the head's products are done and the epilogue has read its scaled rows.
 //
-// Tensor memory (512 columns): [0,128) C_0 B_0^T and [128,256) C_1 B_1^T (fp32);
-// [256,384) the scores P'_0, P'_1 (bf16; at the start of a run this range holds
-// CBoff in fp32); [384,512) the accumulators Y_0, Y_1.  With chunk_len 128 the
-// two score/accumulator slots alternate between consecutive heads instead.
+// Tensor memory (512 columns): [0,128) P_0, P_1 (bf16); CBoff (bf16, A
+// operand of a TS product) in [256,288) and [320,352); two accumulator
+// buffers {Y_0, Y_1} at [384,512) and [128,256), alternating between heads.  At the start of a run
+// the fp32 C B^T tiles pass through them (C_0 B_0^T -> [384,512), C_1 B_1^T ->
+// [128,256), CBoff -> [256,384)), so a run starts once the accumulators of the
+// previous heads are read.
 //
-// Roles (22 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..17 scores
-// (one 32 x 32 block each: lane quarter warp % 4, column block (warp - 2) / 4),
-// warps 18..21 epilogue (y = u_t Y, each warp staging its 32 rows in shared
-// memory and writing them with its own TMA store).
+// Roles (14 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 score /
+// scale warps (two 32 x 32 score blocks each at the start of a run: lane
+// quarter warp % 4, column blocks 2 (warp - 2) / 4 + {0, 1}; x scaling per
+// head), warps 10..13 epilogue (y = u_t Y + D_h x, each warp staging its 32
+// rows, 32 columns at a time, and writing them with its own TMA stores).
 #include <cmath>
 
 #include "common.cuh"
@@ -52,39 +59,37 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 704;
+constexpr int kThreads = 448;
 constexpr int kRows = 128;
-constexpr int kScoreWarps = 16;
+constexpr int kScoreWarps = 8;
 constexpr int kScoreThreads = 32 * kScoreWarps;
 constexpr int kEpiWarp0 = 2 + kScoreWarps;
 constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 512;
-constexpr uint32_t kColCB = 0, kColP = 256, kColTmp = 256, kColAcc = 384;
-constexpr int kGStride = 384;  // floats per factor buffer: g0 [0,128), g1 [128,384)
-// Tiles whose decay range reaches this go to the block-factored kernel: the
-// factors g_s and D_h / u_t here stay below e^64.
-constexpr float kSteep = 64.f;
+constexpr uint32_t kColP = 0, kColOff = 256;
+// packed CBoff: 32-column block cb (16 bf16 pairs) within the fp32 range that
+// the two score warps of column blocks {2 (cb / 2), 2 (cb / 2) + 1} read
+__device__ __forceinline__ uint32_t off_col(int cb) { return kColOff + (cb >> 1) * 64 + (cb & 1) * 16; }
+// accumulator buffer ab of a head (hit & 1)
+__device__ __forceinline__ uint32_t acc_col(int ab) { return ab == 0 ? 384u : 128u; }
 
 struct Smem5 {
-    uint32_t c_off, b_off, stage_off, stage_bytes, x_rel, s_rel, l_rel, dt_rel;
-    uint32_t y_off, g_off, e_off, flag_off, bar_off, total;
+    uint32_t c_off, b_off, stage_off, stage_bytes, x_rel, s_rel, l_rel, g_rel;
+    uint32_t y_off, bar_off, total;
 };
 
 __host__ __device__ inline Smem5 scan5_smem(int Q, int N) {
     Smem5 s;
     s.c_off = 0;
-    s.b_off = up1k(Q * N * 2);                                      // C rows of the chunk
-    s.stage_off = s.b_off + up1k(umax(kRows * N * 2, kRows * kRows * 2));  // B rows / CBoff
+    s.b_off = up1k(Q * N * 2);                    // C rows of the chunk
+    s.stage_off = s.b_off + up1k(kRows * N * 2);  // B rows of one tile
     s.x_rel = 0;
     s.s_rel = Q * 128;
     s.l_rel = s.s_rel + up1k(64 * N * 2);
-    s.dt_rel = s.l_rel + Q * 4;
-    s.stage_bytes = up1k(s.dt_rel + Q * 4);
+    s.g_rel = s.l_rel + Q * 4;  // g (Q floats), then the per-tile steep flags
+    s.stage_bytes = up1k(s.g_rel + chunk_gq(Q) * 4);
     s.y_off = s.stage_off + 2 * s.stage_bytes;  // y staging: 128 rows x 128 bytes
-    s.g_off = s.y_off + kRows * 128;
-    s.e_off = s.g_off + 2 * kGStride * 4;
-    s.flag_off = s.e_off + 2 * kRows * 4;
-    s.bar_off = s.flag_off + 16;
+    s.bar_off = s.y_off + kRows * 128;
     s.total = s.bar_off + 256 + 1024;
     return s;
 }
@@ -97,7 +102,7 @@ __device__ __forceinline__ uint64_t c_desc(uint32_t base, int k, int kk, int Q, 
 }
 
 // Items (b, c, h) in order, h fastest; a run = consecutive items of one
-// (b, c, group).  Returns the run length starting at item i (< i1).
+// (b, c, group).  Returns the run starting at item i (< i1).
 struct Run {
     int b, c, h, g, len;
 };
@@ -113,11 +118,23 @@ __device__ __forceinline__ Run run_at(long long i, long long i1, const Dims &d) 
     return r;
 }
 
+// fp32 32 x 32 block (one TMEM row per lane) -> bf16 pairs, all columns or,
+// for a block on the diagonal, columns e <= lane only.
+template <bool kDiag>
+__device__ __forceinline__ void mask_pack(const float (&v)[32], int lane, uint32_t (&pk)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float a = (!kDiag || 2 * e <= lane) ? v[2 * e] : 0.f;
+        const float b = (!kDiag || 2 * e + 1 <= lane) ? v[2 * e + 1] : 0.f;
+        pk[e] = pack_bf16x2(a, b);
+    }
+}
+
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_s,
-                   const __grid_constant__ CUtensorMap tm_y, Dims d, const float *__restrict__ dtq,
+                   const __grid_constant__ CUtensorMap tm_y, Dims d, const float *__restrict__ gq,
                    const float *__restrict__ Dskip, const float *__restrict__ lcum,
                    int *__restrict__ nsteep, long long *__restrict__ steep_items, int max_steep,
                    unsigned int *err) {
@@ -126,21 +143,19 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int Q = d.Q;
     const bool two = Q == 2 * kRows;  // two tiles per chunk
+    const int ntile = two ? 2 : 1;
+    const int ngq = chunk_gq(Q);
     const Smem5 L = scan5_smem(Q, N);
     uint8_t *sC = smem + L.c_off;
-    uint8_t *sB = smem + L.b_off;  // B rows of one tile, then CBoff (bf16)
+    uint8_t *sB = smem + L.b_off;  // B rows of one tile
     uint8_t *sY = smem + L.y_off;  // y staging, 32 rows per epilogue warp
-    float *sG = reinterpret_cast<float *>(smem + L.g_off);   // [2][kGStride] per-token factors
-    float *sE = reinterpret_cast<float *>(smem + L.e_off);   // [2][128] row factors u_t
-    int *sFlag = reinterpret_cast<int *>(smem + L.flag_off);  // [2] tile left to the list
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *ld_c = bars + 0, *ld_b1 = bars + 1, *b0_free = bars + 2, *cb_full = bars + 3;
-    uint64_t *cvt_done = bars + 4, *cb_smem_free = bars + 5;
-    uint64_t *head_full = bars + 6, *head_free = bars + 8, *gsync = bars + 10;  // [2] each
-    uint64_t *scores_ready = bars + 12, *p_free = bars + 14;                  // [2] each
-    uint64_t *acc_full = bars + 16, *acc_free = bars + 18;                    // [2] each
-    uint64_t *scaled_ready = bars + 20, *done = bars + 21;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 22);
+    uint64_t *cvt_done = bars + 5, *cb_smem_free = bars + 6;
+    uint64_t *head_full = bars + 7, *head_free = bars + 9, *ready = bars + 11;  // [2] each
+    uint64_t *acc_full = bars + 13, *acc_free = bars + 15;                     // [2] each
+    uint64_t *done = bars + 17;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 18);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int kSlabs = N >= 64 ? N / 64 : 1;
@@ -159,14 +174,13 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         mbar_init(cb_smem_free, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&head_full[i], 1);
-            mbar_init(&head_free[i], 1);
-            mbar_init(&gsync[i], kScoreThreads);
-            mbar_init(&scores_ready[i], kScoreThreads);
-            mbar_init(&p_free[i], 1);
+            // the head's products (one commit) and the epilogue, which reads the
+            // head's scaled rows, l and g
+            mbar_init(&head_free[i], 1 + kEpiThreads);
+            mbar_init(&ready[i], kScoreThreads);
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_free[i], kEpiThreads);
         }
-        mbar_init(scaled_ready, kScoreThreads);
         mbar_init(done, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_c);
@@ -193,7 +207,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 // C of the chunk and B of tile 0, once the previous run's MMAs are done
                 if (!mbar_wait(cb_smem_free, (si & 1) ^ 1, err)) break;
                 mbar_expect_tx(ld_c, uint32_t(Q) * N * 2 + uint32_t(kRows) * N * 2);
-                for (int k = 0; k < Q / kRows; ++k)
+                for (int k = 0; k < ntile; ++k)
                     for (int sl = 0; sl < kSlabs; ++sl)
                         tma_load_3d(sC + sl * Q * 128 + k * kRows * kRB, &tm_c, ld_c, sl * 64, R.g,
                                     trow0 + k * kRows);
@@ -211,16 +225,16 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     const int h = R.h + hi;
                     if (!mbar_wait(&head_free[st], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
                     uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
-                    mbar_expect_tx(&head_full[st], uint32_t(Q) * 128 + 64u * N * 2 + 2u * Q * 4);
-                    for (int k = 0; k < Q / kRows; ++k)
+                    mbar_expect_tx(&head_full[st], uint32_t(Q) * 128 + 64u * N * 2 + uint32_t(Q + ngq) * 4);
+                    for (int k = 0; k < ntile; ++k)
                         tma_load_3d(stage + L.x_rel + k * kRows * 128, &tm_x, &head_full[st], 0, h,
                                     trow0 + k * kRows);
                     const int srow = ((R.b * d.nc + R.c) * d.H + h) * 64;
                     for (int sl = 0; sl < kSlabs; ++sl)
                         tma_load_2d(stage + L.s_rel + sl * 64 * 128, &tm_s, &head_full[st], sl * 64, srow);
-                    const int64_t lo = off_lq(d, R.b, h, R.c);
-                    bulk_load(stage + L.l_rel, lcum + lo, Q * 4, &head_full[st]);
-                    bulk_load(stage + L.dt_rel, dtq + lo, Q * 4, &head_full[st]);
+                    bulk_load(stage + L.l_rel, lcum + off_lq(d, R.b, h, R.c), Q * 4, &head_full[st]);
+                    bulk_load(stage + L.g_rel, gq + ((int64_t(R.b) * d.H + h) * d.nc + R.c) * ngq, ngq * 4,
+                              &head_full[st]);
                 }
             }
             // drain: the last loads issued must have landed before the CTA exits
@@ -245,70 +259,64 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             for (long long i = i0; i < i1 && ok; ++si) {
                 const Run R = run_at(i, i1, d);
                 i += R.len;
-                if (!mbar_wait(ld_c, si & 1, err)) break;
+                // the fp32 C B^T tiles pass through the accumulator columns: wait
+                // until the epilogue has read the previous heads' accumulators
+                for (uint32_t j = 1; j <= 2 && j <= hit && ok; ++j) {
+                    const uint32_t hh = hit - j;
+                    ok = mbar_wait(&acc_free[hh & 1], (hh >> 1) & 1, err);
+                }
+                if (!ok || !mbar_wait(ld_c, si & 1, err)) break;
                 tc_fence_after();
-                // C_0 B_0^T and, for two tiles, CBoff = C_1 B_0^T (fp32, score range)
+                // C_0 B_0^T -> [384,512) and, for two tiles, CBoff = C_1 B_0^T -> [256,384)
                 for (int kk = 0; kk < N / 16; ++kk)
-                    mma_bf16_ss(tmem + kColCB, c_desc(ca, 0, kk, Q, N), kmajor_desc(ba, kk, kRows, N), idCB,
-                                kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + acc_col(0), c_desc(ca, 0, kk, Q, N), kmajor_desc(ba, kk, kRows, N),
+                                idCB, kk > 0 ? 1u : 0u);
                 if (two) {
                     for (int kk = 0; kk < N / 16; ++kk)
-                        mma_bf16_ss(tmem + kColTmp, c_desc(ca, 1, kk, Q, N), kmajor_desc(ba, kk, kRows, N),
+                        mma_bf16_ss(tmem + kColOff, c_desc(ca, 1, kk, Q, N), kmajor_desc(ba, kk, kRows, N),
                                     idCB, kk > 0 ? 1u : 0u);
                     mma_commit(b0_free);
                     if (!mbar_wait(ld_b1, si & 1, err)) break;
                     tc_fence_after();
+                    // C_1 B_1^T -> [128,256)
                     for (int kk = 0; kk < N / 16; ++kk)
-                        mma_bf16_ss(tmem + kColCB + kRows, c_desc(ca, 1, kk, Q, N),
+                        mma_bf16_ss(tmem + acc_col(1), c_desc(ca, 1, kk, Q, N),
                                     kmajor_desc(ba, kk, kRows, N), idCB, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(cb_full);
+                // the scores of this run exist once the score warps have converted them
+                if (!mbar_wait(cvt_done, si & 1, err)) break;
+                tc_fence_after();
                 for (int hi = 0; hi < R.len; ++hi, ++hit) {
-                    const int st = hit & 1;
+                    const int st = hit & 1, ab = hit & 1;
                     const uint32_t hp = (hit >> 1) & 1;
                     const uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
                     const uint32_t xa = smem_u32(stage + L.x_rel);
                     const uint32_t sa = smem_u32(stage + L.s_rel);
-                    // tile 0 (or, for chunk_len 128, the slot of this head)
-                    const int k0 = two ? 0 : st;
-                    const uint32_t n0 = two ? (hit & 1) : hp;  // parity of this slot's use
-                    if (!mbar_wait(&head_full[st], hp, err) ||
-                        !mbar_wait(&acc_free[k0], n0 ^ 1, err)) { ok = false; break; }
+                    if (!mbar_wait(&head_full[st], hp, err) || !mbar_wait(&ready[st], hp, err) ||
+                        !mbar_wait(&acc_free[ab], hp ^ 1, err)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t acc0 = tmem + kColAcc + k0 * 64;
-                    // Y_0 = C_0 s_in^T ...
-                    for (int kk = 0; kk < N / 16; ++kk)
-                        mma_bf16_ss(acc0, c_desc(ca, 0, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS,
+                    const uint32_t acc = tmem + acc_col(ab);
+                    // Y_0 = C_0 s_in^T + P_0 X''_0 and Y_1 = C_1 s_in^T + CBoff X''_0 + P_1 X''_1,
+                    // interleaved so that consecutive products go to different
+                    // accumulators and one need not wait for the previous to finish
+                    for (int kk = 0; kk < N / 16; ++kk) {
+                        mma_bf16_ss(acc, c_desc(ca, 0, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS,
                                     kk > 0 ? 1u : 0u);
-                    // ... + P'_0 X_0
-                    if (!mbar_wait(&scores_ready[k0], n0, err)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int kk = 0; kk < kRows / 16; ++kk)
-                        mma_bf16_ts(acc0, tmem + kColP + k0 * 64 + kk * 8,
-                                    smem_desc(xa + kk * 2048, 16, 1024, kSw128), idX, 1u);
-                    mma_commit(&p_free[k0]);
-                    mma_commit(&acc_full[k0]);
-                    if (two) {
-                        const uint32_t acc1 = tmem + kColAcc + 64;
-                        if (!mbar_wait(&acc_free[1], (hit & 1) ^ 1, err) ||
-                            !mbar_wait(&scores_ready[1], hit & 1, err)) { ok = false; break; }
-                        tc_fence_after();
-                        // Y_1 = P'_1 X_1 ...
-                        for (int kk = 0; kk < kRows / 16; ++kk)
-                            mma_bf16_ts(acc1, tmem + kColP + 64 + kk * 8,
-                                        smem_desc(xa + kRows * 128 + kk * 2048, 16, 1024, kSw128), idX,
+                        if (two)
+                            mma_bf16_ss(acc + 64, c_desc(ca, 1, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS,
                                         kk > 0 ? 1u : 0u);
-                        mma_commit(&p_free[1]);
-                        // ... + CBoff X' + C_1 S'^T (operands scaled in place by the score warps)
-                        if (!mbar_wait(scaled_ready, hit & 1, err)) { ok = false; break; }
-                        tc_fence_after();
-                        for (int kk = 0; kk < kRows / 16; ++kk)
-                            mma_bf16_ss(acc1, kmajor_desc(ba, kk, kRows, kRows),
-                                        smem_desc(xa + kk * 2048, 16, 1024, kSw128), idX, 1u);
-                        for (int kk = 0; kk < N / 16; ++kk)
-                            mma_bf16_ss(acc1, c_desc(ca, 1, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS, 1u);
-                        mma_commit(&acc_full[1]);
                     }
+                    for (int kk = 0; kk < kRows / 16; ++kk) {
+                        const uint64_t x0 = smem_desc(xa + kk * 2048, 16, 1024, kSw128);
+                        mma_bf16_ts(acc, tmem + kColP + kk * 8, x0, idX, 1u);
+                        if (two) mma_bf16_ts(acc + 64, tmem + off_col(kk >> 1) + (kk & 1) * 8, x0, idX, 1u);
+                    }
+                    if (two)
+                        for (int kk = 0; kk < kRows / 16; ++kk)
+                            mma_bf16_ts(acc + 64, tmem + kColP + 64 + kk * 8,
+                                        smem_desc(xa + kRows * 128 + kk * 2048, 16, 1024, kSw128), idX, 1u);
+                    mma_commit(&acc_full[ab]);
                     mma_commit(&head_free[st]);
                 }
                 if (ok) mma_commit(cb_smem_free);
@@ -317,12 +325,10 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             mbar_wait(done, 0, nullptr);
         }
     } else if (warp < kEpiWarp0) {
-        // ================================ scores ================================
-        const int sid = tid - 64;            // 0..511
+        // ============================ scores / scaling ==========================
+        const int sid = tid - 64;            // 0..255
         const int qd = warp & 3;             // TMEM lane quarter of this warp
-        const int cb = (warp - 2) >> 2;      // 32-column block of the tile
-        const int t_local = qd * 32 + lane;  // row of the tile
-        const int j0 = cb * 32;              // first column of the block
+        const int cb0 = 2 * ((warp - 2) >> 2);  // first of its two 32-column blocks
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
         uint32_t si = 0, hit = 0;
         bool ok = true;
@@ -331,23 +337,44 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             i += R.len;
             if (!mbar_wait(cb_full, si & 1, err)) break;
             tc_fence_after();
-            if (two) {
-                // CBoff fp32 -> bf16, into shared memory as a K-major, 128B-swizzled
-                // A operand: this thread packs row t_local, columns [j0, j0 + 32)
-                uint8_t *slab = sB + (cb >> 1) * (kRows * 128);
-                float v[32];
-                tmem_ld32(tmem + lane_base + kColTmp + j0, v);
+            // ---- masked scores of this run: fp32 C B^T -> bf16 P_k, CBoff ----
+            // block (qd, cb) of a tile: below the diagonal all columns, on it the
+            // causal half, above it zeros.  P ([0,128)) overlaps no fp32 source;
+            // CBoff is packed in place, each warp within its own source columns.
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, (cb & 1) * 4 + c4)) =
-                        make_uint4(pack_bf16x2(v[8 * c4], v[8 * c4 + 1]),
-                                   pack_bf16x2(v[8 * c4 + 2], v[8 * c4 + 3]),
-                                   pack_bf16x2(v[8 * c4 + 4], v[8 * c4 + 5]),
-                                   pack_bf16x2(v[8 * c4 + 6], v[8 * c4 + 7]));
-                fence_proxy_async_smem();
+            for (int k = 0; k < 2; ++k) {
+                if (k == 1 && !two) break;
+                const uint32_t src = acc_col(k);  // C_0 B_0^T, C_1 B_1^T
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int cb = cb0 + bb;
+                    uint32_t pk[16];
+                    if (cb > qd) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else {
+                        float v[32];
+                        tmem_ld32(tmem + lane_base + src + cb * 32, v);
+                        if (cb < qd) mask_pack<false>(v, lane, pk);
+                        else mask_pack<true>(v, lane, pk);
+                    }
+                    tmem_st16(tmem + lane_base + kColP + k * 64 + cb * 16, pk);
+                }
             }
-            // every score thread is done with the CBoff range before any score
-            // (same tensor-memory columns) is written
+            if (two) {
+                // CBoff in place: packed block cb goes to the first half of this
+                // warp's own fp32 range (off_col), so no other warp's source is
+                // overwritten; one block at a time, each read before it is replaced
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    float v[32];
+                    uint32_t pk[16];
+                    tmem_ld32(tmem + lane_base + kColOff + (cb0 + bb) * 32, v);
+                    mask_pack<false>(v, lane, pk);
+                    tmem_st16(tmem + lane_base + off_col(cb0 + bb), pk);
+                }
+            }
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(cvt_done);
             if (!mbar_wait(cvt_done, si & 1, err)) break;
@@ -357,161 +384,105 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 const uint32_t hp = (hit >> 1) & 1;
                 const int h = R.h + hi;
                 uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
-                const float *sl_ = reinterpret_cast<const float *>(stage + L.l_rel);
-                const float *sdt = reinterpret_cast<const float *>(stage + L.dt_rel);
-                float *gb = sG + st * kGStride;
+                const float *gb = reinterpret_cast<const float *>(stage + L.g_rel);
                 if (!mbar_wait(&head_full[st], hp, err)) { ok = false; break; }
-                const float l127 = sl_[kRows - 1];
-                // per-token factors: g0_s = exp(-l_s) dt_s (tile 0), and for two
-                // tiles g1_s = exp(l_127 - l_s) dt_s (s < 128: X' factors; s >= 128:
-                // tile-1 column factors).  Exponents are clamped at 80: beyond
-                // kSteep the tile is left to the list anyway.
-                if (sid < kRows) {
-                    gb[sid] = __expf(fminf(-sl_[sid], 80.f)) * sdt[sid];
-                } else if (two && sid < 3 * kRows) {
-                    const int s = sid - kRows;
-                    gb[kRows + s] = __expf(fminf(l127 - sl_[s], 80.f)) * sdt[s];
-                }
-                mbar_arrive(&gsync[st]);
-                if (!mbar_wait(&gsync[st], hp, err)) { ok = false; break; }
-                const bool steep0 = -l127 >= kSteep;
-                const bool steep1 = two && (l127 - sl_[Q - 1] >= kSteep);
-                if ((sid == 0 && steep0) || (sid == 1 && steep1)) {
+                if (sid < ntile && gb[Q + sid] != 0.f) {
+                    // steep tile: left to the block-factored scan
                     const int idx = atomicAdd(nsteep, 1);
                     if (idx < max_steep)
                         steep_items[idx] = ((long long)R.b << 40) | ((long long)R.c << 24) |
                                            ((long long)sid << 16) | h;
                 }
-                const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
-                const int ntile = two ? 2 : 1;
-                for (int k = 0; k < ntile; ++k) {
-                    const int slot = two ? k : st;
-                    const uint32_t use = two ? (hit & 1) : hp;
-                    const int t0 = k * kRows;
-                    const float r = k == 0 ? 0.f : l127;
-                    // row factors for the epilogue (its previous use of this slot
-                    // has ended once the slot's accumulator is free)
-                    if (sid < kRows) {
-                        if (!mbar_wait(&acc_free[slot], use ^ 1, err)) { ok = false; break; }
-                        sE[slot * kRows + sid] = __expf(sl_[t0 + sid] - r);
-                        if (sid == 0) sFlag[slot] = k == 0 ? steep0 : steep1;
-                    }
-                    if (!mbar_wait(&p_free[slot], use ^ 1, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const float *gcol = gb + (k == 0 ? 0 : 2 * kRows) + j0;  // factors of this block
-                    const uint32_t pcol = tmem + lane_base + kColP + slot * 64 + (j0 >> 1);
-                    const uint32_t cbcol = tmem + lane_base + kColCB + k * kRows + j0;
-                    if (j0 > qd * 32) {
-                        // block above the diagonal
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                        tmem_st16(pcol, pk);
-                    } else if (j0 < qd * 32) {
-                        // block entirely below the diagonal: column factors only
-                        float v[32];
-                        tmem_ld32(cbcol, v);
-                        const float4 *g4 = reinterpret_cast<const float4 *>(gcol);
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float4 gg = g4[e];
-                            pk[2 * e] = pack_bf16x2(v[4 * e] * gg.x, v[4 * e + 1] * gg.y);
-                            pk[2 * e + 1] = pack_bf16x2(v[4 * e + 2] * gg.z, v[4 * e + 3] * gg.w);
-                        }
-                        tmem_st16(pcol, pk);
-                    } else {
-                        // block on the diagonal (warp-uniform branch): row lane of the
-                        // block sees sources 0..lane; D_h / u_t sits on the diagonal
-                        const float dfac = Dh * __expf(fminf(r - sl_[t0 + t_local], 80.f));
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            float v[16];
-                            tmem_ld16(cbcol + 16 * hf, v);
-                            const float4 *g4 = reinterpret_cast<const float4 *>(gcol + 16 * hf);
-                            uint32_t pk[8];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float4 gg = g4[e];
-                                const int c0 = 16 * hf + 4 * e;  // column within the block
-                                float p0 = c0 <= lane ? v[4 * e] * gg.x : 0.f;
-                                float p1 = c0 + 1 <= lane ? v[4 * e + 1] * gg.y : 0.f;
-                                float p2 = c0 + 2 <= lane ? v[4 * e + 2] * gg.z : 0.f;
-                                float p3 = c0 + 3 <= lane ? v[4 * e + 3] * gg.w : 0.f;
-                                if (c0 == lane) p0 += dfac;
-                                if (c0 + 1 == lane) p1 += dfac;
-                                if (c0 + 2 == lane) p2 += dfac;
-                                if (c0 + 3 == lane) p3 += dfac;
-                                pk[2 * e] = pack_bf16x2(p0, p1);
-                                pk[2 * e + 1] = pack_bf16x2(p2, p3);
-                            }
-                            tmem_st8(pcol + 8 * hf, pk);
-                        }
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(&scores_ready[slot]);
-                }
-                if (!ok) break;
-                if (two) {
-                    // X' = g1 o X_0 and S' = exp(l_127) s_in, in place, once this
-                    // head's tile-0 products (which read them unscaled) are done
-                    if (!mbar_wait(&p_free[0], hit & 1, err)) { ok = false; break; }
-                    scale_chunks(stage + L.x_rel, kRows * 8, sid, kScoreThreads,
-                                 [&](int k) { return gb[kRows + (k >> 3)]; });
-                    const float el = __expf(l127);
-                    scale_chunks(stage + L.s_rel, 64 * N * 2 / 16, sid, kScoreThreads,
-                                 [&](int) { return el; });
-                    fence_proxy_async_smem();
-                    mbar_arrive(scaled_ready);
-                }
+                // X'' = g o X in place (every row of the chunk) and, for r != 0,
+                // S' = e^r s_in, which directly follows x in the stage
+                const float r = gb[Q + 2];
+                const float er = __expf(r);
+                scale_chunks(stage + L.x_rel, r != 0.f ? Q * 8 + 8 * N : Q * 8, sid, kScoreThreads,
+                             [&](int kc) { return kc < Q * 8 ? gb[kc >> 3] : er; });
+                fence_proxy_async_smem();
+                mbar_arrive(&ready[st]);
             }
         }
     } else {
         // =============================== epilogue ===============================
-        // y_t = u_t Y[t]: each warp stages its 32 rows (128B swizzle) and writes
-        // them with its own TMA store, so the warps never wait on one another
+        // y_t = u_t Y[t] + (D_h / g_t) X''_t with u_t = exp(l_t - r): the skip term
+        // D_h x_t comes from the head's scaled rows (the cumsum kernel flags a
+        // tile with a zero dt as steep, so g_t > 0 here).  Per tile, each thread
+        // reads its scaled x row, l and g (the stage is released after the last
+        // tile's) and its accumulator row in two halves.  Each warp stages
+        // its 32 rows and writes them with its own TMA stores, so the warps never
+        // wait on one another.
         const int qd = warp & 3;
         const int t_local = qd * 32 + lane;
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
-        uint8_t *sYw = sY + qd * 32 * 128;
-        uint32_t hit = 0;
+        uint8_t *sYw = sY + qd * 32 * 128;  // two 32 x 32 bf16 blocks per warp
+        uint32_t hit = 0, nst = 0;
         bool ok = true;
         for (long long i = i0; i < i1 && ok;) {
             const Run R = run_at(i, i1, d);
             i += R.len;
             for (int hi = 0; hi < R.len && ok; ++hi, ++hit) {
                 const int h = R.h + hi;
-                const int ntile = two ? 2 : 1;
-                for (int k = 0; k < ntile; ++k) {
-                    const int slot = two ? k : (hit & 1);
-                    const uint32_t use = two ? (hit & 1) : ((hit >> 1) & 1);
-                    if (!mbar_wait(&acc_full[slot], use, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const bool store = !sFlag[slot];
-                    const float ut = sE[slot * kRows + t_local];
-                    // this warp's previous TMA store has finished reading the staging rows
-                    if (lane == 0) bulk_wait_read();
-                    __syncwarp();
+                const int ab = hit & 1, st = hit & 1;
+                const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
+                if (!mbar_wait(&acc_full[ab], (hit >> 1) & 1, err)) { ok = false; break; }
+                tc_fence_after();
+                const uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
+                const float *lb = reinterpret_cast<const float *>(stage + L.l_rel);
+                const float *gb = reinterpret_cast<const float *>(stage + L.g_rel);
 #pragma unroll
-                    for (int p0 = 0; p0 < 64; p0 += 16) {
-                        uint32_t a[16];
-                        tmem_ld16_nowait(tmem + lane_base + kColAcc + slot * 64 + p0, a);
+                for (int k = 0; k < 2; ++k) {
+                    if (k == 1 && !two) break;
+                    const int t = k * kRows + t_local;
+                    // this tile's scaled x row, l and g from the stage; its
+                    // accumulator row in two 32-column halves, one wait each
+                    const uint8_t *xrow = stage + L.x_rel + t * 128;
+                    uint4 xr[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        xr[q] = *reinterpret_cast<const uint4 *>(xrow + ((q ^ (t & 7)) << 4));
+                    const float u = __expf(lb[t] - gb[Q + 2]);
+                    const bool store = gb[Q + k] == 0.f;
+                    const float dg = store ? Dh / gb[t] : 0.f;
+                    // the stage goes back to the producer after the last tile's reads
+                    if (k == ntile - 1) mbar_arrive(&head_free[st]);
+                    const int row = R.b * d.T + R.c * Q + k * kRows + qd * 32;
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t a[32];
+                        tmem_ld32_nowait(tmem + lane_base + acc_col(ab) + k * 64 + hf * 32, a);
                         tmem_wait_ld();
-                        uint32_t o[8];
+                        if (k == ntile - 1 && hf == 1) {
+                            // the accumulator buffer goes back to the MMAs
+                            tc_fence_before();
+                            mbar_arrive(&acc_free[ab]);
+                        }
+                        if (!store) continue;
+                        // staged (64-byte swizzle) in one of this warp's two blocks
+                        // and written by its own TMA store
+                        uint8_t *blk = sYw + (nst & 1) * (32 * 64);
+                        // the store that used this block two stores ago has read it
+                        if (lane == 0) bulk_wait_read_1();
+                        __syncwarp();
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            o[e] = pack_bf16x2(ut * __uint_as_float(a[2 * e]), ut * __uint_as_float(a[2 * e + 1]));
-                        *reinterpret_cast<uint4 *>(sY + sw128_off(t_local, p0 / 8)) = make_uint4(o[0], o[1], o[2], o[3]);
-                        *reinterpret_cast<uint4 *>(sY + sw128_off(t_local, p0 / 8 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&acc_free[slot]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0 && store) {
-                        tma_store_3d(&tm_y, sYw, 0, h, R.b * d.T + R.c * Q + k * kRows + qd * 32);
-                        bulk_commit();
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 xv = xr[4 * hf + q];
+                            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                            const uint32_t *ah = a + 8 * q;
+                            uint32_t o[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                o[e] = pack_bf16x2(fmaf(u, __uint_as_float(ah[2 * e]), dg * bf16lo(xw[e])),
+                                                   fmaf(u, __uint_as_float(ah[2 * e + 1]), dg * bf16hi(xw[e])));
+                            *reinterpret_cast<uint4 *>(blk + sw64_off(lane, q)) = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&tm_y, blk, 32 * hf, h, row);
+                            bulk_commit();
+                        }
+                        ++nst;
                     }
                 }
             }
@@ -524,7 +495,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
 }
 
 template <int N>
-cudaError_t launch5(const Dims &d, const CUtensorMap *maps, const float *dtq, const float *D,
+cudaError_t launch5(const Dims &d, const CUtensorMap *maps, const float *gq, const float *D,
                     const float *l, int *nsteep, long long *items, int max_items,
                     unsigned int *err, cudaStream_t stream) {
     const Smem5 L = scan5_smem(d.Q, N);
@@ -534,7 +505,7 @@ cudaError_t launch5(const Dims &d, const CUtensorMap *maps, const float *dtq, co
     const int sms = device_sm_count();
     const int grid = n_items < sms ? int(n_items) : sms;
     chunk_scan5_kernel<N><<<grid, kThreads, L.total, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], d, dtq, D, l, nsteep, items, max_items, err);
+        maps[0], maps[1], maps[2], maps[3], maps[4], d, gq, D, l, nsteep, items, max_items, err);
     return cudaGetLastError();
 }
 
@@ -549,7 +520,7 @@ bool tc_chunk_scan5_supported(const Dims &d) {
 
 int chunk_scan5_max_steep(const Dims &d) { return d.B * d.nc * d.H * (d.Q / kRows); }
 
-cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *dtq, const void *Bm,
+cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq, const void *Bm,
                                   const void *Cm, const float *D, const float *l,
                                   const void *s_in_bf16, void *y, int *nsteep, long long *items,
                                   unsigned int *err, cudaStream_t stream) {
@@ -564,18 +535,18 @@ cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *dtq
     const uint64_t sdims[2] = {uint64_t(d.N), uint64_t(d.B) * d.nc * d.H * d.P};
     const uint64_t sstr[1] = {uint64_t(d.N) * 2};
     const uint32_t sbox[2] = {nbox, 64};
-    const uint32_t ybox[3] = {64, 1, 32};  // one epilogue warp's 32 rows
+    const uint32_t ybox[3] = {32, 1, 32};  // 32 columns of one epilogue warp's 32 rows
     CUtensorMap maps[5];
     if (!make_tmap_bf16(&maps[0], 3, Cm, bcdims, bcstr, bcbox, rb) ||
         !make_tmap_bf16(&maps[1], 3, Bm, bcdims, bcstr, bcbox, rb) ||
         !make_tmap_bf16(&maps[2], 3, x, xdims, xstr, xbox, 128) ||
         !make_tmap_bf16(&maps[3], 2, s_in_bf16, sdims, sstr, sbox, rb) ||
-        !make_tmap_bf16(&maps[4], 3, y, xdims, xstr, ybox, 128))
+        !make_tmap_bf16(&maps[4], 3, y, xdims, xstr, ybox, 64))
         return cudaErrorInvalidValue;
     const int max_items = chunk_scan5_max_steep(d);
     switch (d.N) {
-        case 16: return launch5<16>(d, maps, dtq, D, l, nsteep, items, max_items, err, stream);
-        case 128: return launch5<128>(d, maps, dtq, D, l, nsteep, items, max_items, err, stream);
+        case 16: return launch5<16>(d, maps, gq, D, l, nsteep, items, max_items, err, stream);
+        case 128: return launch5<128>(d, maps, gq, D, l, nsteep, items, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -7,9 +7,18 @@
 
 namespace ssd {
 
-// ssd_chunk_cumsum: dt, A -> l, w, dtq, beta [B,H,nc,Q], alpha [B,H,nc]
+// ssd_chunk_cumsum: dt, A -> l, w, dtq, beta [B,H,nc,Q], alpha [B,H,nc] and,
+// if gq != nullptr (chunk_len 128 / 256), per (b, h, c) the chunk-wide scan's
+// token factors g_s = exp(-l_s) dt_s (Q floats) followed by one steep flag per
+// 128-token tile (1.0 when the tile is left to the block-factored scan) and
+// padding: chunk_gq(Q) floats in all
+__host__ __device__ constexpr int chunk_gq(int Q) { return Q + 4; }
+// a 128-token tile k is steep when -l at its last token reaches this (the
+// chunk-wide scan's factors exp(-l_s) would exceed e^72), or when one of its
+// dt is 0 (the skip term is recovered from the scaled rows as D / g)
+constexpr float kScanSteep = 72.f;
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
-                                float *w, float *dtq, float *beta, float *alpha,
+                                float *w, float *dtq, float *beta, float *alpha, float *gq,
                                 cudaStream_t stream);
 
 // ssd_state_passing: states [B,nc,H,P,N] (fp32 or bf16 per states_bf16), alpha
@@ -57,11 +66,12 @@ cudaError_t launch_chunk_scan_tc4(const Dims &d, const void *x, const float *dtq
                                   const float *D, const float *l, const void *s_in_bf16, void *y,
                                   const long long *items, const int *nitems, int max_items,
                                   unsigned int *err, cudaStream_t stream);
-// chunk-wide tensor-core scan: one accumulator per 128-row tile; tiles with a
-// decay range >= 64 are appended to (nsteep, items) for the kernel above
+// chunk-wide tensor-core scan: masked scores shared by the heads of a group,
+// one accumulator per 128-row tile; tiles that the cumsum kernel flagged as
+// steep are appended to (nsteep, items) for the kernel above
 bool tc_chunk_scan5_supported(const Dims &d);
 int chunk_scan5_max_steep(const Dims &d);
-cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *dtq, const void *Bm,
+cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq, const void *Bm,
                                   const void *Cm, const float *D, const float *l,
                                   const void *s_in_bf16, void *y, int *nsteep, long long *items,
                                   unsigned int *err, cudaStream_t stream);

@@ -59,6 +59,7 @@ struct Plan {
     bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
     bool scan5;     // chunk-wide scan, steep tiles finished by the block-factored scan
     size_t steep_offset;  // scan5: item counter (256 bytes) + packed steep items
+    size_t gq_offset;     // scan5: per-token column factors [B,H,nc,chunk_gq(Q)]
     ssd_workspace_layout_t ws;
 };
 
@@ -113,6 +114,8 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
     plan->steep_offset = off;
     if (plan->scan5) off = align_up(off + kAlign + sizeof(long long) * size_t(ssd::chunk_scan5_max_steep(d)));
+    plan->gq_offset = off;
+    if (plan->scan5) off = align_up(off + al * ssd::chunk_gq(d.Q));
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
     w.launches = (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
@@ -158,6 +161,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     void *s_in = ws + pl.ws.s_in_offset;
     int *nsteep = reinterpret_cast<int *>(ws + pl.steep_offset);
     long long *steep_items = reinterpret_cast<long long *>(ws + pl.steep_offset + kAlign);
+    float *gq = pl.scan5 ? reinterpret_cast<float *>(ws + pl.gq_offset) : nullptr;
     for (int stage = 0; stage < 4; ++stage) {
         if (only_stage >= 0 && stage != only_stage) continue;
         cudaError_t e = cudaSuccess;
@@ -166,7 +170,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 // the steep-tile list of the chunk-wide scan starts empty each call
                 if (pl.scan5) e = cudaMemsetAsync(nsteep, 0, sizeof(int), stream);
                 if (e == cudaSuccess)
-                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, stream);
+                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.fused ? ssd::launch_state_fused(d, x, Bm, w, alpha, init_state, s_in, fin, err, stream)
@@ -183,7 +187,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                 if (pl.scan5) {
                     // chunk-wide scan, then the block-factored scan over the tiles
                     // it listed as steep (an empty list costs one short launch)
-                    e = ssd::launch_chunk_scan_tc5(d, x, dtq, Bm, Cm, D, l, s_in, y, nsteep,
+                    e = ssd::launch_chunk_scan_tc5(d, x, gq, Bm, Cm, D, l, s_in, y, nsteep,
                                                    steep_items, err, stream);
                     if (e == cudaSuccess)
                         e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,

@@ -65,14 +65,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 // Bounded wait for the phase with the given parity to complete.  Also gives
 // up early once another wait on the device has failed.
+// The error word lives in global memory: it is polled only once a wait has
+// lasted kErrPollNs, so an ordinary wait never has a global load in flight
+// when its phase completes.
+constexpr uint64_t kErrPollNs = 20000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0) {
-            if (device_failed(err)) return false;
-            if (global_ns() - t0 > kWaitLimitNs) break;
+            const uint64_t el = global_ns() - t0;
+            if (el > kWaitLimitNs) break;
+            if (el > kErrPollNs && (i & 255u) == 0 && device_failed(err)) return false;
         }
     }
     if (err) atomicOr(err, 1u);

@@ -122,6 +122,42 @@ def test_no_skip_term(oracle):
     check_full(inp, oracle)
 
 
+@pytest.mark.parametrize("dstate", [16, 128])
+def test_decay_range_across_the_chunk(oracle, dstate):
+    """Per-token decays of about e^-0.4 (head 0): each 128-token tile spans ~e^-51
+    but the 256-token chunk ~e^-102, so the chunk-wide scan moves its reference
+    to the middle of the chunk; head 1 stays below the threshold, head 2 exceeds
+    it inside a tile (block-factored path), head 3 barely decays."""
+    inp = make_inputs(2, 1024, 4, 64, dstate, 1, 256, dtype="bf16", seed=19, init_state=True, h0_std=1.0)
+    rng = np.random.default_rng(19)
+    inp.dt = rng.uniform(0.3, 0.5, size=inp.dt.shape).astype(np.float32)
+    inp.A = np.array([-1.0, -0.5, -2.0, -0.01], dtype=np.float32)
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    for h in range(4):
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
+    # the carried state reaches the first tokens of every chunk
+    yc = y[:, 256::256, 0][:, :, None]
+    yrc = yr[:, 256::256, 0][:, :, None]
+    assert rel(yc, yrc) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("chunk_len", [128, 256])
+def test_zero_dt_tokens(oracle, chunk_len):
+    """dt = 0 on a run of tokens (the state holds, only D x reaches y there) and on
+    every token of one head (y = C h0 + D x); the other tokens keep their dt."""
+    inp = make_inputs(2, 1024, 4, 64, 128, 1, chunk_len, dtype="bf16", seed=17, init_state=True)
+    inp.dt[0, 100:260, 1] = 0.0
+    inp.dt[1, 300:301, 0] = 0.0
+    inp.dt[:, :, 3] = 0.0
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    for h in range(4):
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
+
+
 def test_final_state_may_alias_init_state(oracle):
     inp = make_inputs(1, 512, 4, 64, 128, 2, 256, dtype="bf16", seed=5, init_state=True)
     a = to_dev(inp)
