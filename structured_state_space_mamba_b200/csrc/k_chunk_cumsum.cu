@@ -40,8 +40,12 @@ __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
                     float *__restrict__ l_out, float *__restrict__ w_out,
                     float *__restrict__ dtq_out, float *__restrict__ beta_out,
-                    float *__restrict__ alpha_out, float *__restrict__ gq_out) {
+                    float *__restrict__ alpha_out, float *__restrict__ gq_out,
+                    int *__restrict__ nsteep) {
     constexpr int Q = 32 * E;
+    // the chunk-wide scan's steep-tile list starts empty (that kernel runs after
+    // this one in stream order)
+    if (nsteep && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *nsteep = 0;
     __shared__ float s_dt[Q][kHeads + 1];
     const int c = blockIdx.x, b = blockIdx.z;
     const int h0 = blockIdx.y * kHeads;
@@ -118,13 +122,13 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
 
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *dtq, float *beta, float *alpha, float *gq,
-                                cudaStream_t stream) {
+                                int *nsteep, cudaStream_t stream) {
     dim3 grid(d.nc, (d.H + kHeads - 1) / kHeads, d.B);
     switch (d.Q) {
-        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
-        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
-        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
-        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq); break;
+        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
+        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
+        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
+        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

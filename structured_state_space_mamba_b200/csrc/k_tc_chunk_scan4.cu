@@ -124,6 +124,7 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                    unsigned int *err) {
     if (device_failed(err)) return;  // an earlier wait expired: skip all work
     if (items) units = min(*nitems, units);  // list mode: the listed (b, c, tile, head) items
+    if (int(blockIdx.x) >= units) return;    // no unit for this CTA (units are strided by the grid)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int Q = d.Q;

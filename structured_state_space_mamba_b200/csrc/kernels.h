@@ -7,7 +7,8 @@
 
 namespace ssd {
 
-// ssd_chunk_cumsum: dt, A -> l, w, dtq, beta [B,H,nc,Q], alpha [B,H,nc] and,
+// ssd_chunk_cumsum: dt, A -> l, w, dtq, beta [B,H,nc,Q], alpha [B,H,nc]; sets
+// *nsteep = 0 when nsteep != nullptr; and,
 // if gq != nullptr (chunk_len 128 / 256), per (b, h, c) the chunk-wide scan's
 // token factors g_s = exp(-l_s) dt_s (Q floats) followed by one steep flag per
 // 128-token tile (1.0 when the tile is left to the block-factored scan) and
@@ -19,6 +20,7 @@ __host__ __device__ constexpr int chunk_gq(int Q) { return Q + 4; }
 constexpr float kScanSteep = 72.f;
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *dtq, float *beta, float *alpha, float *gq,
+                                int *nsteep,
                                 cudaStream_t stream);
 
 // ssd_state_passing: states [B,nc,H,P,N] (fp32 or bf16 per states_bf16), alpha

@@ -167,10 +167,9 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
         cudaError_t e = cudaSuccess;
         switch (stage) {
             case SSD_STAGE_CHUNK_CUMSUM:
-                // the steep-tile list of the chunk-wide scan starts empty each call
-                if (pl.scan5) e = cudaMemsetAsync(nsteep, 0, sizeof(int), stream);
-                if (e == cudaSuccess)
-                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq, stream);
+                // also empties the chunk-wide scan's steep-tile list
+                e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq,
+                                             pl.scan5 ? nsteep : nullptr, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.fused ? ssd::launch_state_fused(d, x, Bm, w, alpha, init_state, s_in, fin, err, stream)
