@@ -29,22 +29,27 @@
 // block-factored kernel of k_tc_chunk_scan4.cu finishes in a second launch.
 //
 // Work: the (b, c, h) items are split into one contiguous range per CTA
-// (persistent grid), walked in order.  Per head the chunk's x rows, s_in, l and
-// the factors g are loaded once (double buffered); a stage is released when
-// the head's products are done and the epilogue has read its scaled rows.
+// (persistent grid), walked in order.  Per head the chunk's x rows and s_in
+// go through a ring of three stages (l and g through a ring of their own); a
+// run's start borrows two stages of the ring for C_0 and the B tiles, so a
+// stage is reused three uses later, once the use's products are done and the
+// epilogue has read the head's scaled rows.  C_1 stays in its own buffer for
+// the run.
 //
-// Tensor memory (512 columns): [0,128) P_0, P_1 (bf16); CBoff (bf16, A
-// operand of a TS product) in [256,288) and [320,352); two accumulator
-// buffers {Y_0, Y_1} at [384,512) and [128,256), alternating between heads.  At the start of a run
-// the fp32 C B^T tiles pass through them (C_0 B_0^T -> [384,512), C_1 B_1^T ->
-// [128,256), CBoff -> [256,384)), so a run starts once the accumulators of the
-// previous heads are read.
+// Tensor memory (512 columns): [0,128) P_0, P_1 (bf16); [256,384) CBoff and
+// C_0 (bf16 A operands of TS products: CBoff in [256,288) and [320,352), C_0 in
+// [288,320) and [352,384)); two accumulator buffers {Y_0, Y_1} at [384,512) and
+// [128,256), alternating between heads.  At the start of a run the fp32 C B^T
+// tiles pass through them (C_0 B_0^T -> [384,512), C_1 B_1^T -> [128,256),
+// CBoff -> [256,384)), so a run starts once the accumulators of the previous
+// heads are read.
 //
 // Roles (14 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..9 score /
-// scale warps (two 32 x 32 score blocks each at the start of a run: lane
-// quarter warp % 4, column blocks 2 (warp - 2) / 4 + {0, 1}; x scaling per
-// head), warps 10..13 epilogue (y = u_t Y + D_h x, each warp staging its 32
-// rows, 32 columns at a time, and writing them with its own TMA stores).
+// scale warps (at the start of a run two 32 x 32 score blocks each -- lane
+// quarter warp % 4, column blocks 2 (warp - 2) / 4 + {0, 1} -- and half of
+// C_0's row; x scaling per head), warps 10..13 epilogue (y = u_t Y + D_h x,
+// each warp staging its 32 rows, 32 columns at a time, and writing them with
+// its own TMA stores).
 #include <cmath>
 
 #include "common.cuh"
@@ -66,39 +71,36 @@ constexpr int kScoreThreads = 32 * kScoreWarps;
 constexpr int kEpiWarp0 = 2 + kScoreWarps;
 constexpr int kEpiThreads = 128;
 constexpr int kTmemCols = 512;
+constexpr int kStages = 3;  // x / s_in stages (a run's start borrows two)
 constexpr uint32_t kColP = 0, kColOff = 256;
 // packed CBoff: 32-column block cb (16 bf16 pairs) within the fp32 range that
 // the two score warps of column blocks {2 (cb / 2), 2 (cb / 2) + 1} read
 __device__ __forceinline__ uint32_t off_col(int cb) { return kColOff + (cb >> 1) * 64 + (cb & 1) * 16; }
 // accumulator buffer ab of a head (hit & 1)
 __device__ __forceinline__ uint32_t acc_col(int ab) { return ab == 0 ? 384u : 128u; }
+// C_0 (bf16, A operand of the C_0 S'^T products), K step kk: the second half of
+// each score warp pair's CBoff source range, free once CBoff is packed
+__device__ __forceinline__ uint32_t c0_col(int kk) { return kColOff + 32 + (kk >> 2) * 64 + (kk & 3) * 8; }
 
 struct Smem5 {
-    uint32_t c_off, b_off, stage_off, stage_bytes, x_rel, s_rel, l_rel, g_rel;
-    uint32_t y_off, bar_off, total;
+    uint32_t c1_off, stage_off, stage_bytes, s_rel, lg_off, lg_bytes, y_off, bar_off, total;
 };
 
+// C_1 (tile 1 of C, for the C_1 S'^T products) stays for the whole run; a stage
+// holds a head's x rows and s_in, or at a run's start C_0 (first stage) and the
+// B tiles (second); l and g ride in a ring of their own.
 __host__ __device__ inline Smem5 scan5_smem(int Q, int N) {
     Smem5 s;
-    s.c_off = 0;
-    s.b_off = up1k(Q * N * 2);                    // C rows of the chunk
-    s.stage_off = s.b_off + up1k(kRows * N * 2);  // B rows of one tile
-    s.x_rel = 0;
+    s.c1_off = 0;
+    s.stage_off = Q == 2 * kRows ? up1k(kRows * N * 2) : 0;
     s.s_rel = Q * 128;
-    s.l_rel = s.s_rel + up1k(64 * N * 2);
-    s.g_rel = s.l_rel + Q * 4;  // g (Q floats), then the per-tile steep flags
-    s.stage_bytes = up1k(s.g_rel + chunk_gq(Q) * 4);
-    s.y_off = s.stage_off + 2 * s.stage_bytes;  // y staging: 128 rows x 128 bytes
+    s.stage_bytes = umax(up1k(s.s_rel + 64 * N * 2), up1k(kRows * N * 2));
+    s.lg_off = s.stage_off + kStages * s.stage_bytes;
+    s.lg_bytes = (Q * 4 + chunk_gq(Q) * 4 + 127) & ~127u;  // l (Q floats), then g, flags, r
+    s.y_off = up1k(s.lg_off + kStages * s.lg_bytes);  // y staging: 128 rows x 128 bytes
     s.bar_off = s.y_off + kRows * 128;
     s.total = s.bar_off + 256 + 1024;
     return s;
-}
-
-// A operand: rows [128 k, 128 k + 128) of the C tile of Q rows, K step kk.
-__device__ __forceinline__ uint64_t c_desc(uint32_t base, int k, int kk, int Q, int n) {
-    if (n >= 64)
-        return smem_desc(base + (kk >> 2) * Q * 128 + k * kRows * 128 + (kk & 3) * 32, 16, 1024, kSw128);
-    return smem_desc(base + k * kRows * row_bytes(n) + kk * 32, 16, 8 * row_bytes(n), kmajor_swz(n));
 }
 
 // Items (b, c, h) in order, h fastest; a run = consecutive items of one
@@ -146,16 +148,19 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     const int ntile = two ? 2 : 1;
     const int ngq = chunk_gq(Q);
     const Smem5 L = scan5_smem(Q, N);
-    uint8_t *sC = smem + L.c_off;
-    uint8_t *sB = smem + L.b_off;  // B rows of one tile
-    uint8_t *sY = smem + L.y_off;  // y staging, 32 rows per epilogue warp
+    uint8_t *sC1 = smem + L.c1_off;  // C_1 (two tiles only)
+    uint8_t *sY = smem + L.y_off;    // y staging, 32 rows per epilogue warp
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *ld_c = bars + 0, *ld_b1 = bars + 1, *b0_free = bars + 2, *cb_full = bars + 3;
-    uint64_t *cvt_done = bars + 5, *cb_smem_free = bars + 6;
-    uint64_t *head_full = bars + 7, *head_free = bars + 9, *ready = bars + 11;  // [2] each
-    uint64_t *acc_full = bars + 13, *acc_free = bars + 15;                     // [2] each
-    uint64_t *done = bars + 17;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 18);
+    uint64_t *cvt_done = bars + 4, *cb_smem_free = bars + 5;
+    uint64_t *head_full = bars + 6, *stage_free = bars + 9, *ready = bars + 12;  // [kStages] each
+    uint64_t *acc_full = bars + 15, *acc_free = bars + 17;                      // [2] each
+    uint64_t *done = bars + 19;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 20);
+    auto stage_at = [&](uint32_t use) { return smem + L.stage_off + (use % kStages) * L.stage_bytes; };
+    auto lg_at = [&](uint32_t use) {
+        return reinterpret_cast<float *>(smem + L.lg_off + (use % kStages) * L.lg_bytes);
+    };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int kSlabs = N >= 64 ? N / 64 : 1;
@@ -172,12 +177,14 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         mbar_init(cb_full, 1);
         mbar_init(cvt_done, kScoreThreads);
         mbar_init(cb_smem_free, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             mbar_init(&head_full[i], 1);
-            // the head's products (one commit) and the epilogue, which reads the
-            // head's scaled rows, l and g
-            mbar_init(&head_free[i], 1 + kEpiThreads);
+            // the use's products (one commit) and the epilogue, which reads a
+            // head's scaled rows
+            mbar_init(&stage_free[i], 1 + kEpiThreads);
             mbar_init(&ready[i], kScoreThreads);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_free[i], kEpiThreads);
         }
@@ -195,70 +202,80 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // Every role walks the same sequence of stage uses: per run, two for its
+    // start (C_0, then the B tiles), then one per head.
     if (warp == 0) {
         // =============================== producer ===============================
         if (lane == 0) {
-            uint32_t si = 0, hit = 0;
+            uint32_t si = 0, use = 0;
             bool ok = true;
             for (long long i = i0; i < i1 && ok; ++si) {
                 const Run R = run_at(i, i1, d);
                 i += R.len;
                 const int trow0 = R.b * d.T + R.c * Q;
-                // C of the chunk and B of tile 0, once the previous run's MMAs are done
-                if (!mbar_wait(cb_smem_free, (si & 1) ^ 1, err)) break;
-                mbar_expect_tx(ld_c, uint32_t(Q) * N * 2 + uint32_t(kRows) * N * 2);
-                for (int k = 0; k < ntile; ++k)
-                    for (int sl = 0; sl < kSlabs; ++sl)
-                        tma_load_3d(sC + sl * Q * 128 + k * kRows * kRB, &tm_c, ld_c, sl * 64, R.g,
-                                    trow0 + k * kRows);
-                for (int sl = 0; sl < kSlabs; ++sl)
-                    tma_load_3d(sB + sl * kRows * 128, &tm_b, ld_c, sl * 64, R.g, trow0);
+                // C_0 and B_0 into the next two stages, C_1 into its own buffer
+                // once the previous run's products are done
+                const uint32_t uc = use, ub = use + 1;
+                use += 2;
+                if (!mbar_wait(&stage_free[uc % kStages], ((uc / kStages) & 1) ^ 1, err) ||
+                    !mbar_wait(&stage_free[ub % kStages], ((ub / kStages) & 1) ^ 1, err) ||
+                    !mbar_wait(cb_smem_free, (si & 1) ^ 1, err))
+                    break;
+                uint8_t *sc0 = stage_at(uc), *sb = stage_at(ub);
+                // these two uses carry no head: their head_full phases pass at once
+                mbar_arrive(&head_full[uc % kStages]);
+                mbar_arrive(&head_full[ub % kStages]);
+                mbar_expect_tx(ld_c, uint32_t(ntile + 1) * kRows * N * 2);
+                for (int sl = 0; sl < kSlabs; ++sl) {
+                    tma_load_3d(sc0 + sl * kRows * 128, &tm_c, ld_c, sl * 64, R.g, trow0);
+                    tma_load_3d(sb + sl * kRows * 128, &tm_b, ld_c, sl * 64, R.g, trow0);
+                    if (two) tma_load_3d(sC1 + sl * kRows * 128, &tm_c, ld_c, sl * 64, R.g, trow0 + kRows);
+                }
                 if (two) {
                     // B of tile 1 into the same place once the tile-0 products are done
                     if (!mbar_wait(b0_free, si & 1, err)) break;
                     mbar_expect_tx(ld_b1, uint32_t(kRows) * N * 2);
                     for (int sl = 0; sl < kSlabs; ++sl)
-                        tma_load_3d(sB + sl * kRows * 128, &tm_b, ld_b1, sl * 64, R.g, trow0 + kRows);
+                        tma_load_3d(sb + sl * kRows * 128, &tm_b, ld_b1, sl * 64, R.g, trow0 + kRows);
                 }
-                for (int hi = 0; hi < R.len; ++hi, ++hit) {
-                    const int st = hit & 1;
+                for (int hi = 0; hi < R.len; ++hi, ++use) {
+                    const int st = use % kStages;
                     const int h = R.h + hi;
-                    if (!mbar_wait(&head_free[st], ((hit >> 1) & 1) ^ 1, err)) { ok = false; break; }
-                    uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
+                    if (!mbar_wait(&stage_free[st], ((use / kStages) & 1) ^ 1, err)) { ok = false; break; }
+                    uint8_t *stage = stage_at(use);
+                    float *lg = lg_at(use);
                     mbar_expect_tx(&head_full[st], uint32_t(Q) * 128 + 64u * N * 2 + uint32_t(Q + ngq) * 4);
                     for (int k = 0; k < ntile; ++k)
-                        tma_load_3d(stage + L.x_rel + k * kRows * 128, &tm_x, &head_full[st], 0, h,
-                                    trow0 + k * kRows);
+                        tma_load_3d(stage + k * kRows * 128, &tm_x, &head_full[st], 0, h, trow0 + k * kRows);
                     const int srow = ((R.b * d.nc + R.c) * d.H + h) * 64;
                     for (int sl = 0; sl < kSlabs; ++sl)
                         tma_load_2d(stage + L.s_rel + sl * 64 * 128, &tm_s, &head_full[st], sl * 64, srow);
-                    bulk_load(stage + L.l_rel, lcum + off_lq(d, R.b, h, R.c), Q * 4, &head_full[st]);
-                    bulk_load(stage + L.g_rel, gq + ((int64_t(R.b) * d.H + h) * d.nc + R.c) * ngq, ngq * 4,
+                    bulk_load(lg, lcum + off_lq(d, R.b, h, R.c), Q * 4, &head_full[st]);
+                    bulk_load(lg + Q, gq + ((int64_t(R.b) * d.H + h) * d.nc + R.c) * ngq, ngq * 4,
                               &head_full[st]);
                 }
             }
-            // drain: the last loads issued must have landed before the CTA exits
-            for (uint32_t k = 0; k < 2 && k < hit; ++k) {
-                const uint32_t i = hit - 1 - k;
-                mbar_wait(&head_full[i & 1], (i >> 1) & 1, nullptr);
-            }
-            if (si > 0) {
-                mbar_wait(ld_c, (si - 1) & 1, nullptr);
-                if (two) mbar_wait(ld_b1, (si - 1) & 1, nullptr);
+            // drain: every use issued has been consumed (so its loads landed)
+            for (uint32_t k = 1; k <= kStages && k <= use; ++k) {
+                const uint32_t u = use - k;
+                mbar_wait(&stage_free[u % kStages], (u / kStages) & 1, nullptr);
             }
         }
     } else if (warp == 1) {
         // =============================== MMA issuer =============================
         if (lane == 0) {
-            uint32_t si = 0, hit = 0;
+            uint32_t si = 0, hit = 0, use = 0;
             bool ok = true;
-            const uint32_t ca = smem_u32(sC), ba = smem_u32(sB);
+            const uint32_t c1a = smem_u32(sC1);
             const uint32_t idCB = idesc_bf16_f32(kRows, kRows, 0, 0);
             const uint32_t idX = idesc_bf16_f32(kRows, 64, 0, 1);
             const uint32_t idS = idesc_bf16_f32(kRows, 64, 0, 0);
             for (long long i = i0; i < i1 && ok; ++si) {
                 const Run R = run_at(i, i1, d);
                 i += R.len;
+                const uint32_t uc = use, ub = use + 1;
+                use += 2;
+                const uint32_t c0a = smem_u32(stage_at(uc)), ba = smem_u32(stage_at(ub));
                 // the fp32 C B^T tiles pass through the accumulator columns: wait
                 // until the epilogue has read the previous heads' accumulators
                 for (uint32_t j = 1; j <= 2 && j <= hit && ok; ++j) {
@@ -269,42 +286,46 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 tc_fence_after();
                 // C_0 B_0^T -> [384,512) and, for two tiles, CBoff = C_1 B_0^T -> [256,384)
                 for (int kk = 0; kk < N / 16; ++kk)
-                    mma_bf16_ss(tmem + acc_col(0), c_desc(ca, 0, kk, Q, N), kmajor_desc(ba, kk, kRows, N),
+                    mma_bf16_ss(tmem + acc_col(0), kmajor_desc(c0a, kk, kRows, N), kmajor_desc(ba, kk, kRows, N),
                                 idCB, kk > 0 ? 1u : 0u);
                 if (two) {
                     for (int kk = 0; kk < N / 16; ++kk)
-                        mma_bf16_ss(tmem + kColOff, c_desc(ca, 1, kk, Q, N), kmajor_desc(ba, kk, kRows, N),
-                                    idCB, kk > 0 ? 1u : 0u);
+                        mma_bf16_ss(tmem + kColOff, kmajor_desc(c1a, kk, kRows, N),
+                                    kmajor_desc(ba, kk, kRows, N), idCB, kk > 0 ? 1u : 0u);
                     mma_commit(b0_free);
                     if (!mbar_wait(ld_b1, si & 1, err)) break;
                     tc_fence_after();
                     // C_1 B_1^T -> [128,256)
                     for (int kk = 0; kk < N / 16; ++kk)
-                        mma_bf16_ss(tmem + acc_col(1), c_desc(ca, 1, kk, Q, N),
+                        mma_bf16_ss(tmem + acc_col(1), kmajor_desc(c1a, kk, kRows, N),
                                     kmajor_desc(ba, kk, kRows, N), idCB, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(cb_full);
-                // the scores of this run exist once the score warps have converted them
+                // the scores of this run (and C_0 in tensor memory) exist once the
+                // score warps have converted them; the run's two stages go back
                 if (!mbar_wait(cvt_done, si & 1, err)) break;
                 tc_fence_after();
-                for (int hi = 0; hi < R.len; ++hi, ++hit) {
-                    const int st = hit & 1, ab = hit & 1;
-                    const uint32_t hp = (hit >> 1) & 1;
-                    const uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
-                    const uint32_t xa = smem_u32(stage + L.x_rel);
+                // (the epilogue does not read them: its share is arrived here; both
+                // stages' previous uses were released before C_0 and B landed)
+                mma_commit(&stage_free[uc % kStages]);
+                mma_commit(&stage_free[ub % kStages]);
+                mbar_arrive_cnt(&stage_free[uc % kStages], kEpiThreads);
+                mbar_arrive_cnt(&stage_free[ub % kStages], kEpiThreads);
+                for (int hi = 0; hi < R.len; ++hi, ++hit, ++use) {
+                    const int st = use % kStages, ab = hit & 1;
+                    const uint32_t sp = (use / kStages) & 1, hp = (hit >> 1) & 1;
+                    const uint8_t *stage = stage_at(use);
+                    const uint32_t xa = smem_u32(stage);
                     const uint32_t sa = smem_u32(stage + L.s_rel);
-                    if (!mbar_wait(&head_full[st], hp, err) || !mbar_wait(&ready[st], hp, err) ||
+                    if (!mbar_wait(&head_full[st], sp, err) || !mbar_wait(&ready[st], sp, err) ||
                         !mbar_wait(&acc_free[ab], hp ^ 1, err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t acc = tmem + acc_col(ab);
-                    // Y_0 = C_0 s_in^T + P_0 X''_0 and Y_1 = C_1 s_in^T + CBoff X''_0 + P_1 X''_1,
-                    // interleaved so that consecutive products go to different
-                    // accumulators and one need not wait for the previous to finish
+                    // Y_0 = C_0 S'^T + P_0 X''_0 and Y_1 = C_1 S'^T + CBoff X''_0 + P_1 X''_1
                     for (int kk = 0; kk < N / 16; ++kk) {
-                        mma_bf16_ss(acc, c_desc(ca, 0, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS,
-                                    kk > 0 ? 1u : 0u);
+                        mma_bf16_ts(acc, tmem + c0_col(kk), kmajor_desc(sa, kk, 64, N), idS, kk > 0 ? 1u : 0u);
                         if (two)
-                            mma_bf16_ss(acc + 64, c_desc(ca, 1, kk, Q, N), kmajor_desc(sa, kk, 64, N), idS,
+                            mma_bf16_ss(acc + 64, kmajor_desc(c1a, kk, kRows, N), kmajor_desc(sa, kk, 64, N), idS,
                                         kk > 0 ? 1u : 0u);
                     }
                     for (int kk = 0; kk < kRows / 16; ++kk) {
@@ -317,7 +338,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                             mma_bf16_ts(acc + 64, tmem + kColP + 64 + kk * 8,
                                         smem_desc(xa + kRows * 128 + kk * 2048, 16, 1024, kSw128), idX, 1u);
                     mma_commit(&acc_full[ab]);
-                    mma_commit(&head_free[st]);
+                    mma_commit(&stage_free[st]);
                 }
                 if (ok) mma_commit(cb_smem_free);
             }
@@ -330,12 +351,14 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         const int qd = warp & 3;             // TMEM lane quarter of this warp
         const int cb0 = 2 * ((warp - 2) >> 2);  // first of its two 32-column blocks
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
-        uint32_t si = 0, hit = 0;
+        uint32_t si = 0, use = 0;
         bool ok = true;
         for (long long i = i0; i < i1 && ok; ++si) {
             const Run R = run_at(i, i1, d);
             i += R.len;
-            if (!mbar_wait(cb_full, si & 1, err)) break;
+            const uint32_t uc = use;
+            use += 2;
+            if (!mbar_wait(cb_full, si & 1, err) || !mbar_wait(ld_c, si & 1, err)) break;
             tc_fence_after();
             // ---- masked scores of this run: fp32 C B^T -> bf16 P_k, CBoff ----
             // block (qd, cb) of a tile: below the diagonal all columns, on it the
@@ -374,18 +397,52 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     tmem_st16(tmem + lane_base + off_col(cb0 + bb), pk);
                 }
             }
+            // C_0 into the second half of this warp's range: row t, K half cb0 / 2
+            // (one 128-byte swizzled slab row, or the 32-byte row for N = 16)
+            {
+                const int t = qd * 32 + lane;
+                const uint8_t *sc0 = stage_at(uc);
+                if (N >= 64) {
+                    const uint8_t *row = sc0 + (cb0 >> 1) * kRows * 128 + t * 128;
+                    uint32_t cw[32];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((q ^ (t & 7)) << 4));
+                        cw[4 * q] = v.x;
+                        cw[4 * q + 1] = v.y;
+                        cw[4 * q + 2] = v.z;
+                        cw[4 * q + 3] = v.w;
+                    }
+                    tmem_st16(tmem + lane_base + c0_col(4 * (cb0 >> 1)), cw);
+                    tmem_st16(tmem + lane_base + c0_col(4 * (cb0 >> 1)) + 16, cw + 16);
+                } else if (cb0 == 0) {
+                    uint32_t cw[8];
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(sc0 + swz_off(t * kRB + q * 16, kRB));
+                        cw[4 * q] = v.x;
+                        cw[4 * q + 1] = v.y;
+                        cw[4 * q + 2] = v.z;
+                        cw[4 * q + 3] = v.w;
+                    }
+                    tmem_st8(tmem + lane_base + c0_col(0), cw);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(cvt_done);
+            // the run's start uses carry no head: their ready phases pass at once
+            mbar_arrive(&ready[uc % kStages]);
+            mbar_arrive(&ready[(uc + 1) % kStages]);
             if (!mbar_wait(cvt_done, si & 1, err)) break;
             tc_fence_after();
-            for (int hi = 0; hi < R.len; ++hi, ++hit) {
-                const int st = hit & 1;
-                const uint32_t hp = (hit >> 1) & 1;
+            for (int hi = 0; hi < R.len; ++hi, ++use) {
+                const int st = use % kStages;
+                const uint32_t sp = (use / kStages) & 1;
                 const int h = R.h + hi;
-                uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
-                const float *gb = reinterpret_cast<const float *>(stage + L.g_rel);
-                if (!mbar_wait(&head_full[st], hp, err)) { ok = false; break; }
+                uint8_t *stage = stage_at(use);
+                const float *gb = lg_at(use) + Q;
+                if (!mbar_wait(&head_full[st], sp, err)) { ok = false; break; }
                 if (sid < ntile && gb[Q + sid] != 0.f) {
                     // steep tile: left to the block-factored scan
                     const int idx = atomicAdd(nsteep, 1);
@@ -397,7 +454,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 // S' = e^r s_in, which directly follows x in the stage
                 const float r = gb[Q + 2];
                 const float er = __expf(r);
-                scale_chunks(stage + L.x_rel, r != 0.f ? Q * 8 + 8 * N : Q * 8, sid, kScoreThreads,
+                scale_chunks(stage, r != 0.f ? Q * 8 + 8 * N : Q * 8, sid, kScoreThreads,
                              [&](int kc) { return kc < Q * 8 ? gb[kc >> 3] : er; });
                 fence_proxy_async_smem();
                 mbar_arrive(&ready[st]);
@@ -416,27 +473,28 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         const int t_local = qd * 32 + lane;
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
         uint8_t *sYw = sY + qd * 32 * 128;  // two 32 x 32 bf16 blocks per warp
-        uint32_t hit = 0, nst = 0;
+        uint32_t hit = 0, nst = 0, use = 0;
         bool ok = true;
         for (long long i = i0; i < i1 && ok;) {
             const Run R = run_at(i, i1, d);
             i += R.len;
-            for (int hi = 0; hi < R.len && ok; ++hi, ++hit) {
+            use += 2;  // the run's start uses: released by the MMA issuer
+            for (int hi = 0; hi < R.len && ok; ++hi, ++hit, ++use) {
                 const int h = R.h + hi;
-                const int ab = hit & 1, st = hit & 1;
+                const int ab = hit & 1, st = use % kStages;
                 const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
                 if (!mbar_wait(&acc_full[ab], (hit >> 1) & 1, err)) { ok = false; break; }
                 tc_fence_after();
-                const uint8_t *stage = smem + L.stage_off + st * L.stage_bytes;
-                const float *lb = reinterpret_cast<const float *>(stage + L.l_rel);
-                const float *gb = reinterpret_cast<const float *>(stage + L.g_rel);
+                const uint8_t *stage = stage_at(use);
+                const float *lb = lg_at(use);
+                const float *gb = lb + Q;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     if (k == 1 && !two) break;
                     const int t = k * kRows + t_local;
                     // this tile's scaled x row, l and g from the stage; its
                     // accumulator row in two 32-column halves, one wait each
-                    const uint8_t *xrow = stage + L.x_rel + t * 128;
+                    const uint8_t *xrow = stage + t * 128;
                     uint4 xr[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q)
@@ -445,7 +503,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     const bool store = gb[Q + k] == 0.f;
                     const float dg = store ? Dh / gb[t] : 0.f;
                     // the stage goes back to the producer after the last tile's reads
-                    if (k == ntile - 1) mbar_arrive(&head_free[st]);
+                    if (k == ntile - 1) mbar_arrive(&stage_free[st]);
                     const int row = R.b * d.T + R.c * Q + k * kRows + qd * 32;
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
