@@ -103,6 +103,14 @@ __host__ __device__ inline Smem5 scan5_smem(int Q, int N) {
     return s;
 }
 
+// Start-address step (in 16-byte units) of K step kk in a K-major operand of
+// `rows` rows, relative to K step 0 (the layouts of kmajor_desc).
+template <int N>
+__device__ __forceinline__ uint64_t kdesc_step_n(int kk, int rows) {
+    if (N >= 64) return uint64_t(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
+    return uint64_t((kk * 32) >> 4);
+}
+
 // Items (b, c, h) in order, h fastest; a run = consecutive items of one
 // (b, c, group).  Returns the run starting at item i (< i1).
 struct Run {
@@ -267,6 +275,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             uint32_t si = 0, hit = 0, use = 0;
             bool ok = true;
             const uint32_t c1a = smem_u32(sC1);
+            const uint64_t c1d = kmajor_desc(c1a, 0, kRows, N);
             const uint32_t idCB = idesc_bf16_f32(kRows, kRows, 0, 0);
             const uint32_t idX = idesc_bf16_f32(kRows, 64, 0, 1);
             const uint32_t idS = idesc_bf16_f32(kRows, 64, 0, 0);
@@ -321,22 +330,31 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         !mbar_wait(&acc_free[ab], hp ^ 1, err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t acc = tmem + acc_col(ab);
-                    // Y_0 = C_0 S'^T + P_0 X''_0 and Y_1 = C_1 S'^T + CBoff X''_0 + P_1 X''_1
+                    // Y_0 = C_0 S'^T + P_0 X''_0 and Y_1 = C_1 S'^T + CBoff X''_0 + P_1 X''_1.
+                    // Descriptors are formed once per head; each K step adds a
+                    // constant to the start-address field (no carry: every
+                    // address stays inside shared memory).
+                    const uint64_t xd = smem_desc(xa, 16, 1024, kSw128);
+                    const uint64_t sd = kmajor_desc(sa, 0, 64, N);
+#pragma unroll
                     for (int kk = 0; kk < N / 16; ++kk) {
-                        mma_bf16_ts(acc, tmem + c0_col(kk), kmajor_desc(sa, kk, 64, N), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ts(acc, tmem + c0_col(kk), sd + kdesc_step_n<N>(kk, 64), idS, kk > 0 ? 1u : 0u);
                         if (two)
-                            mma_bf16_ss(acc + 64, kmajor_desc(c1a, kk, kRows, N), kmajor_desc(sa, kk, 64, N), idS,
+                            mma_bf16_ss(acc + 64, c1d + kdesc_step_n<N>(kk, kRows), sd + kdesc_step_n<N>(kk, 64), idS,
                                         kk > 0 ? 1u : 0u);
                     }
+#pragma unroll
                     for (int kk = 0; kk < kRows / 16; ++kk) {
-                        const uint64_t x0 = smem_desc(xa + kk * 2048, 16, 1024, kSw128);
+                        const uint64_t x0 = xd + uint64_t(kk * (2048 >> 4));
                         mma_bf16_ts(acc, tmem + kColP + kk * 8, x0, idX, 1u);
                         if (two) mma_bf16_ts(acc + 64, tmem + off_col(kk >> 1) + (kk & 1) * 8, x0, idX, 1u);
                     }
-                    if (two)
+                    if (two) {
+#pragma unroll
                         for (int kk = 0; kk < kRows / 16; ++kk)
                             mma_bf16_ts(acc + 64, tmem + kColP + 64 + kk * 8,
-                                        smem_desc(xa + kRows * 128 + kk * 2048, 16, 1024, kSw128), idX, 1u);
+                                        xd + uint64_t((kRows * 128 + kk * 2048) >> 4), idX, 1u);
+                    }
                     mma_commit(&acc_full[ab]);
                     mma_commit(&stage_free[st]);
                 }
