@@ -44,6 +44,12 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # ---------------------------------------------------------------------------
 # algorithmic work (chunked algorithm; compulsory bytes only)
 # ---------------------------------------------------------------------------
+# DRAM bytes (read + write) of one launch of the dominant kernel on a workload,
+# from one ncu capture of the current kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum); workloads without such a capture report None.
+NCU_TRAFFIC = {("mamba2_2p7b", "ssd_chunk_scan"): 412_230_912}
+
+
 def work_model(cfg, final_state=True, lay=None):
     B, T, H, P, N, G, Q = (cfg[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
                                             "ngroups", "chunk_len"))
@@ -66,19 +72,24 @@ def work_model(cfg, final_state=True, lay=None):
     s_sz = 2 if (lay is None or lay.states_dtype == 1) else 4
     sin_sz = 2 if (lay is None or lay.s_in_dtype == 1) else 4
     fused = bool(lay is not None and lay.fused_state)
+    # the chunk-wide scan (one launch more than the four-stage sequence) reads l
+    # and the per-token factors g [B,H,nc,Q+4] instead of l, dtq and beta
+    chunkwide = bool(lay is not None and lay.launches == (3 if fused else 4) + 1)
+    gq_bytes = B * H * nc * (Q + 4) * 4
     h0_bytes = state_bytes if cfg.get("init_state") else 0
     fin_bytes = state_bytes if final_state else 0
     per_kernel = {
-        # dt, A -> l, w, dtq, beta, alpha
-        "ssd_chunk_cumsum": dt_bytes + H * 4 + 4 * lq + B * H * nc * 4,
+        # dt, A -> l, w, dtq, beta, alpha (and g for the chunk-wide scan)
+        "ssd_chunk_cumsum": dt_bytes + H * 4 + 4 * lq + B * H * nc * 4 + (gq_bytes if chunkwide else 0),
         # x, B, w -> S  (fused: x, B, w, alpha, h0 -> s_in, final)
         "ssd_chunk_state": (x_bytes + bc_bytes // 2 + lq + B * H * nc * 4 + h0_bytes
                             + st_elems * sin_sz + fin_bytes) if fused
                            else (x_bytes + bc_bytes // 2 + lq + st_elems * s_sz),
         "ssd_state_passing": 0 if fused else (st_elems * s_sz + B * H * nc * 4 + h0_bytes
                                               + st_elems * sin_sz + fin_bytes),
-        # x, B, C, l, dtq, beta, s_in, D -> y
-        "ssd_chunk_scan": 2 * x_bytes + bc_bytes + 3 * lq + st_elems * sin_sz + H * 4,
+        # x, B, C, l, (g | dtq, beta), s_in, D -> y
+        "ssd_chunk_scan": (2 * x_bytes + bc_bytes + (lq + gq_bytes if chunkwide else 3 * lq)
+                           + st_elems * sin_sz + H * 4),
     }
     per_kernel_flops = {
         "ssd_chunk_state": 2 * B * nc * H * Q * N * P,
@@ -378,7 +389,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
         "config": config_block(cfg, args.workload),
         "roofline": {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None if args.batch is not None else NCU_TRAFFIC.get((args.workload, top)),
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"},
         "path_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": t_step * 1e6,
                           "frac": t_roof / t_step, "flops": wm["flops"],
