@@ -412,6 +412,135 @@ def run_gpu(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# decode step (ssd_step): one token per (batch, head) on a resident state
+# ---------------------------------------------------------------------------
+DECODE = dict(batch=64, nheads=80, headdim=64, dstate=128, ngroups=1, dtype="bf16")
+DECODE_METRIC = "SSD decode-step tokens/sec on 1 B200 and % of HBM roofline"
+
+
+def decode_inputs(cfg, seed=2000):
+    """One decode token per batch row, drawn like the scan's inputs, and a state
+    drawn N(0, 0.1^2) (resident on the device between steps)."""
+    from structured_state_space_mamba_b200.inputs import make_inputs
+    inp = make_inputs(cfg["batch"], 1, cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["ngroups"], 1,
+                      dtype=cfg["dtype"], seed=seed, init_state=True, h0_std=0.1)
+    return dict(x=inp.x[:, 0], dt=inp.dt[:, 0], A=inp.A, B=inp.B[:, 0], C=inp.C[:, 0], D=inp.D,
+                state=inp.h0)
+
+
+def decode_cpu_baseline(v, budget_s=8.0):
+    """The oracle's fp64 step on the host, repeated for about budget_s."""
+    import oracle
+    n, t0 = 0, time.perf_counter()
+    state = v["state"]
+    while time.perf_counter() - t0 < budget_s:
+        _, state = oracle.ssd_step(state, v["x"], v["dt"], v["A"], v["B"], v["C"], D=v["D"])
+        n += 1
+    sec = time.perf_counter() - t0
+    bsz = v["x"].shape[0]
+    return {"value": n * bsz / sec, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"fp64 numpy step over the full decode shape, {n} steps in {sec:.1f} s"}
+
+
+def run_decode(args, rank, world, local_rank):
+    import torch
+    from structured_state_space_mamba_b200 import binding
+    cfg = dict(DECODE)
+    if args.batch is not None:
+        cfg["batch"] = args.batch
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    v = decode_inputs(cfg, seed=2000 + rank)
+    sd = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
+    esz = 2 if cfg["dtype"] == "bf16" else 4
+    t = lambda a, ty=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(ty)  # noqa: E731
+    x, dt, A, B, C, D = t(v["x"], sd), t(v["dt"]), t(v["A"]), t(v["B"], sd), t(v["C"], sd), t(v["D"])
+    state = t(v["state"])
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.step(state, x, dt, A, B, C, D=D, out=y)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(val):
+        if world == 1:
+            return val
+        tt = torch.tensor([val], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        return float(tt.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    clocks = clk.summary()
+    # end to end: each step copies the token's inputs in from pinned host memory
+    # and reads y back (the state stays on the device, as in a generation loop)
+    hx, hdt, hB, hC = (a.cpu().pin_memory() for a in (x, dt, B, C))
+    hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(a.numel() * a.element_size() for a in (hx, hdt, hB, hC))
+    d2h = hy.numel() * hy.element_size()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(hx, non_blocking=True)
+        dt.copy_(hdt, non_blocking=True)
+        B.copy_(hB, non_blocking=True)
+        C.copy_(hC, non_blocking=True)
+        step()
+        hy.copy_(y, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    if rank != 0:
+        return
+    bsz, H, P, N, G = cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["ngroups"]
+    # algorithmic bytes of one step: the fp32 state read and written, x, y, dt, A, D, B, C
+    step_bytes = 2 * bsz * H * P * N * 4 + 2 * bsz * H * P * esz + bsz * H * 4 + 2 * H * 4 + 2 * bsz * G * N * esz
+    t_step = ms / args.steps * 1e-3
+    peaks, peak_src = load_peaks()
+    achieved = step_bytes / t_step / 1e9
+    value = world * bsz * args.steps / (ms * 1e-3)
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg["dtype"], "data": "synthetic",
+        "config": {"workload": f"decode_2p7b: one token, B={bsz} H={H} P={P} N={N} G={G} {cfg['dtype']}, "
+                               "fp32 state resident",
+                   "batch": bsz, "nheads": H, "headdim": P, "dstate": N, "ngroups": G,
+                   "l2": "no flush: the fp32 state exceeds L2 (126 MB)" if 2 * bsz * H * P * N * 4 > 126e6
+                         else "state smaller than L2", "parallelism": "replicas"},
+        "roofline": {"bound": "hbm", "kernel": "ssd_step", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"},
+        "gpu_launches": args.steps,
+        "e2e": {"value": world * bsz * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = decode_cpu_baseline(v)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -424,6 +553,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode step (ssd_step) on its own shape instead of the scan")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -445,7 +576,10 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, cfg, rank, world, local_rank)
+        if args.decode:
+            run_decode(args, rank, world, local_rank)
+        else:
+            run_gpu(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
             import torch

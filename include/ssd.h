@@ -156,6 +156,8 @@ SSD_API ssd_status_t ssd_forward_static(const ssd_dims_t *dims, const void *x, c
  *   stage 2  ssd_state_passing  states, alpha, init_state -> s_in, final_state_out
  *            (fused_state layouts: nothing)
  *   stage 3  ssd_chunk_scan     x, dt, B, C, D, l, s_in   -> y_out
+ *            (chunk_len 128/256 bf16 layouts: the chunk-wide scan, then the
+ *            list-mode scan of the tiles it left, two launches)
  * Any other stage value returns SSD_ERR_INVALID_DIM.
  */
 typedef enum {
@@ -171,6 +173,40 @@ SSD_API ssd_status_t ssd_forward_stage(int stage, const ssd_dims_t *dims, const 
                                        const float *init_state, void *y_out,
                                        float *final_state_out, void *workspace,
                                        size_t workspace_bytes, void *stream);
+
+/*
+ * ssd_step -- one token of the recurrence for every (batch, head): the decode
+ * step.  The recurrent form of the scalar-identity SSM (akillness.github.io
+ * "State Space Duality and Mamba-2: Unifying Transformers and Semiseparable
+ * Matrices", "Mathematical Foundations: From State Spaces to Semiseparable
+ * Matrices"), with dt on the decay and the input as in ssd_forward:
+ *   state <- exp(dt_t A_h) state + dt_t x_t B_t^T      (in place)
+ *   y_t    = state C_t + D_h x_t                       (with the new state)
+ * A generation loop calls it once per new token on the state that
+ * ssd_forward's final_state_out left behind.
+ *
+ *   dims       seqlen must be 1 (else SSD_ERR_INVALID_DIM); batch, nheads,
+ *              headdim, dstate, ngroups, dtype as for ssd_forward, with
+ *              headdim, dstate <= 256 (any value, no chunk rule)
+ *   x_t        [B, H, P]     dtype
+ *   dt_t       [B, H]        fp32 step sizes
+ *   A          [H]           fp32
+ *   B_t, C_t   [B, G, N]     dtype
+ *   D          [H]           fp32, or NULL for no skip term
+ *   state      [B, H, P, N]  fp32, read and overwritten with the new state;
+ *                            16-byte alignment and dstate in {16, 32, 64,
+ *                            128, 256} take the vectorised kernel, anything
+ *                            else a scalar one
+ *   y_t        [B, H, P]     dtype, written; must not alias the inputs
+ *   stream                   cudaStream_t
+ * The caller owns every buffer (device pointers).  Asynchronous, no
+ * allocation, one kernel launch; argument errors come back before the launch,
+ * a failed launch as SSD_ERR_CUDA.  Accuracy against the fp64 step: the bounds
+ * of ssd_forward, per call.
+ */
+SSD_API ssd_status_t ssd_step(const ssd_dims_t *dims, const void *x_t, const float *dt_t,
+                              const float *A, const void *B_t, const void *C_t, const float *D,
+                              float *state, void *y_t, void *stream);
 
 /* Bytes of workspace one call needs (0 if the arguments are invalid). */
 SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);

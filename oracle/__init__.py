@@ -27,7 +27,7 @@ import numpy as np
 
 from . import build as _build
 
-__all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "default_threads"]
+__all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "ssd_step", "default_threads"]
 
 
 class _Dims(ctypes.Structure):
@@ -164,3 +164,33 @@ def ssd_chunked(x, dt, A, B, C, chunk_len, D=None, h0=None, intermediates=False)
     if intermediates:
         return y, fin, dict(l=l, w=w, alpha=alpha, S=S, s_in=s_in[:, :nc])
     return y, fin
+
+
+def ssd_step(state, x, dt, A, B, C, D=None):
+    """One token of the recurrence for every (batch, head) in fp64 (numpy): the
+    decode step.  Per batch b, head h, group g = h // (H // G):
+        state' = exp(dt A_h) state + dt x B^T,   y = state' C + D_h x
+    (akillness.github.io "State Space Duality and Mamba-2", "Mathematical
+    Foundations": the recurrent form, one token).
+
+    state [B,H,P,N]; x [B,H,P]; dt [B,H]; A, D [H]; B, C [B,G,N].
+    Returns (y [B,H,P], new_state [B,H,P,N]) as float64 arrays; ``state`` is
+    not modified.
+    """
+    h = _f64(state)
+    x, dt, A, B, C, D = (_f64(v) for v in (x, dt, A, B, C, D))
+    bsz, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if h.shape != (bsz, H, P, N) or dt.shape != (bsz, H) or A.shape != (H,) or C.shape != B.shape:
+        raise ValueError("state [B,H,P,N], x [B,H,P], dt [B,H], A [H], B and C [B,G,N]")
+    if H % G:
+        raise ValueError("nheads must be a multiple of ngroups")
+    group = np.arange(H) // (H // G)        # head -> group
+    Bh = B[:, group, :]                     # [B,H,N]
+    Ch = C[:, group, :]
+    decay = np.exp(dt * A[None, :])         # [B,H]
+    new = decay[:, :, None, None] * h + (dt[:, :, None] * x)[:, :, :, None] * Bh[:, :, None, :]
+    y = np.einsum("bhpn,bhn->bhp", new, Ch)
+    if D is not None:
+        y = y + D[None, :, None] * x
+    return y, new

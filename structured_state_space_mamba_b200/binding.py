@@ -22,7 +22,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
 
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
            "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
-           "ssd_forward_static")
+           "ssd_forward_static", "ssd_step")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -75,6 +75,8 @@ def load():
     lib.ssd_forward_ws.restype = ctypes.c_int
     lib.ssd_forward_static.argtypes = lib.ssd_forward.argtypes
     lib.ssd_forward_static.restype = ctypes.c_int
+    lib.ssd_step.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, fp, vp, vp]
+    lib.ssd_step.restype = ctypes.c_int
     lib.ssd_forward_stage.argtypes = [ctypes.c_int] + lib.ssd_forward_ws.argtypes
     lib.ssd_forward_stage.restype = ctypes.c_int
     lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
@@ -219,6 +221,47 @@ def forward_static(x, dt, A, B, C, D=None, chunk_len=256, init_state=None,
 
 
 STATIC_SCRATCH_BYTES = 64 << 20  # SSD_STATIC_SCRATCH_BYTES in include/ssd.h
+
+
+def step(state, x, dt, A, B, C, D=None, out=None, stream=None):
+    """One decode step through ``ssd_step``: ``state`` [B,H,P,N] float32 is
+    updated in place to exp(dt A) state + dt x B^T and y = state C + D x is
+    returned.  x [B,H,P], B/C [B,G,N] (float32 or bfloat16, one dtype);
+    dt [B,H], A [H], D [H] float32."""
+    if not x.is_cuda:
+        raise ValueError("ssd.step runs on CUDA tensors only")
+    dev = x.device
+    for name, t in (("state", state), ("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D)):
+        if t is None:
+            continue
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, x on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if x.dtype not in (torch.float32, torch.bfloat16) or B.dtype != x.dtype or C.dtype != x.dtype:
+        raise ValueError("x, B and C must share a dtype: float32 or bfloat16")
+    for name, t in (("state", state), ("dt", dt), ("A", A), ("D", D)):
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32")
+    bsz, H, P = x.shape
+    if B.dim() != 3 or B.shape[0] != bsz or C.shape != B.shape:
+        raise ValueError("B and C must be [batch, ngroups, dstate]")
+    G, N = B.shape[1], B.shape[2]
+    if dt.shape != (bsz, H) or A.shape != (H,) or state.shape != (bsz, H, P, N):
+        raise ValueError("dt must be [batch, nheads], A [nheads], state [batch, nheads, headdim, dstate]")
+    if D is not None and D.shape != (H,):
+        raise ValueError("D must be [nheads]")
+    dims = make_dims(bsz, 1, H, P, N, G, x.dtype)
+    y = out if out is not None else torch.empty_like(x)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = load().ssd_step(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                             _ptr(state), _ptr(y), ctypes.c_void_p(stream))
+    _check(st)
+    return y
 
 
 def device_status(device=None) -> int:

@@ -163,3 +163,31 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         binding.forward(x, torch.zeros(1, 64, 2), torch.zeros(2), torch.zeros(1, 64, 1, 16),
                         torch.zeros(1, 64, 1, 16), chunk_len=64)
+
+
+def test_step_argument_checks(lib):
+    """ssd_step validates before any CUDA call (the pointers are never touched)."""
+    f = ctypes.c_void_p(FAKE)
+
+    def call(d, **kw):
+        v = dict(x=f, dt=f, A=f, B=f, C=f, D=None, state=f, y=f)
+        v.update(kw)
+        return lib.ssd_step(ctypes.byref(d) if d is not None else None, v["x"], v["dt"], v["A"],
+                            v["B"], v["C"], v["D"], v["state"], v["y"], None)
+
+    assert call(None) == 1
+    for name in ("x", "dt", "A", "B", "C", "state", "y"):
+        assert call(binding.make_dims(2, 1, 4, 64, 128, 2, "bf16"), **{name: None}) == 1, name
+    assert call(binding.make_dims(2, 2, 4, 64, 128, 2, "bf16")) == 2       # seqlen must be 1
+    assert call(binding.make_dims(2, 1, 4, 64, 128, 3, "bf16")) == 2       # H % G
+    assert call(binding.make_dims(2, 1, 4, 300, 128, 2, "f32")) == 3       # headdim > 256
+    bad = binding.make_dims(2, 1, 4, 64, 128, 2, "bf16")
+    bad.dtype = 7
+    assert call(bad) == 3
+
+
+def test_binding_step_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.step(torch.zeros(1, 2, 16, 16), torch.zeros(1, 2, 16), torch.zeros(1, 2),
+                     torch.zeros(2), torch.zeros(1, 1, 16), torch.zeros(1, 1, 16))

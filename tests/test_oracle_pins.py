@@ -16,7 +16,9 @@ semiseparable matrix, and closed forms computed here with plain numpy:
 * T = 1 hand formula;
 * split sequence with the state carried across the split (the constant-size
   recurrent state of the recurrent mode);
-* linearity in x, superposition in (x, h0), group sharing, head permutation.
+* linearity in x, superposition in (x, h0), group sharing, head permutation;
+* the decode step: T single steps == the recurrence over T tokens, and one step
+  == the same hand formula written element by element.
 """
 import json
 import os
@@ -294,3 +296,64 @@ def test_golden_rejects_planted_mistakes(oracle):
             if case["name"] == "unit_step" and v == "no_dt_input":
                 continue  # dt = 1 makes that mistake invisible; the other cases catch it
             assert np.max(np.abs(yv - np.array(case["y"]))) > 1e-3, (case["name"], v)
+
+
+# --------------------------------------------------------------------------
+# the decode step (one token of the recurrence)
+# --------------------------------------------------------------------------
+def test_steps_equal_recurrence(oracle):
+    """Applying ssd_step token by token reproduces the recurrence oracle."""
+    inp = small(seed=21, T=17, H=6, G=3)
+    y_ref, fin_ref = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    state = inp.h0.astype(np.float64)
+    ys = []
+    for t in range(inp.x.shape[1]):
+        y_t, state = oracle.ssd_step(state, inp.x[:, t], inp.dt[:, t], inp.A, inp.B[:, t], inp.C[:, t],
+                                     D=inp.D)
+        ys.append(y_t)
+    assert rel_err(np.stack(ys, axis=1), y_ref) < 1e-12
+    assert rel_err(state, fin_ref) < 1e-12
+
+
+def test_step_hand_formula_elementwise(oracle):
+    """One step written out element by element with scalar loops (no numpy
+    broadcasting): group map, decay, input outer product, readout and skip."""
+    rng = np.random.default_rng(22)
+    bsz, H, P, N, G = 2, 4, 3, 5, 2
+    state = rng.standard_normal((bsz, H, P, N))
+    x = rng.standard_normal((bsz, H, P))
+    dt = rng.uniform(0.01, 0.5, size=(bsz, H))
+    A = -rng.uniform(0.1, 4.0, size=H)
+    B = rng.standard_normal((bsz, G, N))
+    C = rng.standard_normal((bsz, G, N))
+    D = rng.standard_normal(H)
+    y, new = oracle.ssd_step(state, x, dt, A, B, C, D=D)
+    import math
+    for b in range(bsz):
+        for h in range(H):
+            g = h // (H // G)
+            a = math.exp(dt[b, h] * A[h])
+            for p in range(P):
+                acc = 0.0
+                for n in range(N):
+                    s_new = a * state[b, h, p, n] + dt[b, h] * x[b, h, p] * B[b, g, n]
+                    assert abs(new[b, h, p, n] - s_new) <= 1e-13 * max(1.0, abs(s_new))
+                    acc += s_new * C[b, g, n]
+                want = acc + D[h] * x[b, h, p]
+                assert abs(y[b, h, p] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_step_dt_zero_and_no_skip(oracle):
+    """dt = 0 leaves the state and reads it out; D = None drops the skip term."""
+    rng = np.random.default_rng(23)
+    state = rng.standard_normal((1, 2, 3, 4))
+    x = rng.standard_normal((1, 2, 3))
+    B = rng.standard_normal((1, 1, 4))
+    C = rng.standard_normal((1, 1, 4))
+    D = np.array([0.5, -2.0])
+    y, new = oracle.ssd_step(state, x, np.zeros((1, 2)), np.array([-1.0, -3.0]), B, C, D=D)
+    assert np.array_equal(new, state)
+    np.testing.assert_allclose(y, np.einsum("bhpn,n->bhp", state, C[0, 0]) + D[None, :, None] * x,
+                               rtol=1e-14, atol=1e-14)
+    y0, _ = oracle.ssd_step(state, x, np.zeros((1, 2)), np.array([-1.0, -3.0]), B, C)
+    np.testing.assert_allclose(y0, np.einsum("bhpn,n->bhp", state, C[0, 0]), rtol=1e-14, atol=1e-14)
