@@ -50,6 +50,23 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 NCU_TRAFFIC = {("mamba2_2p7b", "ssd_chunk_scan"): 412_230_912}
 
 
+def max_over_ranks(value, world, device):
+    """The largest of every rank's `value` (a time); every rank gets it.  One
+    all-reduce over the job's process group (NCCL on GPUs, gloo on CPUs)."""
+    if world == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, units_per_rank_step, steps, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank does the same work)."""
+    return world * units_per_rank_step * steps / (ms * 1e-3)
+
+
 def work_model(cfg, final_state=True, lay=None):
     B, T, H, P, N, G, Q = (cfg[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
                                             "ngroups", "chunk_len"))
@@ -275,12 +292,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    def max_ms(v):
+        return max_over_ranks(v, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -310,7 +323,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        return max_over_ranks(e0.elapsed_time(e1))
+        return max_ms(e0.elapsed_time(e1))
 
     # ---- timed region: K back-to-back steps -------------------------------
     with ClockSampler(local_rank) as clk:
@@ -368,13 +381,13 @@ def run_gpu(args, cfg, rank, world, local_rank):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_ms = max_ms(f0.elapsed_time(f1))
     barrier()
 
     if rank != 0:
         return
     tokens_step = inp.x.shape[0] * inp.x.shape[1]
-    value = world * tokens_step * args.steps / (ms_total * 1e-3)
+    value = job_rate(world, tokens_step, args.steps, ms_total)
     wm = work_model(cfg, final_state=want_final, lay=lay)
     peaks, peak_src = load_peaks()
     top = max(kern_ms, key=kern_ms.get)
@@ -403,7 +416,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "gpu_launches": args.steps * lay.launches,
         "tensor_core": bool(lay.tensor_core),
         "fused_state": bool(lay.fused_state),
-        "e2e": {"value": world * tokens_step * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_rate(world, tokens_step, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
     }
@@ -467,12 +480,8 @@ def run_decode(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(val):
-        if world == 1:
-            return val
-        tt = torch.tensor([val], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        return float(tt.item())
+    def max_ms(v):
+        return max_over_ranks(v, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -487,7 +496,7 @@ def run_decode(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_ms(e0.elapsed_time(e1))
     clocks = clk.summary()
     # end to end: each step copies the token's inputs in from pinned host memory
     # and reads y back (the state stays on the device, as in a generation loop)
@@ -509,7 +518,7 @@ def run_decode(args, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_ms = max_ms(f0.elapsed_time(f1))
     if rank != 0:
         return
     bsz, H, P, N, G = cfg["batch"], cfg["nheads"], cfg["headdim"], cfg["dstate"], cfg["ngroups"]
@@ -518,7 +527,7 @@ def run_decode(args, rank, world, local_rank):
     t_step = ms / args.steps * 1e-3
     peaks, peak_src = load_peaks()
     achieved = step_bytes / t_step / 1e9
-    value = world * bsz * args.steps / (ms * 1e-3)
+    value = job_rate(world, bsz, args.steps, ms)
     line = {
         "metric": DECODE_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -532,7 +541,7 @@ def run_decode(args, rank, world, local_rank):
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"},
         "gpu_launches": args.steps,
-        "e2e": {"value": world * bsz * args.steps / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_rate(world, bsz, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,
     }
