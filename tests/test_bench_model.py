@@ -1,0 +1,68 @@
+"""Host-side accounting of bench.py (CPU): the algorithmic bytes behind the
+roofline fractions and the L2 timing policy."""
+import pytest
+
+import bench
+from structured_state_space_mamba_b200 import binding
+from structured_state_space_mamba_b200.inputs import WORKLOADS
+
+MB = 1e6
+
+
+def layout(cfg):
+    d = binding.make_dims(cfg["batch"], cfg["seqlen"], cfg["nheads"], cfg["headdim"], cfg["dstate"],
+                          cfg["ngroups"], cfg["dtype"])
+    return binding.workspace_layout(d, cfg["chunk_len"])
+
+
+def test_scan_bytes_of_the_2p7b_layer_by_hand():
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    lay = layout(cfg)
+    wm = bench.work_model(cfg, True, lay)
+    B, T, H, P, N, Q = 4, 4096, 80, 64, 128, 256
+    nc = T // Q
+    x = B * T * H * P * 2                       # bf16 x (and y)
+    bc = 2 * B * T * N * 2                      # bf16 B and C, one group
+    l_g = B * H * nc * Q * 4 + B * H * nc * (Q + 4) * 4
+    s_in = B * nc * H * P * N * 2               # bf16 state entering each chunk
+    assert wm["per_kernel_bytes"]["ssd_chunk_scan"] == 2 * x + bc + l_g + s_in + H * 4
+    assert wm["per_kernel_bytes"]["ssd_chunk_scan"] / MB == pytest.approx(438.4, abs=0.1)
+    # chunk_state reads x, B and w and writes the bf16 chunk states
+    assert wm["per_kernel_bytes"]["ssd_chunk_state"] / MB == pytest.approx(261.1, abs=0.1)
+    # compulsory bytes: x and y, B and C, dt, A and D, the final fp32 state
+    comp = 2 * x + bc + B * T * H * 4 + 2 * H * 4 + B * H * P * N * 4
+    assert wm["bytes"] == comp
+
+
+def test_fused_layout_has_no_state_passing_traffic():
+    cfg = dict(WORKLOADS["mamba2_130m"])
+    lay = layout(cfg)
+    assert lay.fused_state == 1
+    wm = bench.work_model(cfg, True, lay)
+    assert wm["per_kernel_bytes"]["ssd_state_passing"] == 0
+
+
+def test_flops_count_the_causal_products_once():
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    wm = bench.work_model(cfg, True, layout(cfg))
+    B, T, H, P, N, G, Q = 4, 4096, 80, 64, 128, 1, 256
+    nc = T // Q
+    per_bch = Q * (Q + 1) * P + 4 * Q * N * P
+    per_bcg = Q * (Q + 1) * N
+    assert wm["flops"] == B * nc * (H * per_bch + G * per_bcg)
+
+
+@pytest.mark.parametrize("name, flush", [("mamba2_2p7b", False), ("long_g8", False),
+                                         ("mamba2_130m", True), ("tiny_f32", True)])
+def test_l2_policy(name, flush):
+    got, note = bench.l2_policy(WORKLOADS[name], 126 * 1024 * 1024)
+    assert got is flush
+    assert ("flushed" in note) is flush
+
+
+def test_traffic_figure_only_for_the_captured_kernel():
+    assert set(bench.NCU_TRAFFIC) == {("mamba2_2p7b", "ssd_chunk_scan")}
+    # the capture moved somewhat less than the algorithmic bytes (part of y still in L2)
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    algo = bench.work_model(cfg, True, layout(cfg))["per_kernel_bytes"]["ssd_chunk_scan"]
+    assert 0.8 * algo < bench.NCU_TRAFFIC[("mamba2_2p7b", "ssd_chunk_scan")] <= algo
