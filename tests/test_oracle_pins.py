@@ -357,3 +357,44 @@ def test_step_dt_zero_and_no_skip(oracle):
                                rtol=1e-14, atol=1e-14)
     y0, _ = oracle.ssd_step(state, x, np.zeros((1, 2)), np.array([-1.0, -3.0]), B, C)
     np.testing.assert_allclose(y0, np.einsum("bhpn,n->bhp", state, C[0, 0]), rtol=1e-14, atol=1e-14)
+
+
+def _step_variant(kind, state, x, dt, A, B, C, D):
+    """A numpy step with one plausible mistake planted (or none: 'correct')."""
+    H, G = x.shape[1], B.shape[1]
+    group = np.arange(H) // (H // G)
+    if kind == "group_modulo":          # head h -> group h % G instead of h // (H/G)
+        group = np.arange(H) % G
+    Bh, Ch = B[:, group, :], C[:, group, :]
+    decay = np.exp(dt * A[None, :])
+    if kind == "decay_without_dt":
+        decay = np.exp(np.broadcast_to(A[None, :], dt.shape))
+    inp = dt[:, :, None] * x
+    if kind == "no_dt_input":
+        inp = x
+    new = decay[:, :, None, None] * state + inp[:, :, :, None] * Bh[:, :, None, :]
+    read = state if kind == "read_before_update" else new
+    y = np.einsum("bhpn,bhn->bhp", read, Ch) + D[None, :, None] * x
+    return y, new
+
+
+def test_step_pins_reject_planted_mistakes(oracle):
+    """The steps-equal-recurrence pin fails for each planted mistake and holds
+    for the unmutated step (and for the oracle's own)."""
+    inp = small(seed=24, T=9, H=4, G=2)
+    y_ref, fin_ref = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    args64 = [np.asarray(a, np.float64) for a in (inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, inp.h0)]
+    x, dt, A, B, C, D, h0 = args64
+
+    def run(kind):
+        state, ys = h0, []
+        for t in range(x.shape[1]):
+            y_t, state = _step_variant(kind, state, x[:, t], dt[:, t], A, B[:, t], C[:, t], D)
+            ys.append(y_t)
+        return np.stack(ys, axis=1), state
+
+    y, fin = run("correct")
+    assert rel_err(y, y_ref) < 1e-12 and rel_err(fin, fin_ref) < 1e-12
+    for kind in ("group_modulo", "decay_without_dt", "no_dt_input", "read_before_update"):
+        yv, fv = run(kind)
+        assert rel_err(yv, y_ref) > 1e-3, kind
