@@ -126,6 +126,95 @@ def test_chunked_intermediates_consistent(oracle):
 
 
 # --------------------------------------------------------------------------
+# every intermediate of the chunked form, pinned to the recurrence
+# --------------------------------------------------------------------------
+# Each stage output of the chunked algorithm (aifetchly blog "Mamba-2
+# Architecture", "The Chunked SSD Algorithm", steps 1-2) is a state of the
+# recurrence over some token range, so the token-by-token oracle -- itself
+# pinned above to the explicit T x T dual matrix and the hand-worked 3x3 case
+# -- fixes all of them without restating their formulas:
+#   S_c      = final state of the recurrence over chunk c alone, from zero;
+#   s_in[c]  = final state of the recurrence over tokens [0, cQ), from h0;
+#   alpha_c  = final state over chunk c with x = 0, from an all-ones state;
+#   w_s      = final state over chunk c with x zero except at token s, from
+#              zero, divided by x_s[p] B_s[n] (the state is w_s x_s B_s^T).
+
+_PIN_Q = 8
+
+
+def _slice_t(inp, t0, t1):
+    return (inp.x[:, t0:t1], inp.dt[:, t0:t1], inp.A, inp.B[:, t0:t1], inp.C[:, t0:t1])
+
+
+def _intermediate_pins(oracle, inp, Q, it):
+    """Check (w, S, alpha, s_in) of the chunked form against recurrence runs;
+    returns the largest relative error of each."""
+    bsz, T, H, P = inp.x.shape
+    N = inp.B.shape[3]
+    nc = T // Q
+    h0 = inp.h0.astype(np.float64)
+    errs = {"S": 0.0, "s_in": 0.0, "alpha": 0.0, "w": 0.0}
+    for c in range(nc):
+        t0, t1 = c * Q, (c + 1) * Q
+        _, S_ref = oracle.ssd_recurrent(*_slice_t(inp, t0, t1))
+        errs["S"] = max(errs["S"], rel_err(it["S"][:, c], S_ref))
+        if c == 0:
+            s_ref = h0
+        else:
+            _, s_ref = oracle.ssd_recurrent(*_slice_t(inp, 0, t0), h0=h0)
+        errs["s_in"] = max(errs["s_in"], rel_err(it["s_in"][:, c], s_ref))
+        a = _slice_t(inp, t0, t1)
+        _, ones_fin = oracle.ssd_recurrent(np.zeros_like(a[0]), *a[1:],
+                                           h0=np.ones((bsz, H, P, N)))
+        errs["alpha"] = max(errs["alpha"],
+                            rel_err(it["alpha"][:, :, c][..., None, None] * np.ones((P, N)),
+                                    ones_fin))
+        x64 = a[0].astype(np.float64)
+        B64 = a[3].astype(np.float64)
+        r = H // inp.B.shape[2]
+        for s in range(Q):
+            xs = np.zeros_like(x64)
+            xs[:, s] = x64[:, s]
+            _, fin_s = oracle.ssd_recurrent(xs, *a[1:])
+            # fin_s[b,h,p,n] = w_s x_s[b,h,p] B_s[b,g(h),n]: read w at (p, n) = (0, 0)
+            denom = x64[:, s, :, 0] * np.repeat(B64[:, s, :, 0], r, axis=1)  # [b,h]
+            w_ref = fin_s[:, :, 0, 0] / denom
+            errs["w"] = max(errs["w"], rel_err(it["w"][:, :, c, s], w_ref))
+    return errs
+
+
+def test_chunked_intermediates_pinned_to_recurrence(oracle):
+    """Every chunk's S, s_in, alpha and every token's w equal the recurrence
+    states that define them (fp64, 1e-12)."""
+    inp = small(seed=4, T=24)
+    a, kw = args(inp)
+    _, _, it = oracle.ssd_chunked(*a, _PIN_Q, intermediates=True, **kw)
+    errs = _intermediate_pins(oracle, inp, _PIN_Q, it)
+    for k, e in errs.items():
+        assert e < 1e-12, (k, e)
+
+
+def test_intermediate_pins_reject_planted_mistakes(oracle):
+    """The pins above fail for plausible mistakes in the stage outputs: a flipped
+    sign in w's exponent, S and s_in taken one chunk off, and alpha without
+    the exponential's last term."""
+    inp = small(seed=4, T=24)
+    a, kw = args(inp)
+    _, _, it = oracle.ssd_chunked(*a, _PIN_Q, intermediates=True, **kw)
+    l = it["l"]
+    dtc = inp.dt.astype(np.float64).transpose(0, 2, 1).reshape(l.shape)
+    planted = {
+        "w": dict(it, w=np.exp(l - l[..., -1:]) * dtc),              # exp(l_s - l_last) dt_s
+        "S": dict(it, S=np.roll(it["S"], 1, axis=1)),               # chunk offset off by one
+        "s_in": dict(it, s_in=np.roll(it["s_in"], -1, axis=1)),     # next chunk's state
+        "alpha": dict(it, alpha=np.exp(l[..., -2])),                # decay of Q-1 tokens
+    }
+    for key, bent in planted.items():
+        errs = _intermediate_pins(oracle, inp, _PIN_Q, bent)
+        assert errs[key] > 1e-3, (key, errs)
+
+
+# --------------------------------------------------------------------------
 # closed forms
 # --------------------------------------------------------------------------
 def test_A_zero_is_causal_linear_attention(oracle):
