@@ -47,7 +47,15 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # DRAM bytes (read + write) of one launch of the dominant kernel on a workload,
 # from one ncu capture of the current kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum); workloads without such a capture report None.
-NCU_TRAFFIC = {("mamba2_2p7b", "ssd_chunk_scan"): 412_230_912}
+# Keyed by (workload, kernel, library version): a capture stands only for the
+# build it was taken from, so a rebuilt kernel reports traffic None until it is
+# captured again.
+NCU_TRAFFIC = {("mamba2_2p7b", "ssd_chunk_scan", "ssd-b200 0.1.0 sm_100a"): 412_230_912}
+
+
+def ncu_traffic(workload, kernel):
+    from structured_state_space_mamba_b200 import binding
+    return NCU_TRAFFIC.get((workload, kernel, binding.version()))
 
 
 def max_over_ranks(value, world, device):
@@ -108,12 +116,20 @@ def work_model(cfg, final_state=True, lay=None):
         "ssd_chunk_scan": (2 * x_bytes + bc_bytes + (lq + gq_bytes if chunkwide else 3 * lq)
                            + st_elems * sin_sz + H * 4),
     }
+    # the compulsory bytes (above) that each kernel moves itself: the roofline
+    # fraction of a kernel counts only these; workspace traffic is its loss
+    per_kernel_comp = {
+        "ssd_chunk_cumsum": dt_bytes + H * 4,
+        "ssd_chunk_state": x_bytes + bc_bytes // 2 + ((h0_bytes + fin_bytes) if fused else 0),
+        "ssd_state_passing": 0 if fused else h0_bytes + fin_bytes,
+        "ssd_chunk_scan": 2 * x_bytes + bc_bytes + H * 4,
+    }
     per_kernel_flops = {
         "ssd_chunk_state": 2 * B * nc * H * Q * N * P,
         "ssd_chunk_scan": B * nc * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * flops_bcg),
     }
     return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
-                per_kernel_flops=per_kernel_flops)
+                per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops)
 
 
 def load_peaks():
@@ -128,15 +144,30 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
+def gpu_identity(device_index):
+    """nvidia-smi's id of the torch device: its UUID ("GPU-..."), which names the
+    same physical GPU whatever CUDA_VISIBLE_DEVICES maps (nvidia-smi's own
+    indices follow PCI order and ignore it); the PCI bus id if no UUID is known."""
+    import torch
+    p = torch.cuda.get_device_properties(device_index)
+    u = str(getattr(p, "uuid", "") or "")
+    if u:
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+
+
 class ClockSampler:
-    def __init__(self, index=0):
+    """Samples the SM clock and the clock-event reasons of ONE GPU, named by its
+    nvidia-smi id (gpu_identity), while the timed region runs."""
+
+    def __init__(self, gpu_id):
         self.proc = None
-        self.index = index
+        self.gpu_id = str(gpu_id)
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index),
+                ["nvidia-smi", "-i", self.gpu_id,
                  "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
@@ -179,7 +210,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu_id}
 
 
 # ---------------------------------------------------------------------------
@@ -234,7 +265,9 @@ def run_reference(args, cfg, rank):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference", "config": config_block(cfg, args.workload),
+            "data": "synthetic", "impl": "reference",
+            "config": config_block(cfg, args.workload,
+                                   l2_policy(cfg, device_l2_bytes(int(os.environ.get("LOCAL_RANK", "0"))))[1]),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": th, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -256,6 +289,20 @@ def l2_policy(cfg, l2_bytes):
                        f"L2 {l2_bytes / 1e6:.0f} MB)")
     return True, (f"L2 flushed before every timed step by a {2 * l2_bytes / 1e6:.0f} MB write outside "
                   f"the step's events (x and y {x_bytes / 1e6:.0f} MB each, L2 {l2_bytes / 1e6:.0f} MB)")
+
+
+def device_l2_bytes(device_index=0):
+    """L2 size of the GPU the run uses (the fallback when no GPU is visible);
+    both arms build config.l2 from it, so identical workloads get identical
+    config blocks."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            return int(getattr(torch.cuda.get_device_properties(device_index), "L2_cache_size", 0)
+                       or L2_FALLBACK_BYTES)
+    except Exception:  # noqa: BLE001 -- the note is informational
+        pass
+    return L2_FALLBACK_BYTES
 
 
 def config_block(cfg, name, l2_note=None):
@@ -329,7 +376,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
             graph.replay()
         torch.cuda.synchronize()
 
-    l2_bytes = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or L2_FALLBACK_BYTES
+    l2_bytes = device_l2_bytes(local_rank)
     flush, l2_note = l2_policy(cfg, l2_bytes)
     flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if flush else None
 
@@ -360,7 +407,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         return max_ms(e0.elapsed_time(e1))
 
     # ---- timed region: K back-to-back steps -------------------------------
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(gpu_identity(local_rank)) as clk:
         ms_direct = timed(step)
         ms_graph = timed(graph.replay) if graph is not None else None
     clocks = clk.summary()
@@ -426,9 +473,14 @@ def run_gpu(args, cfg, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     top = max(kern_ms, key=kern_ms.get)
     bound = "hbm"
-    achieved = wm["per_kernel_bytes"][top] / (kern_ms[top] * 1e-3) / 1e9
-    peak = peaks["hbm_gbs"]
     t_step = ms_total / args.steps * 1e-3
+    # the kernel's time inside the timed step: its share of the per-stage event
+    # times applied to the step (stage-by-stage launches carry launch gaps that
+    # the graph-replayed step does not, so their sum exceeds the step)
+    share = kern_ms[top] / sum(kern_ms.values())
+    t_top = share * t_step
+    achieved = wm["per_kernel_comp"][top] / t_top / 1e9
+    peak = peaks["hbm_gbs"]
     t_roof = max(wm["flops"] / (peaks["bf16_tflops"] * 1e12), wm["bytes"] / (peaks["hbm_gbs"] * 1e9))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -437,8 +489,14 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "config": config_block(cfg, args.workload, l2_note),
         "roofline": {"bound": bound, "kernel": top, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None if args.batch is not None else NCU_TRAFFIC.get((args.workload, top)),
-                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"},
+                     "traffic": None if args.batch is not None else ncu_traffic(args.workload, top),
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                     "bytes": "compulsory bytes the kernel moves (inputs it reads, outputs it "
+                              "writes); workspace traffic counts against it",
+                     "compulsory_bytes": wm["per_kernel_comp"][top],
+                     "kernel_us_in_step": t_top * 1e6, "kernel_share_of_step": share,
+                     "bytes_incl_workspace": wm["per_kernel_bytes"][top],
+                     "frac_incl_workspace": wm["per_kernel_bytes"][top] / t_top / 1e9 / peak},
         "path_roofline": {"t_roof_us": t_roof * 1e6, "t_step_us": t_step * 1e6,
                           "frac": t_roof / t_step, "flops": wm["flops"],
                           "compulsory_bytes": wm["bytes"],
@@ -521,7 +579,7 @@ def run_decode(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(gpu_identity(local_rank)) as clk:
         barrier()
         torch.cuda.synchronize()
         e0.record(stream)

@@ -24,8 +24,13 @@
  *    returned BEFORE anything is launched; launch errors come back as
  *    SSD_ERR_CUDA.  Errors of kernels that already ran surface, as usual in
  *    CUDA, on the next synchronising call.
- *  - Re-entrant: no global mutable state except a per-device cache of device
- *    properties.
+ *  - Shared state: a per-device cache of device properties; one device-side
+ *    error word per device (set by an expired bounded wait, read and cleared by
+ *    ssd_device_status); and the static scratch array of ssd_forward_static,
+ *    which every call of that entry point on a device shares, so that such
+ *    calls overlapping in time race (see ssd_forward_static).  The other entry
+ *    points keep no state between calls and may run concurrently on
+ *    different streams with separate outputs and workspaces.
  */
 #ifndef SSD_H_
 #define SSD_H_

@@ -60,9 +60,42 @@ def test_l2_policy(name, flush):
     assert ("flushed" in note) is flush
 
 
-def test_traffic_figure_only_for_the_captured_kernel():
-    assert set(bench.NCU_TRAFFIC) == {("mamba2_2p7b", "ssd_chunk_scan")}
-    # the capture moved somewhat less than the algorithmic bytes (part of y still in L2)
+def test_traffic_figure_only_for_the_captured_kernel_and_build():
+    keys = set(bench.NCU_TRAFFIC)
+    assert all(len(k) == 3 for k in keys)
     cfg = dict(WORKLOADS["mamba2_2p7b"])
-    algo = bench.work_model(cfg, True, layout(cfg))["per_kernel_bytes"]["ssd_chunk_scan"]
-    assert 0.8 * algo < bench.NCU_TRAFFIC[("mamba2_2p7b", "ssd_chunk_scan")] <= algo
+    wm = bench.work_model(cfg, True, layout(cfg))
+    for (wl, kern, ver), traffic in bench.NCU_TRAFFIC.items():
+        # a capture moves at least the kernel's compulsory bytes and, with L2
+        # hits, at most somewhat more than its workspace-inclusive bytes
+        assert wl in WORKLOADS
+        w = bench.work_model(dict(WORKLOADS[wl]), True, layout(dict(WORKLOADS[wl])))
+        assert 0.8 * w["per_kernel_comp"][kern] < traffic <= 1.2 * w["per_kernel_bytes"][kern]
+    # a build the capture was not taken from reports no traffic figure
+    assert bench.NCU_TRAFFIC.get(("mamba2_2p7b", "ssd_chunk_scan", "some other build")) is None
+    assert wm["per_kernel_comp"]["ssd_chunk_scan"] <= wm["per_kernel_bytes"]["ssd_chunk_scan"]
+
+
+def test_kernel_roofline_counts_compulsory_bytes_only():
+    """The scan's roofline bytes are the compulsory bytes it moves itself (x in,
+    y out, B, C and D in); the chunk states it reads are not among them."""
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    wm = bench.work_model(cfg, True, layout(cfg))
+    B, T, H, P, N = 4, 4096, 80, 64, 128
+    x = B * T * H * P * 2
+    bc = 2 * B * T * N * 2
+    assert wm["per_kernel_comp"]["ssd_chunk_scan"] == 2 * x + bc + H * 4
+    assert wm["per_kernel_comp"]["ssd_chunk_cumsum"] == B * T * H * 4 + H * 4
+
+
+def test_both_arms_build_the_same_config_block():
+    """The reference arm and the GPU arm describe one workload with one config
+    block when they see the same L2 size."""
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    cfg.setdefault("final_state", True)
+    l2 = 133 * 1000 * 1000
+    a = bench.config_block(cfg, "mamba2_2p7b", bench.l2_policy(cfg, l2)[1])
+    b = bench.config_block(cfg, "mamba2_2p7b", bench.l2_policy(cfg, l2)[1])
+    assert a == b
+    # without a GPU the helper falls back to the nominal L2 size
+    assert bench.device_l2_bytes() > 0
