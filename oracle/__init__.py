@@ -27,7 +27,8 @@ import numpy as np
 
 from . import build as _build
 
-__all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "ssd_step", "default_threads"]
+__all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "ssd_step", "default_threads",
+           "dt_transform", "gated_rmsnorm", "ssd_block"]
 
 
 class _Dims(ctypes.Structure):
@@ -194,3 +195,51 @@ def ssd_step(state, x, dt, A, B, C, D=None):
     if D is not None:
         y = y + D[None, :, None] * x
     return y, new
+
+
+# ---------------------------------------------------------------------------
+# the scan's neighbours in the Mamba-2 block (aifetchly blog "Mamba-2
+# Architecture: State Space Duality Explained", "Step 2: Full Mamba-2 Block with
+# Gated Projections": softplus on dt before the SSD call; the SSD output gated by
+# silu of the z branch; RMSNorm over d_inner = H * P; akillness.github.io "State
+# Space Duality and Mamba-2", the block diagram: "Element-wise Gating", RMSNorm)
+# ---------------------------------------------------------------------------
+def dt_transform(dt, dt_bias=None, softplus=False):
+    """The step size the scan uses: dt + dt_bias[h], then softplus if asked,
+    softplus(v) = log(1 + exp(v)), in fp64.  dt [B,T,H]; dt_bias [H] or None."""
+    v = _f64(dt).copy()
+    if dt_bias is not None:
+        v = v + _f64(dt_bias)[None, None, :]
+    if softplus:
+        # log(1 + e^v) = max(v, 0) + log(1 + e^-|v|): the same number, without overflow
+        v = np.maximum(v, 0.0) + np.log1p(np.exp(-np.abs(v)))
+    return v
+
+
+def gated_rmsnorm(y, z=None, weight=None, eps=1e-5):
+    """The block's output side, in fp64: g = y * silu(z) (silu(z) = z / (1 +
+    e^-z); no gate when z is None), then RMSNorm over each token's H * P values,
+    out = g / sqrt(mean(g^2) + eps) * weight (weight [H*P]; no norm when weight is
+    None).  y, z [B,T,H,P].  Returns (out [B,T,H,P], rstd [B,T] or None)."""
+    g = _f64(y)
+    if z is not None:
+        zz = _f64(z)
+        g = g * (zz / (1.0 + np.exp(-zz)))
+    if weight is None:
+        return g, None
+    bsz, T, H, P = g.shape
+    flat = g.reshape(bsz, T, H * P)
+    rstd = 1.0 / np.sqrt(np.mean(flat * flat, axis=-1) + float(eps))
+    out = flat * rstd[..., None] * _f64(weight)[None, None, :]
+    return out.reshape(bsz, T, H, P), rstd
+
+
+def ssd_block(x, dt, A, B, C, D=None, h0=None, dt_bias=None, dt_softplus=False, z=None,
+              norm_weight=None, norm_eps=1e-5, units=None, nthreads=0):
+    """The scan with its neighbours, in the block's order: dt_transform, the
+    recurrence (ssd_recurrent), gated_rmsnorm.  Returns (out, final_state,
+    rstd)."""
+    dte = dt_transform(dt, dt_bias, dt_softplus)
+    y, fin = ssd_recurrent(x, dte, A, B, C, D=D, h0=h0, units=units, nthreads=nthreads)
+    out, rstd = gated_rmsnorm(y, z, norm_weight, norm_eps)
+    return out, fin, rstd
