@@ -50,7 +50,7 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # Keyed by (workload, kernel, library version): a capture stands only for the
 # build it was taken from, so a rebuilt kernel reports traffic None until it is
 # captured again.
-NCU_TRAFFIC = {("mamba2_2p7b", "ssd_chunk_scan", "ssd-b200 0.1.0 sm_100a"): 412_230_912}
+NCU_TRAFFIC = {}
 
 
 def ncu_traffic(workload, kernel):
@@ -103,6 +103,25 @@ def work_model(cfg, final_state=True, lay=None):
     gq_bytes = B * H * nc * (Q + 4) * 4
     h0_bytes = state_bytes if cfg.get("init_state") else 0
     fin_bytes = state_bytes if final_state else 0
+    if lay is not None and getattr(lay, "single_pass", 0):
+        # cumsum (fused mode): dt, A -> l and g (dtq and beta only for chunks with
+        # a steep tile); the single-pass kernel: x, B, C, l, g, D, h0 -> y, final
+        # (its per-(b, h) state slots stay in L2: B*H*P*N*4 bytes, each written
+        # and read once per chunk); the block-factored scan: only listed tiles
+        per_kernel = {
+            "ssd_chunk_cumsum": dt_bytes + H * 4 + lq + gq_bytes,
+            "ssd_chunk_fused": (2 * x_bytes + bc_bytes + lq + gq_bytes + H * 4 + h0_bytes + fin_bytes),
+            "ssd_chunk_scan_steep": 0,
+        }
+        per_kernel_comp = {
+            "ssd_chunk_cumsum": dt_bytes + H * 4,
+            "ssd_chunk_fused": 2 * x_bytes + bc_bytes + H * 4 + h0_bytes + fin_bytes,
+            "ssd_chunk_scan_steep": 0,
+        }
+        per_kernel_flops = {"ssd_chunk_fused": flops}
+        return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
+                    per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops,
+                    stages=("ssd_chunk_cumsum", "ssd_chunk_fused", None, "ssd_chunk_scan_steep"))
     per_kernel = {
         # dt, A -> l, w, dtq, beta, alpha (and g for the chunk-wide scan)
         "ssd_chunk_cumsum": dt_bytes + H * 4 + 4 * lq + B * H * nc * 4 + (gq_bytes if chunkwide else 0),
@@ -129,7 +148,8 @@ def work_model(cfg, final_state=True, lay=None):
         "ssd_chunk_scan": B * nc * (H * (Q * (Q + 1) * P + 2 * Q * N * P) + G * flops_bcg),
     }
     return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
-                per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops)
+                per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops,
+                stages=("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan"))
 
 
 def load_peaks():
@@ -420,8 +440,11 @@ def run_gpu(args, cfg, rank, world, local_rank):
     # ---- per-kernel durations: the same steps, one stage per launch ---------
     # A GPU-side sleep before each step lets the host enqueue all four stages
     # (and the events between them) first, so no host launch gap lands inside
-    # an event pair.
-    nst = len(binding.STAGES)
+    # an event pair.  Stage names follow the call's layout (the single-pass
+    # layout runs stages 1-3 of the four-kernel sequence as one kernel, plus the
+    # block-factored scan of the listed steep tiles).
+    names = work_model(cfg, final_state=want_final, lay=lay)["stages"]
+    nst = len(names)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
@@ -432,9 +455,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
             step(stage=s)
             ev[k][s + 1].record(stream)
     torch.cuda.synchronize()
-    kern_ms = {binding.STAGES[s]: statistics.mean(ev[k][s].elapsed_time(ev[k][s + 1])
-                                                  for k in range(args.steps))
-               for s in range(nst)}
+    kern_ms = {names[s]: statistics.mean(ev[k][s].elapsed_time(ev[k][s + 1]) for k in range(args.steps))
+               for s in range(nst) if names[s] is not None}
     barrier()
 
     # ---- end to end through the public call, host buffers ------------------
@@ -508,6 +530,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "gpu_launches": args.steps * lay.launches,
         "tensor_core": bool(lay.tensor_core),
         "fused_state": bool(lay.fused_state),
+        "single_pass": bool(lay.single_pass),
+        "scan_engine": binding.SCAN_ENGINES.get(lay.scan_engine, lay.scan_engine),
         "e2e": {"value": job_rate(world, tokens_step, args.steps, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clocks,

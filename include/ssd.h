@@ -51,7 +51,7 @@ extern "C" {
 typedef enum {
     SSD_OK = 0,
     SSD_ERR_NULL_ARG = 1,       /* a required pointer is NULL                    */
-    SSD_ERR_INVALID_DIM = 2,    /* a size is <= 0, H % G != 0, T % chunk_len != 0 */
+    SSD_ERR_INVALID_DIM = 2,    /* a size is <= 0 or H % G != 0                  */
     SSD_ERR_UNSUPPORTED = 3,    /* sizes outside the supported set (see below)   */
     SSD_ERR_MISALIGNED = 4,     /* a pointer is not 16-byte aligned              */
     SSD_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed          */
@@ -75,7 +75,11 @@ typedef struct {
 
 /*
  * Supported sizes (anything else returns SSD_ERR_UNSUPPORTED):
- *   chunk_len in {32, 64, 128, 256}, seqlen % chunk_len == 0 (else INVALID_DIM);
+ *   chunk_len in {32, 64, 128, 256}; any seqlen >= 1 -- when seqlen is not a
+ *   multiple of chunk_len the full chunks run as below and the last
+ *   seqlen mod chunk_len tokens run as the recurrence itself from the state the
+ *   full chunks leave (one more launch), which needs dstate in {8, 16, 32, 64}
+ *   or a multiple of 64 and headdim * max(1, dstate / 64) <= 1024;
  *   1 <= headdim <= 256, 1 <= dstate <= 256; nheads % ngroups == 0;
  *   SSD_BF16 additionally: headdim % 8 == 0 and dstate % 8 == 0.
  * The tensor-core path runs for SSD_BF16 with headdim == 64,
@@ -213,6 +217,59 @@ SSD_API ssd_status_t ssd_step(const ssd_dims_t *dims, const void *x_t, const flo
                               const float *A, const void *B_t, const void *C_t, const float *D,
                               float *state, void *y_t, void *stream);
 
+/*
+ * ssd_forward_block -- the scan together with its neighbours in the Mamba-2
+ * block (aifetchly blog "Mamba-2 Architecture: State Space Duality Explained",
+ * "Step 2: Full Mamba-2 Block with Gated Projections": softplus on dt before the
+ * SSD call; the SSD output gated by silu of the z branch, then RMSNorm over the
+ * token's d_inner = H * P values; akillness.github.io "State Space Duality and
+ * Mamba-2", the block diagram: "Element-wise Gating", RMSNorm):
+ *
+ *   dt_eff = softplus(dt + dt_bias)        (each part only when requested)
+ *   y      = the scan of ssd_forward with dt_eff
+ *   g      = y * silu(z),  silu(z) = z / (1 + e^-z)            (if z != NULL)
+ *   rstd_t = 1 / sqrt(mean over the token's H*P values of g^2 + norm_eps)
+ *   y_out  = g * rstd_t * norm_weight  (norm_apply != 0)
+ *          = g * norm_weight           (norm_apply == 0: rstd_t goes to
+ *                                       rstd_out and the caller applies it; it
+ *                                       is one factor per token, so it can be
+ *                                       applied to the rows of the next linear
+ *                                       layer's output instead)
+ *          = g                         (norm_weight == NULL)
+ *
+ *   opts       NULL = no neighbours (then this is ssd_forward_ws);
+ *              dt_bias [H] fp32 or NULL; dt_softplus nonzero for softplus;
+ *              z [B, T, H, P] dtype or NULL; norm_weight [H * P] fp32 or NULL;
+ *              norm_eps > 0 when norm_weight is given (else
+ *              SSD_ERR_INVALID_DIM); rstd_out [B, T] fp32 (required when
+ *              norm_weight is given and norm_apply == 0, else SSD_ERR_NULL_ARG;
+ *              optional otherwise); reserved0 must be 0.
+ *   workspace  ssd_block_workspace_bytes bytes, 256-byte aligned, or NULL:
+ *              then it is allocated stream-ordered on `stream` and released
+ *              before return, as in ssd_forward.
+ * Every other argument is that of ssd_forward.  The final state is the scan's.
+ * Accuracy: the bounds of ssd_forward, on y_out against the same chain in fp64.
+ */
+typedef struct {
+    const float *dt_bias;
+    int32_t dt_softplus;
+    int32_t norm_apply;
+    const void *z;
+    const float *norm_weight;
+    float norm_eps;
+    int32_t reserved0;
+    float *rstd_out;
+} ssd_block_opts_t;
+
+SSD_API size_t ssd_block_workspace_bytes(const ssd_dims_t *dims, int chunk_len,
+                                         const ssd_block_opts_t *opts);
+SSD_API ssd_status_t ssd_forward_block(const ssd_dims_t *dims, const void *x, const float *dt,
+                                       const float *A, const void *Bm, const void *Cm,
+                                       const float *D, int chunk_len, const float *init_state,
+                                       void *y_out, float *final_state_out,
+                                       const ssd_block_opts_t *opts, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace one call needs (0 if the arguments are invalid). */
 SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
 
@@ -235,7 +292,29 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * per-chunk states then never
  * reach memory, the states region is empty (states_offset == s_in_offset) and
  * stage 2 of ssd_forward_stage does nothing.
+ * `single_pass` is 1 when chunk state, state passing and chunk scan run as ONE
+ * kernel (bf16, headdim 64, dstate 128, chunk_len 128 / 256, an even number of
+ * heads per group, and at least 40% as many (batch, head pair) chains as the
+ * GPU has SMs): each chunk's state is carried to the next through an fp32
+ * slot per (batch, head) in the workspace, so neither the per-chunk states nor
+ * the incoming states reach memory (w, alpha and states are not written, s_in
+ * only for chunks with a tile the block-factored scan finishes).  Stage 1 of
+ * ssd_forward_stage then runs that kernel, stage 2 nothing, and stage 3 the
+ * block-factored scan of the tiles it listed.  `scan_engine` names the kernel
+ * that computes y.  `chunk_len` is the chunk length the kernels run with: the
+ * caller's, except that SSD_BF16 with chunk_len 64 runs the tensor-core
+ * kernels with 128-token chunks (their tile height; two of the caller's chunks
+ * per tile, the same recurrence), and the arrays above then describe 128-token
+ * chunks (nc = T / 128).
  */
+typedef enum {
+    SSD_ENGINE_SIMT = 0,            /* chunk scan on the CUDA cores                     */
+    SSD_ENGINE_TILE = 1,            /* tensor-core scan, one 128-row tile per work item */
+    SSD_ENGINE_BLOCK_FACTORED = 2,  /* tensor-core scan, block-factored decay           */
+    SSD_ENGINE_CHUNK_WIDE = 3,      /* tensor-core scan, whole chunk, shared scores     */
+    SSD_ENGINE_SINGLE_PASS = 4      /* chunk state + state passing + scan in one kernel */
+} ssd_scan_engine_t;
+
 typedef struct {
     size_t total_bytes;
     size_t l_offset, w_offset, dtq_offset, beta_offset, alpha_offset, states_offset, s_in_offset;
@@ -244,6 +323,9 @@ typedef struct {
     int32_t launches;
     int32_t states_dtype; /* element type of states: SSD_F32 or SSD_BF16 */
     int32_t fused_state;
+    int32_t single_pass;  /* 1: stages 1-3 run as one kernel (see below)   */
+    int32_t scan_engine;  /* ssd_scan_engine_t of the chunk scan            */
+    int32_t chunk_len;    /* chunk length the kernels use (see below)       */
 } ssd_workspace_layout_t;
 
 SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,

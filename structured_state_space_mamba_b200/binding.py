@@ -22,7 +22,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
 
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
            "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
-           "ssd_forward_static", "ssd_step")
+           "ssd_forward_static", "ssd_step", "ssd_forward_block", "ssd_block_workspace_bytes")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -41,7 +41,20 @@ class WorkspaceLayout(ctypes.Structure):
                 ("states_offset", ctypes.c_size_t), ("s_in_offset", ctypes.c_size_t),
                 ("s_in_dtype", ctypes.c_int32), ("tensor_core", ctypes.c_int32),
                 ("launches", ctypes.c_int32), ("states_dtype", ctypes.c_int32),
-                ("fused_state", ctypes.c_int32)]
+                ("fused_state", ctypes.c_int32), ("single_pass", ctypes.c_int32),
+                ("scan_engine", ctypes.c_int32), ("chunk_len", ctypes.c_int32)]
+
+
+# ssd_scan_engine_t: which kernel computes y
+SCAN_ENGINES = {0: "simt", 1: "tile", 2: "block_factored", 3: "chunk_wide", 4: "single_pass"}
+
+
+class BlockOpts(ctypes.Structure):
+    """ssd_block_opts_t: the scan's neighbours in the Mamba-2 block."""
+    _fields_ = [("dt_bias", ctypes.c_void_p), ("dt_softplus", ctypes.c_int32),
+                ("norm_apply", ctypes.c_int32), ("z", ctypes.c_void_p),
+                ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float),
+                ("reserved0", ctypes.c_int32), ("rstd_out", ctypes.c_void_p)]
 
 
 class SSDError(RuntimeError):
@@ -79,6 +92,11 @@ def load():
     lib.ssd_step.restype = ctypes.c_int
     lib.ssd_forward_stage.argtypes = [ctypes.c_int] + lib.ssd_forward_ws.argtypes
     lib.ssd_forward_stage.restype = ctypes.c_int
+    lib.ssd_forward_block.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp, vp, fp,
+                                      ctypes.POINTER(BlockOpts), vp, ctypes.c_size_t, vp]
+    lib.ssd_forward_block.restype = ctypes.c_int
+    lib.ssd_block_workspace_bytes.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(BlockOpts)]
+    lib.ssd_block_workspace_bytes.restype = ctypes.c_size_t
     lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
     lib.ssd_workspace_bytes.restype = ctypes.c_size_t
     lib.ssd_workspace_layout.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]
@@ -186,6 +204,58 @@ def forward(x, dt, A, B, C, D=None, chunk_len=256, init_state=None, return_final
     if return_final_state or final_out is not None:
         return y, fin
     return y
+
+
+def forward_block(x, dt, A, B, C, D=None, chunk_len=256, init_state=None, dt_bias=None,
+                  dt_softplus=False, z=None, norm_weight=None, norm_eps=1e-5, norm_apply=True,
+                  return_rstd=False, return_final_state=False, out=None, final_out=None,
+                  workspace=None, stream=None):
+    """The scan with its block neighbours through ``ssd_forward_block``:
+    softplus(dt + dt_bias) as the step size, then y * silu(z) and RMSNorm over
+    each token's H * P values with ``norm_weight`` [H*P] float32.  With
+    ``norm_apply=False`` the output is the gated, weighted y and the per-token
+    factor rstd [B, T] is returned for the caller to apply.
+    Returns ``out`` plus, as asked, the final state and rstd (in that order)."""
+    dims = _validate(x, dt, A, B, C, D, init_state)
+    dev = x.device
+    for name, t in (("dt_bias", dt_bias), ("norm_weight", norm_weight)):
+        if t is not None and (t.device != dev or t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {dev}")
+    if z is not None and (z.device != dev or z.dtype != x.dtype or z.shape != x.shape or not z.is_contiguous()):
+        raise ValueError("z must be a contiguous tensor like x")
+    y = out if out is not None else torch.empty_like(x)
+    fin = final_out
+    if fin is None and return_final_state:
+        fin = torch.empty((dims.batch, dims.nheads, dims.headdim, dims.dstate),
+                          dtype=torch.float32, device=dev)
+    rstd = None
+    if norm_weight is not None and (return_rstd or not norm_apply):
+        rstd = torch.empty((dims.batch, dims.seqlen), dtype=torch.float32, device=dev)
+    opts = BlockOpts(dt_bias=None if dt_bias is None else dt_bias.data_ptr(),
+                     dt_softplus=1 if dt_softplus else 0, norm_apply=1 if norm_apply else 0,
+                     z=None if z is None else z.data_ptr(),
+                     norm_weight=None if norm_weight is None else norm_weight.data_ptr(),
+                     norm_eps=float(norm_eps), reserved0=0,
+                     rstd_out=None if rstd is None else rstd.data_ptr())
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = load().ssd_forward_block(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                      _ptr(D), int(chunk_len), _ptr(init_state), _ptr(y), _ptr(fin),
+                                      ctypes.byref(opts), _ptr(workspace), wsz, ctypes.c_void_p(stream))
+    _check(st)
+    res = [y]
+    if return_final_state or final_out is not None:
+        res.append(fin)
+    if rstd is not None:
+        res.append(rstd)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def block_workspace_bytes(dims: Dims, chunk_len: int, dt_transform: bool) -> int:
+    opts = BlockOpts(dt_softplus=1 if dt_transform else 0)
+    return int(load().ssd_block_workspace_bytes(ctypes.byref(dims), int(chunk_len), ctypes.byref(opts)))
 
 
 def forward_ws(*args, **kwargs):

@@ -15,6 +15,18 @@
 //             block-factored scan), then r.  The reference r is 0, or l[127]
 //             when -l[Q-1] reaches kScanSteep but neither tile's own decay
 //             range does
+//   fused mode (the single-pass kernel of k_tc_chunk_fused.cu): the same gq
+//             layout with a reference that also keeps the chunk state exact --
+//             r = 0 or l[127] as above, otherwise r = l[Q-1] (then every
+//             g_s <= dt_s); a tile is flagged only when a factor it needs,
+//             u_t = exp(l_t - r) or g_s, would reach e^kScanSteep (a zero dt
+//             is handled by the scan itself); w and alpha are not written, and
+//             dtq and beta only for chunks with a flagged tile (the
+//             block-factored scan reads them); the pairs' chain flags are
+//             reset to 0
+// With a dt bias or softplus requested (the Mamba-2 block's dt preprocessing),
+// every use above takes dt_eff = softplus(dt + dt_bias) (or dt + dt_bias), and
+// dt_eff is also written in dt's layout for the scans that read dt directly.
 // The decay between tokens s <= t of one chunk is exp(l[t] - l[s]): the
 // segment-sum mask L of akillness.github.io "State Space Duality and Mamba-2",
 // "The Scalar-Identity Structural Constraint" (the product of the a_k is
@@ -41,11 +53,18 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
                     float *__restrict__ l_out, float *__restrict__ w_out,
                     float *__restrict__ dtq_out, float *__restrict__ beta_out,
                     float *__restrict__ alpha_out, float *__restrict__ gq_out,
-                    int *__restrict__ nsteep) {
+                    int *__restrict__ nsteep, unsigned int *__restrict__ chain_flags,
+                    const float *__restrict__ dt_bias, int dt_softplus, float *__restrict__ dt_eff) {
     constexpr int Q = 32 * E;
+    const bool fused = chain_flags != nullptr;
     // the chunk-wide scan's steep-tile list starts empty (that kernel runs after
     // this one in stream order)
     if (nsteep && (blockIdx.x | blockIdx.y | blockIdx.z | threadIdx.x) == 0) *nsteep = 0;
+    // fused mode: the chain flags of this CTA's 4 head pairs start at 0
+    if (fused && blockIdx.x == 0 && threadIdx.x < kHeads / 2) {
+        const int pair = blockIdx.y * (kHeads / 2) + threadIdx.x;
+        if (pair < d.H / 2) chain_flags[int64_t(blockIdx.z) * (d.H / 2) + pair] = 0u;
+    }
     __shared__ float s_dt[Q][kHeads + 1];
     const int c = blockIdx.x, b = blockIdx.z;
     const int h0 = blockIdx.y * kHeads;
@@ -58,10 +77,23 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
         const int j = threadIdx.x % kHeads;
         const int i0 = threadIdx.x / kHeads;
         float v[kIters];
+        const float bias = (dt_bias && h0 + j < d.H) ? __ldg(dt_bias + h0 + j) : 0.f;
 #pragma unroll
         for (int k = 0; k < kIters; ++k) {
             const int i = i0 + k * (kThreads / kHeads);
             v[k] = h0 + j < d.H ? __ldg(dt + off_dt(d, b, t0 + i) + h0 + j) : 0.f;
+        }
+        if (dt_bias || dt_softplus) {
+            // the step size the scan uses: softplus(dt + dt_bias), written as
+            // max(v, 0) + log1p(e^-|v|) (no overflow for large v)
+#pragma unroll
+            for (int k = 0; k < kIters; ++k) {
+                if (h0 + j >= d.H) continue;
+                float e = v[k] + bias;
+                if (dt_softplus) e = fmaxf(e, 0.f) + log1pf(expf(-fabsf(e)));
+                v[k] = e;
+                if (dt_eff) dt_eff[off_dt(d, b, t0 + i0 + k * (kThreads / kHeads)) + h0 + j] = e;
+            }
         }
 #pragma unroll
         for (int k = 0; k < kIters; ++k) s_dt[i0 + k * (kThreads / kHeads)][j] = v[k];
@@ -71,7 +103,7 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
     if (h >= d.H) return;
     const float a = __ldg(A + h);
     const int64_t base = off_lq(d, b, h, c);
-    float lv[E], dts[E];
+    float lv[E], dts[E], bend[E];
     float carry = 0.f;
 #pragma unroll
     for (int k = 0; k < E; ++k) {
@@ -83,15 +115,51 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
             if (lane >= o) incl += n;
         }
         lv[k] = carry + incl;
-        const float blk_end = __shfl_sync(0xffffffffu, lv[k], 31);  // l at token 32k+31
+        bend[k] = __shfl_sync(0xffffffffu, lv[k], 31);  // l at token 32k+31
         l_out[base + 32 * k + lane] = lv[k];
-        dtq_out[base + 32 * k + lane] = dts[k];
-        beta_out[base + 32 * k + lane] = __expf(blk_end - lv[k]) * dts[k];
-        carry = blk_end;
+        carry = bend[k];
     }
     const float last = carry;  // l[Q-1]
+    if (fused && E >= 4) {
+        float *g = gq_out + ((int64_t(b) * d.H + h) * d.nc + c) * chunk_gq(Q);
+        // r = 0, or l[127] when only the whole chunk's decay reaches the limit,
+        // else l[Q-1] (every g_s <= dt_s: the chunk state stays exact)
+        const float l127 = __shfl_sync(0xffffffffu, lv[3], 31);
+        float r;
+        if (-last < kScanSteep) r = 0.f;
+        else if (E == 8 && -l127 < kScanSteep && l127 - last < kScanSteep) r = l127;
+        else r = last;
+        bool any = false;
 #pragma unroll
-    for (int k = 0; k < E; ++k) w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
+        for (int k = 0; k < E; ++k) {
+            g[32 * k + lane] = __expf(fminf(r - lv[k], 80.f)) * dts[k];
+            if ((k & 3) == 3) {  // last 32 tokens of a 128-token tile
+                const float lfirst = __shfl_sync(0xffffffffu, lv[k - 3], 0);
+                const bool steep = lfirst - r >= kScanSteep || r - bend[k] >= kScanSteep;
+                any |= steep;
+                if (lane == 0) g[Q + (k >> 2)] = steep ? 1.f : 0.f;
+            }
+        }
+        if (lane == 0) {
+            if (E == 4) g[Q + 1] = 0.f;
+            g[Q + 2] = r;
+            g[Q + 3] = 0.f;
+        }
+        if (any) {  // the block-factored scan recomputes this chunk's flagged tiles
+#pragma unroll
+            for (int k = 0; k < E; ++k) {
+                dtq_out[base + 32 * k + lane] = dts[k];
+                beta_out[base + 32 * k + lane] = __expf(bend[k] - lv[k]) * dts[k];
+            }
+        }
+        return;
+    }
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        dtq_out[base + 32 * k + lane] = dts[k];
+        beta_out[base + 32 * k + lane] = __expf(bend[k] - lv[k]) * dts[k];
+        w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
+    }
     if (lane == 0) alpha_out[off_alpha(d, b, h, c)] = __expf(last);
     if (gq_out && E >= 4) {
         float *g = gq_out + ((int64_t(b) * d.H + h) * d.nc + c) * chunk_gq(Q);
@@ -122,13 +190,15 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
 
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *dtq, float *beta, float *alpha, float *gq,
-                                int *nsteep, cudaStream_t stream) {
+                                int *nsteep, unsigned int *chain_flags, const float *dt_bias,
+                                int dt_softplus, float *dt_eff, cudaStream_t stream) {
+    if (chain_flags && (d.Q < 128 || !gq)) return cudaErrorInvalidValue;
     dim3 grid(d.nc, (d.H + kHeads - 1) / kHeads, d.B);
     switch (d.Q) {
-        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
-        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
-        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
-        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep); break;
+        case 32: chunk_cumsum_kernel<1><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, chain_flags, dt_bias, dt_softplus, dt_eff); break;
+        case 64: chunk_cumsum_kernel<2><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, chain_flags, dt_bias, dt_softplus, dt_eff); break;
+        case 128: chunk_cumsum_kernel<4><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, chain_flags, dt_bias, dt_softplus, dt_eff); break;
+        case 256: chunk_cumsum_kernel<8><<<grid, kThreads, 0, stream>>>(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, chain_flags, dt_bias, dt_softplus, dt_eff); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -1,0 +1,809 @@
+// k_tc_chunk_fused.cu -- the whole chunked SSD forward pass after the cumsum in
+// ONE persistent tensor-core kernel: chunk state, state passing and chunk scan.
+//
+// For batch b, head h (group g), chunk c with incoming state s_in_c (P x N):
+//   y_t = exp(l_t) C_t s_in_c^T + sum_{s <= t in c} exp(l_t - l_s) dt_s (C_t . B_s) x_s + D_h x_t
+//   s_in_{c+1} = exp(l_last) s_in_c + sum_{s in c} exp(l_last - l_s) dt_s x_s B_s^T
+// (the chunked SSD algorithm -- aifetchly blog "Mamba-2 Architecture: State
+// Space Duality Explained", "The Chunked SSD Algorithm", steps 1 and 2: the
+// masked product (L o C B^T) X inside the chunk, the chunk state and the
+// hand-off between chunks; the decay between s and t is exp(l_t - l_s) with l
+// the cumulative log-decay, akillness.github.io "State Space Duality and
+// Mamba-2", "The Scalar-Identity Structural Constraint").
+//
+// With the chunk's reference r (chosen by the cumsum kernel so that no factor
+// overflows), u_t = exp(l_t - r), g_s = exp(r - l_s) dt_s and X''_s = g_s x_s,
+// every decay factorises as exp(l_t - l_s) dt_s = u_t g_s, and with the state
+// in reference units S' = e^r s_in (kept transposed, P x N per head, in TMEM):
+//   per 128-token tile k of the chunk (S'_0 = e^r s_in_c):
+//     Y_k    = (C_k B_k^T o M) X''_k + C_k S'_k^T,   y_t = u_t Y_k[t] + D_h x_t
+//     S'_k+1 = S'_k + X''_k^T B_k
+//   s_in_{c+1} = exp(l_last - r) S'_end.
+// The masked scores C_k B_k^T o M do not depend on the head, so the work is
+// organised by PAIRS of heads of one group: every product has N = 128 (two
+// heads x P = 64) and the scores are built once for both heads.  A chain is the
+// chunk sequence of one (b, head pair); its state stays in tensor memory from
+// chunk to chunk while one CTA walks it (rescaled to each chunk's reference).
+// With G CTAs (G <= chains), CTA k takes the k-th G-th of the chain-major
+// (chain, chunk) list: at least one chain's length, so it holds at most one
+// chain that began on CTA k - 1.  It walks that chain last, after a state hand-
+// off through the chain's fp32 slot in global memory (release / acquire flag,
+// bounded wait), and the chain it shares with CTA k + 1 first.  x is read once
+// and y written once; no chunk state reaches HBM.
+//
+// Tiles the cumsum kernel flagged as steep (a factor would pass e^72) are not
+// stored here: the state path stays exact (r keeps every g_s <= 1 there), the
+// kernel writes s_in_c in bf16 for the listed chunk, and the block-factored
+// scan (k_tc_chunk_scan4.cu, list mode) computes those tiles' y afterwards.
+//
+// Per tile (128 tokens of one chunk of one chain), on the tensor cores:
+//   CB  C_k B_k^T      -> Y buffer (fp32), packed to bf16 P in TMEM by the
+//                         score warps with the causal mask (diagonal included)
+//   Z   X''_k^T B_k    -> ACC += (M = 128: both heads' P rows, N = dstate)
+//   PX  P X''_k        -> Y buffer (N = 128: both heads)
+//   CS  C_k S'^T       -> Y buffer += (S' read back from ACC, written into the
+//                         tile's B region once Z has read it)
+// Tensor memory (512 columns): Y buffers [0,128) and [128,256) alternating per
+// tile, ACC [256, 256 + N), P buffers [384,448) and [448,512).
+//
+// Roles (14 warps, at most four per SM sub-partition, so 128 registers each):
+// warp 0 TMA producer; warp 1 MMA issuer; warps 2-5 scale x by g, then convert
+// the scores; warps 6-9 state (chain in/out, S' read-back); warps 10-13
+// epilogue (y = u Y + D x, staged and TMA-stored).
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+#include "tc_scan_common.cuh"
+#include "tma_host.h"
+
+namespace ssd {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 480;
+constexpr int kRows = 128;
+constexpr uint32_t kColAcc = 256;
+__device__ __forceinline__ uint32_t ycol(int yb) { return yb ? 128u : 0u; }
+__device__ __forceinline__ uint32_t pcol(int yb) { return yb ? 448u : 384u; }
+constexpr int kBarState = 1;  // named barrier of the four state warps
+
+// Shared memory: a ring of kCBStages slots {C_k, B_k} (L2-resident inputs,
+// released once the tile's products are done; S'_k goes into the B_k half once
+// Z has read it) and a deeper ring of kXStages slots for the pair's x rows (the
+// HBM stream: x, scaled in place to X'', then overwritten row by row with y
+// and written out from there); barriers.
+template <int NS>
+struct FusedLayout {
+    static constexpr int kSlabs = NS / 64;
+    static constexpr uint32_t kCB = uint32_t(kRows) * NS * 2;  // C_k or B_k
+    static constexpr uint32_t kCBSlot = 2 * kCB;
+    static constexpr uint32_t kX = 2u * kRows * 128;            // x of the pair
+    static constexpr int kCBStages = 2;
+    static constexpr int kXStages = NS >= 128 ? 3 : 4;
+    static constexpr uint32_t kXOff = kCBStages * kCBSlot;
+    static constexpr uint32_t kBar = kXOff + kXStages * kX;
+    static constexpr uint32_t kTotal = kBar + 256 + 1024;
+};
+
+// Work assignment.  The (chain, chunk) items, chain = (b, head pair p), are
+// listed chain-major; CTA k takes items [k I / G, (k + 1) I / G) (I items, G
+// CTAs, with G <= the number of chains, so every range holds at least one
+// chain's worth of chunks).  A range is cut into segments, each a run of chunks
+// [c0, c1) of one chain, processed in this order: the range's LAST chain
+// (starting at chunk 0), the chains in the middle (whole), and last the range's
+// FIRST chain, which continues from chunk c0 > 0 the chain whose beginning is
+// the first segment processed by CTA k - 1.  So the one segment of a CTA that
+// needs a state from another CTA runs last, and the segment that supplies it
+// runs first on its CTA; the state crosses between them once, through the
+// chain's fp32 slot in global memory (flag = chunks published).
+struct Seg {
+    int b, p, c0, c1;
+};
+struct Range {
+    int cf, cfc, cl, clc;  // first chain and its first chunk; last chain and its end chunk
+    int nseg;
+};
+__device__ __forceinline__ Range cta_range(const Dims &d) {
+    const long long chains = (long long)d.B * (d.H / 2);
+    const long long items = chains * d.nc;
+    const long long i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
+    Range r;
+    r.cf = int(i0 / d.nc);
+    r.cfc = int(i0 % d.nc);
+    r.cl = int((i1 - 1) / d.nc);
+    r.clc = int((i1 - 1) % d.nc) + 1;
+    r.nseg = r.cf == r.cl ? 1 : r.cl - r.cf + 1;
+    return r;
+}
+__device__ __forceinline__ Seg seg_at(const Range &r, int s, const Dims &d) {
+    const int np = d.H / 2;
+    int ch, c0, c1;
+    if (r.cf == r.cl) {
+        ch = r.cf; c0 = r.cfc; c1 = r.clc;
+    } else if (s == 0) {
+        ch = r.cl; c0 = 0; c1 = r.clc;
+    } else if (s < r.cl - r.cf) {
+        ch = r.cf + s; c0 = 0; c1 = d.nc;
+    } else {
+        ch = r.cf; c0 = r.cfc; c1 = d.nc;
+    }
+    Seg g;
+    g.b = ch / np;
+    g.p = ch % np;
+    g.c0 = c0;
+    g.c1 = c1;
+    return g;
+}
+
+// Walks the CTA's tiles in order (segment, chunk, tile): roles that prefetch
+// the next tile's per-token factors keep one walker a tile ahead.
+struct TileWalk {
+    int sg, c, k;
+    Seg T;
+    bool valid;
+    __device__ __forceinline__ void start(const Range &R, const Dims &d) {
+        sg = 0;
+        k = 0;
+        valid = R.nseg > 0;
+        if (valid) {
+            T = seg_at(R, 0, d);
+            c = T.c0;
+        }
+    }
+    __device__ __forceinline__ void next(const Range &R, const Dims &d, int ntile) {
+        if (!valid) return;
+        if (++k < ntile) return;
+        k = 0;
+        if (++c < T.c1) return;
+        if (++sg < R.nseg) {
+            T = seg_at(R, sg, d);
+            c = T.c0;
+        } else {
+            valid = false;
+        }
+    }
+};
+
+// fp32 32 x 32 block (one TMEM row per lane) -> bf16 pairs, all columns or,
+// on the diagonal, columns e <= lane only.
+template <bool kDiag>
+__device__ __forceinline__ void mask_pack(const uint32_t (&v)[32], int lane, uint32_t (&pk)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float a = (!kDiag || 2 * e <= lane) ? __uint_as_float(v[2 * e]) : 0.f;
+        const float b = (!kDiag || 2 * e + 1 <= lane) ? __uint_as_float(v[2 * e + 1]) : 0.f;
+        pk[e] = pack_bf16x2(a, b);
+    }
+}
+
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int *f) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(unsigned int *f, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+// Bounded wait until *f >= want (the predecessor ticket has published); sets
+// bit 0 of *err and returns false after kWaitLimitNs, or early once another
+// wait on the device has failed.
+__device__ __noinline__ bool wait_flag(const unsigned int *f, unsigned int want, unsigned int *err) {
+    if (ld_acquire(f) >= want) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(64);
+        if (ld_acquire(f) >= want) return true;
+        if ((i & 15u) == 0) {
+            const uint64_t el = global_ns() - t0;
+            if (el > kWaitLimitNs) break;
+            if (el > kErrPollNs && device_failed(err)) return false;
+        }
+    }
+    if (err) atomicOr(err, 1u);
+    return false;
+}
+
+template <int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
+                   Dims d, const __nv_bfloat16 *__restrict__ x, const float *__restrict__ gq,
+                   const float *__restrict__ lcum, const float *__restrict__ Dskip,
+                   const float *__restrict__ h0, float *__restrict__ fin, float *__restrict__ chain,
+                   unsigned int *__restrict__ flags, __nv_bfloat16 *__restrict__ s_in,
+                   int *__restrict__ nsteep, long long *__restrict__ steep_items, int max_steep,
+                   unsigned int *err) {
+    using L = FusedLayout<NS>;
+    constexpr int kCBS = L::kCBStages, kXS = L::kXStages;
+    if (device_failed(err)) return;  // an earlier wait expired: skip all work
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint64_t *cb_full = bars, *cb_free = cb_full + kCBS;                        // [kCBS]
+    uint64_t *x_full = cb_free + kCBS, *scaled = x_full + kXS, *x_free = scaled + kXS;  // [kXS]
+    uint64_t *cbm_done = x_free + kXS, *p_ready = cbm_done + 2, *acc_full = p_ready + 2,
+             *y_free = acc_full + 2;                                             // [2]
+    uint64_t *acc_ready = y_free + 2, *z_done = acc_ready + 1, *sp_ready = z_done + 1, *done = sp_ready + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
+    volatile int *state_ok = reinterpret_cast<volatile int *>(done + 2);
+    auto cb_at = [&](uint32_t kt) { return smem + (kt % kCBS) * L::kCBSlot; };
+    auto x_at = [&](uint32_t kt) { return smem + L::kXOff + (kt % kXS) * L::kX; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int Q = d.Q, ntile = Q / kRows, ngq = chunk_gq(Q);
+    const int np = d.H / 2;
+    const Range R = cta_range(d);
+
+    if (tid == 0) {
+        for (int i = 0; i < kCBS; ++i) {
+            mbar_init(&cb_full[i], 1);
+            mbar_init(&cb_free[i], 1);  // the tile's products
+        }
+        for (int i = 0; i < kXS; ++i) {
+            mbar_init(&x_full[i], 1);
+            mbar_init(&scaled[i], 128);
+            mbar_init(&x_free[i], 4);  // the 4 epilogue warps' y stores have read the slot
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&cbm_done[i], 1);
+            mbar_init(&p_ready[i], 128);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&y_free[i], 128);
+        }
+        mbar_init(acc_ready, 128);
+        mbar_init(z_done, 1);
+        mbar_init(sp_ready, 128);
+        mbar_init(done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_c);
+        tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_y);
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    // Every role walks the same sequence: segments 0 .. R.nseg - 1, chunks
+    // c0 .. c1 - 1 of each, tiles 0 .. ntile - 1 of each chunk (tile counter kt;
+    // C/B slot kt % kCBS, x slot kt % kXS, Y and P buffers kt % 2).
+    if (warp == 0 || warp == 14) {
+        // ============================ producers (TMA) =============================
+        // warp 0: the pair's x rows into the x ring; warp 14: C_k and B_k into the
+        // C/B ring.  Separate threads, so the deeper x ring runs ahead of C/B.
+        if (lane == 0) {
+            const bool xp = warp == 0;
+            uint32_t kt = 0;
+            bool ok = true;
+            for (int sg = 0; sg < R.nseg && ok; ++sg) {
+                const Seg T = seg_at(R, sg, d);
+                const int g = (2 * T.p) / d.r;
+                for (int c = T.c0; c < T.c1 && ok; ++c)
+                    for (int k = 0; k < ntile; ++k) {
+                        const int row = T.b * d.T + c * Q + k * kRows;
+                        if (xp) {
+                            if (!mbar_wait(&x_free[kt % kXS], ((kt / kXS) & 1) ^ 1, err)) { ok = false; break; }
+                            uint8_t *xs = x_at(kt);
+                            uint64_t *fb = &x_full[kt % kXS];
+                            mbar_expect_tx(fb, L::kX);
+                            tma_load_3d(xs, &tm_x, fb, 0, 2 * T.p, row);
+                            tma_load_3d(xs + kRows * 128, &tm_x, fb, 0, 2 * T.p + 1, row);
+                        } else {
+                            if (!mbar_wait(&cb_free[kt % kCBS], ((kt / kCBS) & 1) ^ 1, err)) { ok = false; break; }
+                            uint8_t *cs = cb_at(kt);
+                            uint64_t *fb = &cb_full[kt % kCBS];
+                            mbar_expect_tx(fb, L::kCBSlot);
+#pragma unroll
+                            for (int sl = 0; sl < L::kSlabs; ++sl) {
+                                tma_load_3d(cs + sl * kRows * 128, &tm_c, fb, sl * 64, g, row);
+                                tma_load_3d(cs + L::kCB + sl * kRows * 128, &tm_b, fb, sl * 64, g, row);
+                            }
+                        }
+                        ++kt;
+                    }
+            }
+            // every load issued has landed before the CTA exits
+            const uint32_t depth = xp ? kXS : kCBS;
+            for (uint32_t i = kt > depth ? kt - depth : 0; i < kt; ++i)
+                mbar_wait(xp ? &x_full[i % kXS] : &cb_full[i % kCBS], (i / depth) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer ===============================
+        if (lane == 0) {
+            const uint32_t idCB = idesc_bf16_f32(kRows, kRows, 0, 0);
+            const uint32_t idZ = idesc_bf16_f32(128, NS, 1, 1);
+            const uint32_t idPX = idesc_bf16_f32(kRows, 128, 0, 1);
+            const uint32_t idCS = idesc_bf16_f32(kRows, 128, 0, 0);
+            // one tile of lookahead: C_{k+1} B_{k+1}^T is issued between tile k's
+            // Z and its C S'^T, so tile k+1's score conversion overlaps tile k's
+            // state hand-off
+            uint32_t ntot = 0;
+            for (int sg = 0; sg < R.nseg; ++sg) {
+                const Seg T = seg_at(R, sg, d);
+                ntot += uint32_t(T.c1 - T.c0) * ntile;
+            }
+            auto issue_cb = [&](uint32_t t) -> bool {
+                const int yb = t & 1;
+                if (!mbar_wait(&cb_full[t % kCBS], (t / kCBS) & 1, err) ||
+                    !mbar_wait(&y_free[yb], ((t >> 1) & 1) ^ 1, err))
+                    return false;
+                tc_fence_after();
+                const uint32_t cA = smem_u32(cb_at(t)), bA = cA + L::kCB;
+#pragma unroll
+                for (int kk = 0; kk < NS / 16; ++kk)
+                    mma_bf16_ss(tmem + ycol(yb), kmajor_desc(cA, kk, kRows, NS), kmajor_desc(bA, kk, kRows, NS),
+                                idCB, kk > 0 ? 1u : 0u);
+                mma_commit(&cbm_done[yb]);
+                return true;
+            };
+            bool ok = ntot == 0 || issue_cb(0);
+            for (uint32_t kt = 0; kt < ntot && ok; ++kt) {
+                const uint32_t cs = kt % kCBS, xs = kt % kXS, xph = (kt / kXS) & 1;
+                const int yb = kt & 1;
+                const uint32_t yph = (kt >> 1) & 1;
+                const uint32_t cA = smem_u32(cb_at(kt)), bA = cA + L::kCB, xA = smem_u32(x_at(kt));
+                const uint32_t yacc = tmem + ycol(yb);
+                // Y = P X''_k (needs no state)
+                if (!mbar_wait(&scaled[xs], xph, err) || !mbar_wait(&p_ready[yb], yph, err)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    mma_bf16_ts(yacc, tmem + pcol(yb) + kk * 8, smem_desc(xA + kk * 2048, kRows * 128, 1024, kSw128),
+                                idPX, kk > 0 ? 1u : 0u);
+                // Z: ACC (= S'_k, kept there by the state warps) += X''_k^T B_k
+                if (!mbar_wait(acc_ready, kt & 1, err)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    mma_bf16_ss(tmem + kColAcc, smem_desc(xA + kk * 2048, kRows * 128, 1024, kSw128),
+                                smem_desc(bA + kk * 2048, kRows * 128, 1024, kSw128), idZ, 1u);
+                mma_commit(z_done);
+                if (kt + 1 < ntot && !issue_cb(kt + 1)) { ok = false; break; }
+                // Y += C_k S'_k^T, S'_k (bf16) written by the state warps into the
+                // tile's B region once Z has read B_k
+                if (!mbar_wait(sp_ready, kt & 1, err)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < NS / 16; ++kk)
+                    mma_bf16_ss(yacc, kmajor_desc(cA, kk, kRows, NS), kmajor_desc(bA, kk, 128, NS), idCS, 1u);
+                mma_commit(&acc_full[yb]);
+                mma_commit(&cb_free[cs]);
+            }
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);
+        }
+    } else if (warp < 6) {
+        // ========================= scale x, then the scores =========================
+        // Per tile: X''_s = g_s x_s in place (16-byte chunk ci of the pair's x
+        // region lies in row ci / 8: head ci / 1024, token (ci / 8) % 128; the
+        // swizzle only permutes chunks within a row), then fp32 C_k B_k^T -> bf16 P
+        // with the causal mask (diagonal included): warp qd owns rows 32 qd ..
+        // 32 qd + 31; a column block above the diagonal is zero.
+        const int i = tid - 2 * 32;  // 0..127
+        const int qd = warp & 3;
+        const uint32_t lane_base = uint32_t(qd * 32) << 16;
+        // g_s of this thread's 16 rows for tile w (both heads)
+        auto load_g = [&](const TileWalk &w, float (&gv)[16]) {
+            const float *g0 = gq + ((int64_t(w.T.b) * d.H + 2 * w.T.p) * d.nc + w.c) * ngq;
+            const float *g1 = g0 + int64_t(d.nc) * ngq;  // head 2p + 1
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+                gv[jj] = __ldg((jj < 8 ? g0 : g1) + w.k * kRows + (i >> 3) + 16 * (jj & 7));
+        };
+        TileWalk cur, nxt;
+        cur.start(R, d);
+        nxt = cur;
+        nxt.next(R, d, ntile);
+        float gv[16];
+        if (cur.valid) load_g(cur, gv);
+        bool ok = true;
+        for (uint32_t kt = 0; cur.valid && ok; ++kt, cur.next(R, d, ntile), nxt.next(R, d, ntile)) {
+            {
+                // the next tile's factors load while this tile is scaled and scored
+                float gn[16];
+                if (nxt.valid) load_g(nxt, gn);
+                if (!mbar_wait(&x_full[kt % kXS], (kt / kXS) & 1, err)) { ok = false; break; }
+                uint4 *q = reinterpret_cast<uint4 *>(x_at(kt));
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint4 v[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) v[jj] = q[i + 128 * (8 * half + jj)];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const float sc = gv[8 * half + jj];
+                        uint4 o;
+                        o.x = pack_bf16x2(bf16lo(v[jj].x) * sc, bf16hi(v[jj].x) * sc);
+                        o.y = pack_bf16x2(bf16lo(v[jj].y) * sc, bf16hi(v[jj].y) * sc);
+                        o.z = pack_bf16x2(bf16lo(v[jj].z) * sc, bf16hi(v[jj].z) * sc);
+                        o.w = pack_bf16x2(bf16lo(v[jj].w) * sc, bf16hi(v[jj].w) * sc);
+                        q[i + 128 * (8 * half + jj)] = o;
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) gv[jj] = gn[jj];
+                fence_proxy_async_smem();
+                mbar_arrive(&scaled[kt % kXS]);
+            }
+            // ---- masked scores: two blocks' loads in flight per wait ----
+            const int yb = kt & 1;
+            if (!mbar_wait(&cbm_done[yb], (kt >> 1) & 1, err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t src = tmem + lane_base + ycol(yb), dst = tmem + lane_base + pcol(yb);
+#pragma unroll
+            for (int cb = 0; cb < 4; cb += 2) {
+                uint32_t v0[32], v1[32];
+                if (cb <= qd) tmem_ld32_nowait(src + cb * 32, v0);
+                if (cb + 1 <= qd) tmem_ld32_nowait(src + (cb + 1) * 32, v1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int bb = 0; bb < 2; ++bb) {
+                    const int cbb = cb + bb;
+                    uint32_t pk[16];
+                    if (cbb > qd) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else if (cbb < qd) {
+                        mask_pack<false>(bb ? v1 : v0, lane, pk);
+                    } else {
+                        mask_pack<true>(bb ? v1 : v0, lane, pk);
+                    }
+                    tmem_st16(dst + cbb * 16, pk);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_ready[yb]);
+        }
+    } else if (warp < 10) {
+        // ================================= state =================================
+        // Thread m owns ACC row m: head 2p + m / 64, state row p = m % 64.  sp
+        // holds S'_k of the current tile (bf16 pairs of row m) until Z has read
+        // B_k; it then goes into the tile's B region as the K-major operand of
+        // C_k S'_k^T (slab n / 64, 16-byte chunk (n % 64) / 8 of row m, 128-byte
+        // swizzle).
+        const int m = 32 * (warp & 3) + lane;
+        const int jh = m >> 6, p = m & 63;
+        const uint32_t tacc = tmem + (uint32_t(32 * (warp & 3)) << 16) + kColAcc;
+        uint32_t kt = 0;
+        bool ok = true;
+        uint32_t sp[NS / 2];
+        auto pack32 = [&](int seg, const float (&v)[32]) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) sp[seg * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        };
+        auto put_bf16_row = [&](__nv_bfloat16 *dst, const float (&v)[32]) {
+            uint4 *o = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+                o[qq] = make_uint4(pack_bf16x2(v[8 * qq], v[8 * qq + 1]), pack_bf16x2(v[8 * qq + 2], v[8 * qq + 3]),
+                                   pack_bf16x2(v[8 * qq + 4], v[8 * qq + 5]), pack_bf16x2(v[8 * qq + 6], v[8 * qq + 7]));
+        };
+        for (int sg = 0; sg < R.nseg && ok; ++sg) {
+            const Seg T = seg_at(R, sg, d);
+            const int h = 2 * T.p + jh;
+            const int64_t row_off = ((int64_t(T.b) * d.H + h) * d.P + p) * NS;
+            // ---- ticket start: S'_0 = e^r s_in_c0 from h0 or the chain slot ----
+            {
+                const float *gqh = gq + ((int64_t(T.b) * d.H + h) * d.nc + T.c0) * ngq;
+                const bool steep = __ldg(gqh + Q) != 0.f || (ntile == 2 && __ldg(gqh + Q + 1) != 0.f);
+                const float er = __expf(__ldg(gqh + Q + 2));
+                const float *src = nullptr;
+                if (T.c0 == 0) {
+                    src = h0 ? h0 + row_off : nullptr;
+                } else {
+                    if (m == 0)
+                        *state_ok = wait_flag(flags + int64_t(T.b) * np + T.p, unsigned(T.c0), err) ? 1 : 0;
+                    named_barrier(kBarState, 128);
+                    if (!*state_ok) { ok = false; break; }
+                    __threadfence();
+                    src = chain + row_off;
+                }
+                __nv_bfloat16 *sin_row = steep ? s_in + off_state(d, T.b, T.c0, h) + int64_t(p) * NS : nullptr;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    // half a row per round trip: 16 loads in flight
+                    float v[NS / 2];
+                    if (src) {
+#pragma unroll
+                        for (int q4 = 0; q4 < NS / 8; ++q4) {
+                            const float4 *s4 = reinterpret_cast<const float4 *>(src) + hf * (NS / 8) + q4;
+                            const float4 t4 = T.c0 == 0 ? __ldg(s4) : __ldcg(s4);
+                            v[4 * q4] = t4.x; v[4 * q4 + 1] = t4.y; v[4 * q4 + 2] = t4.z; v[4 * q4 + 3] = t4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < NS / 2; ++e) v[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int sg = 0; sg < NS / 64; ++sg) {
+                        float *vv = v + sg * 32;
+                        const int seg = hf * (NS / 64) + sg;
+                        if (sin_row) put_bf16_row(sin_row + seg * 32, *reinterpret_cast<const float(*)[32]>(vv));
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) vv[e] *= er;
+                        tmem_st16(tacc + seg * 32, reinterpret_cast<const uint32_t *>(vv));
+                        tmem_st16(tacc + seg * 32 + 16, reinterpret_cast<const uint32_t *>(vv + 16));
+                        pack32(seg, *reinterpret_cast<const float(*)[32]>(vv));
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(acc_ready);
+            }
+            for (int c = T.c0; c < T.c1 && ok; ++c) {
+                const float *gqh = gq + ((int64_t(T.b) * d.H + h) * d.nc + c) * ngq;
+                const float r = __ldg(gqh + Q + 2);
+                for (int k = 0; k < ntile; ++k, ++kt) {
+                    // Z has read B_k: S'_k into the tile's B region for C_k S'_k^T
+                    if (!mbar_wait(z_done, kt & 1, err)) { ok = false; break; }
+                    tc_fence_after();
+                    {
+                        uint8_t *bq = cb_at(kt) + L::kCB;
+#pragma unroll
+                        for (int ch = 0; ch < NS / 8; ++ch)
+                            *reinterpret_cast<uint4 *>(bq + (ch >> 3) * (kRows * 128) + m * 128 +
+                                                       (((ch & 7) ^ (m & 7)) << 4)) =
+                                make_uint4(sp[4 * ch], sp[4 * ch + 1], sp[4 * ch + 2], sp[4 * ch + 3]);
+                        fence_proxy_async_smem();
+                        mbar_arrive(sp_ready);
+                    }
+                    if (k + 1 < ntile) {
+                        // S'_{k+1} = ACC (the chunk's reference is unchanged)
+#pragma unroll
+                        for (int seg = 0; seg < NS / 32; ++seg) {
+                            float v[32];
+                            tmem_ld32(tacc + seg * 32, v);
+                            pack32(seg, v);
+                        }
+                        tc_fence_before();
+                        mbar_arrive(acc_ready);
+                        continue;
+                    }
+                    // last tile of chunk c: s_in_{c+1} = exp(l_last - r) ACC
+                    const float ul = __expf(__ldg(lcum + off_lq(d, T.b, h, c) + Q - 1) - r);
+                    if (c + 1 < T.c1) {
+                        // next chunk of this ticket: S'_0 = e^{r_{c+1}} s_in_{c+1}, in place
+                        const float *gqn = gqh + ngq;
+                        const float en = __expf(__ldg(gqn + Q + 2));
+                        const bool steep_n = __ldg(gqn + Q) != 0.f || (ntile == 2 && __ldg(gqn + Q + 1) != 0.f);
+                        __nv_bfloat16 *sin_row = steep_n ? s_in + off_state(d, T.b, c + 1, h) + int64_t(p) * NS : nullptr;
+#pragma unroll
+                        for (int seg = 0; seg < NS / 32; ++seg) {
+                            float v[32];
+                            tmem_ld32(tacc + seg * 32, v);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) v[e] *= ul;
+                            if (sin_row) put_bf16_row(sin_row + seg * 32, v);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) v[e] *= en;
+                            tmem_st16(tacc + seg * 32, reinterpret_cast<const uint32_t *>(v));
+                            tmem_st16(tacc + seg * 32 + 16, reinterpret_cast<const uint32_t *>(v + 16));
+                            pack32(seg, v);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(acc_ready);
+                        continue;
+                    }
+                    // ticket end: the state leaves through the chain slot (or final_state)
+                    const bool last = c + 1 == d.nc;
+                    float *dst = last ? (fin ? fin + row_off : nullptr) : chain + row_off;
+#pragma unroll
+                    for (int seg = 0; seg < NS / 32; ++seg) {
+                        float v[32];
+                        tmem_ld32(tacc + seg * 32, v);
+                        if (dst) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4) {
+                                const float4 o = make_float4(v[4 * q4] * ul, v[4 * q4 + 1] * ul, v[4 * q4 + 2] * ul,
+                                                             v[4 * q4 + 3] * ul);
+                                if (last) reinterpret_cast<float4 *>(dst)[seg * 8 + q4] = o;
+                                else __stcg(reinterpret_cast<float4 *>(dst) + seg * 8 + q4, o);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    if (!last) {
+                        __threadfence();
+                        named_barrier(kBarState, 128);
+                        if (m == 0) st_release(flags + int64_t(T.b) * np + T.p, unsigned(T.c1));
+                    }
+                }
+            }
+        }
+    } else {
+        // ================================ epilogue ================================
+        // y_t = u_t Y[t] + D_h x_t with u_t = exp(l_t - r); the skip term comes
+        // from the scaled row as (D_h / g_t) X''_t, or from x in global memory
+        // where g_t is below 1e-30 (a zero dt).  The x rows are read first and
+        // the stage goes back to the producer; each warp then stages its 32 rows
+        // per head (128-byte swizzle) in its own blocks of the y staging area and
+        // writes them with its own TMA stores.
+        const int qd = warp & 3;
+        const int t = qd * 32 + lane;
+        const uint32_t lane_base = uint32_t(qd * 32) << 16;
+        // this row's factors of a tile (both heads), loaded one tile ahead
+        struct Raw {
+            float stp[2], gt[2], lt[2], r[2];
+        };
+        auto load_raw = [&](const TileWalk &w, Raw &e) {
+#pragma unroll
+            for (int jh = 0; jh < 2; ++jh) {
+                const int h = 2 * w.T.p + jh;
+                const float *gqh = gq + ((int64_t(w.T.b) * d.H + h) * d.nc + w.c) * ngq;
+                e.stp[jh] = __ldg(gqh + Q + w.k);
+                e.gt[jh] = __ldg(gqh + w.k * kRows + t);
+                e.lt[jh] = __ldg(lcum + off_lq(d, w.T.b, h, w.c) + w.k * kRows + t);
+                e.r[jh] = __ldg(gqh + Q + 2);
+            }
+        };
+        TileWalk cur, nxt;
+        cur.start(R, d);
+        nxt = cur;
+        nxt.next(R, d, ntile);
+        Raw ecur;
+        if (cur.valid) load_raw(cur, ecur);
+        uint32_t kt = 0;
+        bool ok = true;
+        for (; cur.valid && ok; ++kt, cur.next(R, d, ntile), nxt.next(R, d, ntile)) {
+                    const Seg T = cur.T;
+                    const int c = cur.c, k = cur.k;
+                    Raw enx;
+                    if (nxt.valid) load_raw(nxt, enx);
+                    const int yb = kt & 1;
+                    const int tok = c * Q + k * kRows + t;  // token within the sequence
+                    float u[2], dg[2];
+                    bool stp[2], fb[2];
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        const float Dh = Dskip ? __ldg(Dskip + 2 * T.p + jh) : 0.f;
+                        stp[jh] = ecur.stp[jh] != 0.f;
+                        u[jh] = __expf(ecur.lt[jh] - ecur.r[jh]);
+                        fb[jh] = !(ecur.gt[jh] >= 1e-30f) && Dh != 0.f;
+                        dg[jh] = (fb[jh] || Dh == 0.f) ? 0.f : Dh / ecur.gt[jh];
+                    }
+                    ecur = enx;
+                    if (!mbar_wait(&acc_full[yb], (kt >> 1) & 1, err)) { ok = false; break; }
+                    tc_fence_after();
+                    // this row's scaled x, head by head; y_t is then written over it in
+                    // place (each thread owns its row), and the x slot is written out
+                    uint8_t *xslot = x_at(kt);
+#pragma unroll
+                    for (int jh = 0; jh < 2; ++jh) {
+                        if (stp[jh]) continue;  // computed by the block-factored scan
+                        uint8_t *yrow = xslot + jh * (kRows * 128) + t * 128;
+                        uint4 xr[8];
+                        if (fb[jh]) {
+                            // raw x from global memory (rare): D_h x_t
+                            const uint4 *gx = reinterpret_cast<const uint4 *>(x + off_x(d, T.b, tok, 2 * T.p + jh));
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) xr[q] = __ldg(gx + q);
+                            dg[jh] = __ldg(Dskip + 2 * T.p + jh);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                xr[q] = *reinterpret_cast<const uint4 *>(yrow + ((q ^ (t & 7)) << 4));
+                        }
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            uint32_t a[32];
+                            tmem_ld32_nowait(tmem + lane_base + ycol(yb) + 64 * jh + 32 * hf, a);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int q = 4 * hf + qq;
+                                const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+                                uint32_t o[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    o[e] = pack_bf16x2(
+                                        fmaf(u[jh], __uint_as_float(a[8 * qq + 2 * e]), dg[jh] * bf16lo(xw[e])),
+                                        fmaf(u[jh], __uint_as_float(a[8 * qq + 2 * e + 1]), dg[jh] * bf16hi(xw[e])));
+                                *reinterpret_cast<uint4 *>(yrow + ((q ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&y_free[yb]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int row = T.b * d.T + c * Q + k * kRows + qd * 32;
+#pragma unroll
+                        for (int jh = 0; jh < 2; ++jh) {
+                            if (stp[jh]) {
+                                if (qd == 0) {
+                                    const int idx = atomicAdd(nsteep, 1);
+                                    if (idx < max_steep)
+                                        steep_items[idx] = ((long long)T.b << 40) | ((long long)c << 24) |
+                                                           ((long long)k << 16) | (2 * T.p + jh);
+                                }
+                                continue;
+                            }
+                            // this warp's 32 rows of head jh: 4 KB, 1024-byte aligned
+                            tma_store_3d(&tm_y, xslot + jh * (kRows * 128) + qd * 4096, 0, 2 * T.p + jh, row);
+                        }
+                        bulk_commit();
+                        // the previous tile's stores have read their slot: it goes back
+                        if (kt > 0) {
+                            bulk_wait_read_1();
+                            mbar_arrive(&x_free[(kt - 1) % kXS]);
+                        }
+                    }
+                    __syncwarp();
+        }
+        if (lane == 0) {
+            bulk_wait_all();
+            if (kt > 0) mbar_arrive(&x_free[(kt - 1) % kXS]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int NS>
+cudaError_t launch_fused(const Dims &d, const CUtensorMap *maps, const __nv_bfloat16 *x, const float *gq,
+                         const float *l, const float *D, const float *h0, float *fin, float *chain,
+                         unsigned int *flags, __nv_bfloat16 *s_in, int *nsteep, long long *items,
+                         int max_items, unsigned int *err, cudaStream_t stream) {
+    using L = FusedLayout<NS>;
+    if (!smem_attr_once(reinterpret_cast<const void *>(chunk_fused_kernel<NS>), int(L::kTotal)))
+        return cudaErrorInvalidValue;
+    // one CTA per SM (shared memory), at most one per chain
+    const long long chains = (long long)d.B * (d.H / 2);
+    const int sms = device_sm_count();
+    const int grid = chains < sms ? int(chains) : sms;
+    chunk_fused_kernel<NS><<<grid, kThreads, L::kTotal, stream>>>(maps[0], maps[1], maps[2], maps[3], d, x, gq,
+                                                                  l, D, h0, fin, chain, flags, s_in, nsteep,
+                                                                  items, max_items, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_chunk_fused_supported(const Dims &d) {
+    const bool n_ok = d.N == 64 || d.N == 128;
+    return d.P == 64 && n_ok && (d.Q == 128 || d.Q == 256) && d.r % 2 == 0 &&
+           (long long)d.B * d.T < (1ll << 31) && (long long)d.nc * d.B * (d.H / 2) < (1ll << 40);
+}
+
+size_t chunk_fused_chain_bytes(const Dims &d) { return size_t(d.B) * d.H * d.P * d.N * sizeof(float); }
+size_t chunk_fused_flag_bytes(const Dims &d) { return size_t(d.B) * (d.H / 2) * sizeof(unsigned int); }
+
+cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
+                               const float *D, const float *l, const float *h0, void *y, float *fin,
+                               float *chain, unsigned int *flags, void *s_in_bf16, int *nsteep,
+                               long long *items, int max_items, unsigned int *err, cudaStream_t stream) {
+    const uint64_t bcdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
+    const uint64_t bcstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
+    const uint32_t bcbox[3] = {64, 1, uint32_t(kRows)};
+    const uint64_t xdims[3] = {uint64_t(d.P), uint64_t(d.H), uint64_t(d.B) * d.T};
+    const uint64_t xstr[2] = {uint64_t(d.P) * 2, uint64_t(d.H) * d.P * 2};
+    const uint32_t xbox[3] = {64, 1, uint32_t(kRows)};
+    const uint32_t ybox[3] = {64, 1, 32};  // one epilogue warp's 32 rows of one head
+    CUtensorMap maps[4];
+    if (!make_tmap_bf16(&maps[0], 3, Cm, bcdims, bcstr, bcbox, 128) ||
+        !make_tmap_bf16(&maps[1], 3, Bm, bcdims, bcstr, bcbox, 128) ||
+        !make_tmap_bf16(&maps[2], 3, x, xdims, xstr, xbox, 128) ||
+        !make_tmap_bf16(&maps[3], 3, y, xdims, xstr, ybox, 128))
+        return cudaErrorInvalidValue;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+    __nv_bfloat16 *sb = static_cast<__nv_bfloat16 *>(s_in_bf16);
+    switch (d.N) {
+        case 64: return launch_fused<64>(d, maps, xb, gq, l, D, h0, fin, chain, flags, sb, nsteep, items,
+                                         max_items, err, stream);
+        case 128: return launch_fused<128>(d, maps, xb, gq, l, D, h0, fin, chain, flags, sb, nsteep, items,
+                                           max_items, err, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ssd

@@ -18,10 +18,22 @@ __host__ __device__ constexpr int chunk_gq(int Q) { return Q + 4; }
 // chunk-wide scan's factors exp(-l_s) would exceed e^72), or when one of its
 // dt is 0 (the skip term is recovered from the scaled rows as D / g)
 constexpr float kScanSteep = 72.f;
+// chain_flags != nullptr selects the fused mode (chunk_len 128 / 256, gq
+// required): the reference and flags of the single-pass kernel, no w / alpha,
+// dtq and beta only for chunks with a flagged tile, and the (b, head pair)
+// chain flags [B, H/2] reset to 0.
+// dt_bias [H] (or nullptr) and dt_softplus select the block's dt transform,
+// softplus(dt + dt_bias); dt_eff (or nullptr) receives it in dt's layout.
 cudaError_t launch_chunk_cumsum(const Dims &d, const float *dt, const float *A, float *l,
                                 float *w, float *dtq, float *beta, float *alpha, float *gq,
-                                int *nsteep,
-                                cudaStream_t stream);
+                                int *nsteep, unsigned int *chain_flags, const float *dt_bias,
+                                int dt_softplus, float *dt_eff, cudaStream_t stream);
+
+// The block's output side in place on y [B,T,H,P]: g = y * silu(z) (z may be
+// nullptr), then with a weight w [H*P] the RMSNorm factor rstd per token
+// (written to rstd_out if non-null) and out = g * rstd * w (apply) or g * w.
+cudaError_t launch_gate_norm(const Dims &d, bool bf16, void *y, const void *z, const float *w, float eps,
+                             bool apply, float *rstd_out, cudaStream_t stream);
 
 // ssd_state_passing: states [B,nc,H,P,N] (fp32 or bf16 per states_bf16), alpha
 // -> s_in [B,nc,H,P,N] (fp32 or bf16 per s_in_bf16), final state [B,H,P,N] fp32
@@ -77,5 +89,28 @@ cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq,
                                   const void *Cm, const float *D, const float *l,
                                   const void *s_in_bf16, void *y, int *nsteep, long long *items,
                                   unsigned int *err, cudaStream_t stream);
+
+// The whole pass after the cumsum in one persistent kernel (bf16, P = 64,
+// N in {64, 128}, chunk_len 128 / 256, an even number of heads per group):
+// chunk state, state passing through per-(b, h) fp32 slots `chain` [B,H,P,N]
+// with flags [B, H/2], and chunk scan.  Tiles flagged steep by the cumsum are
+// appended to (nsteep, items) for the block-factored scan, with s_in (bf16
+// [B,nc,H,P,N]) written for their chunks.
+bool tc_chunk_fused_supported(const Dims &d);
+size_t chunk_fused_chain_bytes(const Dims &d);
+size_t chunk_fused_flag_bytes(const Dims &d);
+cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
+                               const float *D, const float *l, const float *h0, void *y, float *fin,
+                               float *chain, unsigned int *flags, void *s_in_bf16, int *nsteep,
+                               long long *items, int max_items, unsigned int *err, cudaStream_t stream);
+
+// The last T mod chunk_len tokens of every (b, h) as the recurrence, from
+// h_in (the full chunks' final state, or the initial state; nullptr = zeros),
+// with the block's dt transform when dt_bias / dt_softplus are given; writes y
+// of those tokens and, if fin != nullptr, the final state.
+bool tail_supported(const Dims &d);
+cudaError_t launch_tail(const Dims &d, bool bf16, int t_begin, const void *x, const float *dt,
+                        const float *dt_bias, int dt_softplus, const float *A, const void *Bm, const void *Cm,
+                        const float *D, const float *h_in, void *y, float *fin, cudaStream_t stream);
 
 }  // namespace ssd

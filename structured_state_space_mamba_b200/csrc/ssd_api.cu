@@ -50,6 +50,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool misaligned(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u); }
 
 constexpr int kB200Sms = 148;
+constexpr int kMinChainNum = 2, kMinChainDen = 5;  // single-pass kernel: chains >= 40% of SMs
 
 struct Plan {
     Dims d;
@@ -58,8 +59,14 @@ struct Plan {
     bool tc_scan;   // tcgen05 chunk scan (consumes bf16 s_in)
     bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
     bool scan5;     // chunk-wide scan, steep tiles finished by the block-factored scan
-    size_t steep_offset;  // scan5: item counter (256 bytes) + packed steep items
-    size_t gq_offset;     // scan5: per-token column factors [B,H,nc,chunk_gq(Q)]
+    bool single;    // the single-pass kernel (chunk state + state passing + scan)
+    int tile_chunks = 1;  // caller chunks per chunk of the plan (2: chunk_len 64 run as 128)
+    int t_full = 0;       // tokens in full chunks; the tail [t_full, T) runs in the tail kernel
+    size_t mid_offset = 0;  // tail: fp32 state after the full chunks [B,H,P,N]
+    size_t steep_offset;  // scan5 / single: item counter (256 bytes) + packed steep items
+    size_t gq_offset;     // scan5 / single: per-token column factors [B,H,nc,chunk_gq(Q)]
+    size_t chain_offset;  // single: per-(b, h) fp32 state slots [B,H,P,N]
+    size_t flag_offset;   // single: per-(b, head pair) chain flags [B, H/2]
     ssd_workspace_layout_t ws;
 };
 
@@ -73,7 +80,6 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     if (a.nheads % a.ngroups != 0) return SSD_ERR_INVALID_DIM;
     if (chunk_len != 32 && chunk_len != 64 && chunk_len != 128 && chunk_len != 256)
         return SSD_ERR_UNSUPPORTED;
-    if (a.seqlen % chunk_len != 0) return SSD_ERR_INVALID_DIM;
     if (a.headdim > 256 || a.dstate > 256) return SSD_ERR_UNSUPPORTED;
     if (a.dtype == SSD_BF16 && (a.headdim % 8 != 0 || a.dstate % 8 != 0)) return SSD_ERR_UNSUPPORTED;
     // grid limits (blockIdx.y / .z <= 65535) and 32-bit token indices
@@ -86,6 +92,25 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     d.B = int(a.batch); d.T = int(a.seqlen); d.H = int(a.nheads); d.P = int(a.headdim);
     d.N = int(a.dstate); d.G = int(a.ngroups); d.Q = chunk_len; d.nc = int(nc);
     d.r = d.H / d.G;
+    // chunk_len 64 on the tensor cores: their tile is 128 rows (the full TMEM
+    // lane range of a one-CTA MMA), so the chunked algorithm runs with 128-token
+    // chunks -- two of the caller's chunks per tile, whose hand-off then happens
+    // inside the tile's masked product.  The result is the same recurrence (the
+    // chunk length only sets the blocking); the workspace arrays then describe
+    // 128-token chunks.
+    if (a.dtype == SSD_BF16 && d.Q == 64 && d.T % 128 == 0) {
+        Dims d2 = d;
+        d2.Q = 128;
+        d2.nc = d.T / 128;
+        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2)) {
+            d = d2;
+            plan->tile_chunks = 2;
+        }
+    }
+    // a length that is not a multiple of chunk_len: the chunked kernels take the
+    // full chunks (they index rows with the true T), the tail kernel the rest
+    plan->t_full = d.nc * d.Q;
+    if (plan->t_full < d.T && !ssd::tail_supported(d)) return SSD_ERR_UNSUPPORTED;
     plan->d = d;
     plan->bf16 = a.dtype == SSD_BF16;
     plan->tc_state = plan->bf16 && ssd::tc_chunk_state_supported(d);
@@ -94,6 +119,12 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     // those units fill most of the GPU's 148 SMs in one wave
     plan->fused = plan->tc_state && plan->tc_scan && ssd::tc_state_fused_supported(d, kB200Sms);
     plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d) && ssd::tc_chunk_scan4_supported(d);
+    // the single-pass kernel walks each (b, head pair) chain chunk by chunk: used
+    // when the chains fill at least kMinChainFrac of the SMs (fewer chains leave
+    // most SMs idle, and the four-kernel sequence is faster there)
+    plan->single = plan->scan5 && ssd::tc_chunk_fused_supported(d) &&
+                   int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
+    if (plan->single) plan->fused = false;
 
     ssd_workspace_layout_t &w = plan->ws;
     std::memset(&w, 0, sizeof(w));
@@ -108,7 +139,7 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.alpha_offset = off; off = align_up(off + al);
     w.states_offset = off;
     w.states_dtype = plan->tc_state ? SSD_BF16 : SSD_F32;
-    if (!plan->fused) off = align_up(off + st * (plan->tc_state ? 2 : 4));
+    if (!plan->fused && !plan->single) off = align_up(off + st * (plan->tc_state ? 2 : 4));
     w.s_in_offset = off;
     w.s_in_dtype = plan->tc_scan ? SSD_BF16 : SSD_F32;
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
@@ -116,10 +147,23 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     if (plan->scan5) off = align_up(off + kAlign + sizeof(long long) * size_t(ssd::chunk_scan5_max_steep(d)));
     plan->gq_offset = off;
     if (plan->scan5) off = align_up(off + al * ssd::chunk_gq(d.Q));
+    plan->chain_offset = off;
+    if (plan->single) off = align_up(off + ssd::chunk_fused_chain_bytes(d));
+    plan->flag_offset = off;
+    if (plan->single) off = align_up(off + ssd::chunk_fused_flag_bytes(d));
+    plan->mid_offset = off;
+    if (plan->t_full < d.T) off = align_up(off + size_t(d.B) * d.H * d.P * d.N * sizeof(float));
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
-    w.launches = (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
+    w.launches = d.nc == 0 ? 0 : plan->single ? 3 : (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
+    if (plan->t_full < d.T) w.launches += 1;
     w.fused_state = plan->fused ? 1 : 0;
+    w.single_pass = plan->single ? 1 : 0;
+    w.chunk_len = d.Q;
+    w.scan_engine = plan->scan5 ? (plan->single ? SSD_ENGINE_SINGLE_PASS : SSD_ENGINE_CHUNK_WIDE)
+                    : plan->tc_scan ? (ssd::tc_chunk_scan4_supported(d) ? SSD_ENGINE_BLOCK_FACTORED
+                                                                        : SSD_ENGINE_TILE)
+                                    : SSD_ENGINE_SIMT;
     return SSD_OK;
 }
 
@@ -142,11 +186,48 @@ bool inject_launch_failure() {
     return v && std::strcmp(v, "launch") == 0;
 }
 
+// The block neighbours of one call (ssd_forward_block); all off for the plain
+// entry points.
+struct Neighbours {
+    const float *dt_bias = nullptr;
+    int softplus = 0;
+    const void *z = nullptr;
+    const float *norm_w = nullptr;
+    float eps = 0.f;
+    bool apply = false;
+    float *rstd = nullptr;
+    float *dt_eff = nullptr;  // workspace copy of the transformed dt, dt's layout
+    bool transform() const { return dt_bias || softplus; }
+    bool output() const { return z || norm_w; }
+};
+
 ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A, const void *Bm,
                  const void *Cm, const float *D, const float *init_state, void *y,
-                 float *fin, char *ws, cudaStream_t stream, int only_stage = -1) {
+                 float *fin, char *ws, cudaStream_t stream, int only_stage = -1,
+                 const Neighbours *nb = nullptr) {
     if (inject_launch_failure()) return SSD_ERR_CUDA;
     const Dims &d = pl.d;
+    const Neighbours none;
+    if (!nb) nb = &none;
+    // with a tail, the full chunks' final state goes to the workspace and the
+    // tail kernel continues from it
+    const bool tail = pl.t_full < d.T;
+    float *fin_user = fin;
+    float *mid = tail ? reinterpret_cast<float *>(ws + pl.mid_offset) : nullptr;
+    if (tail) fin = mid;
+    // after the scan: the tail tokens (recurrence from the full chunks' state),
+    // then the block's gate and norm over every token
+    auto finish_scan = [&]() -> cudaError_t {
+        cudaError_t e2 = cudaSuccess;
+        if (tail)
+            e2 = ssd::launch_tail(d, pl.bf16, pl.t_full, x, dt, nb->dt_bias, nb->softplus, A, Bm, Cm, D,
+                                  d.nc > 0 ? mid : init_state, y, fin_user, stream);
+        if (e2 == cudaSuccess && nb->output())
+            e2 = ssd::launch_gate_norm(d, pl.bf16, y, nb->z, nb->norm_w, nb->eps, nb->apply, nb->rstd, stream);
+        return e2;
+    };
+    // the scans that read dt themselves take the transformed copy
+    const float *dt_scan = nb->transform() ? nb->dt_eff : dt;
     unsigned int *err = nullptr;
     if (pl.tc_state || pl.tc_scan) {
         err = device_error_word();
@@ -162,14 +243,46 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     int *nsteep = reinterpret_cast<int *>(ws + pl.steep_offset);
     long long *steep_items = reinterpret_cast<long long *>(ws + pl.steep_offset + kAlign);
     float *gq = pl.scan5 ? reinterpret_cast<float *>(ws + pl.gq_offset) : nullptr;
+    float *chain = pl.single ? reinterpret_cast<float *>(ws + pl.chain_offset) : nullptr;
+    unsigned int *flags = pl.single ? reinterpret_cast<unsigned int *>(ws + pl.flag_offset) : nullptr;
     for (int stage = 0; stage < 4; ++stage) {
         if (only_stage >= 0 && stage != only_stage) continue;
         cudaError_t e = cudaSuccess;
+        if (d.nc == 0) {
+            // shorter than one chunk: the tail kernel does everything
+            if (stage == SSD_STAGE_CHUNK_SCAN) e = finish_scan();
+            if (e != cudaSuccess) return SSD_ERR_CUDA;
+            continue;
+        }
+        if (pl.single) {
+            // cumsum (fused mode), the single-pass kernel, the block-factored scan
+            // over the tiles it listed as steep
+            switch (stage) {
+                case SSD_STAGE_CHUNK_CUMSUM:
+                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, flags,
+                                                 nb->dt_bias, nb->softplus, nullptr, stream);
+                    break;
+                case SSD_STAGE_CHUNK_STATE:
+                    e = ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags, s_in,
+                                                nsteep, steep_items, ssd::chunk_scan5_max_steep(d), err, stream);
+                    break;
+                case SSD_STAGE_STATE_PASSING:
+                    break;
+                case SSD_STAGE_CHUNK_SCAN:
+                    e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, steep_items, nsteep,
+                                                   ssd::chunk_scan5_max_steep(d), err, stream);
+                    if (e == cudaSuccess) e = finish_scan();
+                    break;
+            }
+            if (e != cudaSuccess) return SSD_ERR_CUDA;
+            continue;
+        }
         switch (stage) {
             case SSD_STAGE_CHUNK_CUMSUM:
                 // also empties the chunk-wide scan's steep-tile list
                 e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq,
-                                             pl.scan5 ? nsteep : nullptr, stream);
+                                             pl.scan5 ? nsteep : nullptr, nullptr, nb->dt_bias,
+                                             nb->softplus, nb->transform() ? nb->dt_eff : nullptr, stream);
                 break;
             case SSD_STAGE_CHUNK_STATE:
                 e = pl.fused ? ssd::launch_state_fused(d, x, Bm, w, alpha, init_state, s_in, fin, err, stream)
@@ -197,10 +310,11 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                             ? (ssd::tc_chunk_scan4_supported(d)
                                    ? ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
                                                                 nullptr, nullptr, 0, err, stream)
-                                   : ssd::launch_chunk_scan_tc(d, x, dt, Bm, Cm, D, l, s_in, y, err, stream))
-                            : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt, Bm, Cm, D, l,
+                                   : ssd::launch_chunk_scan_tc(d, x, dt_scan, Bm, Cm, D, l, s_in, y, err, stream))
+                            : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt_scan, Bm, Cm, D, l,
                                                           static_cast<const float *>(s_in), y, stream);
                 }
+                if (e == cudaSuccess) e = finish_scan();
                 break;
         }
         if (e != cudaSuccess) return SSD_ERR_CUDA;
@@ -284,6 +398,56 @@ ssd_status_t ssd_forward(const ssd_dims_t *dims, const void *x, const float *dt,
     return s;
 }
 
+size_t ssd_block_workspace_bytes(const ssd_dims_t *dims, int chunk_len, const ssd_block_opts_t *opts) {
+    Plan pl;
+    if (make_plan(dims, chunk_len, &pl) != SSD_OK) return 0;
+    size_t total = pl.ws.total_bytes;
+    if (opts && (opts->dt_bias || opts->dt_softplus))
+        total = align_up(total + size_t(pl.d.B) * pl.d.T * pl.d.H * sizeof(float));
+    return total;
+}
+
+ssd_status_t ssd_forward_block(const ssd_dims_t *dims, const void *x, const float *dt, const float *A,
+                               const void *Bm, const void *Cm, const float *D, int chunk_len,
+                               const float *init_state, void *y_out, float *final_state_out,
+                               const ssd_block_opts_t *opts, void *workspace, size_t workspace_bytes,
+                               void *stream) {
+    Plan pl;
+    ssd_status_t s = make_plan(dims, chunk_len, &pl);
+    if (s != SSD_OK) return s;
+    s = check_tensors(pl, x, dt, A, Bm, Cm, D, init_state, y_out, final_state_out);
+    if (s != SSD_OK) return s;
+    Neighbours nb;
+    if (opts) {
+        if (opts->reserved0 != 0) return SSD_ERR_INVALID_DIM;
+        const void *ptrs[] = {opts->dt_bias, opts->z, opts->norm_weight, opts->rstd_out};
+        for (const void *p : ptrs)
+            if (misaligned(p)) return SSD_ERR_MISALIGNED;
+        if (opts->norm_weight && !(opts->norm_eps > 0.f)) return SSD_ERR_INVALID_DIM;
+        if (opts->norm_weight && !opts->norm_apply && !opts->rstd_out) return SSD_ERR_NULL_ARG;
+        nb.dt_bias = opts->dt_bias;
+        nb.softplus = opts->dt_softplus ? 1 : 0;
+        nb.z = opts->z;
+        nb.norm_w = opts->norm_weight;
+        nb.eps = opts->norm_eps;
+        nb.apply = opts->norm_apply != 0;
+        nb.rstd = opts->norm_weight ? opts->rstd_out : nullptr;
+    }
+    const size_t need = ssd_block_workspace_bytes(dims, chunk_len, opts);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = workspace;
+    if (ws) {
+        if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return SSD_ERR_WORKSPACE;
+    } else if (cudaMallocAsync(&ws, need, st) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_WORKSPACE;
+    }
+    if (nb.transform()) nb.dt_eff = reinterpret_cast<float *>(static_cast<char *>(ws) + pl.ws.total_bytes);
+    s = run(pl, x, dt, A, Bm, Cm, D, init_state, y_out, final_state_out, static_cast<char *>(ws), st, -1, &nb);
+    if (!workspace && cudaFreeAsync(ws, st) != cudaSuccess && s == SSD_OK) s = SSD_ERR_CUDA;
+    return s;
+}
+
 const char *ssd_status_string(ssd_status_t status) {
     switch (status) {
         case SSD_OK: return "SSD_OK: success";
@@ -317,6 +481,6 @@ ssd_status_t ssd_device_status(void *stream) {
     return SSD_OK;
 }
 
-const char *ssd_version(void) { return "ssd-b200 0.1.0 sm_100a"; }
+const char *ssd_version(void) { return "ssd-b200 0.2.0 sm_100a"; }
 
 }  // extern "C"

@@ -15,29 +15,51 @@ def layout(cfg):
     return binding.workspace_layout(d, cfg["chunk_len"])
 
 
-def test_scan_bytes_of_the_2p7b_layer_by_hand():
-    cfg = dict(WORKLOADS["mamba2_2p7b"])
+def test_scan_bytes_of_the_long_context_layer_by_hand():
+    """Four-kernel sequence (few (batch, head pair) chains): the chunk-wide scan
+    reads x, B, C, l, g and the bf16 s_in, and writes y."""
+    cfg = dict(WORKLOADS["long_g8"])
     lay = layout(cfg)
+    assert lay.single_pass == 0
     wm = bench.work_model(cfg, True, lay)
-    B, T, H, P, N, Q = 4, 4096, 80, 64, 128, 256
+    B, T, H, P, N, G, Q = 1, 65536, 32, 64, 128, 8, 256
     nc = T // Q
-    x = B * T * H * P * 2                       # bf16 x (and y)
-    bc = 2 * B * T * N * 2                      # bf16 B and C, one group
+    x = B * T * H * P * 2
+    bc = 2 * B * T * G * N * 2
     l_g = B * H * nc * Q * 4 + B * H * nc * (Q + 4) * 4
-    s_in = B * nc * H * P * N * 2               # bf16 state entering each chunk
+    s_in = B * nc * H * P * N * 2
     assert wm["per_kernel_bytes"]["ssd_chunk_scan"] == 2 * x + bc + l_g + s_in + H * 4
-    assert wm["per_kernel_bytes"]["ssd_chunk_scan"] / MB == pytest.approx(438.4, abs=0.1)
-    # chunk_state reads x, B and w and writes the bf16 chunk states
-    assert wm["per_kernel_bytes"]["ssd_chunk_state"] / MB == pytest.approx(261.1, abs=0.1)
-    # compulsory bytes: x and y, B and C, dt, A and D, the final fp32 state
-    comp = 2 * x + bc + B * T * H * 4 + 2 * H * 4 + B * H * P * N * 4
+    assert wm["stages"] == ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
+    comp = 2 * x + bc + B * T * H * 4 + 2 * H * 4 + 2 * B * H * P * N * 4  # h0 and final
     assert wm["bytes"] == comp
 
 
-def test_fused_layout_has_no_state_passing_traffic():
-    cfg = dict(WORKLOADS["mamba2_130m"])
+def test_single_pass_bytes_of_the_2p7b_layer_by_hand():
+    """The 2.7B-shaped layer runs the single-pass kernel: it moves the compulsory
+    bytes (x, B, C in; y, final state out) plus the cumsum's l and g."""
+    cfg = dict(WORKLOADS["mamba2_2p7b"])
     lay = layout(cfg)
-    assert lay.fused_state == 1
+    assert lay.single_pass == 1 and lay.launches == 3
+    assert binding.SCAN_ENGINES[lay.scan_engine] == "single_pass"
+    wm = bench.work_model(cfg, True, lay)
+    B, T, H, P, N, Q = 4, 4096, 80, 64, 128, 256
+    nc = T // Q
+    x = B * T * H * P * 2
+    bc = 2 * B * T * N * 2
+    fin = B * H * P * N * 4
+    comp = 2 * x + bc + B * T * H * 4 + 2 * H * 4 + fin
+    assert wm["bytes"] == comp
+    assert wm["per_kernel_comp"]["ssd_chunk_fused"] == 2 * x + bc + H * 4 + fin
+    l_g = B * H * nc * Q * 4 + B * H * nc * (Q + 4) * 4
+    assert wm["per_kernel_bytes"]["ssd_chunk_fused"] == wm["per_kernel_comp"]["ssd_chunk_fused"] + l_g
+    assert wm["stages"][1] == "ssd_chunk_fused" and wm["stages"][2] is None
+
+
+def test_fused_layout_has_no_state_passing_traffic():
+    # the 130M-shaped layer at dstate 64: one wave of (batch, head pair) units
+    cfg = dict(WORKLOADS["mamba2_130m"], dstate=64)
+    lay = layout(cfg)
+    assert lay.fused_state == 1 and lay.single_pass == 0
     wm = bench.work_model(cfg, True, lay)
     assert wm["per_kernel_bytes"]["ssd_state_passing"] == 0
 
@@ -61,10 +83,6 @@ def test_l2_policy(name, flush):
 
 
 def test_traffic_figure_only_for_the_captured_kernel_and_build():
-    keys = set(bench.NCU_TRAFFIC)
-    assert all(len(k) == 3 for k in keys)
-    cfg = dict(WORKLOADS["mamba2_2p7b"])
-    wm = bench.work_model(cfg, True, layout(cfg))
     for (wl, kern, ver), traffic in bench.NCU_TRAFFIC.items():
         # a capture moves at least the kernel's compulsory bytes and, with L2
         # hits, at most somewhat more than its workspace-inclusive bytes
@@ -72,20 +90,20 @@ def test_traffic_figure_only_for_the_captured_kernel_and_build():
         w = bench.work_model(dict(WORKLOADS[wl]), True, layout(dict(WORKLOADS[wl])))
         assert 0.8 * w["per_kernel_comp"][kern] < traffic <= 1.2 * w["per_kernel_bytes"][kern]
     # a build the capture was not taken from reports no traffic figure
-    assert bench.NCU_TRAFFIC.get(("mamba2_2p7b", "ssd_chunk_scan", "some other build")) is None
-    assert wm["per_kernel_comp"]["ssd_chunk_scan"] <= wm["per_kernel_bytes"]["ssd_chunk_scan"]
+    assert bench.NCU_TRAFFIC.get(("mamba2_2p7b", "ssd_chunk_fused", "some other build")) is None
 
 
 def test_kernel_roofline_counts_compulsory_bytes_only():
-    """The scan's roofline bytes are the compulsory bytes it moves itself (x in,
+    """A scan's roofline bytes are the compulsory bytes it moves itself (x in,
     y out, B, C and D in); the chunk states it reads are not among them."""
-    cfg = dict(WORKLOADS["mamba2_2p7b"])
+    cfg = dict(WORKLOADS["long_g8"])
     wm = bench.work_model(cfg, True, layout(cfg))
-    B, T, H, P, N = 4, 4096, 80, 64, 128
+    B, T, H, P, N, G = 1, 65536, 32, 64, 128, 8
     x = B * T * H * P * 2
-    bc = 2 * B * T * N * 2
+    bc = 2 * B * T * G * N * 2
     assert wm["per_kernel_comp"]["ssd_chunk_scan"] == 2 * x + bc + H * 4
     assert wm["per_kernel_comp"]["ssd_chunk_cumsum"] == B * T * H * 4 + H * 4
+    assert wm["per_kernel_comp"]["ssd_chunk_scan"] < wm["per_kernel_bytes"]["ssd_chunk_scan"]
 
 
 def test_both_arms_build_the_same_config_block():

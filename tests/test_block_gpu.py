@@ -1,0 +1,110 @@
+"""GPU parity of ssd_forward_block (the scan with its Mamba-2 block neighbours:
+softplus(dt + dt_bias), the silu gate and RMSNorm over H * P) against the fp64
+oracle's ssd_block, element by element.
+
+Inputs: x, B, C, D, h0 as for the scan; the raw dt drawn U(-7, -2) (softplus maps
+it to about [1e-3, 0.13], the scan's own dt range), dt_bias U(-0.5, 0.5), z
+N(0, 1) in the storage dtype, norm weight 1 + 0.1 N(0, 1).  Tolerance: that of
+the scan, on the block's output (max abs error / max |reference|).
+"""
+import numpy as np
+import pytest
+import torch
+
+from structured_state_space_mamba_b200 import binding
+from structured_state_space_mamba_b200.inputs import make_inputs, round_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+DEV = torch.device("cuda:0")
+
+
+def rel(a, b):
+    return float(np.max(np.abs(a - b)) / max(np.max(np.abs(b)), 1e-30))
+
+
+def neighbours(inp, seed):
+    rng = np.random.default_rng(seed)
+    bsz, T, H, P = inp.x.shape
+    dt_raw = rng.uniform(-7.0, -2.0, size=(bsz, T, H)).astype(np.float32)
+    bias = rng.uniform(-0.5, 0.5, size=(H,)).astype(np.float32)
+    z = rng.standard_normal((bsz, T, H, P))
+    z = (round_to_bf16(z) if inp.dtype == "bf16" else z).astype(np.float32)
+    w = (1.0 + 0.1 * rng.standard_normal(H * P)).astype(np.float32)
+    return dt_raw, bias, z, w
+
+
+def run(inp, dt_raw, bias, z, w, apply, eps=1e-5):
+    tt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    t = lambda a, ty=torch.float32: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV).to(ty)  # noqa: E731
+    res = binding.forward_block(t(inp.x, tt), t(dt_raw), t(inp.A), t(inp.B, tt), t(inp.C, tt), D=t(inp.D),
+                                chunk_len=inp.chunk_len, init_state=t(inp.h0), dt_bias=t(bias),
+                                dt_softplus=True, z=t(z, tt), norm_weight=t(w), norm_eps=eps,
+                                norm_apply=apply, return_rstd=True, return_final_state=True)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    return [r.double().cpu().numpy() for r in res]
+
+
+SHAPES = [
+    # a length that is not a multiple of chunk_len: the tail kernel applies the dt transform itself
+    dict(batch=1, seqlen=600, nheads=8, headdim=64, dstate=128, ngroups=2, chunk_len=256, dtype="bf16"),
+    # the single-pass kernel (64 chains)
+    dict(batch=1, seqlen=512, nheads=128, headdim=64, dstate=128, ngroups=1, chunk_len=256, dtype="bf16"),
+    # the four-kernel sequence with the chunk-wide scan
+    dict(batch=1, seqlen=512, nheads=8, headdim=64, dstate=128, ngroups=2, chunk_len=128, dtype="bf16"),
+    # the first tensor-core scan (dstate 64) and the CUDA-core fp32 path: both read dt themselves
+    dict(batch=2, seqlen=512, nheads=6, headdim=64, dstate=64, ngroups=3, chunk_len=128, dtype="bf16"),
+    dict(batch=2, seqlen=256, nheads=4, headdim=16, dstate=16, ngroups=1, chunk_len=64, dtype="f32"),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("apply", [True, False])
+def test_block_against_oracle(oracle, shape, apply):
+    inp = make_inputs(**shape, seed=41, init_state=True)
+    dt_raw, bias, z, w = neighbours(inp, 42)
+    out, fin, rstd = run(inp, dt_raw, bias, z, w, apply)
+    ref, fref, rref = oracle.ssd_block(inp.x, dt_raw, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0, dt_bias=bias,
+                                       dt_softplus=True, z=z, norm_weight=w, norm_eps=1e-5)
+    tol = TOL[inp.dtype]
+    assert np.isfinite(out).all()
+    assert rel(fin, fref) <= tol
+    assert rel(rstd, rref) <= tol
+    if apply:
+        assert rel(out, ref) <= tol, rel(out, ref)
+    else:
+        # the output is g * w; the caller's per-token rstd finishes the norm
+        assert rel(out * rstd[:, :, None, None], ref) <= tol
+
+
+def test_block_gate_only_and_dt_only(oracle):
+    shape = SHAPES[0]
+    inp = make_inputs(**shape, seed=43, init_state=False)
+    dt_raw, bias, z, _ = neighbours(inp, 44)
+    tt = torch.bfloat16
+    t = lambda a, ty=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(DEV).to(ty)  # noqa: E731
+    # gate only, no norm, no dt transform: y * silu(z)
+    y = binding.forward_block(t(inp.x, tt), t(inp.dt), t(inp.A), t(inp.B, tt), t(inp.C, tt), D=t(inp.D),
+                              chunk_len=shape["chunk_len"], z=t(z, tt))
+    ref, _, _ = oracle.ssd_block(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, z=z)
+    assert rel(y.double().cpu().numpy(), ref) <= TOL["bf16"]
+    # dt transform only: the plain scan of softplus(dt + bias)
+    y2 = binding.forward_block(t(inp.x, tt), t(dt_raw), t(inp.A), t(inp.B, tt), t(inp.C, tt), D=t(inp.D),
+                               chunk_len=shape["chunk_len"], dt_bias=t(bias), dt_softplus=True)
+    ref2, _, _ = oracle.ssd_block(inp.x, dt_raw, inp.A, inp.B, inp.C, D=inp.D, dt_bias=bias, dt_softplus=True)
+    torch.cuda.synchronize()
+    assert rel(y2.double().cpu().numpy(), ref2) <= TOL["bf16"]
+
+
+def test_block_without_neighbours_equals_forward():
+    inp = make_inputs(**SHAPES[0], seed=45, init_state=True)
+    tt = torch.bfloat16
+    t = lambda a, ty=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(DEV).to(ty)  # noqa: E731
+    args = (t(inp.x, tt), t(inp.dt), t(inp.A), t(inp.B, tt), t(inp.C, tt))
+    y0, f0 = binding.forward(*args, D=t(inp.D), chunk_len=256, init_state=t(inp.h0), return_final_state=True)
+    y1, f1 = binding.forward_block(*args, D=t(inp.D), chunk_len=256, init_state=t(inp.h0),
+                                   return_final_state=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1) and torch.equal(f0, f1)

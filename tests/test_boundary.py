@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_struct_sizes_match_header(lib):
     assert ctypes.sizeof(binding.Dims) == 6 * 8 + 2 * 4
-    assert ctypes.sizeof(binding.WorkspaceLayout) == 8 * 8 + 6 * 4  # 5 int32 + padding
+    assert ctypes.sizeof(binding.WorkspaceLayout) == 8 * 8 + 8 * 4  # 8 int32 fields
 
 
 def test_status_strings(lib):
@@ -81,29 +81,62 @@ def test_workspace_layout(lib):
 
 
 def test_fused_state_layout_for_many_head_pairs(lib):
-    """0.6 x 148 <= (batch x head pairs) <= 148 SMs: chunk_state and state_passing
-    run as one kernel, so no states region is reserved and one launch fewer is
-    made; with more units than SMs, or far fewer, they stay separate."""
-    d = binding.make_dims(batch=8, seqlen=2048, nheads=24, headdim=64, dstate=128, ngroups=1,
+    """0.6 x 148 <= (batch x head pairs) <= 148 SMs at a dstate the single-pass
+    kernel does not take: chunk_state and state_passing run as one kernel, so no
+    states region is reserved and one launch fewer is made."""
+    d = binding.make_dims(batch=8, seqlen=2048, nheads=24, headdim=64, dstate=64, ngroups=1,
                           dtype="bf16")
     lay = binding.workspace_layout(d, 256)
-    assert lay.fused_state == 1 and lay.launches == 4 and lay.tensor_core == 1
+    assert lay.fused_state == 1 and lay.single_pass == 0 and lay.tensor_core == 1
     assert lay.states_offset == lay.s_in_offset
-    few = binding.workspace_layout(binding.make_dims(batch=1, seqlen=65536, nheads=32, headdim=64,
-                                                     dstate=128, ngroups=8, dtype="bf16"), 256)
-    assert few.fused_state == 0 and few.launches == 5
-    assert few.s_in_offset > few.states_offset
-    many = binding.workspace_layout(binding.make_dims(batch=4, seqlen=4096, nheads=80, headdim=64,
-                                                      dstate=128, ngroups=1, dtype="bf16"), 256)
-    assert many.fused_state == 0 and many.launches == 5
     # N = 32 keeps the one-launch scan
     n32 = binding.workspace_layout(binding.make_dims(batch=2, seqlen=1024, nheads=8, headdim=64,
                                                      dstate=32, ngroups=1, dtype="bf16"), 256)
-    assert n32.launches == 4
+    assert n32.launches == 4 and n32.single_pass == 0
+
+
+def test_single_pass_layout_selection(lib):
+    """bf16, P = 64, N = 128, chunk_len 128 / 256 and enough (batch, head pair)
+    chains (>= 40% of the 148 SMs) run the single-pass kernel: three launches,
+    no chunk-state region; few chains keep the four-kernel sequence."""
+    for b, h, q in ((4, 80, 256), (8, 24, 256), (8, 32, 128), (4, 32, 256)):
+        lay = binding.workspace_layout(binding.make_dims(batch=b, seqlen=4096, nheads=h, headdim=64,
+                                                         dstate=128, ngroups=1, dtype="bf16"), q)
+        assert lay.single_pass == 1 and lay.launches == 3, (b, h, q)
+        assert lay.fused_state == 0 and lay.states_offset == lay.s_in_offset
+        assert binding.SCAN_ENGINES[lay.scan_engine] == "single_pass"
+    few = binding.workspace_layout(binding.make_dims(batch=1, seqlen=65536, nheads=32, headdim=64,
+                                                     dstate=128, ngroups=8, dtype="bf16"), 256)
+    assert few.single_pass == 0 and few.launches == 5
+    assert binding.SCAN_ENGINES[few.scan_engine] == "chunk_wide"
+    assert few.s_in_offset > few.states_offset
+    # an odd number of heads per group or dstate 64: not taken
+    for kw, q in ((dict(nheads=81, ngroups=1), 256), (dict(nheads=80, ngroups=1, dstate=64), 256)):
+        args = dict(batch=4, seqlen=4096, headdim=64, dstate=128, dtype="bf16")
+        args.update(kw)
+        assert binding.workspace_layout(binding.make_dims(**args), q).single_pass == 0, (kw, q)
+    # chunk_len 64 runs with 128-token chunks (two per tensor-core tile)
+    lay = binding.workspace_layout(binding.make_dims(batch=4, seqlen=4096, nheads=80, headdim=64,
+                                                     dstate=128, ngroups=1, dtype="bf16"), 64)
+    assert lay.single_pass == 1 and lay.chunk_len == 128
+
+
+def test_chunk_len_64_on_the_tensor_cores(lib):
+    """bf16 chunk_len 64 takes the tensor-core kernels with 128-token chunks when
+    T is a multiple of 128; otherwise, and for fp32, it keeps chunk_len 64."""
+    for n in (16, 32, 64, 128, 256):
+        lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), 64)
+        assert lay.tensor_core == 1 and lay.chunk_len == 128, n
+        assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", n
+    odd = binding.workspace_layout(binding.make_dims(2, 960, 8, 64, 128, 1, "bf16"), 64)
+    assert odd.chunk_len == 64
+    f32 = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, 128, 1, "f32"), 64)
+    assert f32.chunk_len == 64 and f32.tensor_core == 0
 
 
 @pytest.mark.parametrize("kw,chunk,code", [
-    (dict(seqlen=500), 128, 2),          # T % chunk_len != 0
+    (dict(seqlen=500), 128, 0),          # T % chunk_len != 0: the tail kernel takes the rest
+    (dict(seqlen=500, dtype="f32", dstate=24), 128, 3),  # ... with a dstate it cannot split
     (dict(nheads=6, ngroups=4), 128, 2),  # H % G != 0
     (dict(batch=0), 128, 2),
     (dict(dstate=-1), 128, 2),
@@ -142,7 +175,7 @@ def test_misaligned_pointer(lib, name):
 
 
 def test_bad_dims_before_pointers(lib):
-    assert call_forward(lib, dims(seqlen=100)) == 2
+    assert call_forward(lib, dims(nheads=6, ngroups=4)) == 2
     assert lib.ssd_forward(None, None, None, None, None, None, None, 128, None, None, None,
                            None) == 1
 
@@ -191,3 +224,38 @@ def test_binding_step_rejects_cpu_tensors():
     with pytest.raises(ValueError, match="CUDA"):
         binding.step(torch.zeros(1, 2, 16, 16), torch.zeros(1, 2, 16), torch.zeros(1, 2),
                      torch.zeros(2), torch.zeros(1, 1, 16), torch.zeros(1, 1, 16))
+
+
+def test_block_argument_checks(lib):
+    """ssd_forward_block rejects a deferred norm without rstd_out, a norm eps
+    <= 0, a misaligned neighbour pointer and a nonzero reserved field before
+    anything is launched or allocated."""
+    d = dims()
+    f = ctypes.c_void_p(FAKE)
+
+    def call(**kw):
+        o = binding.BlockOpts(**kw)
+        return lib.ssd_forward_block(ctypes.byref(d), f, f, f, f, f, None, 128, None, f, None,
+                                     ctypes.byref(o), None, 0, None)
+
+    assert call(norm_weight=FAKE, norm_eps=1e-5, norm_apply=0) == 1       # no rstd_out
+    assert call(norm_weight=FAKE, norm_eps=0.0, norm_apply=1) == 2         # eps <= 0
+    assert call(z=FAKE + 4) == 4
+    assert call(dt_bias=FAKE + 8) == 4
+    assert call(reserved0=1) == 2
+    # the dt transform adds one fp32 [B, T, H] array to the workspace
+    base = binding.workspace_bytes(d, 128)
+    assert binding.block_workspace_bytes(d, 128, False) == base
+    assert binding.block_workspace_bytes(d, 128, True) >= base + 2 * 512 * 8 * 4
+
+
+def test_ragged_length_layout(lib):
+    """A length that is not a multiple of chunk_len: the full chunks keep their
+    kernels, one launch more runs the tail, and the workspace holds the state
+    between them; shorter than one chunk, only the tail kernel runs."""
+    full = binding.workspace_layout(dims(seqlen=512), 128)
+    ragged = binding.workspace_layout(dims(seqlen=600), 128)
+    assert ragged.launches == full.launches + 1
+    assert ragged.total_bytes >= full.total_bytes + 2 * 8 * 64 * 128 * 4
+    short = binding.workspace_layout(dims(seqlen=100), 128)
+    assert short.launches == 1

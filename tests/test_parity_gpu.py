@@ -106,11 +106,13 @@ def test_bf16_shapes(oracle, shape, h0):
 
 
 def test_tensor_core_path_selected():
-    """bf16 with P = 64 runs the tcgen05 kernels (chunk_len >= 128 for the scan)."""
+    """bf16 with P = 64 runs the tcgen05 kernels for every chunk_len (64 as
+    128-token chunks) and dstate, and the scan engine is a tensor-core one."""
     for n in (16, 32, 64, 128, 256):
-        for q in (128, 256):
+        for q in (64, 128, 256):
             lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
             assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
+            assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (n, q)
     lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 32, 64, 1, "bf16"), 128)
     assert lay.tensor_core == 0
 
@@ -251,7 +253,7 @@ def test_workspace_entry_point_and_intermediates(oracle):
 # fused chunk_state + state_passing (enough (batch, head pair) units)
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("shape", [
-    dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=128, ngroups=1, chunk_len=128),
+    dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=64, ngroups=1, chunk_len=128),
     dict(batch=2, seqlen=256, nheads=96, headdim=64, dstate=64, ngroups=2, chunk_len=128),
     dict(batch=2, seqlen=512, nheads=90, headdim=64, dstate=16, ngroups=1, chunk_len=256),
     dict(batch=1, seqlen=256, nheads=93, headdim=64, dstate=32, ngroups=3, chunk_len=128),
@@ -267,7 +269,7 @@ def test_fused_state_path(oracle, shape, h0):
 
 def test_fused_state_intermediates(oracle):
     """s_in written by the fused kernel, against the fp64 chunked form."""
-    shape = dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=128, ngroups=1)
+    shape = dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=64, ngroups=1)
     inp = make_inputs(**shape, chunk_len=128, dtype="bf16", seed=18, init_state=True)
     a = to_dev(inp)
     lay = binding.workspace_layout(binding.make_dims(**shape, dtype="bf16"), 128)
@@ -282,6 +284,119 @@ def test_fused_state_intermediates(oracle):
     s_in = ws[lay.s_in_offset: lay.s_in_offset + 2 * n].view(torch.bfloat16)
     s_in = s_in.double().cpu().numpy().reshape(it["s_in"].shape)
     assert rel(s_in, it["s_in"]) < 2e-2
+
+
+# ---------------------------------------------------------------------------
+# the single-pass kernel (chunk state + state passing + scan in one launch)
+# ---------------------------------------------------------------------------
+def single_pass(shape):
+    d = binding.make_dims(**{k: shape[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
+                                                     "ngroups")}, dtype="bf16")
+    return binding.workspace_layout(d, shape["chunk_len"]).single_pass == 1
+
+
+SINGLE_SHAPES = [
+    # fewer (batch, pair) chains than SMs: one CTA walks each chain
+    dict(batch=1, seqlen=512, nheads=128, headdim=64, dstate=128, ngroups=1, chunk_len=256),
+    dict(batch=2, seqlen=1024, nheads=64, headdim=64, dstate=128, ngroups=4, chunk_len=128),
+    # more chains than SMs: tickets round-robin, states handed between CTAs
+    dict(batch=4, seqlen=1024, nheads=80, headdim=64, dstate=128, ngroups=1, chunk_len=256),
+    dict(batch=3, seqlen=768, nheads=112, headdim=64, dstate=128, ngroups=2, chunk_len=128),
+]
+
+
+@pytest.mark.parametrize("shape", SINGLE_SHAPES)
+@pytest.mark.parametrize("h0", [False, True])
+def test_single_pass_shapes(oracle, shape, h0):
+    assert single_pass(shape)
+    inp = make_inputs(**shape, dtype="bf16", seed=31, init_state=h0)
+    check_full(inp, oracle)
+
+
+def test_single_pass_no_skip_no_final(oracle):
+    shape = SINGLE_SHAPES[2]
+    inp = make_inputs(**shape, dtype="bf16", seed=32, init_state=True)
+    inp.D = None
+    check_full(inp, oracle, final=False)
+
+
+@pytest.mark.parametrize("shape", [SINGLE_SHAPES[0], SINGLE_SHAPES[3]])
+def test_single_pass_steep_and_zero_dt(oracle, shape):
+    """Per head: a decay steep enough that tiles go to the block-factored scan,
+    a decay range across the chunk (reference moved to the middle), zero dt on
+    a run of tokens, and a gentle decay, all in one launch."""
+    assert single_pass(shape)
+    inp = make_inputs(**shape, dtype="bf16", seed=33, init_state=True, h0_std=1.0)
+    rng = np.random.default_rng(33)
+    H = shape["nheads"]
+    A = inp.A.copy()
+    dt = inp.dt.copy()
+    A[0::4] = -16.0                                      # steep: tiles listed
+    dt[:, :, 0::4] = rng.uniform(0.2, 1.0, size=dt[:, :, 0::4].shape)
+    A[1::4] = -1.0                                       # ~e^-0.4 per token
+    dt[:, :, 1::4] = rng.uniform(0.3, 0.5, size=dt[:, :, 1::4].shape)
+    dt[:, 100:260, 2::4] = 0.0                           # zero dt: skip term only
+    A[3::4] = -0.01
+    inp.A, inp.dt = A.astype(np.float32), dt.astype(np.float32)
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    assert np.isfinite(y).all() and np.isfinite(f).all()
+    for h in range(min(H, 8)):
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
+    assert rel(y, yr) <= TOL["bf16"] and rel(f, fr) <= TOL["bf16"]
+
+
+def test_single_pass_final_aliases_init(oracle):
+    shape = SINGLE_SHAPES[2]
+    inp = make_inputs(**shape, dtype="bf16", seed=34, init_state=True)
+    a = to_dev(inp)
+    h = a["init_state"].clone()
+    y, _ = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=shape["chunk_len"],
+                           init_state=h, final_out=h)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    assert rel(y.double().cpu().numpy(), yr) <= 2e-2
+    assert rel(h.double().cpu().numpy(), fr) <= 2e-2
+
+
+def test_single_pass_repeated_calls_deterministic():
+    inp = make_inputs(**SINGLE_SHAPES[3], dtype="bf16", seed=35, init_state=True)
+    y1, f1 = run_gpu(inp)
+    y2, f2 = run_gpu(inp)
+    np.testing.assert_array_equal(y1, y2)
+    np.testing.assert_array_equal(f1, f2)
+
+
+# ---------------------------------------------------------------------------
+# lengths that are not a multiple of chunk_len: full chunks, then the tail
+# kernel from the state they leave (or from h0 when there is no full chunk)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [
+    dict(batch=2, seqlen=1000, nheads=8, headdim=64, dstate=128, ngroups=2, chunk_len=256, dtype="bf16"),
+    dict(batch=1, seqlen=600, nheads=128, headdim=64, dstate=128, ngroups=1, chunk_len=256, dtype="bf16"),
+    dict(batch=2, seqlen=100, nheads=4, headdim=64, dstate=64, ngroups=1, chunk_len=128, dtype="bf16"),
+    dict(batch=1, seqlen=700, nheads=2, headdim=64, dstate=256, ngroups=1, chunk_len=256, dtype="bf16"),
+    dict(batch=1, seqlen=300, nheads=2, headdim=16, dstate=16, ngroups=1, chunk_len=64, dtype="f32"),
+    dict(batch=2, seqlen=200, nheads=3, headdim=32, dstate=8, ngroups=3, chunk_len=32, dtype="f32"),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_ragged_lengths(oracle, shape, h0):
+    inp = make_inputs(**shape, seed=51, init_state=h0)
+    check_full(inp, oracle)
+
+
+def test_ragged_length_with_final_aliasing_init(oracle):
+    inp = make_inputs(2, 1000, 8, 64, 128, 2, 256, dtype="bf16", seed=52, init_state=True)
+    a = to_dev(inp)
+    h = a["init_state"].clone()
+    y, _ = binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=256,
+                           init_state=h, final_out=h)
+    torch.cuda.synchronize()
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    assert rel(y.double().cpu().numpy(), yr) <= 2e-2
+    assert rel(h.double().cpu().numpy(), fr) <= 2e-2
 
 
 # ---------------------------------------------------------------------------
