@@ -36,20 +36,23 @@
 // kernel writes s_in_c in bf16 for the listed chunk, and the block-factored
 // scan (k_tc_chunk_scan4.cu, list mode) computes those tiles' y afterwards.
 //
-// Per tile (128 tokens of one chunk of one chain), on the tensor cores:
-//   CB  C_k B_k^T      -> Y buffer (fp32), packed to bf16 P in TMEM by the
+// Per tile (128 tokens of one chunk of one chain), on the tensor cores, issued
+// in the order PX(k), Z(k), CB(k+1), CS(k):
+//   CB  C_k B_k^T      -> score buffer (fp32), packed in place to bf16 P by the
 //                         score warps with the causal mask (diagonal included)
 //   Z   X''_k^T B_k    -> ACC += (M = 128: both heads' P rows, N = dstate)
 //   PX  P X''_k        -> Y buffer (N = 128: both heads)
 //   CS  C_k S'^T       -> Y buffer += (S' read back from ACC, written into the
 //                         tile's B region once Z has read it)
 // Tensor memory (512 columns): Y buffers [0,128) and [128,256) alternating per
-// tile, ACC [256, 256 + N), P buffers [384,448) and [448,512).
+// tile, ACC [256, 256 + N), score buffer [384,512).  The Y buffers are released
+// by the epilogue two tiles ahead of their next use, so a slow epilogue does not
+// hold up the next tile's scores.
 //
-// Roles (14 warps, at most four per SM sub-partition, so 128 registers each):
-// warp 0 TMA producer; warp 1 MMA issuer; warps 2-5 scale x by g, then convert
-// the scores; warps 6-9 state (chain in/out, S' read-back); warps 10-13
-// epilogue (y = u Y + D x, staged and TMA-stored).
+// Roles (15 warps, at most four per SM sub-partition, so 128 registers each):
+// warp 0 x producer (TMA); warp 1 MMA issuer; warps 2-5 scale x by g, then
+// convert the scores; warps 6-9 state (chain in/out, S' read-back); warps 10-13
+// epilogue (y = u Y + D x, staged and TMA-stored); warp 14 C / B producer.
 #include <cmath>
 
 #include "common.cuh"
@@ -68,8 +71,14 @@ constexpr int kThreads = 480;
 constexpr int kRows = 128;
 constexpr uint32_t kColAcc = 256;
 __device__ __forceinline__ uint32_t ycol(int yb) { return yb ? 128u : 0u; }
-__device__ __forceinline__ uint32_t pcol(int yb) { return yb ? 448u : 384u; }
+// C_k B_k^T (fp32) and then, packed in place over its first 64 columns, the bf16
+// scores P_k; one buffer: C_{k+1} B_{k+1}^T is issued after P_k X''_k, and the
+// tensor pipe runs a thread's MMAs in issue order
+constexpr uint32_t kColCBP = 384;
 constexpr int kBarState = 1;  // named barrier of the four state warps
+// Descriptor step (16-byte units) to K step kk of a K-major 128-row operand:
+// 128-byte swizzle, 64-element slabs of 128 rows x 128 bytes
+__device__ __forceinline__ uint64_t kstep(int kk) { return uint64_t(((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4); }
 
 // Shared memory: a ring of kCBStages slots {C_k, B_k} (L2-resident inputs,
 // released once the tile's products are done; S'_k goes into the B_k half once
@@ -168,14 +177,13 @@ struct TileWalk {
     }
 };
 
-// fp32 32 x 32 block (one TMEM row per lane) -> bf16 pairs, all columns or,
-// on the diagonal, columns e <= lane only.
-template <bool kDiag>
-__device__ __forceinline__ void mask_pack(const uint32_t (&v)[32], int lane, uint32_t (&pk)[16]) {
+// fp32 32 x 32 block (one TMEM row per lane) -> bf16 pairs, keeping columns
+// e <= lim (lim = 32: all of them, -1: none) and zeroing the rest.
+__device__ __forceinline__ void mask_pack(const uint32_t (&v)[32], int lim, uint32_t (&pk)[16]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
-        const float a = (!kDiag || 2 * e <= lane) ? __uint_as_float(v[2 * e]) : 0.f;
-        const float b = (!kDiag || 2 * e + 1 <= lane) ? __uint_as_float(v[2 * e + 1]) : 0.f;
+        const float a = 2 * e <= lim ? __uint_as_float(v[2 * e]) : 0.f;
+        const float b = 2 * e + 1 <= lim ? __uint_as_float(v[2 * e + 1]) : 0.f;
         pk[e] = pack_bf16x2(a, b);
     }
 }
@@ -322,7 +330,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             const uint32_t idCS = idesc_bf16_f32(kRows, 128, 0, 0);
             // one tile of lookahead: C_{k+1} B_{k+1}^T is issued between tile k's
             // Z and its C S'^T, so tile k+1's score conversion overlaps tile k's
-            // state hand-off
+            // state hand-off (it overwrites P_k only after P_k X''_k in the pipe)
             uint32_t ntot = 0;
             for (int sg = 0; sg < R.nseg; ++sg) {
                 const Seg T = seg_at(R, sg, d);
@@ -330,15 +338,13 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             }
             auto issue_cb = [&](uint32_t t) -> bool {
                 const int yb = t & 1;
-                if (!mbar_wait(&cb_full[t % kCBS], (t / kCBS) & 1, err) ||
-                    !mbar_wait(&y_free[yb], ((t >> 1) & 1) ^ 1, err))
-                    return false;
+                if (!mbar_wait(&cb_full[t % kCBS], (t / kCBS) & 1, err)) return false;
                 tc_fence_after();
                 const uint32_t cA = smem_u32(cb_at(t)), bA = cA + L::kCB;
-#pragma unroll
+                const uint64_t dC = kmajor_desc(cA, 0, kRows, NS), dB = kmajor_desc(bA, 0, kRows, NS);
+#pragma unroll 1
                 for (int kk = 0; kk < NS / 16; ++kk)
-                    mma_bf16_ss(tmem + ycol(yb), kmajor_desc(cA, kk, kRows, NS), kmajor_desc(bA, kk, kRows, NS),
-                                idCB, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + kColCBP, dC + kstep(kk), dB + kstep(kk), idCB, kk > 0 ? 1u : 0u);
                 mma_commit(&cbm_done[yb]);
                 return true;
             };
@@ -350,28 +356,32 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 const uint32_t cA = smem_u32(cb_at(kt)), bA = cA + L::kCB, xA = smem_u32(x_at(kt));
                 const uint32_t yacc = tmem + ycol(yb);
                 // Y = P X''_k (needs no state)
-                if (!mbar_wait(&scaled[xs], xph, err) || !mbar_wait(&p_ready[yb], yph, err)) { ok = false; break; }
+                // (the Y buffer is free once the epilogue has read tile kt - 2)
+                if (!mbar_wait(&scaled[xs], xph, err) || !mbar_wait(&p_ready[yb], yph, err) ||
+                    !mbar_wait(&y_free[yb], yph ^ 1, err)) { ok = false; break; }
                 tc_fence_after();
-#pragma unroll
+                // X''_k is MN-major (16 tokens = 2048 bytes per K step); B_k too for Z
+                const uint64_t dX = smem_desc(xA, kRows * 128, 1024, kSw128);
+                const uint64_t dBm = smem_desc(bA, kRows * 128, 1024, kSw128);
+#pragma unroll 1
                 for (int kk = 0; kk < kRows / 16; ++kk)
-                    mma_bf16_ts(yacc, tmem + pcol(yb) + kk * 8, smem_desc(xA + kk * 2048, kRows * 128, 1024, kSw128),
-                                idPX, kk > 0 ? 1u : 0u);
+                    mma_bf16_ts(yacc, tmem + kColCBP + kk * 8, dX + kk * 128, idPX, kk > 0 ? 1u : 0u);
                 // Z: ACC (= S'_k, kept there by the state warps) += X''_k^T B_k
                 if (!mbar_wait(acc_ready, kt & 1, err)) { ok = false; break; }
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < kRows / 16; ++kk)
-                    mma_bf16_ss(tmem + kColAcc, smem_desc(xA + kk * 2048, kRows * 128, 1024, kSw128),
-                                smem_desc(bA + kk * 2048, kRows * 128, 1024, kSw128), idZ, 1u);
+                    mma_bf16_ss(tmem + kColAcc, dX + kk * 128, dBm + kk * 128, idZ, 1u);
                 mma_commit(z_done);
                 if (kt + 1 < ntot && !issue_cb(kt + 1)) { ok = false; break; }
                 // Y += C_k S'_k^T, S'_k (bf16) written by the state warps into the
                 // tile's B region once Z has read B_k
                 if (!mbar_wait(sp_ready, kt & 1, err)) { ok = false; break; }
                 tc_fence_after();
-#pragma unroll
+                const uint64_t dC = kmajor_desc(cA, 0, kRows, NS), dS = kmajor_desc(bA, 0, kRows, NS);
+#pragma unroll 1
                 for (int kk = 0; kk < NS / 16; ++kk)
-                    mma_bf16_ss(yacc, kmajor_desc(cA, kk, kRows, NS), kmajor_desc(bA, kk, 128, NS), idCS, 1u);
+                    mma_bf16_ss(yacc, dC + kstep(kk), dS + kstep(kk), idCS, 1u);
                 mma_commit(&acc_full[yb]);
                 mma_commit(&cb_free[cs]);
             }
@@ -410,14 +420,14 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 if (nxt.valid) load_g(nxt, gn);
                 if (!mbar_wait(&x_full[kt % kXS], (kt / kXS) & 1, err)) { ok = false; break; }
                 uint4 *q = reinterpret_cast<uint4 *>(x_at(kt));
-#pragma unroll
+#pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     uint4 v[8];
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) v[jj] = q[i + 128 * (8 * half + jj)];
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) {
-                        const float sc = gv[8 * half + jj];
+                        const float sc = half ? gv[8 + jj] : gv[jj];
                         uint4 o;
                         o.x = pack_bf16x2(bf16lo(v[jj].x) * sc, bf16hi(v[jj].x) * sc);
                         o.y = pack_bf16x2(bf16lo(v[jj].y) * sc, bf16hi(v[jj].y) * sc);
@@ -435,8 +445,10 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             const int yb = kt & 1;
             if (!mbar_wait(&cbm_done[yb], (kt >> 1) & 1, err)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t src = tmem + lane_base + ycol(yb), dst = tmem + lane_base + pcol(yb);
-#pragma unroll
+            // in place: each pass reads two 32-column blocks before it writes their
+            // 16 packed columns, which lie in blocks already read
+            const uint32_t src = tmem + lane_base + kColCBP, dst = src;
+#pragma unroll 1
             for (int cb = 0; cb < 4; cb += 2) {
                 uint32_t v0[32], v1[32];
                 if (cb <= qd) tmem_ld32_nowait(src + cb * 32, v0);
@@ -444,16 +456,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 tmem_wait_ld();
 #pragma unroll
                 for (int bb = 0; bb < 2; ++bb) {
+                    // column block cb + bb of row 32 qd + lane: below the diagonal
+                    // block all kept, on it columns <= lane, above it none
                     const int cbb = cb + bb;
+                    const int lim = cbb < qd ? 32 : (cbb == qd ? lane : -1);
                     uint32_t pk[16];
-                    if (cbb > qd) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    } else if (cbb < qd) {
-                        mask_pack<false>(bb ? v1 : v0, lane, pk);
-                    } else {
-                        mask_pack<true>(bb ? v1 : v0, lane, pk);
-                    }
+                    mask_pack(bb ? v1 : v0, lim, pk);
                     tmem_st16(dst + cbb * 16, pk);
                 }
             }
@@ -474,9 +482,15 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         uint32_t kt = 0;
         bool ok = true;
         uint32_t sp[NS / 2];
-        auto pack32 = [&](int seg, const float (&v)[32]) {
+        // sp = ACC (bf16 pairs): the one unrolled read-back, shared by every path
+        auto load_sp = [&]() {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) sp[seg * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            for (int seg = 0; seg < NS / 32; ++seg) {
+                float v[32];
+                tmem_ld32(tacc + seg * 32, v);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sp[seg * 16 + e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            }
         };
         auto put_bf16_row = [&](__nv_bfloat16 *dst, const float (&v)[32]) {
             uint4 *o = reinterpret_cast<uint4 *>(dst);
@@ -489,7 +503,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             const Seg T = seg_at(R, sg, d);
             const int h = 2 * T.p + jh;
             const int64_t row_off = ((int64_t(T.b) * d.H + h) * d.P + p) * NS;
-            // ---- ticket start: S'_0 = e^r s_in_c0 from h0 or the chain slot ----
+            // ---- ticket start: ACC = S'_0 = e^r s_in_c0 from h0 or the chain slot ----
             {
                 const float *gqh = gq + ((int64_t(T.b) * d.H + h) * d.nc + T.c0) * ngq;
                 const bool steep = __ldg(gqh + Q) != 0.f || (ntile == 2 && __ldg(gqh + Q + 1) != 0.f);
@@ -506,34 +520,28 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     src = chain + row_off;
                 }
                 __nv_bfloat16 *sin_row = steep ? s_in + off_state(d, T.b, T.c0, h) + int64_t(p) * NS : nullptr;
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    // half a row per round trip: 16 loads in flight
-                    float v[NS / 2];
+#pragma unroll 1
+                for (int seg = 0; seg < NS / 32; ++seg) {
+                    float v[32];
                     if (src) {
 #pragma unroll
-                        for (int q4 = 0; q4 < NS / 8; ++q4) {
-                            const float4 *s4 = reinterpret_cast<const float4 *>(src) + hf * (NS / 8) + q4;
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 *s4 = reinterpret_cast<const float4 *>(src) + seg * 8 + q4;
                             const float4 t4 = T.c0 == 0 ? __ldg(s4) : __ldcg(s4);
                             v[4 * q4] = t4.x; v[4 * q4 + 1] = t4.y; v[4 * q4 + 2] = t4.z; v[4 * q4 + 3] = t4.w;
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < NS / 2; ++e) v[e] = 0.f;
+                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
                     }
+                    if (sin_row) put_bf16_row(sin_row + seg * 32, v);
 #pragma unroll
-                    for (int sg = 0; sg < NS / 64; ++sg) {
-                        float *vv = v + sg * 32;
-                        const int seg = hf * (NS / 64) + sg;
-                        if (sin_row) put_bf16_row(sin_row + seg * 32, *reinterpret_cast<const float(*)[32]>(vv));
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) vv[e] *= er;
-                        tmem_st16(tacc + seg * 32, reinterpret_cast<const uint32_t *>(vv));
-                        tmem_st16(tacc + seg * 32 + 16, reinterpret_cast<const uint32_t *>(vv + 16));
-                        pack32(seg, *reinterpret_cast<const float(*)[32]>(vv));
-                    }
+                    for (int e = 0; e < 32; ++e) v[e] *= er;
+                    tmem_st16(tacc + seg * 32, reinterpret_cast<const uint32_t *>(v));
+                    tmem_st16(tacc + seg * 32 + 16, reinterpret_cast<const uint32_t *>(v + 16));
                 }
                 tmem_wait_st();
+                load_sp();
                 tc_fence_before();
                 mbar_arrive(acc_ready);
             }
@@ -554,27 +562,41 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         fence_proxy_async_smem();
                         mbar_arrive(sp_ready);
                     }
-                    if (k + 1 < ntile) {
-                        // S'_{k+1} = ACC (the chunk's reference is unchanged)
+                    if (k + 1 == ntile) {
+                        // last tile of chunk c: s_in_{c+1} = exp(l_last - r) ACC
+                        const float ul = __expf(__ldg(lcum + off_lq(d, T.b, h, c) + Q - 1) - r);
+                        if (c + 1 == T.c1) {
+                            // ticket end: the state leaves through the chain slot (or final_state)
+                            const bool last = c + 1 == d.nc;
+                            float *dst = last ? (fin ? fin + row_off : nullptr) : chain + row_off;
+                            if (dst) {
+#pragma unroll 1
+                                for (int seg = 0; seg < NS / 32; ++seg) {
+                                    float v[32];
+                                    tmem_ld32(tacc + seg * 32, v);
 #pragma unroll
-                        for (int seg = 0; seg < NS / 32; ++seg) {
-                            float v[32];
-                            tmem_ld32(tacc + seg * 32, v);
-                            pack32(seg, v);
+                                    for (int q4 = 0; q4 < 8; ++q4) {
+                                        const float4 o = make_float4(v[4 * q4] * ul, v[4 * q4 + 1] * ul,
+                                                                     v[4 * q4 + 2] * ul, v[4 * q4 + 3] * ul);
+                                        if (last) reinterpret_cast<float4 *>(dst)[seg * 8 + q4] = o;
+                                        else __stcg(reinterpret_cast<float4 *>(dst) + seg * 8 + q4, o);
+                                    }
+                                }
+                            }
+                            tc_fence_before();
+                            if (!last) {
+                                __threadfence();
+                                named_barrier(kBarState, 128);
+                                if (m == 0) st_release(flags + int64_t(T.b) * np + T.p, unsigned(T.c1));
+                            }
+                            continue;
                         }
-                        tc_fence_before();
-                        mbar_arrive(acc_ready);
-                        continue;
-                    }
-                    // last tile of chunk c: s_in_{c+1} = exp(l_last - r) ACC
-                    const float ul = __expf(__ldg(lcum + off_lq(d, T.b, h, c) + Q - 1) - r);
-                    if (c + 1 < T.c1) {
-                        // next chunk of this ticket: S'_0 = e^{r_{c+1}} s_in_{c+1}, in place
+                        // next chunk of this ticket: ACC = S'_0 = e^{r_{c+1}} s_in_{c+1}, in place
                         const float *gqn = gqh + ngq;
                         const float en = __expf(__ldg(gqn + Q + 2));
                         const bool steep_n = __ldg(gqn + Q) != 0.f || (ntile == 2 && __ldg(gqn + Q + 1) != 0.f);
                         __nv_bfloat16 *sin_row = steep_n ? s_in + off_state(d, T.b, c + 1, h) + int64_t(p) * NS : nullptr;
-#pragma unroll
+#pragma unroll 1
                         for (int seg = 0; seg < NS / 32; ++seg) {
                             float v[32];
                             tmem_ld32(tacc + seg * 32, v);
@@ -585,36 +607,13 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                             for (int e = 0; e < 32; ++e) v[e] *= en;
                             tmem_st16(tacc + seg * 32, reinterpret_cast<const uint32_t *>(v));
                             tmem_st16(tacc + seg * 32 + 16, reinterpret_cast<const uint32_t *>(v + 16));
-                            pack32(seg, v);
                         }
                         tmem_wait_st();
-                        tc_fence_before();
-                        mbar_arrive(acc_ready);
-                        continue;
                     }
-                    // ticket end: the state leaves through the chain slot (or final_state)
-                    const bool last = c + 1 == d.nc;
-                    float *dst = last ? (fin ? fin + row_off : nullptr) : chain + row_off;
-#pragma unroll
-                    for (int seg = 0; seg < NS / 32; ++seg) {
-                        float v[32];
-                        tmem_ld32(tacc + seg * 32, v);
-                        if (dst) {
-#pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4) {
-                                const float4 o = make_float4(v[4 * q4] * ul, v[4 * q4 + 1] * ul, v[4 * q4 + 2] * ul,
-                                                             v[4 * q4 + 3] * ul);
-                                if (last) reinterpret_cast<float4 *>(dst)[seg * 8 + q4] = o;
-                                else __stcg(reinterpret_cast<float4 *>(dst) + seg * 8 + q4, o);
-                            }
-                        }
-                    }
+                    // S'_{k+1} = ACC
+                    load_sp();
                     tc_fence_before();
-                    if (!last) {
-                        __threadfence();
-                        named_barrier(kBarState, 128);
-                        if (m == 0) st_release(flags + int64_t(T.b) * np + T.p, unsigned(T.c1));
-                    }
+                    mbar_arrive(acc_ready);
                 }
             }
         }
@@ -622,10 +621,11 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         // ================================ epilogue ================================
         // y_t = u_t Y[t] + D_h x_t with u_t = exp(l_t - r); the skip term comes
         // from the scaled row as (D_h / g_t) X''_t, or from x in global memory
-        // where g_t is below 1e-30 (a zero dt).  The x rows are read first and
-        // the stage goes back to the producer; each warp then stages its 32 rows
-        // per head (128-byte swizzle) in its own blocks of the y staging area and
-        // writes them with its own TMA stores.
+        // where g_t is below 1e-30 (a zero dt).  Each thread owns row t of both
+        // heads and writes y_t over X''_t in the x slot (128-byte swizzle), a
+        // quarter row (head, 32 columns) at a time; each warp then writes its 32
+        // rows per head with its own TMA stores, and the slot goes back to the
+        // producer once those stores have read it.
         const int qd = warp & 3;
         const int t = qd * 32 + lane;
         const uint32_t lane_base = uint32_t(qd * 32) << 16;
@@ -650,7 +650,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         nxt.next(R, d, ntile);
         Raw ecur;
         if (cur.valid) load_raw(cur, ecur);
-        uint32_t kt = 0;
+        uint32_t kt = 0, freed = 0;  // x slots of tiles < freed have gone back
         bool ok = true;
         for (; cur.valid && ok; ++kt, cur.next(R, d, ntile), nxt.next(R, d, ntile)) {
                     const Seg T = cur.T;
@@ -670,44 +670,53 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         dg[jh] = (fb[jh] || Dh == 0.f) ? 0.f : Dh / ecur.gt[jh];
                     }
                     ecur = enx;
+                    // the previous tile's stores have read their slot by now (they were
+                    // issued a tile ago): it goes back to the producer before this
+                    // warp waits for the next accumulator
+                    if (kt > 0) {
+                        if (lane == 0) {
+                            bulk_wait_read();
+                            mbar_arrive(&x_free[(kt - 1) % kXS]);
+                        }
+                        freed = kt;
+                    }
+                    __syncwarp();
                     if (!mbar_wait(&acc_full[yb], (kt >> 1) & 1, err)) { ok = false; break; }
                     tc_fence_after();
-                    // this row's scaled x, head by head; y_t is then written over it in
-                    // place (each thread owns its row), and the x slot is written out
                     uint8_t *xslot = x_at(kt);
-#pragma unroll
-                    for (int jh = 0; jh < 2; ++jh) {
-                        if (stp[jh]) continue;  // computed by the block-factored scan
+#pragma unroll 1
+                    for (int qh = 0; qh < 4; ++qh) {
+                        const int jh = qh >> 1, hf = qh & 1;
+                        if (jh ? stp[1] : stp[0]) continue;  // computed by the block-factored scan
+                        const float uu = jh ? u[1] : u[0];
+                        float dgg = jh ? dg[1] : dg[0];
                         uint8_t *yrow = xslot + jh * (kRows * 128) + t * 128;
-                        uint4 xr[8];
-                        if (fb[jh]) {
+                        uint32_t a[32];
+                        tmem_ld32_nowait(tmem + lane_base + ycol(yb) + 64 * jh + 32 * hf, a);
+                        uint4 xr[4];
+                        if (jh ? fb[1] : fb[0]) {
                             // raw x from global memory (rare): D_h x_t
                             const uint4 *gx = reinterpret_cast<const uint4 *>(x + off_x(d, T.b, tok, 2 * T.p + jh));
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) xr[q] = __ldg(gx + q);
-                            dg[jh] = __ldg(Dskip + 2 * T.p + jh);
+                            for (int q = 0; q < 4; ++q) xr[q] = __ldg(gx + 4 * hf + q);
+                            dgg = __ldg(Dskip + 2 * T.p + jh);
                         } else {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                xr[q] = *reinterpret_cast<const uint4 *>(yrow + ((q ^ (t & 7)) << 4));
+                            for (int q = 0; q < 4; ++q)
+                                xr[q] = *reinterpret_cast<const uint4 *>(yrow + (((4 * hf + q) ^ (t & 7)) << 4));
                         }
+                        tmem_wait_ld();
+                        // chunks 4 hf .. 4 hf + 3 of the row: read above, written here
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            uint32_t a[32];
-                            tmem_ld32_nowait(tmem + lane_base + ycol(yb) + 64 * jh + 32 * hf, a);
-                            tmem_wait_ld();
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+                            uint32_t o[4];
 #pragma unroll
-                            for (int qq = 0; qq < 4; ++qq) {
-                                const int q = 4 * hf + qq;
-                                const uint32_t xw[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
-                                uint32_t o[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    o[e] = pack_bf16x2(
-                                        fmaf(u[jh], __uint_as_float(a[8 * qq + 2 * e]), dg[jh] * bf16lo(xw[e])),
-                                        fmaf(u[jh], __uint_as_float(a[8 * qq + 2 * e + 1]), dg[jh] * bf16hi(xw[e])));
-                                *reinterpret_cast<uint4 *>(yrow + ((q ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                            }
+                            for (int e = 0; e < 4; ++e)
+                                o[e] = pack_bf16x2(fmaf(uu, __uint_as_float(a[8 * q + 2 * e]), dgg * bf16lo(xw[e])),
+                                                   fmaf(uu, __uint_as_float(a[8 * q + 2 * e + 1]), dgg * bf16hi(xw[e])));
+                            *reinterpret_cast<uint4 *>(yrow + (((4 * hf + q) ^ (t & 7)) << 4)) =
+                                make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
                     tc_fence_before();
@@ -731,17 +740,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                             tma_store_3d(&tm_y, xslot + jh * (kRows * 128) + qd * 4096, 0, 2 * T.p + jh, row);
                         }
                         bulk_commit();
-                        // the previous tile's stores have read their slot: it goes back
-                        if (kt > 0) {
-                            bulk_wait_read_1();
-                            mbar_arrive(&x_free[(kt - 1) % kXS]);
-                        }
                     }
                     __syncwarp();
         }
         if (lane == 0) {
             bulk_wait_all();
-            if (kt > 0) mbar_arrive(&x_free[(kt - 1) % kXS]);
+            if (kt > freed) mbar_arrive(&x_free[(kt - 1) % kXS]);
         }
     }
     tc_fence_before();

@@ -69,8 +69,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // lasted kErrPollNs, so an ordinary wait never has a global load in flight
 // when its phase completes.
 constexpr uint64_t kErrPollNs = 20000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
-    if (mbar_try_wait(bar, parity)) return true;
+// The polling loop is one out-of-line copy per module: the many waits of a
+// warp-specialised kernel then share its instructions instead of each
+// inlining its own.
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, unsigned int *err) {
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -82,6 +84,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
     }
     if (err) atomicOr(err, 1u);
     return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, err);
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
