@@ -188,6 +188,15 @@ __device__ __forceinline__ void mask_pack(const uint32_t (&v)[32], int lim, uint
     }
 }
 
+// One arrival per warp on behalf of its 32 threads (the barriers count
+// threads): the warp barrier orders every lane's writes before the arriving
+// lane's release, and the barrier word takes one update instead of 32.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    const unsigned am = __activemask();
+    __syncwarp(am);
+    if ((threadIdx.x & 31) == unsigned(__ffs(am) - 1)) mbar_arrive_cnt(bar, 32);
+}
+
 __device__ __forceinline__ unsigned int ld_acquire(const unsigned int *f) {
     unsigned int v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
@@ -439,7 +448,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) gv[jj] = gn[jj];
                 fence_proxy_async_smem();
-                mbar_arrive(&scaled[kt % kXS]);
+                warp_arrive(&scaled[kt % kXS]);
             }
             // ---- masked scores: two blocks' loads in flight per wait ----
             const int yb = kt & 1;
@@ -467,7 +476,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&p_ready[yb]);
+            warp_arrive(&p_ready[yb]);
         }
     } else if (warp < 10) {
         // ================================= state =================================
@@ -543,7 +552,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 tmem_wait_st();
                 load_sp();
                 tc_fence_before();
-                mbar_arrive(acc_ready);
+                warp_arrive(acc_ready);
             }
             for (int c = T.c0; c < T.c1 && ok; ++c) {
                 const float *gqh = gq + ((int64_t(T.b) * d.H + h) * d.nc + c) * ngq;
@@ -560,7 +569,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                                                        (((ch & 7) ^ (m & 7)) << 4)) =
                                 make_uint4(sp[4 * ch], sp[4 * ch + 1], sp[4 * ch + 2], sp[4 * ch + 3]);
                         fence_proxy_async_smem();
-                        mbar_arrive(sp_ready);
+                        warp_arrive(sp_ready);
                     }
                     if (k + 1 == ntile) {
                         // last tile of chunk c: s_in_{c+1} = exp(l_last - r) ACC
@@ -613,7 +622,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     // S'_{k+1} = ACC
                     load_sp();
                     tc_fence_before();
-                    mbar_arrive(acc_ready);
+                    warp_arrive(acc_ready);
                 }
             }
         }
@@ -720,7 +729,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         }
                     }
                     tc_fence_before();
-                    mbar_arrive(&y_free[yb]);
+                    warp_arrive(&y_free[yb]);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {

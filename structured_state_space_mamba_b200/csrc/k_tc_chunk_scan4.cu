@@ -518,7 +518,7 @@ cudaError_t launch4(const Dims &d, const CUtensorMap *maps, int hpc, const float
 }  // namespace
 
 bool tc_chunk_scan4_supported(const Dims &d) {
-    const bool n_ok = d.N == 16 || d.N == 128;
+    const bool n_ok = d.N == 16 || d.N == 32 || d.N == 64 || d.N == 128;
     return d.P == 64 && n_ok && (d.Q == 128 || d.Q == 256) &&
            scan4_smem(d.Q, d.N).total <= 227 * 1024 &&
            int64_t(d.B) * d.nc * (d.Q / kRows) * d.H < (int64_t(1) << 31);

@@ -120,9 +120,10 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     plan->fused = plan->tc_state && plan->tc_scan && ssd::tc_state_fused_supported(d, kB200Sms);
     plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d) && ssd::tc_chunk_scan4_supported(d);
     // the single-pass kernel walks each (b, head pair) chain chunk by chunk: used
-    // when the chains fill at least kMinChainFrac of the SMs (fewer chains leave
-    // most SMs idle, and the four-kernel sequence is faster there)
-    plan->single = plan->scan5 && ssd::tc_chunk_fused_supported(d) &&
+    // when the chains fill at least kMinChainNum / kMinChainDen of the SMs (fewer
+    // chains leave most SMs idle, and the four-kernel sequence is faster there);
+    // the tiles it lists as steep go to the block-factored scan
+    plan->single = plan->tc_scan && ssd::tc_chunk_scan4_supported(d) && ssd::tc_chunk_fused_supported(d) &&
                    int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
     if (plan->single) plan->fused = false;
 
@@ -144,9 +145,10 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.s_in_dtype = plan->tc_scan ? SSD_BF16 : SSD_F32;
     off = align_up(off + st * (plan->tc_scan ? 2 : 4));
     plan->steep_offset = off;
-    if (plan->scan5) off = align_up(off + kAlign + sizeof(long long) * size_t(ssd::chunk_scan5_max_steep(d)));
+    const bool lists = plan->scan5 || plan->single;  // per-token factors and a steep-tile list
+    if (lists) off = align_up(off + kAlign + sizeof(long long) * size_t(ssd::chunk_scan5_max_steep(d)));
     plan->gq_offset = off;
-    if (plan->scan5) off = align_up(off + al * ssd::chunk_gq(d.Q));
+    if (lists) off = align_up(off + al * ssd::chunk_gq(d.Q));
     plan->chain_offset = off;
     if (plan->single) off = align_up(off + ssd::chunk_fused_chain_bytes(d));
     plan->flag_offset = off;
@@ -160,7 +162,8 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.fused_state = plan->fused ? 1 : 0;
     w.single_pass = plan->single ? 1 : 0;
     w.chunk_len = d.Q;
-    w.scan_engine = plan->scan5 ? (plan->single ? SSD_ENGINE_SINGLE_PASS : SSD_ENGINE_CHUNK_WIDE)
+    w.scan_engine = plan->single ? SSD_ENGINE_SINGLE_PASS
+                    : plan->scan5 ? SSD_ENGINE_CHUNK_WIDE
                     : plan->tc_scan ? (ssd::tc_chunk_scan4_supported(d) ? SSD_ENGINE_BLOCK_FACTORED
                                                                         : SSD_ENGINE_TILE)
                                     : SSD_ENGINE_SIMT;
@@ -242,7 +245,7 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     void *s_in = ws + pl.ws.s_in_offset;
     int *nsteep = reinterpret_cast<int *>(ws + pl.steep_offset);
     long long *steep_items = reinterpret_cast<long long *>(ws + pl.steep_offset + kAlign);
-    float *gq = pl.scan5 ? reinterpret_cast<float *>(ws + pl.gq_offset) : nullptr;
+    float *gq = (pl.scan5 || pl.single) ? reinterpret_cast<float *>(ws + pl.gq_offset) : nullptr;
     float *chain = pl.single ? reinterpret_cast<float *>(ws + pl.chain_offset) : nullptr;
     unsigned int *flags = pl.single ? reinterpret_cast<unsigned int *>(ws + pl.flag_offset) : nullptr;
     for (int stage = 0; stage < 4; ++stage) {

@@ -56,8 +56,9 @@ def test_single_pass_bytes_of_the_2p7b_layer_by_hand():
 
 
 def test_fused_layout_has_no_state_passing_traffic():
-    # the 130M-shaped layer at dstate 64: one wave of (batch, head pair) units
-    cfg = dict(WORKLOADS["mamba2_130m"], dstate=64)
+    # the 130M-shaped layer at dstate 32 (not a single-pass size): one wave of
+    # (batch, head pair) units
+    cfg = dict(WORKLOADS["mamba2_130m"], dstate=32)
     lay = layout(cfg)
     assert lay.fused_state == 1 and lay.single_pass == 0
     wm = bench.work_model(cfg, True, lay)

@@ -84,7 +84,7 @@ def test_fused_state_layout_for_many_head_pairs(lib):
     """0.6 x 148 <= (batch x head pairs) <= 148 SMs at a dstate the single-pass
     kernel does not take: chunk_state and state_passing run as one kernel, so no
     states region is reserved and one launch fewer is made."""
-    d = binding.make_dims(batch=8, seqlen=2048, nheads=24, headdim=64, dstate=64, ngroups=1,
+    d = binding.make_dims(batch=8, seqlen=2048, nheads=24, headdim=64, dstate=32, ngroups=1,
                           dtype="bf16")
     lay = binding.workspace_layout(d, 256)
     assert lay.fused_state == 1 and lay.single_pass == 0 and lay.tensor_core == 1
@@ -96,13 +96,14 @@ def test_fused_state_layout_for_many_head_pairs(lib):
 
 
 def test_single_pass_layout_selection(lib):
-    """bf16, P = 64, N = 128, chunk_len 128 / 256 and enough (batch, head pair)
-    chains (>= 40% of the 148 SMs) run the single-pass kernel: three launches,
-    no chunk-state region; few chains keep the four-kernel sequence."""
-    for b, h, q in ((4, 80, 256), (8, 24, 256), (8, 32, 128), (4, 32, 256)):
+    """bf16, P = 64, N = 64 or 128, chunk_len 128 / 256 and enough (batch, head
+    pair) chains (>= 40% of the 148 SMs) run the single-pass kernel: three
+    launches, no chunk-state region; few chains keep the four-kernel sequence."""
+    for b, h, q, n in ((4, 80, 256, 128), (8, 24, 256, 128), (8, 32, 128, 128), (4, 32, 256, 128),
+                       (4, 80, 256, 64), (8, 24, 128, 64)):
         lay = binding.workspace_layout(binding.make_dims(batch=b, seqlen=4096, nheads=h, headdim=64,
-                                                         dstate=128, ngroups=1, dtype="bf16"), q)
-        assert lay.single_pass == 1 and lay.launches == 3, (b, h, q)
+                                                         dstate=n, ngroups=1, dtype="bf16"), q)
+        assert lay.single_pass == 1 and lay.launches == 3, (b, h, q, n)
         assert lay.fused_state == 0 and lay.states_offset == lay.s_in_offset
         assert binding.SCAN_ENGINES[lay.scan_engine] == "single_pass"
     few = binding.workspace_layout(binding.make_dims(batch=1, seqlen=65536, nheads=32, headdim=64,
@@ -110,8 +111,9 @@ def test_single_pass_layout_selection(lib):
     assert few.single_pass == 0 and few.launches == 5
     assert binding.SCAN_ENGINES[few.scan_engine] == "chunk_wide"
     assert few.s_in_offset > few.states_offset
-    # an odd number of heads per group or dstate 64: not taken
-    for kw, q in ((dict(nheads=81, ngroups=1), 256), (dict(nheads=80, ngroups=1, dstate=64), 256)):
+    # an odd number of heads per group, dstate 32 or 256: not taken
+    for kw, q in ((dict(nheads=81, ngroups=1), 256), (dict(nheads=80, ngroups=1, dstate=32), 256),
+                  (dict(nheads=80, ngroups=1, dstate=256), 256)):
         args = dict(batch=4, seqlen=4096, headdim=64, dstate=128, dtype="bf16")
         args.update(kw)
         assert binding.workspace_layout(binding.make_dims(**args), q).single_pass == 0, (kw, q)

@@ -113,6 +113,10 @@ def test_tensor_core_path_selected():
             lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
             assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
             assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (n, q)
+            # dstate 32 / 64 take the block-factored scan, 256 the per-tile one
+            want = {32: "block_factored", 64: "block_factored", 256: "tile"}.get(n)
+            if want:
+                assert binding.SCAN_ENGINES[lay.scan_engine] == want, (n, q)
     lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 32, 64, 1, "bf16"), 128)
     assert lay.tensor_core == 0
 
@@ -123,7 +127,7 @@ def test_no_skip_term(oracle):
     check_full(inp, oracle)
 
 
-@pytest.mark.parametrize("dstate", [16, 128])
+@pytest.mark.parametrize("dstate", [16, 32, 64, 128])
 def test_decay_range_across_the_chunk(oracle, dstate):
     """Per-token decays of about e^-0.4 (head 0): each 128-token tile spans ~e^-51
     but the 256-token chunk ~e^-102, so the chunk-wide scan moves its reference
@@ -253,8 +257,8 @@ def test_workspace_entry_point_and_intermediates(oracle):
 # fused chunk_state + state_passing (enough (batch, head pair) units)
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("shape", [
-    dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=64, ngroups=1, chunk_len=128),
-    dict(batch=2, seqlen=256, nheads=96, headdim=64, dstate=64, ngroups=2, chunk_len=128),
+    dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=32, ngroups=1, chunk_len=128),
+    dict(batch=2, seqlen=256, nheads=96, headdim=64, dstate=32, ngroups=2, chunk_len=128),
     dict(batch=2, seqlen=512, nheads=90, headdim=64, dstate=16, ngroups=1, chunk_len=256),
     dict(batch=1, seqlen=256, nheads=93, headdim=64, dstate=32, ngroups=3, chunk_len=128),
 ])
@@ -269,7 +273,7 @@ def test_fused_state_path(oracle, shape, h0):
 
 def test_fused_state_intermediates(oracle):
     """s_in written by the fused kernel, against the fp64 chunked form."""
-    shape = dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=64, ngroups=1)
+    shape = dict(batch=3, seqlen=512, nheads=64, headdim=64, dstate=32, ngroups=1)
     inp = make_inputs(**shape, chunk_len=128, dtype="bf16", seed=18, init_state=True)
     a = to_dev(inp)
     lay = binding.workspace_layout(binding.make_dims(**shape, dtype="bf16"), 128)
@@ -302,6 +306,9 @@ SINGLE_SHAPES = [
     # more chains than SMs: tickets round-robin, states handed between CTAs
     dict(batch=4, seqlen=1024, nheads=80, headdim=64, dstate=128, ngroups=1, chunk_len=256),
     dict(batch=3, seqlen=768, nheads=112, headdim=64, dstate=128, ngroups=2, chunk_len=128),
+    # dstate 64: one 64-column slab per operand, a four-stage x ring
+    dict(batch=2, seqlen=1024, nheads=96, headdim=64, dstate=64, ngroups=1, chunk_len=256),
+    dict(batch=4, seqlen=512, nheads=80, headdim=64, dstate=64, ngroups=2, chunk_len=128),
 ]
 
 
@@ -320,7 +327,7 @@ def test_single_pass_no_skip_no_final(oracle):
     check_full(inp, oracle, final=False)
 
 
-@pytest.mark.parametrize("shape", [SINGLE_SHAPES[0], SINGLE_SHAPES[3]])
+@pytest.mark.parametrize("shape", [SINGLE_SHAPES[0], SINGLE_SHAPES[3], SINGLE_SHAPES[5]])
 def test_single_pass_steep_and_zero_dt(oracle, shape):
     """Per head: a decay steep enough that tiles go to the block-factored scan,
     a decay range across the chunk (reference moved to the middle), zero dt on
