@@ -36,8 +36,9 @@
 // kernel writes s_in_c in bf16 for the listed chunk, and the block-factored
 // scan (k_tc_chunk_scan4.cu, list mode) computes those tiles' y afterwards.
 //
-// Per tile (128 tokens of one chunk of one chain), on the tensor cores, issued
-// in the order PX(k), Z(k), CB(k+1), CS(k):
+// Per tile (128 tokens of one chunk of one chain), on the tensor cores, from
+// two issuing threads: PX(k) then CB(k+1) from one, Z(k) then CS(k) from the
+// other (CS(k) once PX(k), which initialises the same Y buffer, is done):
 //   CB  C_k B_k^T      -> score buffer (fp32), packed in place to bf16 P by the
 //                         score warps with the causal mask (diagonal included)
 //   Z   X''_k^T B_k    -> ACC += (M = 128: both heads' P rows, N = dstate)
@@ -49,10 +50,11 @@
 // by the epilogue two tiles ahead of their next use, so a slow epilogue does not
 // hold up the next tile's scores.
 //
-// Roles (15 warps, at most four per SM sub-partition, so 128 registers each):
-// warp 0 x producer (TMA); warp 1 MMA issuer; warps 2-5 scale x by g, then
+// Roles (16 warps, four per SM sub-partition, so 128 registers each): warp 0 x
+// producer (TMA); warp 1 MMA issuer for PX and CB; warps 2-5 scale x by g, then
 // convert the scores; warps 6-9 state (chain in/out, S' read-back); warps 10-13
-// epilogue (y = u Y + D x, staged and TMA-stored); warp 14 C / B producer.
+// epilogue (y = u Y + D x, staged and TMA-stored); warp 14 C / B producer;
+// warp 15 MMA issuer for Z and CS.
 #include <cmath>
 
 #include "common.cuh"
@@ -67,7 +69,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 480;
+constexpr int kThreads = 512;
 constexpr int kRows = 128;
 constexpr uint32_t kColAcc = 256;
 __device__ __forceinline__ uint32_t ycol(int yb) { return yb ? 128u : 0u; }
@@ -95,7 +97,7 @@ struct FusedLayout {
     static constexpr int kXStages = NS >= 128 ? 3 : 4;
     static constexpr uint32_t kXOff = kCBStages * kCBSlot;
     static constexpr uint32_t kBar = kXOff + kXStages * kX;
-    static constexpr uint32_t kTotal = kBar + 256 + 1024;
+    static constexpr uint32_t kTotal = kBar + 512 + 1024;
 };
 
 // Work assignment.  The (chain, chunk) items, chain = (b, head pair p), are
@@ -244,7 +246,8 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     uint64_t *x_full = cb_free + kCBS, *scaled = x_full + kXS, *x_free = scaled + kXS;  // [kXS]
     uint64_t *cbm_done = x_free + kXS, *p_ready = cbm_done + 2, *acc_full = p_ready + 2,
              *y_free = acc_full + 2;                                             // [2]
-    uint64_t *acc_ready = y_free + 2, *z_done = acc_ready + 1, *sp_ready = z_done + 1, *done = sp_ready + 1;
+    uint64_t *px_done = y_free + 2;                                           // [2]
+    uint64_t *acc_ready = px_done + 2, *z_done = acc_ready + 1, *sp_ready = z_done + 1, *done = sp_ready + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
     volatile int *state_ok = reinterpret_cast<volatile int *>(done + 2);
     auto cb_at = [&](uint32_t kt) { return smem + (kt % kCBS) * L::kCBSlot; };
@@ -270,11 +273,12 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             mbar_init(&p_ready[i], 128);
             mbar_init(&acc_full[i], 1);
             mbar_init(&y_free[i], 128);
+            mbar_init(&px_done[i], 1);
         }
         mbar_init(acc_ready, 128);
         mbar_init(z_done, 1);
         mbar_init(sp_ready, 128);
-        mbar_init(done, 1);
+        mbar_init(done, 2);  // both MMA issuers
         fence_mbar_init();
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_b);
@@ -331,15 +335,14 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 mbar_wait(xp ? &x_full[i % kXS] : &cb_full[i % kCBS], (i / depth) & 1, nullptr);
         }
     } else if (warp == 1) {
-        // =============================== MMA issuer ===============================
+        // ====================== MMA issuer: P X'' and C B^T ======================
         if (lane == 0) {
             const uint32_t idCB = idesc_bf16_f32(kRows, kRows, 0, 0);
-            const uint32_t idZ = idesc_bf16_f32(128, NS, 1, 1);
             const uint32_t idPX = idesc_bf16_f32(kRows, 128, 0, 1);
-            const uint32_t idCS = idesc_bf16_f32(kRows, 128, 0, 0);
-            // one tile of lookahead: C_{k+1} B_{k+1}^T is issued between tile k's
-            // Z and its C S'^T, so tile k+1's score conversion overlaps tile k's
-            // state hand-off (it overwrites P_k only after P_k X''_k in the pipe)
+            // one tile of lookahead: C_{k+1} B_{k+1}^T is issued right after P_k
+            // X''_k, so tile k+1's score conversion overlaps tile k's state
+            // hand-off (it overwrites P_k only after P_k X''_k in this thread's
+            // issue order, which the tensor pipe keeps)
             uint32_t ntot = 0;
             for (int sg = 0; sg < R.nseg; ++sg) {
                 const Seg T = seg_at(R, sg, d);
@@ -359,33 +362,53 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
             };
             bool ok = ntot == 0 || issue_cb(0);
             for (uint32_t kt = 0; kt < ntot && ok; ++kt) {
+                const uint32_t xs = kt % kXS, xph = (kt / kXS) & 1;
+                const int yb = kt & 1;
+                const uint32_t yph = (kt >> 1) & 1;
+                const uint32_t xA = smem_u32(x_at(kt));
+                const uint32_t yacc = tmem + ycol(yb);
+                if (!mbar_wait(&scaled[xs], xph, err) || !mbar_wait(&p_ready[yb], yph, err) ||
+                    !mbar_wait(&y_free[yb], yph ^ 1, err)) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t dX = smem_desc(xA, kRows * 128, 1024, kSw128);
+#pragma unroll 1
+                for (int kk = 0; kk < kRows / 16; ++kk)
+                    mma_bf16_ts(yacc, tmem + kColCBP + kk * 8, dX + kk * 128, idPX, kk > 0 ? 1u : 0u);
+                mma_commit(&px_done[yb]);
+                if (kt + 1 < ntot && !issue_cb(kt + 1)) { ok = false; break; }
+            }
+            mma_commit(done);
+            mbar_wait(done, 0, nullptr);
+        }
+    } else if (warp == 15) {
+        // ====================== second MMA issuer: Z and C S'^T ======================
+        if (lane == 0) {
+            const uint32_t idZ = idesc_bf16_f32(128, NS, 1, 1);
+            const uint32_t idCS = idesc_bf16_f32(kRows, 128, 0, 0);
+            uint32_t ntot = 0;
+            for (int sg = 0; sg < R.nseg; ++sg) {
+                const Seg T = seg_at(R, sg, d);
+                ntot += uint32_t(T.c1 - T.c0) * ntile;
+            }
+            bool ok = true;
+            for (uint32_t kt = 0; kt < ntot && ok; ++kt) {
                 const uint32_t cs = kt % kCBS, xs = kt % kXS, xph = (kt / kXS) & 1;
                 const int yb = kt & 1;
                 const uint32_t yph = (kt >> 1) & 1;
                 const uint32_t cA = smem_u32(cb_at(kt)), bA = cA + L::kCB, xA = smem_u32(x_at(kt));
                 const uint32_t yacc = tmem + ycol(yb);
-                // Y = P X''_k (needs no state)
-                // (the Y buffer is free once the epilogue has read tile kt - 2)
-                if (!mbar_wait(&scaled[xs], xph, err) || !mbar_wait(&p_ready[yb], yph, err) ||
-                    !mbar_wait(&y_free[yb], yph ^ 1, err)) { ok = false; break; }
+                // Z: ACC += X''_k^T B_k
+                if (!mbar_wait(&cb_full[cs], (kt / kCBS) & 1, err) || !mbar_wait(&scaled[xs], xph, err) ||
+                    !mbar_wait(acc_ready, kt & 1, err)) { ok = false; break; }
                 tc_fence_after();
-                // X''_k is MN-major (16 tokens = 2048 bytes per K step); B_k too for Z
                 const uint64_t dX = smem_desc(xA, kRows * 128, 1024, kSw128);
                 const uint64_t dBm = smem_desc(bA, kRows * 128, 1024, kSw128);
 #pragma unroll 1
                 for (int kk = 0; kk < kRows / 16; ++kk)
-                    mma_bf16_ts(yacc, tmem + kColCBP + kk * 8, dX + kk * 128, idPX, kk > 0 ? 1u : 0u);
-                // Z: ACC (= S'_k, kept there by the state warps) += X''_k^T B_k
-                if (!mbar_wait(acc_ready, kt & 1, err)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll 1
-                for (int kk = 0; kk < kRows / 16; ++kk)
                     mma_bf16_ss(tmem + kColAcc, dX + kk * 128, dBm + kk * 128, idZ, 1u);
                 mma_commit(z_done);
-                if (kt + 1 < ntot && !issue_cb(kt + 1)) { ok = false; break; }
-                // Y += C_k S'_k^T, S'_k (bf16) written by the state warps into the
-                // tile's B region once Z has read B_k
-                if (!mbar_wait(sp_ready, kt & 1, err)) { ok = false; break; }
+                // Y += C_k S'_k^T once P X''_k (the other issuer) is done
+                if (!mbar_wait(sp_ready, kt & 1, err) || !mbar_wait(&px_done[yb], yph, err)) { ok = false; break; }
                 tc_fence_after();
                 const uint64_t dC = kmajor_desc(cA, 0, kRows, NS), dS = kmajor_desc(bA, 0, kRows, NS);
 #pragma unroll 1
