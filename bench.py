@@ -3,7 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 A step is one ssd_forward call -- the whole hot path (ssd_chunk_cumsum,
-ssd_chunk_state, ssd_state_passing, ssd_chunk_scan) -- over one batch of the
+ssd_chunk_state, ssd_state_passing, ssd_chunk_scan; on this layer the last
+three run as the library's single-pass kernel) -- over one batch of the
 Mamba-2-2.7B-shaped layer (B=4, T=4096, H=80, P=64, N=128, G=1, chunk 256,
 bf16 x/B/C, fp32 dt/A/D, final state returned), seeded synthetic inputs resident
 in HBM.  Every step's inputs and outputs exceed L2 (x and y are 168 MB each,
@@ -50,7 +51,10 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # Keyed by (workload, kernel, library version): a capture stands only for the
 # build it was taken from, so a rebuilt kernel reports traffic None until it is
 # captured again.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/full_chunk_fused_mamba2_2p7b.md: 187.96 MB read + 137.98 MB written
+    ("mamba2_2p7b", "ssd_chunk_fused", "ssd-b200 0.2.1 sm_100a"): 325_942_784,
+}
 
 
 def ncu_traffic(workload, kernel):
@@ -90,6 +94,9 @@ def work_model(cfg, final_state=True, lay=None):
     comp = (2 * x_bytes + bc_bytes + dt_bytes + 2 * H * 4
             + (state_bytes if cfg.get("init_state") else 0)
             + (state_bytes if final_state else 0))
+    if cfg.get("block"):
+        # the block's neighbours: z in, the norm weight [H*P] and dt_bias [H]
+        comp += x_bytes + H * P * 4 + H * 4
     # per-kernel algorithmic bytes (what each kernel must read and write, with the
     # element sizes of this call's workspace layout)
     st_elems = B * nc * H * P * N
@@ -334,7 +341,9 @@ def config_block(cfg, name, l2_note=None):
             "chunk_len": cfg["chunk_len"], "init_state": bool(cfg.get("init_state")),
             "final_state": bool(cfg.get("final_state", True)),
             "l2": l2_note if l2_note is not None else l2_policy(cfg, L2_FALLBACK_BYTES)[1],
-            "parallelism": "replicas"}
+            "parallelism": "replicas",
+            **({"block": "softplus(dt + dt_bias), y * silu(z), RMSNorm over H*P"}
+               if cfg.get("block") else {})}
 
 
 # ---------------------------------------------------------------------------
@@ -365,9 +374,33 @@ def run_gpu(args, cfg, rank, world, local_rank):
     lay = binding.workspace_layout(dims, inp.chunk_len)
     ws = torch.empty(lay.total_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    block = bool(cfg.get("block"))
+    if block:
+        # the block's raw inputs: dt_raw = softplus^-1(dt) - dt_bias, so the scan
+        # sees the workload's own step sizes; z ~ N(0, 1); weight 1 + 0.1 N(0, 1)
+        rng = np.random.default_rng(3000)
+        bias = rng.uniform(-0.5, 0.5, size=inp.A.shape).astype(np.float32)
+        dt_raw = (np.log(np.expm1(inp.dt.astype(np.float64))) - bias[None, None, :]).astype(np.float32)
+        zh = rng.standard_normal(inp.x.shape).astype(np.float32)
+        wn = (1.0 + 0.1 * rng.standard_normal(inp.x.shape[2] * inp.x.shape[3])).astype(np.float32)
+        pinned["dt"] = torch.from_numpy(dt_raw).pin_memory()
+        pinned["z"] = torch.from_numpy(zh).to(tt).pin_memory()
+        d["dt"] = pinned["dt"].to(dev)
+        d["z"] = pinned["z"].to(dev)
+        d["dt_plain"] = torch.from_numpy(inp.dt).to(dev)
+        bias_d = torch.from_numpy(bias).to(dev)
+        wn_d = torch.from_numpy(wn).to(dev)
+        ws_block = torch.empty(binding.block_workspace_bytes(dims, inp.chunk_len, True),
+                               dtype=torch.uint8, device=dev)
 
     def step(stage=None):
-        binding.forward(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+        if block and stage is None:
+            binding.forward_block(d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                                  chunk_len=inp.chunk_len, init_state=d.get("init_state"),
+                                  dt_bias=bias_d, dt_softplus=True, z=d["z"], norm_weight=wn_d,
+                                  out=y, final_out=fin, workspace=ws_block)
+            return
+        binding.forward(d["x"], d["dt_plain"] if block else d["dt"], d["A"], d["B"], d["C"], D=d["D"],
                         chunk_len=inp.chunk_len, init_state=d.get("init_state"), out=y,
                         final_out=fin, workspace=ws, stage=stage)
 
@@ -457,6 +490,20 @@ def run_gpu(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     kern_ms = {names[s]: statistics.mean(ev[k][s].elapsed_time(ev[k][s + 1]) for k in range(args.steps))
                for s in range(nst) if names[s] is not None}
+    if block:
+        # the block's gate and norm (one kernel after the scan): the block step
+        # minus the plain scan's stages, on the same inputs
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev2:
+            torch.cuda._sleep(1_000_000)
+            a.record(stream)
+            step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        blk = statistics.mean(a.elapsed_time(b) for a, b in ev2)
+        kern_ms["ssd_gate_norm"] = max(blk - sum(kern_ms.values()), 1e-6)
     barrier()
 
     # ---- end to end through the public call, host buffers ------------------
@@ -492,6 +539,10 @@ def run_gpu(args, cfg, rank, world, local_rank):
     tokens_step = inp.x.shape[0] * inp.x.shape[1]
     value = job_rate(world, tokens_step, args.steps, ms_total)
     wm = work_model(cfg, final_state=want_final, lay=lay)
+    if block:
+        gn = 3 * inp.x.size * (2 if inp.dtype == "bf16" else 4) + inp.x.shape[2] * inp.x.shape[3] * 4
+        wm["per_kernel_comp"]["ssd_gate_norm"] = gn
+        wm["per_kernel_bytes"]["ssd_gate_norm"] = gn
     peaks, peak_src = load_peaks()
     top = max(kern_ms, key=kern_ms.get)
     bound = "hbm"
@@ -525,9 +576,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
                           "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, "
                                    f"bf16 {peaks['bf16_tflops']} TF/s"},
         "kernels_us": {k: v * 1e3 for k, v in kern_ms.items()},
-        "launch": launch_mode,
+        "launch": launch_mode + (" (ssd_forward_block)" if block else ""),
         "ms_per_step_direct_calls": ms_direct / args.steps,
-        "gpu_launches": args.steps * lay.launches,
+        "gpu_launches": args.steps * (lay.launches + (1 if block else 0)),
         "tensor_core": bool(lay.tensor_core),
         "fused_state": bool(lay.fused_state),
         "single_pass": bool(lay.single_pass),
@@ -681,11 +732,16 @@ def main():
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (ssd_step) on its own shape instead of the scan")
+    ap.add_argument("--block", action="store_true",
+                    help="time ssd_forward_block: softplus(dt + dt_bias), the scan, y * silu(z) "
+                         "and RMSNorm over each token's H * P values")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = dict(WORKLOADS[args.workload])
     cfg.setdefault("final_state", True)
+    if args.block:
+        cfg["block"] = True
     if args.batch is not None:
         cfg["batch"] = args.batch
 

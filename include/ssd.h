@@ -12,8 +12,11 @@
  * Constraint"), evaluated blockwise as the chunked SSD algorithm (aifetchly
  * blog "Mamba-2 Architecture: State Space Duality Explained", section "The
  * Chunked SSD Algorithm"): the masked product (L o C B^T) X inside each chunk of
- * chunk_len tokens, and the state recurrence between chunks.  The kernels are
- * ssd_chunk_cumsum, ssd_chunk_state, ssd_state_passing and ssd_chunk_scan.
+ * chunk_len tokens, and the state recurrence between chunks.  The steps are
+ * ssd_chunk_cumsum, ssd_chunk_state, ssd_state_passing and ssd_chunk_scan; on
+ * the tensor-core path with enough (batch, head pair) chains the last three
+ * run as ONE kernel that carries each chain's state on chip from chunk to
+ * chunk (see single_pass under ssd_workspace_layout).
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers to contiguous row-major memory,
@@ -293,9 +296,9 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * reach memory, the states region is empty (states_offset == s_in_offset) and
  * stage 2 of ssd_forward_stage does nothing.
  * `single_pass` is 1 when chunk state, state passing and chunk scan run as ONE
- * kernel (bf16, headdim 64, dstate 128, chunk_len 128 / 256, an even number of
- * heads per group, and at least 40% as many (batch, head pair) chains as the
- * GPU has SMs): each chunk's state is carried to the next through an fp32
+ * kernel (bf16, headdim 64, dstate 64 or 128, chunk_len 128 / 256 (64 as 128),
+ * an even number of heads per group, and at least 40% as many (batch, head
+ * pair) chains as the GPU has SMs): each chunk's state is carried to the next through an fp32
  * slot per (batch, head) in the workspace, so neither the per-chunk states nor
  * the incoming states reach memory (w, alpha and states are not written, s_in
  * only for chunks with a tile the block-factored scan finishes).  Stage 1 of

@@ -215,7 +215,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     if (warp == 0) {
         // =============================== producer ===============================
         if (lane == 0) {
-            uint32_t si = 0, use = 0;
+            uint32_t si = 0, use = 0, nc_issued = 0, nb1_issued = 0;
             bool ok = true;
             for (long long i = i0; i < i1 && ok; ++si) {
                 const Run R = run_at(i, i1, d);
@@ -224,7 +224,6 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 // C_0 and B_0 into the next two stages, C_1 into its own buffer
                 // once the previous run's products are done
                 const uint32_t uc = use, ub = use + 1;
-                use += 2;
                 if (!mbar_wait(&stage_free[uc % kStages], ((uc / kStages) & 1) ^ 1, err) ||
                     !mbar_wait(&stage_free[ub % kStages], ((ub / kStages) & 1) ^ 1, err) ||
                     !mbar_wait(cb_smem_free, (si & 1) ^ 1, err))
@@ -233,18 +232,21 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 // these two uses carry no head: their head_full phases pass at once
                 mbar_arrive(&head_full[uc % kStages]);
                 mbar_arrive(&head_full[ub % kStages]);
+                use += 2;  // counted once armed (the exit drain waits on every counted use)
                 mbar_expect_tx(ld_c, uint32_t(ntile + 1) * kRows * N * 2);
                 for (int sl = 0; sl < kSlabs; ++sl) {
                     tma_load_3d(sc0 + sl * kRows * 128, &tm_c, ld_c, sl * 64, R.g, trow0);
                     tma_load_3d(sb + sl * kRows * 128, &tm_b, ld_c, sl * 64, R.g, trow0);
                     if (two) tma_load_3d(sC1 + sl * kRows * 128, &tm_c, ld_c, sl * 64, R.g, trow0 + kRows);
                 }
+                ++nc_issued;
                 if (two) {
                     // B of tile 1 into the same place once the tile-0 products are done
                     if (!mbar_wait(b0_free, si & 1, err)) break;
                     mbar_expect_tx(ld_b1, uint32_t(kRows) * N * 2);
                     for (int sl = 0; sl < kSlabs; ++sl)
                         tma_load_3d(sb + sl * kRows * 128, &tm_b, ld_b1, sl * 64, R.g, trow0 + kRows);
+                    ++nb1_issued;
                 }
                 for (int hi = 0; hi < R.len; ++hi, ++use) {
                     const int st = use % kStages;
@@ -263,11 +265,15 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                               &head_full[st]);
                 }
             }
-            // drain: every use issued has been consumed (so its loads landed)
+            // drain: the loads issued have landed before the CTA exits (their own
+            // completion barriers, so this holds on the early-out path too, where
+            // the consumers stop freeing stages)
             for (uint32_t k = 1; k <= kStages && k <= use; ++k) {
                 const uint32_t u = use - k;
-                mbar_wait(&stage_free[u % kStages], (u / kStages) & 1, nullptr);
+                mbar_wait(&head_full[u % kStages], (u / kStages) & 1, nullptr);
             }
+            if (nc_issued > 0) mbar_wait(ld_c, (nc_issued - 1) & 1, nullptr);
+            if (nb1_issued > 0) mbar_wait(ld_b1, (nb1_issued - 1) & 1, nullptr);
         }
     } else if (warp == 1) {
         // =============================== MMA issuer =============================

@@ -484,6 +484,6 @@ ssd_status_t ssd_device_status(void *stream) {
     return SSD_OK;
 }
 
-const char *ssd_version(void) { return "ssd-b200 0.2.0 sm_100a"; }
+const char *ssd_version(void) { return "ssd-b200 0.2.1 sm_100a"; }
 
 }  // extern "C"

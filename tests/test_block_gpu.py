@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from structured_state_space_mamba_b200 import binding
-from structured_state_space_mamba_b200.inputs import make_inputs, round_to_bf16
+from structured_state_space_mamba_b200.inputs import make_inputs, make_workload, round_to_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -108,3 +108,25 @@ def test_block_without_neighbours_equals_forward():
                                    return_final_state=True)
     torch.cuda.synchronize()
     assert torch.equal(y0, y1) and torch.equal(f0, f1)
+
+
+@pytest.mark.parametrize("name", ["mamba2_130m", "mamba2_2p7b"])
+def test_block_full_size_layers(oracle, name):
+    """The block entry point on the benchmark layers, every (batch, head) unit
+    compared: the raw dt is softplus^-1 of the workload's dt minus the bias, so
+    the scan runs on the workload's own step sizes (the single-pass kernel on
+    both layers)."""
+    inp = make_workload(name)
+    rng = np.random.default_rng(46)
+    bias = rng.uniform(-0.5, 0.5, size=inp.A.shape).astype(np.float32)
+    dt_raw = (np.log(np.expm1(inp.dt.astype(np.float64))) - bias[None, None, :]).astype(np.float32)
+    z = round_to_bf16(rng.standard_normal(inp.x.shape)).astype(np.float32)
+    w = (1.0 + 0.1 * rng.standard_normal(inp.x.shape[2] * inp.x.shape[3])).astype(np.float32)
+    out, fin, rstd = run(inp, dt_raw, bias, z, w, True)
+    ref, fref, rref = oracle.ssd_block(inp.x, dt_raw, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0, dt_bias=bias,
+                                       dt_softplus=True, z=z, norm_weight=w, norm_eps=1e-5)
+    tol = TOL[inp.dtype]
+    assert np.isfinite(out).all()
+    assert rel(out, ref) <= tol, rel(out, ref)
+    assert rel(fin, fref) <= tol
+    assert rel(rstd, rref) <= tol
