@@ -10,8 +10,11 @@
 //   out  = g * rstd * w    (apply)   or   g * w    (deferred: the caller applies
 //                                         the per-token rstd, e.g. to the rows of
 //                                         the next projection's output)
-// in place on y.  HBM-bound: one CTA per token reads its y (and z) row once
-// from HBM; the second pass over the row finds it in L1 / L2.
+// in place on y.  HBM-bound: y and z are read once and y written once.  One CTA
+// per token; each thread takes 16-byte vectors of the row (8 bf16 or 4 fp32)
+// at a stride of the block, keeps their g in registers through the block-wide
+// sum of squares, then scales and stores them.  Rows longer than the register
+// cache (or not a whole number of vectors) take a plain two-pass loop.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,50 +23,164 @@ namespace ssd {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kCache = 4;  // vectors a thread keeps in registers
 
 template <typename T>
-__device__ __forceinline__ float gate_value(const T *y, const T *z, int64_t i) {
-    const float v = to_f32<T>(y[i]);
-    if (!z) return v;
-    const float zz = to_f32<T>(z[i]);
-    return v * (zz / (1.f + __expf(-zz)));
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+    static constexpr int n = 8;
+    __device__ static void load(const __nv_bfloat16 *p, float (&v)[8]) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static void store(__nv_bfloat16 *p, const float (&v)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+        *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+template <>
+struct Vec<float> {
+    static constexpr int n = 4;
+    __device__ static void load(const float *p, float (&v)[4]) {
+        const float4 u = *reinterpret_cast<const float4 *>(p);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    }
+    __device__ static void store(float *p, const float (&v)[4]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+};
+
+__device__ __forceinline__ float silu_gate(float y, float z) { return y * (z / (1.f + __expf(-z))); }
+
+// block-wide sum (every thread gets the result)
+__device__ __forceinline__ float block_sum(float v, float *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float t = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0.f;
+    if (threadIdx.x < 32) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (threadIdx.x == 0) red[kThreads / 32] = t;
+    }
+    __syncthreads();
+    return red[kThreads / 32];
 }
 
+// rows of at most kCache vectors per thread, E a multiple of the vector width
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+gate_norm_vec_kernel(T *__restrict__ y, const T *__restrict__ z, const float *__restrict__ w, float eps,
+                     int apply, int E, float *__restrict__ rstd_out) {
+    constexpr int V = Vec<T>::n;
+    __shared__ float red[kThreads / 32 + 1];
+    const int64_t tok = blockIdx.x;
+    T *row = y + tok * E;
+    const T *zr = z ? z + tok * E : nullptr;
+    const int nv = E / V;
+    float g[kCache][V];
+    // all of this thread's loads first, then the arithmetic
+    float zz[kCache][V];
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+        const int v = threadIdx.x + j * kThreads;
+        if (v < nv) {
+            Vec<T>::load(row + v * V, g[j]);
+            if (zr) Vec<T>::load(zr + v * V, zz[j]);
+        }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+        const int v = threadIdx.x + j * kThreads;
+        if (v < nv) {
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                if (zr) g[j][e] = silu_gate(g[j][e], zz[j][e]);
+                ss = fmaf(g[j][e], g[j][e], ss);
+            }
+        }
+    }
+    float scale = 1.f;
+    if (w) {
+        const float rs = rsqrtf(block_sum(ss, red) / float(E) + eps);
+        if (rstd_out && threadIdx.x == 0) rstd_out[tok] = rs;
+        if (apply) scale = rs;
+    }
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+        const int v = threadIdx.x + j * kThreads;
+        if (v < nv) {
+            if (w) {
+                float wv[V];
+#pragma unroll
+                for (int e = 0; e < V; e += 4) {
+                    const float4 q = __ldg(reinterpret_cast<const float4 *>(w + v * V + e));
+                    wv[e] = q.x; wv[e + 1] = q.y; wv[e + 2] = q.z; wv[e + 3] = q.w;
+                }
+#pragma unroll
+                for (int e = 0; e < V; ++e) g[j][e] *= scale * wv[e];
+            }
+            Vec<T>::store(row + v * V, g[j]);
+        }
+    }
+}
+
+// any row: two passes over it (the second finds it in L1 / L2)
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 gate_norm_kernel(T *__restrict__ y, const T *__restrict__ z, const float *__restrict__ w, float eps,
                  int apply, int E, float *__restrict__ rstd_out) {
+    __shared__ float red[kThreads / 32 + 1];
     const int64_t tok = blockIdx.x;
     T *row = y + tok * E;
     const T *zr = z ? z + tok * E : nullptr;
-    __shared__ float red[kThreads / 32];
-    float rs = 1.f;
+    float scale = 1.f;
     if (w) {
         float ss = 0.f;
         for (int i = threadIdx.x; i < E; i += kThreads) {
-            const float g = gate_value<T>(row, zr, i);
+            const float v = to_f32<T>(row[i]);
+            const float g = zr ? silu_gate(v, to_f32<T>(zr[i])) : v;
             ss = fmaf(g, g, ss);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            float v = threadIdx.x < kThreads / 32 ? red[threadIdx.x] : 0.f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (threadIdx.x == 0) red[0] = v;
-        }
-        __syncthreads();
-        rs = rsqrtf(red[0] / float(E) + eps);
+        const float rs = rsqrtf(block_sum(ss, red) / float(E) + eps);
         if (rstd_out && threadIdx.x == 0) rstd_out[tok] = rs;
+        if (apply) scale = rs;
     }
-    const float scale = (w && apply) ? rs : 1.f;
     for (int i = threadIdx.x; i < E; i += kThreads) {
-        float g = gate_value<T>(row, zr, i);
+        const float v = to_f32<T>(row[i]);
+        float g = zr ? silu_gate(v, to_f32<T>(zr[i])) : v;
         if (w) g *= scale * __ldg(w + i);
         row[i] = from_f32<T>(g);
     }
+}
+
+template <typename T>
+cudaError_t launch_typed(int64_t tokens, int E, void *y, const void *z, const float *w, float eps, bool apply,
+                         float *rstd_out, cudaStream_t stream) {
+    const dim3 grid(static_cast<unsigned>(tokens), 1, 1);
+    constexpr int V = Vec<T>::n;
+    // the vector path needs whole 16-byte vectors: E % V == 0 keeps every row
+    // (and the weight) 16-byte aligned, the tensors themselves being aligned
+    if (E % V == 0 && E <= kCache * kThreads * V)
+        gate_norm_vec_kernel<T><<<grid, kThreads, 0, stream>>>(static_cast<T *>(y), static_cast<const T *>(z), w,
+                                                               eps, apply ? 1 : 0, E, rstd_out);
+    else
+        gate_norm_kernel<T><<<grid, kThreads, 0, stream>>>(static_cast<T *>(y), static_cast<const T *>(z), w, eps,
+                                                           apply ? 1 : 0, E, rstd_out);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -73,16 +190,8 @@ cudaError_t launch_gate_norm(const Dims &d, bool bf16, void *y, const void *z, c
     const int64_t tokens = int64_t(d.B) * d.T;
     const int E = d.H * d.P;
     if (tokens <= 0 || tokens > 0x7fffffff) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>(tokens), 1, 1);
-    if (bf16)
-        gate_norm_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-            static_cast<__nv_bfloat16 *>(y), static_cast<const __nv_bfloat16 *>(z), w, eps, apply ? 1 : 0, E,
-            rstd_out);
-    else
-        gate_norm_kernel<float><<<grid, kThreads, 0, stream>>>(static_cast<float *>(y),
-                                                                static_cast<const float *>(z), w, eps,
-                                                                apply ? 1 : 0, E, rstd_out);
-    return cudaGetLastError();
+    return bf16 ? launch_typed<__nv_bfloat16>(tokens, E, y, z, w, eps, apply, rstd_out, stream)
+                : launch_typed<float>(tokens, E, y, z, w, eps, apply, rstd_out, stream);
 }
 
 }  // namespace ssd
