@@ -273,6 +273,41 @@ SSD_API ssd_status_t ssd_forward_block(const ssd_dims_t *dims, const void *x, co
                                        const ssd_block_opts_t *opts, void *workspace,
                                        size_t workspace_bytes, void *stream);
 
+/*
+ * ssd_forward_varlen -- several independent sequences packed along the token
+ * axis of one row (the "varlen" layout): sequence i is tokens
+ * [cu_seqlens[i], cu_seqlens[i+1]) and starts from its own initial state, so
+ * no state crosses a boundary (each sequence is the recurrence of
+ * akillness.github.io "State Space Duality and Mamba-2", "Mathematical
+ * Foundations", on its own tokens).
+ *
+ *   dims        batch must be 1; seqlen = total tokens; other fields as for
+ *               ssd_forward (else SSD_ERR_INVALID_DIM)
+ *   cu_seqlens  HOST array of nseq + 1 offsets: cu_seqlens[0] = 0,
+ *               non-decreasing, cu_seqlens[nseq] = seqlen (empty sequences
+ *               allowed); read during the call only
+ *   x, dt, Bm, Cm, y_out   the packed tensors, layouts as for ssd_forward with
+ *               B = 1; every sequence's slices must stay 16-byte aligned
+ *               (SSD_ERR_MISALIGNED otherwise)
+ *   A, D        [H] fp32 as for ssd_forward (D may be NULL)
+ *   init_states [nseq, H, P, N] fp32, or NULL for zeros
+ *   final_states_out [nseq, H, P, N] fp32, or NULL; an empty sequence's
+ *               final state is its initial state
+ *   workspace   ssd_varlen_workspace_bytes bytes, 256-byte aligned (may be
+ *               NULL when that size is 0)
+ * The sequences run one after another on `stream`, each with the plan its own
+ * length selects (ragged lengths included) and all sharing the workspace.
+ * Every argument is validated before the first launch.  Accuracy as for
+ * ssd_forward, per sequence.
+ */
+SSD_API size_t ssd_varlen_workspace_bytes(const ssd_dims_t *dims, const int64_t *cu_seqlens, int64_t nseq,
+                                          int chunk_len);
+SSD_API ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *cu_seqlens, int64_t nseq,
+                                        const void *x, const float *dt, const float *A, const void *Bm,
+                                        const void *Cm, const float *D, int chunk_len,
+                                        const float *init_states, void *y_out, float *final_states_out,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace one call needs (0 if the arguments are invalid). */
 SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
 

@@ -22,7 +22,8 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
 
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
            "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
-           "ssd_forward_static", "ssd_step", "ssd_forward_block", "ssd_block_workspace_bytes")
+           "ssd_forward_static", "ssd_step", "ssd_forward_block", "ssd_block_workspace_bytes",
+           "ssd_forward_varlen", "ssd_varlen_workspace_bytes")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -97,6 +98,12 @@ def load():
     lib.ssd_forward_block.restype = ctypes.c_int
     lib.ssd_block_workspace_bytes.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(BlockOpts)]
     lib.ssd_block_workspace_bytes.restype = ctypes.c_size_t
+    i64p = ctypes.POINTER(ctypes.c_int64)
+    lib.ssd_forward_varlen.argtypes = [dims_p, i64p, ctypes.c_int64, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp,
+                                       vp, fp, vp, ctypes.c_size_t, vp]
+    lib.ssd_forward_varlen.restype = ctypes.c_int
+    lib.ssd_varlen_workspace_bytes.argtypes = [dims_p, i64p, ctypes.c_int64, ctypes.c_int]
+    lib.ssd_varlen_workspace_bytes.restype = ctypes.c_size_t
     lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
     lib.ssd_workspace_bytes.restype = ctypes.c_size_t
     lib.ssd_workspace_layout.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]
@@ -251,6 +258,56 @@ def forward_block(x, dt, A, B, C, D=None, chunk_len=256, init_state=None, dt_bia
     if rstd is not None:
         res.append(rstd)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def _cu_array(cu_seqlens):
+    import numpy as np
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if isinstance(cu_seqlens, torch.Tensor) else cu_seqlens,
+                                         dtype=np.int64))
+    if cu.ndim != 1 or cu.size < 2:
+        raise ValueError("cu_seqlens must be a 1-D array of nseq + 1 offsets")
+    return cu
+
+
+def varlen_workspace_bytes(dims: Dims, cu_seqlens, chunk_len: int) -> int:
+    cu = _cu_array(cu_seqlens)
+    return int(load().ssd_varlen_workspace_bytes(ctypes.byref(dims), cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                                 cu.size - 1, int(chunk_len)))
+
+
+def forward_varlen(x, dt, A, B, C, cu_seqlens, D=None, chunk_len=256, init_states=None,
+                   return_final_states=False, out=None, final_out=None, workspace=None, stream=None):
+    """Several sequences packed along the token axis through ``ssd_forward_varlen``.
+
+    x [1, T, H, P], dt [1, T, H], B/C [1, T, G, N]; ``cu_seqlens`` (host: a list,
+    a numpy array or a CPU tensor) holds nseq + 1 offsets; ``init_states`` and
+    the final states are [nseq, H, P, N] float32.  Returns y (and the final
+    states)."""
+    cu = _cu_array(cu_seqlens)
+    nseq = cu.size - 1
+    dims = _validate(x, dt, A, B, C, D, None)
+    dev = x.device
+    st_shape = (nseq, dims.nheads, dims.headdim, dims.dstate)
+    if init_states is not None and (init_states.device != dev or init_states.dtype != torch.float32
+                                    or tuple(init_states.shape) != st_shape or not init_states.is_contiguous()):
+        raise ValueError(f"init_states must be a contiguous float32 tensor {st_shape} on {dev}")
+    y = out if out is not None else torch.empty_like(x)
+    fin = final_out
+    if fin is None and return_final_states:
+        fin = torch.empty(st_shape, dtype=torch.float32, device=dev)
+    cu_p = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    if workspace is None:
+        need = int(load().ssd_varlen_workspace_bytes(ctypes.byref(dims), cu_p, nseq, int(chunk_len)))
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        wsz = workspace.numel() * workspace.element_size()
+        st = load().ssd_forward_varlen(ctypes.byref(dims), cu_p, nseq, _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                       _ptr(C), _ptr(D), int(chunk_len), _ptr(init_states), _ptr(y), _ptr(fin),
+                                       _ptr(workspace), wsz, ctypes.c_void_p(stream))
+    _check(st)
+    return (y, fin) if (return_final_states or final_out is not None) else y
 
 
 def block_workspace_bytes(dims: Dims, chunk_len: int, dt_transform: bool) -> int:

@@ -325,6 +325,29 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     return SSD_OK;
 }
 
+// ---------------------------------------------------------------------------
+// varlen: several sequences packed along the token axis of one row
+// ---------------------------------------------------------------------------
+// Validates the packing and makes one plan per non-empty sequence (nothing is
+// launched); `need` gets the largest workspace among them.
+ssd_status_t varlen_plans(const ssd_dims_t *dims, const int64_t *cu, int64_t nseq, int chunk_len,
+                          size_t *need) {
+    if (!dims || !cu) return SSD_ERR_NULL_ARG;
+    if (dims->batch != 1 || nseq < 1 || cu[0] != 0 || cu[nseq] != dims->seqlen) return SSD_ERR_INVALID_DIM;
+    *need = 0;
+    for (int64_t i = 0; i < nseq; ++i) {
+        if (cu[i + 1] < cu[i]) return SSD_ERR_INVALID_DIM;
+        if (cu[i + 1] == cu[i]) continue;
+        ssd_dims_t di = *dims;
+        di.seqlen = cu[i + 1] - cu[i];
+        Plan pl;
+        const ssd_status_t s = make_plan(&di, chunk_len, &pl);
+        if (s != SSD_OK) return s;
+        if (pl.ws.total_bytes > *need) *need = pl.ws.total_bytes;
+    }
+    return SSD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -449,6 +472,67 @@ ssd_status_t ssd_forward_block(const ssd_dims_t *dims, const void *x, const floa
     s = run(pl, x, dt, A, Bm, Cm, D, init_state, y_out, final_state_out, static_cast<char *>(ws), st, -1, &nb);
     if (!workspace && cudaFreeAsync(ws, st) != cudaSuccess && s == SSD_OK) s = SSD_ERR_CUDA;
     return s;
+}
+
+size_t ssd_varlen_workspace_bytes(const ssd_dims_t *dims, const int64_t *cu_seqlens, int64_t nseq,
+                                  int chunk_len) {
+    size_t need = 0;
+    if (varlen_plans(dims, cu_seqlens, nseq, chunk_len, &need) != SSD_OK) return 0;
+    return need;
+}
+
+ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *cu_seqlens, int64_t nseq, const void *x,
+                                const float *dt, const float *A, const void *Bm, const void *Cm, const float *D,
+                                int chunk_len, const float *init_states, void *y_out, float *final_states_out,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+    size_t need = 0;
+    ssd_status_t s = varlen_plans(dims, cu_seqlens, nseq, chunk_len, &need);
+    if (s != SSD_OK) return s;
+    if (!x || !dt || !A || !Bm || !Cm || !y_out) return SSD_ERR_NULL_ARG;
+    const size_t esz = dims->dtype == SSD_BF16 ? 2 : 4;
+    const int64_t H = dims->nheads, P = dims->headdim, N = dims->dstate, G = dims->ngroups;
+    const int64_t st_elems = H * P * N;
+    // every sequence's slices must keep the 16-byte alignment of the whole tensors
+    for (int64_t i = 0; i < nseq; ++i) {
+        const int64_t t0 = cu_seqlens[i];
+        if (cu_seqlens[i + 1] == t0) continue;
+        const char *px = static_cast<const char *>(x) + t0 * H * P * esz;
+        const char *pb = static_cast<const char *>(Bm) + t0 * G * N * esz;
+        const char *pc = static_cast<const char *>(Cm) + t0 * G * N * esz;
+        const char *py = static_cast<const char *>(y_out) + t0 * H * P * esz;
+        const float *pdt = dt + t0 * H;
+        const void *ptrs[] = {px, pb, pc, py, pdt, A, D, init_states, final_states_out};
+        for (const void *p : ptrs)
+            if (misaligned(p)) return SSD_ERR_MISALIGNED;
+    }
+    if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1))))
+        return SSD_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int64_t i = 0; i < nseq; ++i) {
+        const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
+        const float *h0 = init_states ? init_states + i * st_elems : nullptr;
+        float *fin = final_states_out ? final_states_out + i * st_elems : nullptr;
+        if (len == 0) {
+            // an empty sequence leaves its initial state (or zeros)
+            if (fin) {
+                const cudaError_t e = h0 ? cudaMemcpyAsync(fin, h0, st_elems * sizeof(float), cudaMemcpyDeviceToDevice, st)
+                                         : cudaMemsetAsync(fin, 0, st_elems * sizeof(float), st);
+                if (e != cudaSuccess) return SSD_ERR_CUDA;
+            }
+            continue;
+        }
+        ssd_dims_t di = *dims;
+        di.seqlen = len;
+        Plan pl;
+        s = make_plan(&di, chunk_len, &pl);
+        if (s != SSD_OK) return s;
+        // the sequences run one after another on the stream and share the workspace
+        s = run(pl, static_cast<const char *>(x) + t0 * H * P * esz, dt + t0 * H, A,
+                static_cast<const char *>(Bm) + t0 * G * N * esz, static_cast<const char *>(Cm) + t0 * G * N * esz, D,
+                h0, static_cast<char *>(y_out) + t0 * H * P * esz, fin, static_cast<char *>(workspace), st);
+        if (s != SSD_OK) return s;
+    }
+    return SSD_OK;
 }
 
 const char *ssd_status_string(ssd_status_t status) {

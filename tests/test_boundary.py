@@ -8,6 +8,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from structured_state_space_mamba_b200 import binding
@@ -261,3 +263,35 @@ def test_ragged_length_layout(lib):
     assert ragged.total_bytes >= full.total_bytes + 2 * 8 * 64 * 128 * 4
     short = binding.workspace_layout(dims(seqlen=100), 128)
     assert short.launches == 1
+
+
+def test_varlen_argument_checks(lib):
+    """ssd_forward_varlen validates the packing before anything runs: batch 1,
+    cu_seqlens from 0 to seqlen and non-decreasing; the workspace is the
+    largest one of its sequences' plans."""
+    d = binding.make_dims(1, 1000, 8, 64, 128, 2, "bf16")
+    i64 = ctypes.POINTER(ctypes.c_int64)
+
+    def ws(cu, q=256):
+        a = np.asarray(cu, dtype=np.int64)
+        return lib.ssd_varlen_workspace_bytes(ctypes.byref(d), a.ctypes.data_as(i64), a.size - 1, q)
+
+    good = ws([0, 300, 300, 1000])
+    assert good > 0
+    one = binding.make_dims(1, 700, 8, 64, 128, 2, "bf16")
+    assert good == binding.workspace_bytes(one, 256)  # the longest sequence's plan
+    assert ws([0, 300, 999]) == 0                       # does not end at seqlen
+    assert ws([1, 300, 1000]) == 0                      # does not start at 0
+    assert ws([0, 600, 300, 1000]) == 0                 # decreasing
+    d2 = binding.make_dims(2, 1000, 8, 64, 128, 2, "bf16")
+    a = np.asarray([0, 1000], dtype=np.int64)
+    assert lib.ssd_varlen_workspace_bytes(ctypes.byref(d2), a.ctypes.data_as(i64), 1, 256) == 0  # batch != 1
+    # the entry point returns the same errors before touching any pointer
+    bad = np.asarray([0, 600, 300, 1000], dtype=np.int64)
+    st = lib.ssd_forward_varlen(ctypes.byref(d), bad.ctypes.data_as(i64), 3, None, None, None, None, None, None,
+                                256, None, None, None, None, 0, None)
+    assert st == 2  # SSD_ERR_INVALID_DIM
+    cu = np.asarray([0, 300, 1000], dtype=np.int64)
+    st = lib.ssd_forward_varlen(ctypes.byref(d), cu.ctypes.data_as(i64), 2, None, None, None, None, None, None,
+                                256, None, None, None, None, 0, None)
+    assert st == 1  # SSD_ERR_NULL_ARG
