@@ -28,7 +28,7 @@ import numpy as np
 from . import build as _build
 
 __all__ = ["ssd_recurrent", "ssd_quadratic", "ssd_chunked", "ssd_step", "default_threads",
-           "dt_transform", "gated_rmsnorm", "ssd_block"]
+           "dt_transform", "gated_rmsnorm", "ssd_block", "ssd_recurrent_grad"]
 
 
 class _Dims(ctypes.Structure):
@@ -243,3 +243,61 @@ def ssd_block(x, dt, A, B, C, D=None, h0=None, dt_bias=None, dt_softplus=False, 
     y, fin = ssd_recurrent(x, dte, A, B, C, D=D, h0=h0, units=units, nthreads=nthreads)
     out, rstd = gated_rmsnorm(y, z, norm_weight, norm_eps)
     return out, fin, rstd
+
+
+def ssd_recurrent_grad(x, dt, A, B, C, dy, D=None, h0=None, dfinal=None):
+    """Reverse mode of the recurrence, in fp64: the gradients of
+    L = sum(y * dy) + sum(final * dfinal) with respect to every input.
+
+    Forward (per b, h, g = h // (H // G)), as ssd_recurrent:
+        a_t = exp(dt_t A_h),  h_t = a_t h_{t-1} + dt_t x_t B_t^T,  y_t = h_t C_t + D_h x_t
+    Reverse, token by token from the last (G_t = dL/dh_t, with the future's
+    share G' = dL/dh_t through h_{t+1}, starting from dfinal):
+        G_t    = dy_t C_t^T + G'
+        dx_t   = dt_t G_t B_t + D_h dy_t
+        dB_t  += dt_t G_t^T x_t           (summed over the group's heads)
+        dC_t  += h_t^T dy_t               (summed over the group's heads)
+        ddt_t  = x_t . (G_t B_t) + A_h a_t (G_t : h_{t-1})
+        dA_h  += dt_t a_t (G_t : h_{t-1})
+        G'     = a_t G_t                  (dL/dh_{t-1}; dh0 at the end)
+        dD_h  += dy_t . x_t
+    Every forward state is kept (small problems only).  Returns a dict with dx,
+    ddt, dA, dB, dC, dD, dh0 (float64)."""
+    x, dt, A, B, C, D, h0 = _prep(x, dt, A, B, C, D, h0)
+    dy = _f64(dy)
+    bsz, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if dy.shape != x.shape:
+        raise ValueError("dy must be shaped like x")
+    rep = H // G
+    Bh = np.repeat(B, rep, axis=2)  # [B,T,H,N]: each head's B and C
+    Ch = np.repeat(C, rep, axis=2)
+    h = np.zeros((bsz, H, P, N)) if h0 is None else h0.copy()
+    hs = [h]
+    for t in range(T):
+        a = np.exp(dt[:, t, :] * A[None, :])
+        h = a[:, :, None, None] * h + (dt[:, t, :, None, None] * x[:, t, :, :, None]) * Bh[:, t, :, None, :]
+        hs.append(h)  # hs[t + 1] = h_t
+    Gn = np.zeros((bsz, H, P, N)) if dfinal is None else _f64(dfinal).copy()
+    dx = np.zeros_like(x)
+    ddt = np.zeros_like(dt)
+    dA = np.zeros(H)
+    dBh = np.zeros_like(Bh)
+    dCh = np.zeros_like(Ch)
+    Dv = np.zeros(H) if D is None else D
+    for t in range(T - 1, -1, -1):
+        Gt = dy[:, t, :, :, None] * Ch[:, t, :, None, :] + Gn
+        a = np.exp(dt[:, t, :] * A[None, :])
+        hprev = hs[t]
+        GB = np.einsum("bhpn,bhn->bhp", Gt, Bh[:, t])
+        dx[:, t] = dt[:, t, :, None] * GB + Dv[None, :, None] * dy[:, t]
+        dBh[:, t] = dt[:, t, :, None] * np.einsum("bhpn,bhp->bhn", Gt, x[:, t])
+        dCh[:, t] = np.einsum("bhpn,bhp->bhn", hs[t + 1], dy[:, t])
+        gh = np.einsum("bhpn,bhpn->bh", Gt, hprev)
+        ddt[:, t] = np.einsum("bhp,bhp->bh", x[:, t], GB) + A[None, :] * a * gh
+        dA += np.sum(dt[:, t] * a * gh, axis=0)
+        Gn = a[:, :, None, None] * Gt
+    dB = dBh.reshape(bsz, T, G, rep, N).sum(axis=3)
+    dC = dCh.reshape(bsz, T, G, rep, N).sum(axis=3)
+    dD = np.einsum("bthp,bthp->h", dy, x)
+    return dict(dx=dx, ddt=ddt, dA=dA, dB=dB, dC=dC, dD=dD, dh0=Gn)
