@@ -308,6 +308,36 @@ SSD_API ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *c
                                         const float *init_states, void *y_out, float *final_states_out,
                                         void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * ssd_backward -- the gradients of a scalar loss L through ssd_forward: given
+ * dy = dL/dy and dfinal_state = dL/dfinal_state, returns dL/d(every input).
+ * The reverse mode of the recurrence (akillness.github.io "State Space Duality
+ * and Mamba-2", "Mathematical Foundations"): with G_t = dL/dh_t,
+ *   G_t = dy_t C_t^T + exp(dt_{t+1} A_h) G_{t+1},  G_{T-1} = dy_{T-1} C_{T-1}^T + dfinal
+ *   dx_t = dt_t G_t B_t + D_h dy_t,   dB_t = sum_heads dt_t G_t^T x_t,
+ *   dC_t = sum_heads h_t^T dy_t,      dD_h = sum dy_t . x_t,
+ *   ddt_t = x_t . (G_t B_t) + A_h exp(dt_t A_h) (G_t : h_{t-1}),
+ *   dA_h = sum dt_t exp(dt_t A_h) (G_t : h_{t-1}),   dinit = exp(dt_0 A_h) G_0.
+ * Computed with four scans of the library's own chunked forward in fp32 (G
+ * backwards in time, h forwards, and each transposed for dB and dC) plus
+ * element-wise and prefix-sum kernels (k_backward.cu gives the identities).
+ *
+ *   inputs as for ssd_forward; dy [B,T,H,P] dtype; dfinal_state [B,H,P,N] fp32
+ *   or NULL (zero)
+ *   dx [B,T,H,P] dtype; ddt [B,T,H] fp32; dA [H] fp32; dB, dC [B,T,G,N] dtype;
+ *   dD [H] fp32 or NULL (not computed); dinit_state [B,H,P,N] fp32 or NULL
+ * Requires dt_t > 0 for every token (the scan of G takes a_t dy_t / dt_t as its
+ * input).  Scratch memory (about 20 fp32 copies of x's size) is allocated
+ * stream-ordered on `stream` and released before return.  Accuracy: the
+ * gradients' max abs error over their max |value| within 1e-3 of the fp64
+ * reverse mode on fp32-exact inputs.
+ */
+SSD_API ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt, const float *A,
+                                  const void *Bm, const void *Cm, const float *D, int chunk_len,
+                                  const float *init_state, const void *dy, const float *dfinal_state, void *dx,
+                                  float *ddt, float *dA, void *dB, void *dC, float *dD, float *dinit_state,
+                                  void *stream);
+
 /* Bytes of workspace one call needs (0 if the arguments are invalid). */
 SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
 

@@ -23,7 +23,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
            "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
            "ssd_forward_static", "ssd_step", "ssd_forward_block", "ssd_block_workspace_bytes",
-           "ssd_forward_varlen", "ssd_varlen_workspace_bytes")
+           "ssd_forward_varlen", "ssd_varlen_workspace_bytes", "ssd_backward")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -104,6 +104,9 @@ def load():
     lib.ssd_forward_varlen.restype = ctypes.c_int
     lib.ssd_varlen_workspace_bytes.argtypes = [dims_p, i64p, ctypes.c_int64, ctypes.c_int]
     lib.ssd_varlen_workspace_bytes.restype = ctypes.c_size_t
+    lib.ssd_backward.argtypes = [dims_p, vp, fp, fp, vp, vp, fp, ctypes.c_int, fp, vp, fp, vp, fp, fp, vp, vp, fp,
+                                 fp, vp]
+    lib.ssd_backward.restype = ctypes.c_int
     lib.ssd_workspace_bytes.argtypes = [dims_p, ctypes.c_int]
     lib.ssd_workspace_bytes.restype = ctypes.c_size_t
     lib.ssd_workspace_layout.argtypes = [dims_p, ctypes.c_int, ctypes.POINTER(WorkspaceLayout)]
@@ -308,6 +311,32 @@ def forward_varlen(x, dt, A, B, C, cu_seqlens, D=None, chunk_len=256, init_state
                                        _ptr(workspace), wsz, ctypes.c_void_p(stream))
     _check(st)
     return (y, fin) if (return_final_states or final_out is not None) else y
+
+
+def backward(x, dt, A, B, C, dy, D=None, chunk_len=256, init_state=None, dfinal_state=None, stream=None):
+    """Gradients through ``ssd_backward``: returns a dict with dx, ddt, dA, dB,
+    dC, dD (None without D) and dinit_state (None without an initial state)."""
+    dims = _validate(x, dt, A, B, C, D, init_state)
+    dev = x.device
+    if dy.shape != x.shape or dy.dtype != x.dtype or dy.device != dev or not dy.is_contiguous():
+        raise ValueError("dy must be a contiguous tensor like x")
+    if dfinal_state is not None and (dfinal_state.dtype != torch.float32 or not dfinal_state.is_contiguous()
+                                     or tuple(dfinal_state.shape) != (dims.batch, dims.nheads, dims.headdim,
+                                                                      dims.dstate)):
+        raise ValueError("dfinal_state must be a contiguous float32 [batch, nheads, headdim, dstate] tensor")
+    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt), dA=torch.empty_like(A),
+               dB=torch.empty_like(B), dC=torch.empty_like(C),
+               dD=None if D is None else torch.empty_like(D),
+               dinit_state=None if init_state is None else torch.empty_like(init_state))
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = load().ssd_backward(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                 int(chunk_len), _ptr(init_state), _ptr(dy), _ptr(dfinal_state), _ptr(out["dx"]),
+                                 _ptr(out["ddt"]), _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+                                 _ptr(out["dD"]), _ptr(out["dinit_state"]), ctypes.c_void_p(stream))
+    _check(st)
+    return out
 
 
 def block_workspace_bytes(dims: Dims, chunk_len: int, dt_transform: bool) -> int:

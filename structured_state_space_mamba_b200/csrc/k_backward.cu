@@ -1,0 +1,350 @@
+// k_backward.cu -- the element-wise and prefix-sum kernels of the backward
+// pass (ssd_backward in ssd_api.cu, which runs the scans themselves).
+//
+// Reverse mode of h_t = a_t h_{t-1} + dt_t x_t B_t^T, y_t = h_t C_t + D x_t
+// (a_t = exp(dt_t A_h)), per (b, h) with G_t = dL/dh_t and K_t = a_t G_t =
+// dL/dh_{t-1}:
+//   K_t = a_t K_{t+1} + a_t dy_t C_t^T,  K_T = dfinal,  dh0 = K_0
+//   dx_t = dt_t G_t B_t + D dy_t,   dB_t = sum_h dt_t G_t^T x_t,   dC_t = sum_h h_t^T dy_t
+//   ddt_t = x_t . (G_t B_t) + A R_t,   dA = sum dt_t R_t,   dD = sum dy_t . x_t
+// with R_t = K_t : h_{t-1}, which obeys R_0 = dh0 : h0 and
+//   R_{t+1} = R_t + c_t - r_t,  c_t = dt_t x_t . (G_t B_t),  r_t = dy_t . (h_t C_t)
+// (expand K_{t+1} = K_t / a_t - dy_t C_t^T and h_t = a_t h_{t-1} + dt_t x_t B_t^T
+// in K_{t+1} : h_t).  K is the forward recurrence run backwards in time with
+// input a_t dy_t / dt_t against C_t (read out against B_t); its transpose gives
+// dB; h^T read out against dy gives dC.  These kernels build the scans' inputs
+// (reversed in time where needed), and turn the scans' outputs into the
+// gradients.  All of them are HBM-bound element-wise passes; the prefix over
+// tokens is one warp per (b, h).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssd {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ float ld(const T *p, int64_t i) { return to_f32<T>(p[i]); }
+
+__device__ __forceinline__ float decay(const float *dt, const float *A, int64_t i_dt, int h) {
+    return __expf(dt[i_dt] * A[h]);
+}
+
+// scan K (reversed): xr[b,tau,h,p] = a_t dy[b,t,h,p] / dt_t, dtr[b,tau,h] = dt_t,
+// and (per group) Br = C, Cr = B, all at tau = T-1-t
+template <typename T>
+__global__ void prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__restrict__ dt,
+                              const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
+                              float *__restrict__ xr, float *__restrict__ dtr, float *__restrict__ Br,
+                              float *__restrict__ Cr) {
+    const int64_t n_x = int64_t(d.B) * d.T * d.H * d.P;
+    const int64_t n_bc = int64_t(d.B) * d.T * d.G * d.N;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_x + n_bc;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        if (i < n_x) {
+            const int p = int(i % d.P);
+            int64_t r = i / d.P;
+            const int h = int(r % d.H);
+            r /= d.H;
+            const int t = int(r % d.T), b = int(r / d.T);
+            const int tau = d.T - 1 - t;
+            const int64_t idt = off_dt(d, b, t) + h;
+            const float dtt = dt[idt];
+            xr[off_x(d, b, tau, h) + p] = decay(dt, A, idt, h) * ld(dy, i) / dtt;
+            if (p == 0) dtr[off_dt(d, b, tau) + h] = dtt;
+        } else {
+            const int64_t j = i - n_x;
+            const int n = int(j % d.N);
+            int64_t r = j / d.N;
+            const int g = int(r % d.G);
+            r /= d.G;
+            const int t = int(r % d.T), b = int(r / d.T);
+            const int64_t dst = off_bc(d, b, d.T - 1 - t, g) + n;
+            Br[dst] = ld(Cm, j);
+            Cr[dst] = ld(Bm, j);
+        }
+    }
+}
+
+// fp32 copies in the same layout (the scans of the backward run in fp32)
+template <typename T>
+__global__ void to_f32_kernel(const T *__restrict__ src, float *__restrict__ dst, int64_t n) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+        dst[i] = ld(src, i);
+}
+
+// the transposed scans' inputs, one value per (b, t, h, n):
+//   reversed (dB): xb[b,tau,h,n] = a_t C[b,t,g,n] / dt_t
+//   forward  (dC): xc[b,t,h,n]   = B[b,t,g,n]
+// and the per-head rows of the reversed ones:
+//   dyr[b,tau,h,p] = dy[b,t,h,p],  xrr[b,tau,h,p] = x[b,t,h,p]
+template <typename T>
+__global__ void prep_t_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ dy,
+                              const float *__restrict__ dt, const float *__restrict__ A,
+                              const T *__restrict__ Bm, const T *__restrict__ Cm, float *__restrict__ xb,
+                              float *__restrict__ xc, float *__restrict__ dyr, float *__restrict__ xrr) {
+    const int64_t n_n = int64_t(d.B) * d.T * d.H * d.N;
+    const int64_t n_p = int64_t(d.B) * d.T * d.H * d.P;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_n + n_p;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        if (i < n_n) {
+            const int n = int(i % d.N);
+            int64_t r = i / d.N;
+            const int h = int(r % d.H);
+            r /= d.H;
+            const int t = int(r % d.T), b = int(r / d.T);
+            const int g = h / d.r;
+            const int64_t idt = off_dt(d, b, t) + h;
+            const int64_t src = off_bc(d, b, t, g) + n;
+            const int64_t rowr = ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * d.N + n;
+            xb[rowr] = decay(dt, A, idt, h) * ld(Cm, src) / dt[idt];
+            xc[i] = ld(Bm, src);
+        } else {
+            const int64_t j = i - n_n;
+            const int p = int(j % d.P);
+            int64_t r = j / d.P;
+            const int h = int(r % d.H);
+            r /= d.H;
+            const int t = int(r % d.T), b = int(r / d.T);
+            const int64_t dst = off_x(d, b, d.T - 1 - t, h) + p;
+            dyr[dst] = ld(dy, j);
+            xrr[dst] = ld(x, j);
+        }
+    }
+}
+
+// [B, H, P, N] -> [B, H, N, P] (a state as the transposed scans hold it)
+__global__ void transpose_state_kernel(int64_t BH, int P, int N, const float *__restrict__ s,
+                                       float *__restrict__ st) {
+    const int64_t total = BH * P * N;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int n = int(i % N);
+        const int64_t r = i / N;
+        const int p = int(r % P);
+        const int64_t bh = r / P;
+        st[(bh * N + n) * P + p] = s[i];
+    }
+}
+
+// one warp per (b, t, h): u = G_t B_t = yk / a_t (yk from the reversed scan),
+// dx = dt u + D dy, xu = x . u, c = dt xu, r = dy . yh (yh = h_t C_t)
+template <typename T>
+__global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ dy,
+                              const float *__restrict__ dt, const float *__restrict__ A,
+                              const float *__restrict__ D, const float *__restrict__ yk,
+                              const float *__restrict__ yh, T *__restrict__ dx, float *__restrict__ xu,
+                              float *__restrict__ cc, float *__restrict__ rr) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = int64_t(d.B) * d.T * d.H;
+    for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; w < nw;
+         w += (int64_t(gridDim.x) * blockDim.x) >> 5) {
+        const int h = int(w % d.H);
+        const int64_t bt = w / d.H;
+        const int t = int(bt % d.T), b = int(bt / d.T);
+        const int64_t idt = off_dt(d, b, t) + h;
+        const float dtt = dt[idt];
+        const float inv_a = __expf(-dtt * A[h]);
+        const float Dh = D ? D[h] : 0.f;
+        const int64_t row = off_x(d, b, t, h);
+        const int64_t rowr = off_x(d, b, d.T - 1 - t, h);
+        float sx = 0.f, sr = 0.f;
+        for (int p = lane; p < d.P; p += 32) {
+            const float u = yk[rowr + p] * inv_a;
+            const float dyp = ld(dy, row + p);
+            dx[row + p] = from_f32<T>(dtt * u + Dh * dyp);
+            sx = fmaf(ld(x, row + p), u, sx);
+            sr = fmaf(dyp, yh[row + p], sr);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            sx += __shfl_xor_sync(0xffffffffu, sx, o);
+            sr += __shfl_xor_sync(0xffffffffu, sr, o);
+        }
+        if (lane == 0) {
+            xu[idt] = sx;
+            cc[idt] = dtt * sx;
+            rr[idt] = sr;
+        }
+    }
+}
+
+// one block per (b, h): R0 = dh0 : h0 (0 without an initial state)
+__global__ void r0_kernel(int64_t BH, int PN, const float *__restrict__ dh0, const float *__restrict__ h0,
+                          float *__restrict__ R0) {
+    __shared__ float red[kThreads / 32];
+    const int64_t bh = blockIdx.x;
+    float s = 0.f;
+    if (h0)
+        for (int i = threadIdx.x; i < PN; i += blockDim.x) s = fmaf(dh0[bh * PN + i], h0[bh * PN + i], s);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+        R0[bh] = t;
+    }
+}
+
+// one warp per (b, h): R over the tokens in blocks of 32 (a warp prefix sum of
+// c - r), ddt_t = xu_t + A R_t, and this (b, h)'s share of dA = sum dt_t R_t
+__global__ void prefix_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
+                              const float *__restrict__ R0, const float *__restrict__ xu,
+                              const float *__restrict__ cc, const float *__restrict__ rr, float *__restrict__ ddt,
+                              float *__restrict__ dA_part) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = int64_t(d.B) * d.H;
+    for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; w < nw;
+         w += (int64_t(gridDim.x) * blockDim.x) >> 5) {
+        const int h = int(w % d.H), b = int(w / d.H);
+        const float a_h = A[h];
+        float R = R0[w];  // R at the first token of the block
+        float sA = 0.f;
+        for (int t0 = 0; t0 < d.T; t0 += 32) {
+            const int t = t0 + lane;
+            const bool in = t < d.T;
+            const int64_t i = off_dt(d, b, in ? t : 0) + h;
+            const float step = in ? cc[i] - rr[i] : 0.f;
+            // exclusive prefix of the steps: R_t = R + sum_{t0 <= k < t} (c_k - r_k)
+            float incl = step;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float nb = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nb;
+            }
+            const float Rt = R + incl - step;
+            if (in) {
+                ddt[i] = xu[i] + a_h * Rt;
+                sA = fmaf(dt[i], Rt, sA);
+            }
+            R += __shfl_sync(0xffffffffu, incl, 31);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sA += __shfl_xor_sync(0xffffffffu, sA, o);
+        if (lane == 0) dA_part[w] = sA;
+    }
+}
+
+// dA[h] = sum_b dA_part[b, h]; dD[h] = sum_{b,t,p} dy x   (one block per head)
+template <typename T>
+__global__ void head_sums_kernel(Dims d, const float *__restrict__ dA_part, const T *__restrict__ x,
+                                 const T *__restrict__ dy, float *__restrict__ dA, float *__restrict__ dD) {
+    __shared__ float red[kThreads / 32];
+    const int h = blockIdx.x;
+    float s = 0.f;
+    if (dD) {
+        const int64_t rows = int64_t(d.B) * d.T;
+        for (int64_t k = threadIdx.x; k < rows * d.P; k += blockDim.x) {
+            const int64_t row = k / d.P;
+            const int p = int(k % d.P);
+            const int64_t i = (row * d.H + h) * d.P + p;
+            s = fmaf(ld(dy, i), ld(x, i), s);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (dD) {
+            float t = 0.f;
+            for (int i = 0; i < kThreads / 32; ++i) t += red[i];
+            dD[h] = t;
+        }
+        float a = 0.f;
+        for (int b = 0; b < d.B; ++b) a += dA_part[int64_t(b) * d.H + h];
+        dA[h] = a;
+    }
+}
+
+// dB[b,t,g,n] = sum_{h in g} (dt_t / a_t) yb[b,T-1-t,h,n];  dC[b,t,g,n] = sum_{h in g} yc[b,t,h,n]
+template <typename T>
+__global__ void group_sums_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
+                                  const float *__restrict__ yb, const float *__restrict__ yc, T *__restrict__ dB,
+                                  T *__restrict__ dC) {
+    const int64_t total = int64_t(d.B) * d.T * d.G * d.N;
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
+         i += int64_t(gridDim.x) * blockDim.x) {
+        const int n = int(i % d.N);
+        int64_t r = i / d.N;
+        const int g = int(r % d.G);
+        r /= d.G;
+        const int t = int(r % d.T), b = int(r / d.T);
+        float sb = 0.f, sc = 0.f;
+        for (int k = 0; k < d.r; ++k) {
+            const int h = g * d.r + k;
+            const int64_t idt = off_dt(d, b, t) + h;
+            const float f = dt[idt] * __expf(-dt[idt] * A[h]);
+            sb = fmaf(f, yb[((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * d.N + n], sb);
+            sc += yc[((int64_t(b) * d.T + t) * d.H + h) * d.N + n];
+        }
+        dB[i] = from_f32<T>(sb);
+        dC[i] = from_f32<T>(sc);
+    }
+}
+
+unsigned grid_for(int64_t n) {
+    const int64_t g = (n + kThreads - 1) / kThreads;
+    return unsigned(g < 148 * 32 ? (g < 1 ? 1 : g) : 148 * 32);
+}
+
+template <typename T>
+cudaError_t backward_prep_t(const Dims &d, const void *x, const void *dy, const float *dt, const float *A,
+                            const void *Bm, const void *Cm, const BackwardBuffers &w, cudaStream_t s) {
+    const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
+    const T *bb = static_cast<const T *>(Bm), *cc = static_cast<const T *>(Cm);
+    const int64_t nx = int64_t(d.B) * d.T * d.H * d.P, nbc = int64_t(d.B) * d.T * d.G * d.N;
+    const int64_t nn = int64_t(d.B) * d.T * d.H * d.N;
+    prep_k_kernel<T><<<grid_for(nx + nbc), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk, w.ck);
+    prep_t_kernel<T><<<grid_for(nn + nx), kThreads, 0, s>>>(d, xx, dyy, dt, A, bb, cc, w.xb, w.xc, w.dyr, w.xrr);
+    if (w.xf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(xx, w.xf, nx);
+    if (w.dyf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(dyy, w.dyf, nx);
+    if (w.bf) to_f32_kernel<T><<<grid_for(nbc), kThreads, 0, s>>>(bb, w.bf, nbc);
+    if (w.cf) to_f32_kernel<T><<<grid_for(nbc), kThreads, 0, s>>>(cc, w.cf, nbc);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const float *dt, const float *A,
+                            const float *D, const float *h0, const BackwardBuffers &w, void *dx, float *ddt,
+                            float *dA, void *dB, void *dC, float *dD, cudaStream_t s) {
+    const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
+    const int64_t nw = int64_t(d.B) * d.T * d.H;
+    const int64_t BH = int64_t(d.B) * d.H;
+    post_k_kernel<T><<<grid_for(nw * 32), kThreads, 0, s>>>(d, xx, dyy, dt, A, D, w.yk, w.yh, static_cast<T *>(dx),
+                                                           w.xu, w.cc, w.rr);
+    r0_kernel<<<unsigned(BH), kThreads, 0, s>>>(BH, d.P * d.N, w.dh0, h0, w.R0);
+    prefix_kernel<<<grid_for(BH * 32), kThreads, 0, s>>>(d, dt, A, w.R0, w.xu, w.cc, w.rr, ddt, w.dA_part);
+    head_sums_kernel<T><<<unsigned(d.H), kThreads, 0, s>>>(d, w.dA_part, xx, dyy, dA, dD);
+    group_sums_kernel<T><<<grid_for(int64_t(d.B) * d.T * d.G * d.N), kThreads, 0, s>>>(
+        d, dt, A, w.yb, w.yc, static_cast<T *>(dB), static_cast<T *>(dC));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward_prep(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
+                                 const float *A, const void *Bm, const void *Cm, const BackwardBuffers &w,
+                                 cudaStream_t stream) {
+    return bf16 ? backward_prep_t<__nv_bfloat16>(d, x, dy, dt, A, Bm, Cm, w, stream)
+                : backward_prep_t<float>(d, x, dy, dt, A, Bm, Cm, w, stream);
+}
+
+cudaError_t launch_transpose_state(int64_t BH, int P, int N, const float *s, float *st, cudaStream_t stream) {
+    transpose_state_kernel<<<grid_for(BH * P * N), kThreads, 0, stream>>>(BH, P, N, s, st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward_post(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
+                                 const float *A, const float *D, const float *h0, const BackwardBuffers &w,
+                                 void *dx, float *ddt, float *dA, void *dB, void *dC, float *dD,
+                                 cudaStream_t stream) {
+    return bf16 ? backward_post_t<__nv_bfloat16>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream)
+                : backward_post_t<float>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream);
+}
+
+}  // namespace ssd

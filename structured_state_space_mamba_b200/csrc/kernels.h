@@ -113,4 +113,27 @@ cudaError_t launch_tail(const Dims &d, bool bf16, int t_begin, const void *x, co
                         const float *dt_bias, int dt_softplus, const float *A, const void *Bm, const void *Cm,
                         const float *D, const float *h_in, void *y, float *fin, cudaStream_t stream);
 
+// The backward pass's own kernels (the scans run through the forward plans).
+// Buffers, fp32 (reversed = token t stored at T-1-t):
+//   xk [B,T,H,P] a_t dy_t / dt_t reversed;  dtr [B,T,H] dt reversed;
+//   bk, ck [B,T,G,N] C and B reversed      (the scan of K = dL/dh_{t-1})
+//   xb [B,T,H,N] a_t C_t / dt_t reversed;  dyr, xrr [B,T,H,P] dy, x reversed
+//                                          (the transposed scan for dB)
+//   xc [B,T,H,N] B per head                (the transposed forward scan for dC)
+//   xf, dyf [B,T,H,P], bf, cf [B,T,G,N]    fp32 copies (nullptr: the inputs are fp32)
+//   yk, yh [B,T,H,P], yb, yc [B,T,H,N]     the scans' outputs
+//   dh0 [B,H,P,N]; xu, cc, rr [B,T,H]; R0, dA_part [B,H]
+struct BackwardBuffers {
+    float *xk, *dtr, *bk, *ck, *xb, *xc, *dyr, *xrr, *xf, *dyf, *bf, *cf;
+    float *yk, *yh, *yb, *yc, *dh0, *xu, *cc, *rr, *R0, *dA_part;
+};
+cudaError_t launch_backward_prep(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
+                                 const float *A, const void *Bm, const void *Cm, const BackwardBuffers &w,
+                                 cudaStream_t stream);
+cudaError_t launch_transpose_state(int64_t BH, int P, int N, const float *s, float *st, cudaStream_t stream);
+cudaError_t launch_backward_post(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
+                                 const float *A, const float *D, const float *h0, const BackwardBuffers &w,
+                                 void *dx, float *ddt, float *dA, void *dB, void *dC, float *dD,
+                                 cudaStream_t stream);
+
 }  // namespace ssd

@@ -535,6 +535,101 @@ ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *cu_seqlen
     return SSD_OK;
 }
 
+// ---------------------------------------------------------------------------
+// backward: the reverse mode, through four fp32 scans of the forward plans and
+// the element-wise / prefix kernels of k_backward.cu
+// ---------------------------------------------------------------------------
+ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt, const float *A, const void *Bm,
+                          const void *Cm, const float *D, int chunk_len, const float *init_state, const void *dy,
+                          const float *dfinal_state, void *dx, float *ddt, float *dA, void *dB, void *dC,
+                          float *dD, float *dinit_state, void *stream) {
+    Plan pf;
+    ssd_status_t s = make_plan(dims, chunk_len, &pf);
+    if (s != SSD_OK) return s;
+    if (!x || !dt || !A || !Bm || !Cm || !dy || !dx || !ddt || !dA || !dB || !dC) return SSD_ERR_NULL_ARG;
+    {
+        const void *ptrs[] = {x, dt, A, Bm, Cm, D, init_state, dy, dfinal_state, dx, ddt, dA, dB, dC, dD,
+                              dinit_state};
+        for (const void *p : ptrs)
+            if (misaligned(p)) return SSD_ERR_MISALIGNED;
+    }
+    const ssd_dims_t &a = *dims;
+    // the scans of the backward run in fp32: K and h with the forward's shape,
+    // the transposed ones (dB, dC) with headdim and dstate swapped and one group per head
+    ssd_dims_t dk = a;
+    dk.dtype = SSD_F32;
+    ssd_dims_t dtp = dk;
+    dtp.headdim = a.dstate;
+    dtp.dstate = a.headdim;
+    dtp.ngroups = a.nheads;
+    Plan pk, pt;
+    if (make_plan(&dk, chunk_len, &pk) != SSD_OK || make_plan(&dtp, chunk_len, &pt) != SSD_OK)
+        return SSD_ERR_UNSUPPORTED;
+    const bool bf16 = a.dtype == SSD_BF16;
+    const Dims &d = pf.d;
+    const size_t nx = size_t(a.batch) * a.seqlen * a.nheads * a.headdim;
+    const size_t nn = size_t(a.batch) * a.seqlen * a.nheads * a.dstate;
+    const size_t nbc = size_t(a.batch) * a.seqlen * a.ngroups * a.dstate;
+    const size_t ntok = size_t(a.batch) * a.seqlen * a.nheads;
+    const size_t nst = size_t(a.batch) * a.nheads * a.headdim * a.dstate;
+    const size_t nbh = size_t(a.batch) * a.nheads;
+    // one allocation: the buffers, the transposed states and the scans' workspace
+    size_t off = 0;
+    auto take = [&](size_t n) { const size_t o = off; off = align_up(off + n * sizeof(float)); return o; };
+    const size_t o_xk = take(nx), o_dtr = take(ntok), o_bk = take(nbc), o_ck = take(nbc), o_xb = take(nn),
+                 o_xc = take(nn), o_dyr = take(nx), o_xrr = take(nx);
+    const size_t o_xf = bf16 ? take(nx) : 0, o_dyf = bf16 ? take(nx) : 0, o_bf = bf16 ? take(nbc) : 0,
+                 o_cf = bf16 ? take(nbc) : 0;
+    const size_t o_yk = take(nx), o_yh = take(nx), o_yb = take(nn), o_yc = take(nn);
+    const size_t o_dh0 = dinit_state ? 0 : take(nst);
+    const size_t o_xu = take(ntok), o_cc = take(ntok), o_rr = take(ntok), o_R0 = take(nbh), o_dAp = take(nbh);
+    const size_t o_ft = dfinal_state ? take(nst) : 0, o_ht = init_state ? take(nst) : 0;
+    const size_t o_ws = off;
+    off = align_up(off + (pk.ws.total_bytes > pt.ws.total_bytes ? pk.ws.total_bytes : pt.ws.total_bytes));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *buf = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&buf), off, st) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_WORKSPACE;
+    }
+    auto F = [&](size_t o) { return reinterpret_cast<float *>(buf + o); };
+    ssd::BackwardBuffers w;
+    w.xk = F(o_xk); w.dtr = F(o_dtr); w.bk = F(o_bk); w.ck = F(o_ck); w.xb = F(o_xb); w.xc = F(o_xc);
+    w.dyr = F(o_dyr); w.xrr = F(o_xrr);
+    w.xf = bf16 ? F(o_xf) : nullptr; w.dyf = bf16 ? F(o_dyf) : nullptr;
+    w.bf = bf16 ? F(o_bf) : nullptr; w.cf = bf16 ? F(o_cf) : nullptr;
+    w.yk = F(o_yk); w.yh = F(o_yh); w.yb = F(o_yb); w.yc = F(o_yc);
+    w.dh0 = dinit_state ? dinit_state : F(o_dh0);
+    w.xu = F(o_xu); w.cc = F(o_cc); w.rr = F(o_rr); w.R0 = F(o_R0); w.dA_part = F(o_dAp);
+    float *ft = dfinal_state ? F(o_ft) : nullptr, *ht = init_state ? F(o_ht) : nullptr;
+    char *ws = buf + o_ws;
+    const float *xf = bf16 ? w.xf : static_cast<const float *>(x);
+    const float *dyf = bf16 ? w.dyf : static_cast<const float *>(dy);
+    const float *bfp = bf16 ? w.bf : static_cast<const float *>(Bm);
+    const float *cfp = bf16 ? w.cf : static_cast<const float *>(Cm);
+    s = SSD_OK;
+    if (ssd::launch_backward_prep(d, bf16, x, dy, dt, A, Bm, Cm, w, st) != cudaSuccess) s = SSD_ERR_CUDA;
+    if (s == SSD_OK && ft &&
+        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), dfinal_state, ft, st) != cudaSuccess)
+        s = SSD_ERR_CUDA;
+    if (s == SSD_OK && ht &&
+        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), init_state, ht, st) != cudaSuccess)
+        s = SSD_ERR_CUDA;
+    // K = dL/dh_{t-1}, backwards in time: read out against B, final state dh0
+    if (s == SSD_OK) s = run(pk, w.xk, w.dtr, A, w.bk, w.ck, nullptr, dfinal_state, w.yk, w.dh0, ws, st);
+    // h_t C_t (the forward without the skip term)
+    if (s == SSD_OK) s = run(pk, xf, dt, A, bfp, cfp, nullptr, init_state, w.yh, nullptr, ws, st);
+    // K^T read out against x (dB), backwards in time
+    if (s == SSD_OK) s = run(pt, w.xb, w.dtr, A, w.dyr, w.xrr, nullptr, ft, w.yb, nullptr, ws, st);
+    // h^T read out against dy (dC)
+    if (s == SSD_OK) s = run(pt, w.xc, dt, A, xf, dyf, nullptr, ht, w.yc, nullptr, ws, st);
+    if (s == SSD_OK &&
+        ssd::launch_backward_post(d, bf16, x, dy, dt, A, D, init_state, w, dx, ddt, dA, dB, dC, dD, st) != cudaSuccess)
+        s = SSD_ERR_CUDA;
+    if (cudaFreeAsync(buf, st) != cudaSuccess && s == SSD_OK) s = SSD_ERR_CUDA;
+    return s;
+}
+
 const char *ssd_status_string(ssd_status_t status) {
     switch (status) {
         case SSD_OK: return "SSD_OK: success";
