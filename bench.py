@@ -593,6 +593,118 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
 
 # ---------------------------------------------------------------------------
+# backward (ssd_backward): the gradients of every input for one batch
+# ---------------------------------------------------------------------------
+BACKWARD_METRIC = "SSD backward tokens/sec on 1 B200 (gradients of every input) and % of HBM roofline"
+
+
+def backward_launches(inp):
+    """Kernels one ssd_backward call launches: the input preparation, the
+    transposed states, four fp32 scans (each its plan's launches) and the five
+    kernels that finish the gradients."""
+    from structured_state_space_mamba_b200 import binding
+    B_, T, H, P = inp.x.shape
+    G, N = inp.B.shape[2], inp.B.shape[3]
+    fwd = binding.workspace_layout(binding.make_dims(B_, T, H, P, N, G, "f32"), inp.chunk_len).launches
+    tr = binding.workspace_layout(binding.make_dims(B_, T, H, N, P, H, "f32"), inp.chunk_len).launches
+    prep = 2 + (4 if inp.dtype == "bf16" else 0)
+    states = 1 + (1 if inp.h0 is not None else 0)  # dfinal (always given here) and h0
+    return prep + states + 2 * fwd + 2 * tr + 5
+
+
+def run_backward(args, cfg, rank, world, local_rank):
+    import torch
+    from structured_state_space_mamba_b200 import binding
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = make_workload(args.workload, **({"batch": cfg["batch"]} if args.batch else {}))
+    tt = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    rng = np.random.default_rng(4000 + rank)
+    dy_h = rng.standard_normal(inp.x.shape).astype(np.float32)
+    fin_h = rng.standard_normal((inp.x.shape[0], inp.x.shape[2], inp.x.shape[3], inp.B.shape[3])).astype(np.float32)
+    host = dict(x=(inp.x, tt), dt=(inp.dt, torch.float32), A=(inp.A, torch.float32), B=(inp.B, tt),
+                C=(inp.C, tt), D=(inp.D, torch.float32), dy=(dy_h, tt), dfin=(fin_h, torch.float32))
+    if inp.h0 is not None:
+        host["h0"] = (inp.h0, torch.float32)
+    pinned = {k: torch.from_numpy(np.ascontiguousarray(v)).to(ty).pin_memory() for k, (v, ty) in host.items()}
+    d = {k: v.to(dev) for k, v in pinned.items()}
+    stream = torch.cuda.current_stream(dev)
+    outs = {}
+
+    def step():
+        outs["g"] = binding.backward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dy"], D=d["D"],
+                                     chunk_len=inp.chunk_len, init_state=d.get("h0"), dfinal_state=d["dfin"])
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_identity(local_rank)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    clocks = clk.summary()
+    # end to end: inputs and dy in from pinned host memory, every gradient back
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    d2h = 0
+    for _ in range(args.steps):
+        for k, v in pinned.items():
+            d[k].copy_(v, non_blocking=True)
+        step()
+        d2h = 0
+        for g in outs["g"].values():
+            if g is not None:
+                g.cpu()
+                d2h += g.numel() * g.element_size()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
+    if rank != 0:
+        return
+    B_, T, H, P = inp.x.shape
+    G, N = inp.B.shape[2], inp.B.shape[3]
+    esz = 2 if inp.dtype == "bf16" else 4
+    st = B_ * H * P * N * 4
+    # compulsory bytes: x, dy, B, C, dt, A, D, h0, dfinal in; dx, dB, dC, ddt, dA, dD, dinit out
+    comp = (3 * B_ * T * H * P * esz + 4 * B_ * T * G * N * esz + 2 * B_ * T * H * 4 + 4 * H * 4
+            + (2 * st if inp.h0 is not None else 0) + st)
+    t_step = ms / args.steps * 1e-3
+    peaks, peak_src = load_peaks()
+    achieved = comp / t_step / 1e9
+    line = {
+        "metric": BACKWARD_METRIC, "value": job_rate(world, B_ * T, args.steps, ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
+        "data": "synthetic", "config": dict(config_block(cfg, args.workload), backward=True),
+        "roofline": {"bound": "hbm", "kernel": "ssd_backward (whole call)", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                     "compulsory_bytes": comp},
+        "launch": "one ssd_backward call per step (four fp32 scans and the element-wise kernels)",
+        "gpu_launches": args.steps * backward_launches(inp),
+        "e2e": {"value": job_rate(world, B_ * T, args.steps, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
 # decode step (ssd_step): one token per (batch, head) on a resident state
 # ---------------------------------------------------------------------------
 DECODE = dict(batch=64, nheads=80, headdim=64, dstate=128, ngroups=1, dtype="bf16")
@@ -732,6 +844,8 @@ def main():
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (ssd_step) on its own shape instead of the scan")
+    ap.add_argument("--backward", action="store_true",
+                    help="time ssd_backward (the gradients of every input) on the workload")
     ap.add_argument("--block", action="store_true",
                     help="time ssd_forward_block: softplus(dt + dt_bias), the scan, y * silu(z) "
                          "and RMSNorm over each token's H * P values")
@@ -760,6 +874,8 @@ def main():
     try:
         if args.decode:
             run_decode(args, rank, world, local_rank)
+        elif args.backward:
+            run_backward(args, cfg, rank, world, local_rank)
         else:
             run_gpu(args, cfg, rank, world, local_rank)
     finally:
