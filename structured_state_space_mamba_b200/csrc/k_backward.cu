@@ -34,11 +34,11 @@ __device__ __forceinline__ float decay(const float *dt, const float *A, int64_t 
 
 // scan K (reversed): xr[b,tau,h,p] = a_t dy[b,t,h,p] / dt_t, dtr[b,tau,h] = dt_t,
 // and (per group) Br = C, Cr = B, all at tau = T-1-t
-template <typename T>
+template <typename T, typename TS>
 __global__ void prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__restrict__ dt,
                               const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
-                              float *__restrict__ xr, float *__restrict__ dtr, float *__restrict__ Br,
-                              float *__restrict__ Cr) {
+                              TS *__restrict__ xr, float *__restrict__ dtr, TS *__restrict__ Br,
+                              TS *__restrict__ Cr) {
     const int64_t n_x = int64_t(d.B) * d.T * d.H * d.P;
     const int64_t n_bc = int64_t(d.B) * d.T * d.G * d.N;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_x + n_bc;
@@ -52,7 +52,7 @@ __global__ void prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__r
             const int tau = d.T - 1 - t;
             const int64_t idt = off_dt(d, b, t) + h;
             const float dtt = dt[idt];
-            xr[off_x(d, b, tau, h) + p] = decay(dt, A, idt, h) * ld(dy, i) / dtt;
+            xr[off_x(d, b, tau, h) + p] = from_f32<TS>(decay(dt, A, idt, h) * ld(dy, i) / dtt);
             if (p == 0) dtr[off_dt(d, b, tau) + h] = dtt;
         } else {
             const int64_t j = i - n_x;
@@ -62,8 +62,8 @@ __global__ void prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__r
             r /= d.G;
             const int t = int(r % d.T), b = int(r / d.T);
             const int64_t dst = off_bc(d, b, d.T - 1 - t, g) + n;
-            Br[dst] = ld(Cm, j);
-            Cr[dst] = ld(Bm, j);
+            Br[dst] = from_f32<TS>(ld(Cm, j));
+            Cr[dst] = from_f32<TS>(ld(Bm, j));
         }
     }
 }
@@ -80,11 +80,14 @@ __global__ void to_f32_kernel(const T *__restrict__ src, float *__restrict__ dst
 //   forward  (dC): xc[b,t,h,n]   = B[b,t,g,n]
 // and the per-head rows of the reversed ones:
 //   dyr[b,tau,h,p] = dy[b,t,h,p],  xrr[b,tau,h,p] = x[b,t,h,p]
-template <typename T>
-__global__ void prep_t_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ dy,
+template <typename T, typename TS>
+__global__ void prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy,
                               const float *__restrict__ dt, const float *__restrict__ A,
-                              const T *__restrict__ Bm, const T *__restrict__ Cm, float *__restrict__ xb,
-                              float *__restrict__ xc, float *__restrict__ dyr, float *__restrict__ xrr) {
+                              const T *__restrict__ Bm, const T *__restrict__ Cm, TS *__restrict__ xb,
+                              TS *__restrict__ xc, TS *__restrict__ dyr, TS *__restrict__ xrr) {
+    // xb and xc are split along dstate into slices of W columns, slice-major:
+    // slice s holds [B, T, H, W] (each slice is one transposed scan's x)
+    const int64_t slice = int64_t(d.B) * d.T * d.H * W;
     const int64_t n_n = int64_t(d.B) * d.T * d.H * d.N;
     const int64_t n_p = int64_t(d.B) * d.T * d.H * d.P;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_n + n_p;
@@ -98,9 +101,11 @@ __global__ void prep_t_kernel(Dims d, const T *__restrict__ x, const T *__restri
             const int g = h / d.r;
             const int64_t idt = off_dt(d, b, t) + h;
             const int64_t src = off_bc(d, b, t, g) + n;
-            const int64_t rowr = ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * d.N + n;
-            xb[rowr] = decay(dt, A, idt, h) * ld(Cm, src) / dt[idt];
-            xc[i] = ld(Bm, src);
+            const int sl = n / W, nn = n % W;
+            const int64_t rowr = sl * slice + ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * W + nn;
+            const int64_t rowf = sl * slice + ((int64_t(b) * d.T + t) * d.H + h) * W + nn;
+            xb[rowr] = from_f32<TS>(decay(dt, A, idt, h) * ld(Cm, src) / dt[idt]);
+            xc[rowf] = from_f32<TS>(ld(Bm, src));
         } else {
             const int64_t j = i - n_n;
             const int p = int(j % d.P);
@@ -109,14 +114,15 @@ __global__ void prep_t_kernel(Dims d, const T *__restrict__ x, const T *__restri
             r /= d.H;
             const int t = int(r % d.T), b = int(r / d.T);
             const int64_t dst = off_x(d, b, d.T - 1 - t, h) + p;
-            dyr[dst] = ld(dy, j);
-            xrr[dst] = ld(x, j);
+            dyr[dst] = from_f32<TS>(ld(dy, j));
+            xrr[dst] = from_f32<TS>(ld(x, j));
         }
     }
 }
 
-// [B, H, P, N] -> [B, H, N, P] (a state as the transposed scans hold it)
-__global__ void transpose_state_kernel(int64_t BH, int P, int N, const float *__restrict__ s,
+// [B, H, P, N] -> slices of [B, H, W, P] (a state as the transposed scans
+// hold it, dstate split into slices of W rows, slice-major)
+__global__ void transpose_state_kernel(int64_t BH, int P, int N, int W, const float *__restrict__ s,
                                        float *__restrict__ st) {
     const int64_t total = BH * P * N;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
@@ -125,17 +131,18 @@ __global__ void transpose_state_kernel(int64_t BH, int P, int N, const float *__
         const int64_t r = i / N;
         const int p = int(r % P);
         const int64_t bh = r / P;
-        st[(bh * N + n) * P + p] = s[i];
+        const int sl = n / W, nn = n % W;
+        st[sl * BH * W * P + (bh * W + nn) * P + p] = s[i];
     }
 }
 
 // one warp per (b, t, h): u = G_t B_t = yk / a_t (yk from the reversed scan),
 // dx = dt u + D dy, xu = x . u, c = dt xu, r = dy . yh (yh = h_t C_t)
-template <typename T>
+template <typename T, typename TS>
 __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ dy,
                               const float *__restrict__ dt, const float *__restrict__ A,
-                              const float *__restrict__ D, const float *__restrict__ yk,
-                              const float *__restrict__ yh, T *__restrict__ dx, float *__restrict__ xu,
+                              const float *__restrict__ D, const TS *__restrict__ yk,
+                              const TS *__restrict__ yh, T *__restrict__ dx, float *__restrict__ xu,
                               float *__restrict__ cc, float *__restrict__ rr) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = int64_t(d.B) * d.T * d.H;
@@ -152,11 +159,11 @@ __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restri
         const int64_t rowr = off_x(d, b, d.T - 1 - t, h);
         float sx = 0.f, sr = 0.f;
         for (int p = lane; p < d.P; p += 32) {
-            const float u = yk[rowr + p] * inv_a;
+            const float u = ld(yk, rowr + p) * inv_a;
             const float dyp = ld(dy, row + p);
             dx[row + p] = from_f32<T>(dtt * u + Dh * dyp);
             sx = fmaf(ld(x, row + p), u, sx);
-            sr = fmaf(dyp, yh[row + p], sr);
+            sr = fmaf(dyp, ld(yh, row + p), sr);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -262,10 +269,11 @@ __global__ void head_sums_kernel(Dims d, const float *__restrict__ dA_part, cons
 }
 
 // dB[b,t,g,n] = sum_{h in g} (dt_t / a_t) yb[b,T-1-t,h,n];  dC[b,t,g,n] = sum_{h in g} yc[b,t,h,n]
-template <typename T>
-__global__ void group_sums_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
-                                  const float *__restrict__ yb, const float *__restrict__ yc, T *__restrict__ dB,
+template <typename T, typename TS>
+__global__ void group_sums_kernel(Dims d, int W, const float *__restrict__ dt, const float *__restrict__ A,
+                                  const TS *__restrict__ yb, const TS *__restrict__ yc, T *__restrict__ dB,
                                   T *__restrict__ dC) {
+    const int64_t slice = int64_t(d.B) * d.T * d.H * W;
     const int64_t total = int64_t(d.B) * d.T * d.G * d.N;
     for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
          i += int64_t(gridDim.x) * blockDim.x) {
@@ -274,13 +282,14 @@ __global__ void group_sums_kernel(Dims d, const float *__restrict__ dt, const fl
         const int g = int(r % d.G);
         r /= d.G;
         const int t = int(r % d.T), b = int(r / d.T);
+        const int sl = n / W, nn = n % W;
         float sb = 0.f, sc = 0.f;
         for (int k = 0; k < d.r; ++k) {
             const int h = g * d.r + k;
             const int64_t idt = off_dt(d, b, t) + h;
             const float f = dt[idt] * __expf(-dt[idt] * A[h]);
-            sb = fmaf(f, yb[((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * d.N + n], sb);
-            sc += yc[((int64_t(b) * d.T + t) * d.H + h) * d.N + n];
+            sb = fmaf(f, ld(yb, sl * slice + ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * W + nn), sb);
+            sc += ld(yc, sl * slice + ((int64_t(b) * d.T + t) * d.H + h) * W + nn);
         }
         dB[i] = from_f32<T>(sb);
         dC[i] = from_f32<T>(sc);
@@ -292,15 +301,18 @@ unsigned grid_for(int64_t n) {
     return unsigned(g < 148 * 32 ? (g < 1 ? 1 : g) : 148 * 32);
 }
 
-template <typename T>
+template <typename T, typename TS>
 cudaError_t backward_prep_t(const Dims &d, const void *x, const void *dy, const float *dt, const float *A,
                             const void *Bm, const void *Cm, const BackwardBuffers &w, cudaStream_t s) {
     const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
     const T *bb = static_cast<const T *>(Bm), *cc = static_cast<const T *>(Cm);
     const int64_t nx = int64_t(d.B) * d.T * d.H * d.P, nbc = int64_t(d.B) * d.T * d.G * d.N;
     const int64_t nn = int64_t(d.B) * d.T * d.H * d.N;
-    prep_k_kernel<T><<<grid_for(nx + nbc), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk, w.ck);
-    prep_t_kernel<T><<<grid_for(nn + nx), kThreads, 0, s>>>(d, xx, dyy, dt, A, bb, cc, w.xb, w.xc, w.dyr, w.xrr);
+    prep_k_kernel<T, float><<<grid_for(nx + nbc), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk,
+                                                                    w.ck);
+    prep_t_kernel<T, TS><<<grid_for(nn + nx), kThreads, 0, s>>>(d, w.W, xx, dyy, dt, A, bb, cc,
+                                                                static_cast<TS *>(w.xb), static_cast<TS *>(w.xc),
+                                                                static_cast<TS *>(w.dyr), static_cast<TS *>(w.xrr));
     if (w.xf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(xx, w.xf, nx);
     if (w.dyf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(dyy, w.dyf, nx);
     if (w.bf) to_f32_kernel<T><<<grid_for(nbc), kThreads, 0, s>>>(bb, w.bf, nbc);
@@ -308,20 +320,21 @@ cudaError_t backward_prep_t(const Dims &d, const void *x, const void *dy, const 
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, typename TS>
 cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const float *dt, const float *A,
                             const float *D, const float *h0, const BackwardBuffers &w, void *dx, float *ddt,
                             float *dA, void *dB, void *dC, float *dD, cudaStream_t s) {
     const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
     const int64_t nw = int64_t(d.B) * d.T * d.H;
     const int64_t BH = int64_t(d.B) * d.H;
-    post_k_kernel<T><<<grid_for(nw * 32), kThreads, 0, s>>>(d, xx, dyy, dt, A, D, w.yk, w.yh, static_cast<T *>(dx),
-                                                           w.xu, w.cc, w.rr);
+    post_k_kernel<T, float><<<grid_for(nw * 32), kThreads, 0, s>>>(d, xx, dyy, dt, A, D, w.yk, w.yh,
+                                                                  static_cast<T *>(dx), w.xu, w.cc, w.rr);
     r0_kernel<<<unsigned(BH), kThreads, 0, s>>>(BH, d.P * d.N, w.dh0, h0, w.R0);
     prefix_kernel<<<grid_for(BH * 32), kThreads, 0, s>>>(d, dt, A, w.R0, w.xu, w.cc, w.rr, ddt, w.dA_part);
     head_sums_kernel<T><<<unsigned(d.H), kThreads, 0, s>>>(d, w.dA_part, xx, dyy, dA, dD);
-    group_sums_kernel<T><<<grid_for(int64_t(d.B) * d.T * d.G * d.N), kThreads, 0, s>>>(
-        d, dt, A, w.yb, w.yc, static_cast<T *>(dB), static_cast<T *>(dC));
+    group_sums_kernel<T, TS><<<grid_for(int64_t(d.B) * d.T * d.G * d.N), kThreads, 0, s>>>(
+        d, w.W, dt, A, static_cast<const TS *>(w.yb), static_cast<const TS *>(w.yc), static_cast<T *>(dB),
+        static_cast<T *>(dC));
     return cudaGetLastError();
 }
 
@@ -330,12 +343,13 @@ cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const 
 cudaError_t launch_backward_prep(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
                                  const float *A, const void *Bm, const void *Cm, const BackwardBuffers &w,
                                  cudaStream_t stream) {
-    return bf16 ? backward_prep_t<__nv_bfloat16>(d, x, dy, dt, A, Bm, Cm, w, stream)
-                : backward_prep_t<float>(d, x, dy, dt, A, Bm, Cm, w, stream);
+    if (!bf16) return backward_prep_t<float, float>(d, x, dy, dt, A, Bm, Cm, w, stream);
+    return w.scan_bf16 ? backward_prep_t<__nv_bfloat16, __nv_bfloat16>(d, x, dy, dt, A, Bm, Cm, w, stream)
+                       : backward_prep_t<__nv_bfloat16, float>(d, x, dy, dt, A, Bm, Cm, w, stream);
 }
 
-cudaError_t launch_transpose_state(int64_t BH, int P, int N, const float *s, float *st, cudaStream_t stream) {
-    transpose_state_kernel<<<grid_for(BH * P * N), kThreads, 0, stream>>>(BH, P, N, s, st);
+cudaError_t launch_transpose_state(int64_t BH, int P, int N, int W, const float *s, float *st, cudaStream_t stream) {
+    transpose_state_kernel<<<grid_for(BH * P * N), kThreads, 0, stream>>>(BH, P, N, W, s, st);
     return cudaGetLastError();
 }
 
@@ -343,8 +357,11 @@ cudaError_t launch_backward_post(const Dims &d, bool bf16, const void *x, const 
                                  const float *A, const float *D, const float *h0, const BackwardBuffers &w,
                                  void *dx, float *ddt, float *dA, void *dB, void *dC, float *dD,
                                  cudaStream_t stream) {
-    return bf16 ? backward_post_t<__nv_bfloat16>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream)
-                : backward_post_t<float>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream);
+    if (!bf16) return backward_post_t<float, float>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream);
+    return w.scan_bf16
+               ? backward_post_t<__nv_bfloat16, __nv_bfloat16>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD,
+                                                               stream)
+               : backward_post_t<__nv_bfloat16, float>(d, x, dy, dt, A, D, h0, w, dx, ddt, dA, dB, dC, dD, stream);
 }
 
 }  // namespace ssd

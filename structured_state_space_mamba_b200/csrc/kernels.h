@@ -114,23 +114,29 @@ cudaError_t launch_tail(const Dims &d, bool bf16, int t_begin, const void *x, co
                         const float *D, const float *h_in, void *y, float *fin, cudaStream_t stream);
 
 // The backward pass's own kernels (the scans run through the forward plans).
-// Buffers, fp32 (reversed = token t stored at T-1-t):
+// The scans that feed the decay terms (K and h) run in fp32; the transposed
+// ones (dB, dC) hold bf16 when scan_bf16 (they then take the tensor-core
+// plans), fp32 otherwise.  Reversed = token t stored at T-1-t:
 //   xk [B,T,H,P] a_t dy_t / dt_t reversed;  dtr [B,T,H] dt reversed;
-//   bk, ck [B,T,G,N] C and B reversed      (the scan of K = dL/dh_{t-1})
-//   xb [B,T,H,N] a_t C_t / dt_t reversed;  dyr, xrr [B,T,H,P] dy, x reversed
-//                                          (the transposed scan for dB)
-//   xc [B,T,H,N] B per head                (the transposed forward scan for dC)
-//   xf, dyf [B,T,H,P], bf, cf [B,T,G,N]    fp32 copies (nullptr: the inputs are fp32)
-//   yk, yh [B,T,H,P], yb, yc [B,T,H,N]     the scans' outputs
+//   bk, ck [B,T,G,N] C and B reversed       (the scan of K = dL/dh_{t-1})
+//   xb [S][B,T,H,W] a_t C_t / dt_t reversed, dstate in S slices of W columns;
+//   dyr, xrr [B,T,H,P] dy, x reversed       (the transposed scans for dB)
+//   xc [S][B,T,H,W] B per head               (the transposed forward scans for dC)
+//   xf, bf, cf: fp32 copies of x, B, C for the scan of h (nullptr: fp32 inputs);
+//   dyf: fp32 copy of dy for fp32 transposed scans of bf16 inputs
+//   yk, yh [B,T,H,P] fp32, yb, yc [S][B,T,H,W]   the scans' outputs
 //   dh0 [B,H,P,N]; xu, cc, rr [B,T,H]; R0, dA_part [B,H]
 struct BackwardBuffers {
-    float *xk, *dtr, *bk, *ck, *xb, *xc, *dyr, *xrr, *xf, *dyf, *bf, *cf;
-    float *yk, *yh, *yb, *yc, *dh0, *xu, *cc, *rr, *R0, *dA_part;
+    void *xb, *xc, *dyr, *xrr, *yb, *yc;
+    float *xk, *bk, *ck, *yk, *yh;
+    float *dtr, *xf, *dyf, *bf, *cf, *dh0, *xu, *cc, *rr, *R0, *dA_part;
+    int W;           // dstate columns per transposed scan
+    bool scan_bf16;  // transposed-scan buffers in bf16
 };
 cudaError_t launch_backward_prep(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
                                  const float *A, const void *Bm, const void *Cm, const BackwardBuffers &w,
                                  cudaStream_t stream);
-cudaError_t launch_transpose_state(int64_t BH, int P, int N, const float *s, float *st, cudaStream_t stream);
+cudaError_t launch_transpose_state(int64_t BH, int P, int N, int W, const float *s, float *st, cudaStream_t stream);
 cudaError_t launch_backward_post(const Dims &d, bool bf16, const void *x, const void *dy, const float *dt,
                                  const float *A, const float *D, const float *h0, const BackwardBuffers &w,
                                  void *dx, float *ddt, float *dA, void *dB, void *dC, float *dD,

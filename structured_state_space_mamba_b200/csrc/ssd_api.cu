@@ -554,18 +554,34 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
             if (misaligned(p)) return SSD_ERR_MISALIGNED;
     }
     const ssd_dims_t &a = *dims;
-    // the scans of the backward run in fp32: K and h with the forward's shape,
-    // the transposed ones (dB, dC) with headdim and dstate swapped and one group per head
+    const bool bf16 = a.dtype == SSD_BF16;
+    // The scans of the backward: K (= dL/dh_{t-1}, backwards in time) and h with
+    // the forward's shape, in fp32 (their outputs feed the decay terms' prefix
+    // sum, where bf16 outputs lose too much to cancellation), and the transposed
+    // ones for dB and dC with headdim and dstate swapped and one group per head,
+    // dstate split into S slices of W: bf16 on the tensor-core plans when the
+    // inputs are bf16 with headdim 64 and dstate a multiple of 64 (W = 64),
+    // else fp32 (W = dstate).
     ssd_dims_t dk = a;
     dk.dtype = SSD_F32;
-    ssd_dims_t dtp = dk;
-    dtp.headdim = a.dstate;
+    ssd_dims_t dtp = a;
     dtp.dstate = a.headdim;
     dtp.ngroups = a.nheads;
+    bool scan_bf16 = bf16 && a.headdim == 64 && a.dstate % 64 == 0;
     Plan pk, pt;
-    if (make_plan(&dk, chunk_len, &pk) != SSD_OK || make_plan(&dtp, chunk_len, &pt) != SSD_OK)
-        return SSD_ERR_UNSUPPORTED;
-    const bool bf16 = a.dtype == SSD_BF16;
+    if (make_plan(&dk, chunk_len, &pk) != SSD_OK) return SSD_ERR_UNSUPPORTED;
+    if (scan_bf16) {
+        dtp.headdim = 64;
+        if (make_plan(&dtp, chunk_len, &pt) != SSD_OK || !pt.tc_scan) scan_bf16 = false;
+    }
+    if (!scan_bf16) {
+        dtp.headdim = a.dstate;
+        dtp.dtype = SSD_F32;
+        if (make_plan(&dtp, chunk_len, &pt) != SSD_OK) return SSD_ERR_UNSUPPORTED;
+    }
+    const int W = scan_bf16 ? 64 : int(a.dstate);
+    const int S = int(a.dstate) / W;
+    const size_t es = scan_bf16 ? 2 : 4;  // bytes per scan-buffer element
     const Dims &d = pf.d;
     const size_t nx = size_t(a.batch) * a.seqlen * a.nheads * a.headdim;
     const size_t nn = size_t(a.batch) * a.seqlen * a.nheads * a.dstate;
@@ -573,17 +589,23 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
     const size_t ntok = size_t(a.batch) * a.seqlen * a.nheads;
     const size_t nst = size_t(a.batch) * a.nheads * a.headdim * a.dstate;
     const size_t nbh = size_t(a.batch) * a.nheads;
+    const size_t nsl = size_t(a.batch) * a.seqlen * a.nheads * W;        // one slice of xb, xc, yb, yc
+    const size_t nstsl = size_t(a.batch) * a.nheads * W * a.headdim;    // one slice of a transposed state
+    // fp32 copies of bf16 inputs: x, B, C for the scan of h; dy for fp32 transposed scans
+    const bool copies = bf16;
+    const bool dy_copy = bf16 && !scan_bf16;
     // one allocation: the buffers, the transposed states and the scans' workspace
     size_t off = 0;
-    auto take = [&](size_t n) { const size_t o = off; off = align_up(off + n * sizeof(float)); return o; };
-    const size_t o_xk = take(nx), o_dtr = take(ntok), o_bk = take(nbc), o_ck = take(nbc), o_xb = take(nn),
-                 o_xc = take(nn), o_dyr = take(nx), o_xrr = take(nx);
-    const size_t o_xf = bf16 ? take(nx) : 0, o_dyf = bf16 ? take(nx) : 0, o_bf = bf16 ? take(nbc) : 0,
-                 o_cf = bf16 ? take(nbc) : 0;
-    const size_t o_yk = take(nx), o_yh = take(nx), o_yb = take(nn), o_yc = take(nn);
-    const size_t o_dh0 = dinit_state ? 0 : take(nst);
-    const size_t o_xu = take(ntok), o_cc = take(ntok), o_rr = take(ntok), o_R0 = take(nbh), o_dAp = take(nbh);
-    const size_t o_ft = dfinal_state ? take(nst) : 0, o_ht = init_state ? take(nst) : 0;
+    auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes); return o; };
+    const size_t o_xk = take(nx * 4), o_dtr = take(ntok * 4), o_bk = take(nbc * 4), o_ck = take(nbc * 4),
+                 o_xb = take(nn * es), o_xc = take(nn * es), o_dyr = take(nx * es), o_xrr = take(nx * es);
+    const size_t o_xf = copies ? take(nx * 4) : 0, o_dyf = dy_copy ? take(nx * 4) : 0,
+                 o_bf = copies ? take(nbc * 4) : 0, o_cf = copies ? take(nbc * 4) : 0;
+    const size_t o_yk = take(nx * 4), o_yh = take(nx * 4), o_yb = take(nn * es), o_yc = take(nn * es);
+    const size_t o_dh0 = dinit_state ? 0 : take(nst * 4);
+    const size_t o_xu = take(ntok * 4), o_cc = take(ntok * 4), o_rr = take(ntok * 4), o_R0 = take(nbh * 4),
+                 o_dAp = take(nbh * 4);
+    const size_t o_ft = dfinal_state ? take(nst * 4) : 0, o_ht = init_state ? take(nst * 4) : 0;
     const size_t o_ws = off;
     off = align_up(off + (pk.ws.total_bytes > pt.ws.total_bytes ? pk.ws.total_bytes : pt.ws.total_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -593,36 +615,48 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
         return SSD_ERR_WORKSPACE;
     }
     auto F = [&](size_t o) { return reinterpret_cast<float *>(buf + o); };
+    auto V = [&](size_t o) { return static_cast<void *>(buf + o); };
     ssd::BackwardBuffers w;
-    w.xk = F(o_xk); w.dtr = F(o_dtr); w.bk = F(o_bk); w.ck = F(o_ck); w.xb = F(o_xb); w.xc = F(o_xc);
-    w.dyr = F(o_dyr); w.xrr = F(o_xrr);
-    w.xf = bf16 ? F(o_xf) : nullptr; w.dyf = bf16 ? F(o_dyf) : nullptr;
-    w.bf = bf16 ? F(o_bf) : nullptr; w.cf = bf16 ? F(o_cf) : nullptr;
-    w.yk = F(o_yk); w.yh = F(o_yh); w.yb = F(o_yb); w.yc = F(o_yc);
+    w.xk = F(o_xk); w.bk = F(o_bk); w.ck = F(o_ck); w.xb = V(o_xb); w.xc = V(o_xc);
+    w.dyr = V(o_dyr); w.xrr = V(o_xrr); w.yk = F(o_yk); w.yh = F(o_yh); w.yb = V(o_yb); w.yc = V(o_yc);
+    w.dtr = F(o_dtr);
+    w.xf = copies ? F(o_xf) : nullptr; w.dyf = dy_copy ? F(o_dyf) : nullptr;
+    w.bf = copies ? F(o_bf) : nullptr; w.cf = copies ? F(o_cf) : nullptr;
     w.dh0 = dinit_state ? dinit_state : F(o_dh0);
     w.xu = F(o_xu); w.cc = F(o_cc); w.rr = F(o_rr); w.R0 = F(o_R0); w.dA_part = F(o_dAp);
+    w.W = W;
+    w.scan_bf16 = scan_bf16;
     float *ft = dfinal_state ? F(o_ft) : nullptr, *ht = init_state ? F(o_ht) : nullptr;
     char *ws = buf + o_ws;
-    const float *xf = bf16 ? w.xf : static_cast<const float *>(x);
-    const float *dyf = bf16 ? w.dyf : static_cast<const float *>(dy);
-    const float *bfp = bf16 ? w.bf : static_cast<const float *>(Bm);
-    const float *cfp = bf16 ? w.cf : static_cast<const float *>(Cm);
+    // the forward-direction scans read the inputs themselves where their dtype fits
+    const void *xs = copies ? static_cast<const void *>(w.xf) : x;    // the fp32 scan of h
+    const void *bs = copies ? static_cast<const void *>(w.bf) : Bm;
+    const void *cs = copies ? static_cast<const void *>(w.cf) : Cm;
+    const void *xt = scan_bf16 || !bf16 ? x : static_cast<const void *>(w.xf);  // the transposed scans
+    const void *dyt = dy_copy ? static_cast<const void *>(w.dyf) : dy;
     s = SSD_OK;
     if (ssd::launch_backward_prep(d, bf16, x, dy, dt, A, Bm, Cm, w, st) != cudaSuccess) s = SSD_ERR_CUDA;
     if (s == SSD_OK && ft &&
-        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), dfinal_state, ft, st) != cudaSuccess)
+        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), W, dfinal_state, ft, st) !=
+            cudaSuccess)
         s = SSD_ERR_CUDA;
     if (s == SSD_OK && ht &&
-        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), init_state, ht, st) != cudaSuccess)
+        ssd::launch_transpose_state(int64_t(nbh), int(a.headdim), int(a.dstate), W, init_state, ht, st) !=
+            cudaSuccess)
         s = SSD_ERR_CUDA;
     // K = dL/dh_{t-1}, backwards in time: read out against B, final state dh0
     if (s == SSD_OK) s = run(pk, w.xk, w.dtr, A, w.bk, w.ck, nullptr, dfinal_state, w.yk, w.dh0, ws, st);
     // h_t C_t (the forward without the skip term)
-    if (s == SSD_OK) s = run(pk, xf, dt, A, bfp, cfp, nullptr, init_state, w.yh, nullptr, ws, st);
-    // K^T read out against x (dB), backwards in time
-    if (s == SSD_OK) s = run(pt, w.xb, w.dtr, A, w.dyr, w.xrr, nullptr, ft, w.yb, nullptr, ws, st);
-    // h^T read out against dy (dC)
-    if (s == SSD_OK) s = run(pt, w.xc, dt, A, xf, dyf, nullptr, ht, w.yc, nullptr, ws, st);
+    if (s == SSD_OK) s = run(pk, xs, dt, A, bs, cs, nullptr, init_state, w.yh, nullptr, ws, st);
+    for (int sl = 0; sl < S && s == SSD_OK; ++sl) {
+        char *xb = static_cast<char *>(w.xb) + sl * nsl * es, *xc = static_cast<char *>(w.xc) + sl * nsl * es;
+        char *yb = static_cast<char *>(w.yb) + sl * nsl * es, *yc = static_cast<char *>(w.yc) + sl * nsl * es;
+        // K^T read out against x (dB), backwards in time
+        s = run(pt, xb, w.dtr, A, w.dyr, w.xrr, nullptr, ft ? ft + sl * nstsl : nullptr, yb, nullptr, ws, st);
+        // h^T read out against dy (dC)
+        if (s == SSD_OK)
+            s = run(pt, xc, dt, A, xt, dyt, nullptr, ht ? ht + sl * nstsl : nullptr, yc, nullptr, ws, st);
+    }
     if (s == SSD_OK &&
         ssd::launch_backward_post(d, bf16, x, dy, dt, A, D, init_state, w, dx, ddt, dA, dB, dC, dD, st) != cudaSuccess)
         s = SSD_ERR_CUDA;

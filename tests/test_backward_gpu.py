@@ -3,8 +3,11 @@
 
 Inputs as for the scan (bf16 storage rounds x, B, C and dy on the host, so
 both sides see the same values); dy ~ N(0, 1), dfinal ~ N(0, 1).  Every
-gradient is compared in full: max abs error / max |reference| within 1e-3
-(the backward's scans run in fp32).
+gradient is compared in full, max abs error / max |reference|: dx, ddt, dA,
+dD and dinit come from fp32 scans and are within 1e-3 (1e-2 for the
+bf16-stored dx); dB and dC within 2e-2 (the scan's bf16 tolerance) when
+their transposed scans take the bf16 tensor-core plans (bf16, headdim 64,
+dstate a multiple of 64), else 1e-2 (bf16-stored) or 1e-3.
 """
 import numpy as np
 import pytest
@@ -27,6 +30,8 @@ SHAPES = [
     dict(batch=2, seqlen=256, nheads=4, headdim=64, dstate=128, ngroups=2, chunk_len=128, dtype="bf16"),
     dict(batch=1, seqlen=300, nheads=4, headdim=64, dstate=64, ngroups=1, chunk_len=64, dtype="bf16"),
     dict(batch=2, seqlen=96, nheads=2, headdim=16, dstate=16, ngroups=1, chunk_len=32, dtype="f32"),
+    # bf16 inputs whose scans cannot take the tensor-core plans (headdim 32): fp32 scans
+    dict(batch=1, seqlen=160, nheads=4, headdim=32, dstate=32, ngroups=2, chunk_len=64, dtype="bf16"),
     dict(batch=1, seqlen=192, nheads=6, headdim=32, dstate=48, ngroups=3, chunk_len=64, dtype="f32"),
 ]
 
@@ -55,8 +60,14 @@ def test_backward_against_oracle(oracle, shape, extras):
         got = g[n].double().cpu().numpy()
         want = ref["dh0" if n == "dinit_state" else n]
         assert np.isfinite(got).all(), n
+        tc = shape["dtype"] == "bf16" and shape["headdim"] == 64 and shape["dstate"] % 64 == 0
         # bf16 outputs (dx, dB, dC) carry one rounding of their own
-        tol = 1e-2 if (shape["dtype"] == "bf16" and n in ("dx", "dB", "dC")) else TOL
+        if tc and n in ("dB", "dC"):
+            tol = 2e-2
+        elif shape["dtype"] == "bf16" and n in ("dx", "dB", "dC"):
+            tol = 1e-2
+        else:
+            tol = TOL
         assert rel(got, want) <= tol, (n, rel(got, want))
     if not extras:
         assert g["dD"] is None and g["dinit_state"] is None
