@@ -122,8 +122,12 @@ chunk_scan4_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                    const float *__restrict__ Dskip, const float *__restrict__ lcum,
                    const long long *__restrict__ items, const int *__restrict__ nitems,
                    unsigned int *err) {
-    if (device_failed(err)) return;  // an earlier wait expired: skip all work
-    if (items) units = min(*nitems, units);  // list mode: the listed (b, c, tile, head) items
+    // both words are read before either is tested (one memory latency, not two:
+    // an empty list, the usual case in list mode, then costs one round trip)
+    const unsigned int err_word = err ? *reinterpret_cast<const volatile unsigned int *>(err) : 0u;
+    const int listed = items ? *nitems : units;  // list mode: the listed (b, c, tile, head) items
+    if (err_word & 1u) return;               // an earlier wait expired: skip all work
+    units = min(listed, units);
     if (int(blockIdx.x) >= units) return;    // no unit for this CTA (units are strided by the grid)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
