@@ -169,7 +169,8 @@ SSD_API ssd_status_t ssd_forward_static(const ssd_dims_t *dims, const void *x, c
  *            (fused_state layouts: nothing)
  *   stage 3  ssd_chunk_scan     x, dt, B, C, D, l, s_in   -> y_out
  *            (chunk_len 128/256 bf16 layouts: the chunk-wide scan, then the
- *            list-mode scan of the tiles it left, two launches)
+ *            list-mode scan of the tiles it left -- the block-factored kernel,
+ *            or the per-tile kernel for dstate 256 -- two launches)
  * Any other stage value returns SSD_ERR_INVALID_DIM.
  */
 typedef enum {
@@ -372,8 +373,9 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * that computes y.  `chunk_len` is the chunk length the kernels run with: the
  * caller's, except that SSD_BF16 with chunk_len 64 runs the tensor-core
  * kernels with 128-token chunks (their tile height; two of the caller's chunks
- * per tile, the same recurrence), and the arrays above then describe 128-token
- * chunks (nc = T / 128).
+ * per tile, the same recurrence), and so does SSD_BF16 with dstate 256 at
+ * chunk_len 256 (the chunk-wide scan holds one 128-token tile of C at that
+ * dstate); the arrays above then describe 128-token chunks (nc = T / 128).
  */
 typedef enum {
     SSD_ENGINE_SIMT = 0,            /* chunk scan on the CUDA cores                     */

@@ -19,6 +19,10 @@
 //      (tcgen05.ld) into bf16 scores CB * exp(l_t - l_s) * dt_s (s <= t) in
 //      shared memory; UMMA  Y = scores . X (K = s_len) and Z = C s_in^T (K = N)
 //      -> tensor memory; epilogue y = Y + exp(l_t) Z + D x, rounded to bf16.
+// The scores take exp(l_t - l_s) per element, so every decay range is exact:
+// in list mode (one CTA per SM walking packed (b, c, tile, head) items) this
+// kernel finishes the tiles that the chunk-wide scan left as steep where the
+// block-factored kernel has no shared-memory plan (dstate 256).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -77,6 +81,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
                      const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_s,
                      Dims d, int hpc, const float *__restrict__ dt, const float *__restrict__ Dskip,
                      const float *__restrict__ lcum, __nv_bfloat16 *__restrict__ y,
+                     const long long *__restrict__ items, const int *__restrict__ nitems, int max_items,
                      unsigned int *err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -93,18 +98,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 4);
     __shared__ int s_abort;
 
-    const int mt = blockIdx.x, c = blockIdx.y;
-    const int nhb = d.H / hpc;
-    const int b = blockIdx.z / nhb, hb = blockIdx.z % nhb;
-    const int hfirst = hb * hpc;
-    const int g = hfirst / d.r;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, half = warp >> 2;
-    const int s_len = (mt + 1) * kRows;              // source tokens [0, s_len) of the chunk
-    const int trow0 = b * d.T + c * Q;                // first token row of the chunk in [B*T]
     const int t_local = qd * 32 + lane;               // this thread's row within the tile
-    const int t = mt * kRows + t_local;               // ... within the chunk
-
+    // units: the grid's one (b, c, tile, head block), or in list mode the listed
+    // items blockIdx.x, blockIdx.x + gridDim.x, ... (one head each)
+    int nunits = 1;
+    if (items) {
+        const unsigned int err_word = err ? *reinterpret_cast<const volatile unsigned int *>(err) : 0u;
+        const int listed = *nitems;
+        if (err_word & 1u) return;
+        nunits = min(listed, max_items);
+        if (int(blockIdx.x) >= nunits) return;  // uniform: nothing listed for this CTA
+        hpc = 1;
+    }
     if (device_failed(err)) return;  // an earlier wait expired: skip all work
     if (tid == 0) {
         s_abort = 0;
@@ -121,151 +128,178 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
     const uint32_t lane_base = uint32_t(qd * 32) << 16;
+    // phases: bars[0] and bars[1] complete once per unit, bars[2] and bars[3] once per head
+    uint32_t jc = 0, hc = 0;
+    bool issued0 = false;
 
-    // ---- 1. C tile and B rows --------------------------------------------
-    if (tid == 0) {
-        constexpr int slabs = N >= 64 ? N / 64 : 1;
-        const uint32_t bytes = uint32_t(kRows) * N * 2 + uint32_t(s_len) * N * 2;
-        mbar_expect_tx(&bars[0], bytes);
-        for (int sl_i = 0; sl_i < slabs; ++sl_i) {
-            tma_load_3d(sC + sl_i * kRows * 128, &tm_c, &bars[0], sl_i * 64, g, trow0 + mt * kRows);
-            for (int i = 0; i <= mt; ++i)
-                tma_load_3d(sB + sl_i * s_len * 128 + i * kRows * row_bytes(N), &tm_b, &bars[0],
-                            sl_i * 64, g, trow0 + i * kRows);
+    for (int unit = items ? int(blockIdx.x) : 0; unit < nunits && s_abort == 0;
+         unit += items ? int(gridDim.x) : 1, ++jc) {
+        int mt, c, b, hfirst;
+        if (items) {
+            const long long v = items[unit];
+            b = int(v >> 40);
+            c = int((v >> 24) & 0xFFFF);
+            mt = int((v >> 16) & 0xFF);
+            hfirst = int(v & 0xFFFF);
+        } else {
+            const int nhb = d.H / hpc;
+            mt = blockIdx.x;
+            c = blockIdx.y;
+            b = blockIdx.z / nhb;
+            hfirst = (blockIdx.z % nhb) * hpc;
         }
-    }
-    bool ok = mbar_wait(&bars[0], 0, err);
-    // ---- 2. CB = C B^T into TMEM columns [0, s_len) ----------------------------
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kRows, s_len, 0, 0);
-        const uint32_t ca = smem_u32(sC), ba = smem_u32(sB);
-        for (int k = 0; k < N / 16; ++k)
-            mma_bf16_ss(tmem, kmajor_desc(ca, k, kRows, N), kmajor_desc(ba, k, s_len, N), idesc,
-                        k > 0 ? 1u : 0u);
-        mma_commit(&bars[1]);
-    }
-    if (ok && !mbar_wait(&bars[1], 0, err)) ok = false;
-    tc_fence_after();
-    if (!ok) s_abort = 1;
-    __syncthreads();
+        const int g = hfirst / d.r;
+        const int s_len = (mt + 1) * kRows;              // source tokens [0, s_len) of the chunk
+        const int trow0 = b * d.T + c * Q;                // first token row of the chunk in [B*T]
+        const int t = mt * kRows + t_local;               // this thread's row within the chunk
+        const uint32_t jpar = jc & 1;
 
-    for (int hi = 0; hi < hpc && s_abort == 0; ++hi) {
-        const int h = hfirst + hi;
-        const uint32_t par = hi & 1;
-        // ---- 3a. loads for this head ----------------------------------------
+        // ---- 1. C tile and B rows --------------------------------------------
         if (tid == 0) {
             constexpr int slabs = N >= 64 ? N / 64 : 1;
-            const uint32_t bytes = uint32_t(s_len) * 128 + 64u * N * 2;
-            mbar_expect_tx(&bars[2], bytes);
-            for (int i = 0; i <= mt; ++i)
-                tma_load_3d(sX + i * kRows * 128, &tm_x, &bars[2], 0, h, trow0 + i * kRows);
-            const int srow = ((b * d.nc + c) * d.H + h) * 64;
-            for (int sl_i = 0; sl_i < slabs; ++sl_i)
-                tma_load_2d(sS + sl_i * 64 * 128, &tm_s, &bars[2], sl_i * 64, srow);
+            const uint32_t bytes = uint32_t(kRows) * N * 2 + uint32_t(s_len) * N * 2;
+            mbar_expect_tx(&bars[0], bytes);
+            issued0 = true;
+            for (int sl_i = 0; sl_i < slabs; ++sl_i) {
+                tma_load_3d(sC + sl_i * kRows * 128, &tm_c, &bars[0], sl_i * 64, g, trow0 + mt * kRows);
+                for (int i = 0; i <= mt; ++i)
+                    tma_load_3d(sB + sl_i * s_len * 128 + i * kRows * row_bytes(N), &tm_b, &bars[0],
+                                sl_i * 64, g, trow0 + i * kRows);
+            }
         }
-        for (int i = tid; i < s_len; i += kThreads) {
-            sl[i] = __ldg(lcum + off_lq(d, b, h, c) + i);
-            sdt[i] = __ldg(dt + off_dt(d, b, c * Q + i) + h);
+        bool ok = mbar_wait(&bars[0], jpar, err);
+        // ---- 2. CB = C B^T into TMEM columns [0, s_len) ----------------------------
+        if (tid == 0 && ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(kRows, s_len, 0, 0);
+            const uint32_t ca = smem_u32(sC), ba = smem_u32(sB);
+            for (int k = 0; k < N / 16; ++k)
+                mma_bf16_ss(tmem, kmajor_desc(ca, k, kRows, N), kmajor_desc(ba, k, s_len, N), idesc,
+                            k > 0 ? 1u : 0u);
+            mma_commit(&bars[1]);
         }
+        if (ok && !mbar_wait(&bars[1], jpar, err)) ok = false;
+        tc_fence_after();
+        if (!ok) s_abort = 1;
         __syncthreads();
 
-        // ---- 3b. scores = CB * exp(l_t - l_s) * dt_s for s <= t -> bf16 smem
-        {
-            const float lt = sl[t];
-            const int cols = s_len / 2;
-            const int c0 = half * cols;
-            const int tmax = mt * kRows + qd * 32 + 31;  // last row of this warp
+        for (int hi = 0; hi < hpc && s_abort == 0; ++hi, ++hc) {
+            const int h = hfirst + hi;
+            const uint32_t par = hc & 1;
+            // ---- 3a. loads for this head ----------------------------------------
+            if (tid == 0) {
+                constexpr int slabs = N >= 64 ? N / 64 : 1;
+                const uint32_t bytes = uint32_t(s_len) * 128 + 64u * N * 2;
+                mbar_expect_tx(&bars[2], bytes);
+                for (int i = 0; i <= mt; ++i)
+                    tma_load_3d(sX + i * kRows * 128, &tm_x, &bars[2], 0, h, trow0 + i * kRows);
+                const int srow = ((b * d.nc + c) * d.H + h) * 64;
+                for (int sl_i = 0; sl_i < slabs; ++sl_i)
+                    tma_load_2d(sS + sl_i * 64 * 128, &tm_s, &bars[2], sl_i * 64, srow);
+            }
+            for (int i = tid; i < s_len; i += kThreads) {
+                sl[i] = __ldg(lcum + off_lq(d, b, h, c) + i);
+                sdt[i] = __ldg(dt + off_dt(d, b, c * Q + i) + h);
+            }
+            __syncthreads();
+
+            // ---- 3b. scores = CB * exp(l_t - l_s) * dt_s for s <= t -> bf16 smem
+            {
+                const float lt = sl[t];
+                const int cols = s_len / 2;
+                const int c0 = half * cols;
+                const int tmax = mt * kRows + qd * 32 + 31;  // last row of this warp
 #pragma unroll 1
-            for (int s0 = c0; s0 < c0 + cols; s0 += 32) {
-                uint32_t pk[16];
-                if (s0 > tmax) {
+                for (int s0 = c0; s0 < c0 + cols; s0 += 32) {
+                    uint32_t pk[16];
+                    if (s0 > tmax) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else {
+                        float v[32];
+                        tmem_ld32(tmem + lane_base + s0, v);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int s = s0 + 2 * e;
+                            const float a0 = s <= t ? v[2 * e] * __expf(lt - sl[s]) * sdt[s] : 0.f;
+                            const float a1 = s + 1 <= t ? v[2 * e + 1] * __expf(lt - sl[s + 1]) * sdt[s + 1] : 0.f;
+                            pk[e] = pack_bf16x2(a0, a1);
+                        }
+                    }
+                    uint8_t *slab = sP + (s0 >> 6) * (kRows * 128);
+                    const int q0 = (s0 & 63) >> 3;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq)
+                        *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, q0 + qq)) =
+                            make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+
+            // ---- 3c. Y = scores . X,  Z = C . s_in^T -------------------------------
+            if (tid == 0) {
+                if (!mbar_wait(&bars[2], par, err)) {
+                    s_abort = 1;
                 } else {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + s0, v);
+                    tc_fence_after();
+                    const uint32_t pa = smem_u32(sP), xa = smem_u32(sX), ca = smem_u32(sC), sa = smem_u32(sS);
+                    const uint32_t id1 = idesc_bf16_f32(kRows, 64, 0, 1);
+                    for (int k = 0; k < s_len / 16; ++k)
+                        mma_bf16_ss(tmem + kColY, kmajor_desc(pa, k, kRows, 64),
+                                    smem_desc(xa + k * 2048, 16, 1024, kSw128), id1, k > 0 ? 1u : 0u);
+                    const uint32_t id2 = idesc_bf16_f32(kRows, 64, 0, 0);
+                    for (int k = 0; k < N / 16; ++k)
+                        mma_bf16_ss(tmem + kColZ, kmajor_desc(ca, k, kRows, N), kmajor_desc(sa, k, 64, N),
+                                    id2, k > 0 ? 1u : 0u);
+                    mma_commit(&bars[3]);
+                }
+            }
+            __syncthreads();
+            if (s_abort == 0) {
+                // bars[2] (already complete) also makes the TMA-written x rows
+                // visible to this thread's epilogue loads
+                if (!mbar_wait(&bars[2], par, err) || !mbar_wait(&bars[3], par, err)) s_abort = 1;
+            }
+            tc_fence_after();
+            __syncthreads();
+
+            // ---- 3d. epilogue: y = Y + exp(l_t) Z + D x ------------------------------
+            if (s_abort == 0) {
+                const int p0 = half * 32;
+                float yv[32], zv[32];
+                tmem_ld32(tmem + lane_base + kColY + p0, yv);
+                tmem_ld32(tmem + lane_base + kColZ + p0, zv);
+                const float e = __expf(sl[t]);
+                const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
+                uint32_t out[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int s = s0 + 2 * e;
-                        const float a0 = s <= t ? v[2 * e] * __expf(lt - sl[s]) * sdt[s] : 0.f;
-                        const float a1 = s + 1 <= t ? v[2 * e + 1] * __expf(lt - sl[s + 1]) * sdt[s + 1] : 0.f;
-                        pk[e] = pack_bf16x2(a0, a1);
+                for (int qq = 0; qq < 4; ++qq) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(t, (p0 >> 3) + qq));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = qq * 8 + 2 * u;
+                        const float o0 = fmaf(Dh, bf16lo(xw[u]), fmaf(e, zv[i], yv[i]));
+                        const float o1 = fmaf(Dh, bf16hi(xw[u]), fmaf(e, zv[i + 1], yv[i + 1]));
+                        out[qq * 4 + u] = pack_bf16x2(o0, o1);
                     }
                 }
-                uint8_t *slab = sP + (s0 >> 6) * (kRows * 128);
-                const int q0 = (s0 & 63) >> 3;
+                uint4 *dst = reinterpret_cast<uint4 *>(y + off_x(d, b, c * Q + t, h) + p0);
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq)
-                    *reinterpret_cast<uint4 *>(slab + sw128_off(t_local, q0 + qq)) =
-                        make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
+                    dst[qq] = make_uint4(out[4 * qq], out[4 * qq + 1], out[4 * qq + 2], out[4 * qq + 3]);
             }
+            tc_fence_before();
+            __syncthreads();
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- 3c. Y = scores . X,  Z = C . s_in^T -------------------------------
-        if (tid == 0) {
-            if (!mbar_wait(&bars[2], par, err)) {
-                s_abort = 1;
-            } else {
-                tc_fence_after();
-                const uint32_t pa = smem_u32(sP), xa = smem_u32(sX), ca = smem_u32(sC), sa = smem_u32(sS);
-                const uint32_t id1 = idesc_bf16_f32(kRows, 64, 0, 1);
-                for (int k = 0; k < s_len / 16; ++k)
-                    mma_bf16_ss(tmem + kColY, kmajor_desc(pa, k, kRows, 64),
-                                smem_desc(xa + k * 2048, 16, 1024, kSw128), id1, k > 0 ? 1u : 0u);
-                const uint32_t id2 = idesc_bf16_f32(kRows, 64, 0, 0);
-                for (int k = 0; k < N / 16; ++k)
-                    mma_bf16_ss(tmem + kColZ, kmajor_desc(ca, k, kRows, N), kmajor_desc(sa, k, 64, N),
-                                id2, k > 0 ? 1u : 0u);
-                mma_commit(&bars[3]);
-            }
-        }
-        __syncthreads();
-        if (s_abort == 0) {
-            // bars[2] (already complete) also makes the TMA-written x rows
-            // visible to this thread's epilogue loads
-            if (!mbar_wait(&bars[2], par, err) || !mbar_wait(&bars[3], par, err)) s_abort = 1;
-        }
-        tc_fence_after();
-        __syncthreads();
-
-        // ---- 3d. epilogue: y = Y + exp(l_t) Z + D x ------------------------------
-        if (s_abort == 0) {
-            const int p0 = half * 32;
-            float yv[32], zv[32];
-            tmem_ld32(tmem + lane_base + kColY + p0, yv);
-            tmem_ld32(tmem + lane_base + kColZ + p0, zv);
-            const float e = __expf(sl[t]);
-            const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
-            uint32_t out[16];
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(sX + sw128_off(t, (p0 >> 3) + qq));
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int i = qq * 8 + 2 * u;
-                    const float o0 = fmaf(Dh, bf16lo(xw[u]), fmaf(e, zv[i], yv[i]));
-                    const float o1 = fmaf(Dh, bf16hi(xw[u]), fmaf(e, zv[i + 1], yv[i + 1]));
-                    out[qq * 4 + u] = pack_bf16x2(o0, o1);
-                }
-            }
-            uint4 *dst = reinterpret_cast<uint4 *>(y + off_x(d, b, c * Q + t, h) + p0);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-                dst[qq] = make_uint4(out[4 * qq], out[4 * qq + 1], out[4 * qq + 2], out[4 * qq + 3]);
-        }
-        tc_fence_before();
-        __syncthreads();
     }
-    // after an abandoned wait, give copies still in flight a bounded chance to land
+    // after an abandoned wait, give copies still in flight a bounded chance to
+    // land: the unit's C / B loads and its current head's x / s_in loads
     if (tid == 0 && s_abort) {
-        mbar_wait(&bars[0], 0, nullptr);
-        mbar_wait(&bars[2], 0, nullptr);
-        mbar_wait(&bars[2], 1, nullptr);
+        if (issued0) mbar_wait(&bars[0], jc & 1, nullptr);
+        mbar_wait(&bars[2], hc & 1, nullptr);
     }
     tc_fence_before();
     __syncthreads();
@@ -274,16 +308,21 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
 
 template <int N>
 cudaError_t launch_n(const Dims &d, const CUtensorMap *maps, int hpc, const float *dt,
-                     const float *D, const float *l, __nv_bfloat16 *y, unsigned int *err,
-                     cudaStream_t stream) {
+                     const float *D, const float *l, __nv_bfloat16 *y, const long long *items,
+                     const int *nitems, int max_items, unsigned int *err, cudaStream_t stream) {
     const ScanSmem L = scan_smem(d.Q, N);
     // at least 116 KB so that one CTA (which takes all 512 TMEM columns) runs per SM
     const int smem = int(L.total < 116 * 1024 ? 116 * 1024 : L.total);
     if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan_tc_kernel<N>), smem))
         return cudaErrorInvalidValue;
     dim3 grid(d.Q / kRows, d.nc, d.B * (d.H / hpc));
-    chunk_scan_tc_kernel<N><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3],
-                                                                d, hpc, dt, D, l, y, err);
+    if (items) {
+        // one CTA per SM walks the list (most CTAs exit at once when it is short)
+        const int sms = device_sm_count();
+        grid = dim3(max_items < sms ? max_items : sms, 1, 1);
+    }
+    chunk_scan_tc_kernel<N><<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], d, hpc,
+                                                                dt, D, l, y, items, nitems, max_items, err);
     return cudaGetLastError();
 }
 
@@ -304,8 +343,10 @@ bool tc_chunk_scan_supported(const Dims &d) {
 
 cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
                                  const void *Cm, const float *D, const float *l,
-                                 const void *s_in_bf16, void *y, unsigned int *err,
+                                 const void *s_in_bf16, void *y, const long long *items,
+                                 const int *nitems, int max_items, unsigned int *err,
                                  cudaStream_t stream) {
+    if (items && max_items <= 0) return cudaSuccess;
     const uint32_t nbox = uint32_t(d.N >= 64 ? 64 : d.N);
     const int rb = row_bytes(d.N);
     const uint64_t bcdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
@@ -326,11 +367,11 @@ cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, 
     const int hpc = heads_per_cta(d);
     auto *yo = static_cast<__nv_bfloat16 *>(y);
     switch (d.N) {
-        case 16: return launch_n<16>(d, maps, hpc, dt, D, l, yo, err, stream);
-        case 32: return launch_n<32>(d, maps, hpc, dt, D, l, yo, err, stream);
-        case 64: return launch_n<64>(d, maps, hpc, dt, D, l, yo, err, stream);
-        case 128: return launch_n<128>(d, maps, hpc, dt, D, l, yo, err, stream);
-        case 256: return launch_n<256>(d, maps, hpc, dt, D, l, yo, err, stream);
+        case 16: return launch_n<16>(d, maps, hpc, dt, D, l, yo, items, nitems, max_items, err, stream);
+        case 32: return launch_n<32>(d, maps, hpc, dt, D, l, yo, items, nitems, max_items, err, stream);
+        case 64: return launch_n<64>(d, maps, hpc, dt, D, l, yo, items, nitems, max_items, err, stream);
+        case 128: return launch_n<128>(d, maps, hpc, dt, D, l, yo, items, nitems, max_items, err, stream);
+        case 256: return launch_n<256>(d, maps, hpc, dt, D, l, yo, items, nitems, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

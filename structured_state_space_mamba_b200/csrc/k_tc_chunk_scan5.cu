@@ -38,7 +38,8 @@
 //
 // Tensor memory (512 columns): [0,128) P_0, P_1 (bf16); [256,384) CBoff and
 // C_0 (bf16 A operands of TS products: CBoff in [256,288) and [320,352), C_0 in
-// [288,320) and [352,384)); two accumulator buffers {Y_0, Y_1} at [384,512) and
+// [288,320) and [352,384); with dstate 256, which runs 128-token chunks only,
+// C_0 takes all of [256,384)); two accumulator buffers {Y_0, Y_1} at [384,512) and
 // [128,256), alternating between heads.  At the start of a run the fp32 C B^T
 // tiles pass through them (C_0 B_0^T -> [384,512), C_1 B_1^T -> [128,256),
 // CBoff -> [256,384)), so a run starts once the accumulators of the previous
@@ -79,8 +80,13 @@ __device__ __forceinline__ uint32_t off_col(int cb) { return kColOff + (cb >> 1)
 // accumulator buffer ab of a head (hit & 1)
 __device__ __forceinline__ uint32_t acc_col(int ab) { return ab == 0 ? 384u : 128u; }
 // C_0 (bf16, A operand of the C_0 S'^T products), K step kk: the second half of
-// each score warp pair's CBoff source range, free once CBoff is packed
-__device__ __forceinline__ uint32_t c0_col(int kk) { return kColOff + 32 + (kk >> 2) * 64 + (kk & 3) * 8; }
+// each score warp pair's CBoff source range, free once CBoff is packed; with
+// dstate 256 (128-token chunks only, so no CBoff) the whole range [256,384)
+template <int N>
+__device__ __forceinline__ uint32_t c0_col(int kk) {
+    if (N == 256) return kColOff + kk * 8;
+    return kColOff + 32 + (kk >> 2) * 64 + (kk & 3) * 8;
+}
 
 struct Smem5 {
     uint32_t c1_off, stage_off, stage_bytes, s_rel, lg_off, lg_bytes, y_off, bar_off, total;
@@ -344,7 +350,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     const uint64_t sd = kmajor_desc(sa, 0, 64, N);
 #pragma unroll
                     for (int kk = 0; kk < N / 16; ++kk) {
-                        mma_bf16_ts(acc, tmem + c0_col(kk), sd + kdesc_step_n<N>(kk, 64), idS, kk > 0 ? 1u : 0u);
+                        mma_bf16_ts(acc, tmem + c0_col<N>(kk), sd + kdesc_step_n<N>(kk, 64), idS, kk > 0 ? 1u : 0u);
                         if (two)
                             mma_bf16_ss(acc + 64, c1d + kdesc_step_n<N>(kk, kRows), sd + kdesc_step_n<N>(kk, 64), idS,
                                         kk > 0 ? 1u : 0u);
@@ -421,24 +427,29 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                     tmem_st16(tmem + lane_base + off_col(cb0 + bb), pk);
                 }
             }
-            // C_0 into the second half of this warp's range: row t, K half cb0 / 2
-            // (one 128-byte swizzled slab row, or the 32-byte row for N = 16)
+            // C_0 into tensor memory: row t, K half cb0 / 2 (one 128-byte swizzled
+            // slab row per 64 columns of dstate, or the 32-byte row for N = 16)
             {
                 const int t = qd * 32 + lane;
                 const uint8_t *sc0 = stage_at(uc);
                 if (N >= 64) {
-                    const uint8_t *row = sc0 + (cb0 >> 1) * kRows * 128 + t * 128;
-                    uint32_t cw[32];
+                    constexpr int kHalf = kSlabs / 2;  // slabs per K half
+#pragma unroll 1
+                    for (int j = 0; j < kHalf; ++j) {
+                        const int sl = (cb0 >> 1) * kHalf + j;
+                        const uint8_t *row = sc0 + sl * kRows * 128 + t * 128;
+                        uint32_t cw[32];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(row + ((q ^ (t & 7)) << 4));
-                        cw[4 * q] = v.x;
-                        cw[4 * q + 1] = v.y;
-                        cw[4 * q + 2] = v.z;
-                        cw[4 * q + 3] = v.w;
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(row + ((q ^ (t & 7)) << 4));
+                            cw[4 * q] = v.x;
+                            cw[4 * q + 1] = v.y;
+                            cw[4 * q + 2] = v.z;
+                            cw[4 * q + 3] = v.w;
+                        }
+                        tmem_st16(tmem + lane_base + c0_col<N>(4 * sl), cw);
+                        tmem_st16(tmem + lane_base + c0_col<N>(4 * sl) + 16, cw + 16);
                     }
-                    tmem_st16(tmem + lane_base + c0_col(4 * (cb0 >> 1)), cw);
-                    tmem_st16(tmem + lane_base + c0_col(4 * (cb0 >> 1)) + 16, cw + 16);
                 } else if (cb0 == 0) {
                     uint32_t cw[8];
 #pragma unroll
@@ -449,7 +460,7 @@ chunk_scan5_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         cw[4 * q + 2] = v.z;
                         cw[4 * q + 3] = v.w;
                     }
-                    tmem_st8(tmem + lane_base + c0_col(0), cw);
+                    tmem_st8(tmem + lane_base + c0_col<N>(0), cw);
                 }
             }
             tmem_wait_st();
@@ -594,7 +605,9 @@ cudaError_t launch5(const Dims &d, const CUtensorMap *maps, const float *gq, con
 }  // namespace
 
 bool tc_chunk_scan5_supported(const Dims &d) {
-    const bool n_ok = d.N == 16 || d.N == 128;
+    // dstate 256: 128-token chunks only (C_0 takes the tensor memory that CBoff
+    // would need, and C_1 would not fit in shared memory)
+    const bool n_ok = d.N == 16 || d.N == 128 || (d.N == 256 && d.Q == kRows);
     return d.P == 64 && n_ok && (d.Q == 128 || d.Q == 256) &&
            scan5_smem(d.Q, d.N).total <= 227 * 1024 && d.H < 65536 && d.nc < 65536 &&
            d.B < 65536;
@@ -629,6 +642,7 @@ cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq,
     switch (d.N) {
         case 16: return launch5<16>(d, maps, gq, D, l, nsteep, items, max_items, err, stream);
         case 128: return launch5<128>(d, maps, gq, D, l, nsteep, items, max_items, err, stream);
+        case 256: return launch5<256>(d, maps, gq, D, l, nsteep, items, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

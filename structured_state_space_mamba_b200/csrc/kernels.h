@@ -65,9 +65,13 @@ cudaError_t launch_chunk_state_tc(const Dims &d, const void *x, const void *Bm, 
 cudaError_t launch_state_fused(const Dims &d, const void *x, const void *Bm, const float *w,
                                const float *alpha, const float *h0, void *s_in_bf16, float *fin,
                                unsigned int *err, cudaStream_t stream);
+// items == nullptr: every (b, c, tile, head block); otherwise list mode: the
+// *nitems packed (b, c, tile, head) items (at most max_items) that the
+// chunk-wide scan left as steep, walked by one CTA per SM
 cudaError_t launch_chunk_scan_tc(const Dims &d, const void *x, const float *dt, const void *Bm,
                                  const void *Cm, const float *D, const float *l,
-                                 const void *s_in_bf16, void *y, unsigned int *err,
+                                 const void *s_in_bf16, void *y, const long long *items,
+                                 const int *nitems, int max_items, unsigned int *err,
                                  cudaStream_t stream);
 // Persistent warp-specialised variant (dstate <= 128); dtq and beta come from
 // ssd_chunk_cumsum.  Writes y with TMA stores.

@@ -60,7 +60,7 @@ struct Plan {
     bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
     bool scan5;     // chunk-wide scan, steep tiles finished by the block-factored scan
     bool single;    // the single-pass kernel (chunk state + state passing + scan)
-    int tile_chunks = 1;  // caller chunks per chunk of the plan (2: chunk_len 64 run as 128)
+    bool tile_finish;  // scan5's steep tiles go to the per-tile scan (no block-factored plan)
     int t_full = 0;       // tokens in full chunks; the tail [t_full, T) runs in the tail kernel
     size_t mid_offset = 0;  // tail: fp32 state after the full chunks [B,H,P,N]
     size_t steep_offset;  // scan5 / single: item counter (256 bytes) + packed steep items
@@ -102,10 +102,19 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
         Dims d2 = d;
         d2.Q = 128;
         d2.nc = d.T / 128;
-        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2)) {
+        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2)) d = d2;
+    }
+    // dstate 256 at chunk_len 256: the chunk-wide tensor-core scan holds one
+    // 128-token tile of C (C_0 in tensor memory) but not a second, so the chunks
+    // are 128 tokens (the same recurrence, blocked finer; the workspace arrays
+    // then describe 128-token chunks)
+    if (a.dtype == SSD_BF16 && d.N == 256 && d.Q == 256) {
+        Dims d2 = d;
+        d2.Q = 128;
+        d2.nc = d.T / 128;
+        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2) &&
+            ssd::tc_chunk_scan5_supported(d2))
             d = d2;
-            plan->tile_chunks = 2;
-        }
     }
     // a length that is not a multiple of chunk_len: the chunked kernels take the
     // full chunks (they index rows with the true T), the tail kernel the rest
@@ -118,7 +127,11 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     // the fused state kernel walks each (b, head pair) over all chunks: used when
     // those units fill most of the GPU's 148 SMs in one wave
     plan->fused = plan->tc_state && plan->tc_scan && ssd::tc_state_fused_supported(d, kB200Sms);
-    plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d) && ssd::tc_chunk_scan4_supported(d);
+    // the chunk-wide scan leaves steep tiles to the block-factored scan, or (no
+    // shared-memory plan there: dstate 256) to the per-tile scan, whose scores
+    // take every decay exactly
+    plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d);
+    plan->tile_finish = plan->scan5 && !ssd::tc_chunk_scan4_supported(d);
     // the single-pass kernel walks each (b, head pair) chain chunk by chunk: used
     // when the chains fill at least kMinChainNum / kMinChainDen of the SMs (fewer
     // chains leave most SMs idle, and the four-kernel sequence is faster there);
@@ -305,15 +318,19 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                     e = ssd::launch_chunk_scan_tc5(d, x, gq, Bm, Cm, D, l, s_in, y, nsteep,
                                                    steep_items, err, stream);
                     if (e == cudaSuccess)
-                        e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
-                                                       steep_items, nsteep,
-                                                       ssd::chunk_scan5_max_steep(d), err, stream);
+                        e = pl.tile_finish
+                                ? ssd::launch_chunk_scan_tc(d, x, dt_scan, Bm, Cm, D, l, s_in, y, steep_items,
+                                                            nsteep, ssd::chunk_scan5_max_steep(d), err, stream)
+                                : ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
+                                                             steep_items, nsteep,
+                                                             ssd::chunk_scan5_max_steep(d), err, stream);
                 } else {
                     e = pl.tc_scan
                             ? (ssd::tc_chunk_scan4_supported(d)
                                    ? ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y,
                                                                 nullptr, nullptr, 0, err, stream)
-                                   : ssd::launch_chunk_scan_tc(d, x, dt_scan, Bm, Cm, D, l, s_in, y, err, stream))
+                                   : ssd::launch_chunk_scan_tc(d, x, dt_scan, Bm, Cm, D, l, s_in, y, nullptr,
+                                                               nullptr, 0, err, stream))
                             : ssd::launch_chunk_scan_simt(d, pl.bf16, x, dt_scan, Bm, Cm, D, l,
                                                           static_cast<const float *>(s_in), y, stream);
                 }

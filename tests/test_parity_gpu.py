@@ -113,10 +113,13 @@ def test_tensor_core_path_selected():
             lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
             assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
             assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (n, q)
-            # dstate 32 / 64 take the block-factored scan, 256 the per-tile one
-            want = {32: "block_factored", 64: "block_factored", 256: "tile"}.get(n)
+            # dstate 32 / 64 take the block-factored scan, 256 the chunk-wide one
+            # on 128-token chunks
+            want = {32: "block_factored", 64: "block_factored", 256: "chunk_wide"}.get(n)
             if want:
                 assert binding.SCAN_ENGINES[lay.scan_engine] == want, (n, q)
+            if n == 256:
+                assert lay.chunk_len == 128, q
     lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 32, 64, 1, "bf16"), 128)
     assert lay.tensor_core == 0
 
@@ -127,7 +130,7 @@ def test_no_skip_term(oracle):
     check_full(inp, oracle)
 
 
-@pytest.mark.parametrize("dstate", [16, 32, 64, 128])
+@pytest.mark.parametrize("dstate", [16, 32, 64, 128, 256])
 def test_decay_range_across_the_chunk(oracle, dstate):
     """Per-token decays of about e^-0.4 (head 0): each 128-token tile spans ~e^-51
     but the 256-token chunk ~e^-102, so the chunk-wide scan moves its reference
@@ -146,6 +149,39 @@ def test_decay_range_across_the_chunk(oracle, dstate):
     yc = y[:, 256::256, 0][:, :, None]
     yrc = yr[:, 256::256, 0][:, :, None]
     assert rel(yc, yrc) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=2, seqlen=677, nheads=6, headdim=64, dstate=256, ngroups=3, chunk_len=256),
+    dict(batch=1, seqlen=1024, nheads=8, headdim=64, dstate=256, ngroups=1, chunk_len=128),
+    dict(batch=2, seqlen=384, nheads=4, headdim=64, dstate=256, ngroups=2, chunk_len=64),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_dstate_256_chunk_wide(oracle, shape, h0):
+    """dstate 256 on the chunk-wide tensor-core scan at 128-token chunks, for
+    every caller chunk_len, a ragged length (tail kernel) and groups."""
+    inp = make_inputs(**shape, dtype="bf16", seed=23, init_state=h0)
+    d = binding.make_dims(**{k: shape[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
+                                                     "ngroups")}, dtype="bf16")
+    lay = binding.workspace_layout(d, shape["chunk_len"])
+    assert binding.SCAN_ENGINES[lay.scan_engine] == "chunk_wide" and lay.chunk_len == 128
+    check_full(inp, oracle)
+
+
+def test_dstate_256_steep_list(oracle):
+    """Every tile of every head but head 1 decays past the chunk-wide scan's
+    range (at least e^-150 per 128 tokens), so it lists 7 * 2 * 16 = 224 tiles
+    for the per-tile scan, which walks the list with one CTA per SM: more items
+    than CTAs, so most CTAs take two."""
+    inp = make_inputs(2, 2048, 8, 64, 256, 2, 256, dtype="bf16", seed=29, init_state=True, h0_std=1.0)
+    rng = np.random.default_rng(29)
+    inp.dt = rng.uniform(0.3, 0.5, size=inp.dt.shape).astype(np.float32)
+    inp.A = np.array([-4.0, -0.05, -8.0, -16.0, -3.0, -5.0, -6.0, -7.0], dtype=np.float32)
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    for h in range(8):
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
 
 
 @pytest.mark.parametrize("chunk_len", [128, 256])
