@@ -29,7 +29,11 @@
  *    CUDA, on the next synchronising call.
  *  - Shared state: a per-device cache of device properties; one device-side
  *    error word per device (set by an expired bounded wait, read and cleared by
- *    ssd_device_status); and the static scratch array of ssd_forward_static,
+ *    ssd_device_status); a per-device stream-ordered memory pool from which the
+ *    entry points that allocate their own workspace take it (the pool keeps
+ *    its reserved memory between calls, so repeated calls reuse it;
+ *    ssd_workspace_trim returns the unused part); and the static scratch
+ *    array of ssd_forward_static,
  *    which every call of that entry point on a device shares, so that such
  *    calls overlapping in time race (see ssd_forward_static).  The other entry
  *    points keep no state between calls and may run concurrently on
@@ -107,7 +111,8 @@ typedef struct {
  *   stream                   cudaStream_t
  *
  * Intermediates (ssd_workspace_bytes) are allocated stream-ordered on
- * `stream` and released before return (cudaMallocAsync / cudaFreeAsync).
+ * `stream` from the library's workspace pool and released to it before
+ * return (cudaMallocFromPoolAsync / cudaFreeAsync).
  * Accuracy against the fp64 recurrence: max|y - y_ref| / max|y_ref| <= 1e-4
  * for SSD_F32 and <= 2e-2 for SSD_BF16 when every dt_t * A_h <= 0; the same
  * bound holds for the final state.
@@ -319,17 +324,20 @@ SSD_API ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *c
  *   dC_t = sum_heads h_t^T dy_t,      dD_h = sum dy_t . x_t,
  *   ddt_t = x_t . (G_t B_t) + A_h exp(dt_t A_h) (G_t : h_{t-1}),
  *   dA_h = sum dt_t exp(dt_t A_h) (G_t : h_{t-1}),   dinit = exp(dt_0 A_h) G_0.
- * Computed with four scans of the library's own chunked forward in fp32 (G
- * backwards in time, h forwards, and each transposed for dB and dC) plus
- * element-wise and prefix-sum kernels (k_backward.cu gives the identities).
+ * Computed with four scans of the library's own chunked forward (G backwards
+ * in time and h forwards, in fp32; each transposed for dB and dC, on the bf16
+ * tensor-core plans when the inputs are bf16 with headdim 64 and dstate a
+ * multiple of 64, in fp32 otherwise) plus element-wise and prefix-sum kernels
+ * (k_backward.cu gives the identities).
  *
  *   inputs as for ssd_forward; dy [B,T,H,P] dtype; dfinal_state [B,H,P,N] fp32
  *   or NULL (zero)
  *   dx [B,T,H,P] dtype; ddt [B,T,H] fp32; dA [H] fp32; dB, dC [B,T,G,N] dtype;
  *   dD [H] fp32 or NULL (not computed); dinit_state [B,H,P,N] fp32 or NULL
  * Requires dt_t > 0 for every token (the scan of G takes a_t dy_t / dt_t as its
- * input).  Scratch memory (about 20 fp32 copies of x's size) is allocated
- * stream-ordered on `stream` and released before return.  Accuracy: the
+ * input) and nheads <= 12288 (else SSD_ERR_UNSUPPORTED).  Scratch memory
+ * (about 20 fp32 copies of x's size) is allocated stream-ordered on `stream`
+ * from the library's workspace pool and released to it before return.  Accuracy: the
  * gradients' max abs error over their max |value| within 1e-3 of the fp64
  * reverse mode on fp32-exact inputs.
  */
@@ -406,13 +414,21 @@ SSD_API ssd_status_t ssd_workspace_layout(const ssd_dims_t *dims, int chunk_len,
  * device-side error word of the current device: SSD_ERR_DEVICE_TIMEOUT if a
  * bounded wait inside a tensor-core kernel expired since the last query (that
  * kernel skipped its remaining work, so its outputs are incomplete), SSD_ERR_CUDA
- * if the synchronisation reported an error, SSD_OK otherwise.  This is the only
- * entry point that blocks the host.
+ * if the synchronisation reported an error, SSD_OK otherwise.  With
+ * ssd_workspace_trim, the only entry points that block the host.
  */
 SSD_API ssd_status_t ssd_device_status(void *stream);
 
 /* Static description of a status code (never NULL). */
 SSD_API const char *ssd_status_string(ssd_status_t status);
+
+/*
+ * ssd_workspace_trim -- synchronise the current device, then return to the
+ * system the workspace memory that the library's pool on that device holds
+ * but no call is using (the pool otherwise keeps it for the next call).
+ * SSD_ERR_CUDA if the synchronisation or the trim failed.  Blocks the host.
+ */
+SSD_API ssd_status_t ssd_workspace_trim(void);
 
 /* Library version, e.g. "ssd-b200 0.1.0 sm_100a". */
 SSD_API const char *ssd_version(void);

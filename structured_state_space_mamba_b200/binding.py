@@ -23,7 +23,7 @@ STATUS = {0: "SSD_OK", 1: "SSD_ERR_NULL_ARG", 2: "SSD_ERR_INVALID_DIM", 3: "SSD_
 EXPORTS = ("ssd_forward", "ssd_forward_ws", "ssd_forward_stage", "ssd_workspace_bytes",
            "ssd_workspace_layout", "ssd_device_status", "ssd_status_string", "ssd_version",
            "ssd_forward_static", "ssd_step", "ssd_forward_block", "ssd_block_workspace_bytes",
-           "ssd_forward_varlen", "ssd_varlen_workspace_bytes", "ssd_backward")
+           "ssd_forward_varlen", "ssd_varlen_workspace_bytes", "ssd_backward", "ssd_workspace_trim")
 STAGES = ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
 
 
@@ -117,6 +117,8 @@ def load():
     lib.ssd_device_status.restype = ctypes.c_int
     lib.ssd_version.argtypes = []
     lib.ssd_version.restype = ctypes.c_char_p
+    lib.ssd_workspace_trim.argtypes = []
+    lib.ssd_workspace_trim.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -427,6 +429,14 @@ def device_status(device=None) -> int:
     with torch.cuda.device(dev):
         return int(load().ssd_device_status(
             ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+
+
+def workspace_trim(device=None) -> int:
+    """Synchronise the device and return the library pool's unused workspace
+    memory to the system; 0 (SSD_OK) or an ssd_status_t error code."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return int(load().ssd_workspace_trim())
 
 
 def version() -> str:

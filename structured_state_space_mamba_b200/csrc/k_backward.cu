@@ -28,42 +28,34 @@ constexpr int kThreads = 256;
 template <typename T>
 __device__ __forceinline__ float ld(const T *p, int64_t i) { return to_f32<T>(p[i]); }
 
-__device__ __forceinline__ float decay(const float *dt, const float *A, int64_t i_dt, int h) {
-    return __expf(dt[i_dt] * A[h]);
-}
+// The row kernels below take one (b, t) row per block, blocks striding over
+// the B*T rows; inside a row the indices are 32-bit (a row holds H*N or H*P
+// elements).
 
 // scan K (reversed): xr[b,tau,h,p] = a_t dy[b,t,h,p] / dt_t, dtr[b,tau,h] = dt_t,
 // and (per group) Br = C, Cr = B, all at tau = T-1-t
 template <typename T, typename TS>
-__global__ void prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__restrict__ dt,
-                              const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
-                              TS *__restrict__ xr, float *__restrict__ dtr, TS *__restrict__ Br,
-                              TS *__restrict__ Cr) {
-    const int64_t n_x = int64_t(d.B) * d.T * d.H * d.P;
-    const int64_t n_bc = int64_t(d.B) * d.T * d.G * d.N;
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_x + n_bc;
-         i += int64_t(gridDim.x) * blockDim.x) {
-        if (i < n_x) {
-            const int p = int(i % d.P);
-            int64_t r = i / d.P;
-            const int h = int(r % d.H);
-            r /= d.H;
-            const int t = int(r % d.T), b = int(r / d.T);
-            const int tau = d.T - 1 - t;
-            const int64_t idt = off_dt(d, b, t) + h;
-            const float dtt = dt[idt];
-            xr[off_x(d, b, tau, h) + p] = from_f32<TS>(decay(dt, A, idt, h) * ld(dy, i) / dtt);
-            if (p == 0) dtr[off_dt(d, b, tau) + h] = dtt;
-        } else {
-            const int64_t j = i - n_x;
-            const int n = int(j % d.N);
-            int64_t r = j / d.N;
-            const int g = int(r % d.G);
-            r /= d.G;
-            const int t = int(r % d.T), b = int(r / d.T);
-            const int64_t dst = off_bc(d, b, d.T - 1 - t, g) + n;
-            Br[dst] = from_f32<TS>(ld(Cm, j));
-            Cr[dst] = from_f32<TS>(ld(Bm, j));
+__global__ void __launch_bounds__(kThreads)
+prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__restrict__ dt, const float *__restrict__ A,
+              const T *__restrict__ Bm, const T *__restrict__ Cm, TS *__restrict__ xr, float *__restrict__ dtr,
+              TS *__restrict__ Br, TS *__restrict__ Cr) {
+    for (int64_t row = blockIdx.x; row < int64_t(d.B) * d.T; row += gridDim.x) {
+        const int b = int(row / d.T), t = int(row % d.T);
+        const int tau = d.T - 1 - t;
+        const int64_t sdt = off_dt(d, b, t), ddt_ = off_dt(d, b, tau);
+        const int64_t sx = off_x(d, b, t, 0), dx_ = off_x(d, b, tau, 0);
+        const int HP = d.H * d.P;
+        for (int k = threadIdx.x; k < HP; k += blockDim.x) {
+            const int h = k / d.P;
+            const float dtt = __ldg(dt + sdt + h);
+            xr[dx_ + k] = from_f32<TS>(__expf(dtt * __ldg(A + h)) * ld(dy, sx + k) / dtt);
+        }
+        for (int h = threadIdx.x; h < d.H; h += blockDim.x) dtr[ddt_ + h] = __ldg(dt + sdt + h);
+        const int GN = d.G * d.N;
+        const int64_t sbc = off_bc(d, b, t, 0), dbc = off_bc(d, b, tau, 0);
+        for (int k = threadIdx.x; k < GN; k += blockDim.x) {
+            Br[dbc + k] = from_f32<TS>(ld(Cm, sbc + k));
+            Cr[dbc + k] = from_f32<TS>(ld(Bm, sbc + k));
         }
     }
 }
@@ -81,41 +73,39 @@ __global__ void to_f32_kernel(const T *__restrict__ src, float *__restrict__ dst
 // and the per-head rows of the reversed ones:
 //   dyr[b,tau,h,p] = dy[b,t,h,p],  xrr[b,tau,h,p] = x[b,t,h,p]
 template <typename T, typename TS>
-__global__ void prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy,
-                              const float *__restrict__ dt, const float *__restrict__ A,
-                              const T *__restrict__ Bm, const T *__restrict__ Cm, TS *__restrict__ xb,
-                              TS *__restrict__ xc, TS *__restrict__ dyr, TS *__restrict__ xrr) {
+__global__ void __launch_bounds__(kThreads)
+prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy, const float *__restrict__ dt,
+              const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
+              TS *__restrict__ xb, TS *__restrict__ xc, TS *__restrict__ dyr, TS *__restrict__ xrr) {
     // xb and xc are split along dstate into slices of W columns, slice-major:
     // slice s holds [B, T, H, W] (each slice is one transposed scan's x)
+    extern __shared__ float f_h[];  // a_t / dt_t of this row, per head
     const int64_t slice = int64_t(d.B) * d.T * d.H * W;
-    const int64_t n_n = int64_t(d.B) * d.T * d.H * d.N;
-    const int64_t n_p = int64_t(d.B) * d.T * d.H * d.P;
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n_n + n_p;
-         i += int64_t(gridDim.x) * blockDim.x) {
-        if (i < n_n) {
-            const int n = int(i % d.N);
-            int64_t r = i / d.N;
-            const int h = int(r % d.H);
-            r /= d.H;
-            const int t = int(r % d.T), b = int(r / d.T);
+    for (int64_t row = blockIdx.x; row < int64_t(d.B) * d.T; row += gridDim.x) {
+        const int b = int(row / d.T), t = int(row % d.T);
+        const int tau = d.T - 1 - t;
+        const int64_t sdt = off_dt(d, b, t), sbc = off_bc(d, b, t, 0);
+        const int64_t rowr = off_dt(d, b, tau) * W, rowf = off_dt(d, b, t) * W;  // (b, t', h = 0) * W
+        __syncthreads();  // the previous row's factors are no longer read
+        for (int h = threadIdx.x; h < d.H; h += blockDim.x) {
+            const float dtt = __ldg(dt + sdt + h);
+            f_h[h] = __expf(dtt * __ldg(A + h)) / dtt;
+        }
+        __syncthreads();
+        const int HN = d.H * d.N;
+        for (int k = threadIdx.x; k < HN; k += blockDim.x) {
+            const int h = k / d.N, n = k - h * d.N;
             const int g = h / d.r;
-            const int64_t idt = off_dt(d, b, t) + h;
-            const int64_t src = off_bc(d, b, t, g) + n;
-            const int sl = n / W, nn = n % W;
-            const int64_t rowr = sl * slice + ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * W + nn;
-            const int64_t rowf = sl * slice + ((int64_t(b) * d.T + t) * d.H + h) * W + nn;
-            xb[rowr] = from_f32<TS>(decay(dt, A, idt, h) * ld(Cm, src) / dt[idt]);
-            xc[rowf] = from_f32<TS>(ld(Bm, src));
-        } else {
-            const int64_t j = i - n_n;
-            const int p = int(j % d.P);
-            int64_t r = j / d.P;
-            const int h = int(r % d.H);
-            r /= d.H;
-            const int t = int(r % d.T), b = int(r / d.T);
-            const int64_t dst = off_x(d, b, d.T - 1 - t, h) + p;
-            dyr[dst] = from_f32<TS>(ld(dy, j));
-            xrr[dst] = from_f32<TS>(ld(x, j));
+            const int sl = n / W, nn = n - sl * W;
+            const int64_t o = sl * slice + int64_t(h) * W + nn;
+            xb[o + rowr] = from_f32<TS>(f_h[h] * ld(Cm, sbc + g * d.N + n));
+            xc[o + rowf] = from_f32<TS>(ld(Bm, sbc + g * d.N + n));
+        }
+        const int HP = d.H * d.P;
+        const int64_t sx = off_x(d, b, t, 0), dx_ = off_x(d, b, tau, 0);
+        for (int k = threadIdx.x; k < HP; k += blockDim.x) {
+            dyr[dx_ + k] = from_f32<TS>(ld(dy, sx + k));
+            xrr[dx_ + k] = from_f32<TS>(ld(x, sx + k));
         }
     }
 }
@@ -137,13 +127,14 @@ __global__ void transpose_state_kernel(int64_t BH, int P, int N, int W, const fl
 }
 
 // one warp per (b, t, h): u = G_t B_t = yk / a_t (yk from the reversed scan),
-// dx = dt u + D dy, xu = x . u, c = dt xu, r = dy . yh (yh = h_t C_t)
+// dx = dt u + D dy, xu = x . u, c = dt xu, r = dy . yh (yh = h_t C_t), and the
+// row's share of dD, dd = dy . x
 template <typename T, typename TS>
 __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ dy,
                               const float *__restrict__ dt, const float *__restrict__ A,
                               const float *__restrict__ D, const TS *__restrict__ yk,
                               const TS *__restrict__ yh, T *__restrict__ dx, float *__restrict__ xu,
-                              float *__restrict__ cc, float *__restrict__ rr) {
+                              float *__restrict__ cc, float *__restrict__ rr, float *__restrict__ dd) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = int64_t(d.B) * d.T * d.H;
     for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; w < nw;
@@ -157,23 +148,26 @@ __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restri
         const float Dh = D ? D[h] : 0.f;
         const int64_t row = off_x(d, b, t, h);
         const int64_t rowr = off_x(d, b, d.T - 1 - t, h);
-        float sx = 0.f, sr = 0.f;
+        float sx = 0.f, sr = 0.f, sd = 0.f;
         for (int p = lane; p < d.P; p += 32) {
             const float u = ld(yk, rowr + p) * inv_a;
-            const float dyp = ld(dy, row + p);
+            const float dyp = ld(dy, row + p), xp = ld(x, row + p);
             dx[row + p] = from_f32<T>(dtt * u + Dh * dyp);
-            sx = fmaf(ld(x, row + p), u, sx);
+            sx = fmaf(xp, u, sx);
             sr = fmaf(dyp, ld(yh, row + p), sr);
+            sd = fmaf(dyp, xp, sd);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             sx += __shfl_xor_sync(0xffffffffu, sx, o);
             sr += __shfl_xor_sync(0xffffffffu, sr, o);
+            sd += __shfl_xor_sync(0xffffffffu, sd, o);
         }
         if (lane == 0) {
             xu[idt] = sx;
             cc[idt] = dtt * sx;
             rr[idt] = sr;
+            dd[idt] = sd;
         }
     }
 }
@@ -198,11 +192,13 @@ __global__ void r0_kernel(int64_t BH, int PN, const float *__restrict__ dh0, con
 }
 
 // one warp per (b, h): R over the tokens in blocks of 32 (a warp prefix sum of
-// c - r), ddt_t = xu_t + A R_t, and this (b, h)'s share of dA = sum dt_t R_t
+// c - r), ddt_t = xu_t + A R_t, and this (b, h)'s shares of dA = sum dt_t R_t
+// and of dD = sum dd_t
 __global__ void prefix_kernel(Dims d, const float *__restrict__ dt, const float *__restrict__ A,
                               const float *__restrict__ R0, const float *__restrict__ xu,
-                              const float *__restrict__ cc, const float *__restrict__ rr, float *__restrict__ ddt,
-                              float *__restrict__ dA_part) {
+                              const float *__restrict__ cc, const float *__restrict__ rr,
+                              const float *__restrict__ dd, float *__restrict__ ddt, float *__restrict__ dA_part,
+                              float *__restrict__ dD_part) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = int64_t(d.B) * d.H;
     for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; w < nw;
@@ -210,7 +206,7 @@ __global__ void prefix_kernel(Dims d, const float *__restrict__ dt, const float 
         const int h = int(w % d.H), b = int(w / d.H);
         const float a_h = A[h];
         float R = R0[w];  // R at the first token of the block
-        float sA = 0.f;
+        float sA = 0.f, sD = 0.f;
         for (int t0 = 0; t0 < d.T; t0 += 32) {
             const int t = t0 + lane;
             const bool in = t < d.T;
@@ -227,78 +223,95 @@ __global__ void prefix_kernel(Dims d, const float *__restrict__ dt, const float 
             if (in) {
                 ddt[i] = xu[i] + a_h * Rt;
                 sA = fmaf(dt[i], Rt, sA);
+                sD += dd[i];
             }
             R += __shfl_sync(0xffffffffu, incl, 31);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sA += __shfl_xor_sync(0xffffffffu, sA, o);
-        if (lane == 0) dA_part[w] = sA;
+        for (int o = 16; o > 0; o >>= 1) {
+            sA += __shfl_xor_sync(0xffffffffu, sA, o);
+            sD += __shfl_xor_sync(0xffffffffu, sD, o);
+        }
+        if (lane == 0) {
+            dA_part[w] = sA;
+            dD_part[w] = sD;
+        }
     }
 }
 
-// dA[h] = sum_b dA_part[b, h]; dD[h] = sum_{b,t,p} dy x   (one block per head)
-template <typename T>
-__global__ void head_sums_kernel(Dims d, const float *__restrict__ dA_part, const T *__restrict__ x,
-                                 const T *__restrict__ dy, float *__restrict__ dA, float *__restrict__ dD) {
-    __shared__ float red[kThreads / 32];
-    const int h = blockIdx.x;
-    float s = 0.f;
-    if (dD) {
-        const int64_t rows = int64_t(d.B) * d.T;
-        for (int64_t k = threadIdx.x; k < rows * d.P; k += blockDim.x) {
-            const int64_t row = k / d.P;
-            const int p = int(k % d.P);
-            const int64_t i = (row * d.H + h) * d.P + p;
-            s = fmaf(ld(dy, i), ld(x, i), s);
-        }
+// dA[h] = sum_b dA_part[b, h]; dD[h] = sum_b dD_part[b, h]   (one thread per head)
+__global__ void head_sums_kernel(Dims d, const float *__restrict__ dA_part, const float *__restrict__ dD_part,
+                                 float *__restrict__ dA, float *__restrict__ dD) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= d.H) return;
+    float a = 0.f, s = 0.f;
+    for (int b = 0; b < d.B; ++b) {
+        a += dA_part[int64_t(b) * d.H + h];
+        s += dD_part[int64_t(b) * d.H + h];
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        if (dD) {
-            float t = 0.f;
-            for (int i = 0; i < kThreads / 32; ++i) t += red[i];
-            dD[h] = t;
-        }
-        float a = 0.f;
-        for (int b = 0; b < d.B; ++b) a += dA_part[int64_t(b) * d.H + h];
-        dA[h] = a;
-    }
+    dA[h] = a;
+    if (dD) dD[h] = s;
 }
 
 // dB[b,t,g,n] = sum_{h in g} (dt_t / a_t) yb[b,T-1-t,h,n];  dC[b,t,g,n] = sum_{h in g} yc[b,t,h,n]
+// the heads of a group are split over kParts threads per output (partial sums
+// combined in shared memory), so each row keeps kThreads loads in flight
+constexpr int kParts = 4;
 template <typename T, typename TS>
-__global__ void group_sums_kernel(Dims d, int W, const float *__restrict__ dt, const float *__restrict__ A,
-                                  const TS *__restrict__ yb, const TS *__restrict__ yc, T *__restrict__ dB,
-                                  T *__restrict__ dC) {
+__global__ void __launch_bounds__(kThreads)
+group_sums_kernel(Dims d, int W, const float *__restrict__ dt, const float *__restrict__ A,
+                  const TS *__restrict__ yb, const TS *__restrict__ yc, T *__restrict__ dB, T *__restrict__ dC) {
+    constexpr int kCols = kThreads / kParts;  // outputs per pass
+    __shared__ float red_b[kParts][kCols], red_c[kParts][kCols];
     const int64_t slice = int64_t(d.B) * d.T * d.H * W;
-    const int64_t total = int64_t(d.B) * d.T * d.G * d.N;
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total;
-         i += int64_t(gridDim.x) * blockDim.x) {
-        const int n = int(i % d.N);
-        int64_t r = i / d.N;
-        const int g = int(r % d.G);
-        r /= d.G;
-        const int t = int(r % d.T), b = int(r / d.T);
-        const int sl = n / W, nn = n % W;
-        float sb = 0.f, sc = 0.f;
-        for (int k = 0; k < d.r; ++k) {
-            const int h = g * d.r + k;
-            const int64_t idt = off_dt(d, b, t) + h;
-            const float f = dt[idt] * __expf(-dt[idt] * A[h]);
-            sb = fmaf(f, ld(yb, sl * slice + ((int64_t(b) * d.T + (d.T - 1 - t)) * d.H + h) * W + nn), sb);
-            sc += ld(yc, sl * slice + ((int64_t(b) * d.T + t) * d.H + h) * W + nn);
+    const int col = threadIdx.x % kCols, part = threadIdx.x / kCols;
+    for (int64_t row = blockIdx.x; row < int64_t(d.B) * d.T; row += gridDim.x) {
+        const int b = int(row / d.T), t = int(row % d.T);
+        const int tau = d.T - 1 - t;
+        const int64_t sdt = off_dt(d, b, t), obc = off_bc(d, b, t, 0);
+        const int64_t rowr = off_dt(d, b, tau) * W, rowf = off_dt(d, b, t) * W;
+        const int GN = d.G * d.N;
+        for (int k0 = 0; k0 < GN; k0 += kCols) {
+            const int k = k0 + col;
+            float sb = 0.f, sc = 0.f;
+            if (k < GN) {
+                const int g = k / d.N, n = k - g * d.N;
+                const int sl = n / W, nn = n - sl * W;
+                const int64_t o = sl * slice + nn;
+                for (int j = part; j < d.r; j += kParts) {
+                    const int h = g * d.r + j;
+                    const float dtt = __ldg(dt + sdt + h);
+                    const float f = dtt * __expf(-dtt * __ldg(A + h));
+                    sb = fmaf(f, ld(yb, o + rowr + int64_t(h) * W), sb);
+                    sc += ld(yc, o + rowf + int64_t(h) * W);
+                }
+            }
+            red_b[part][col] = sb;
+            red_c[part][col] = sc;
+            __syncthreads();
+            if (part == 0 && k < GN) {
+                float tb = 0.f, tc = 0.f;
+#pragma unroll
+                for (int q = 0; q < kParts; ++q) {
+                    tb += red_b[q][col];
+                    tc += red_c[q][col];
+                }
+                dB[obc + k] = from_f32<T>(tb);
+                dC[obc + k] = from_f32<T>(tc);
+            }
+            __syncthreads();
         }
-        dB[i] = from_f32<T>(sb);
-        dC[i] = from_f32<T>(sc);
     }
 }
 
 unsigned grid_for(int64_t n) {
     const int64_t g = (n + kThreads - 1) / kThreads;
     return unsigned(g < 148 * 32 ? (g < 1 ? 1 : g) : 148 * 32);
+}
+// blocks for the row kernels (one row per block, striding)
+unsigned grid_rows(const Dims &d) {
+    const int64_t rows = int64_t(d.B) * d.T;
+    return unsigned(rows < 148 * 64 ? (rows < 1 ? 1 : rows) : 148 * 64);
 }
 
 template <typename T, typename TS>
@@ -307,10 +320,9 @@ cudaError_t backward_prep_t(const Dims &d, const void *x, const void *dy, const 
     const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
     const T *bb = static_cast<const T *>(Bm), *cc = static_cast<const T *>(Cm);
     const int64_t nx = int64_t(d.B) * d.T * d.H * d.P, nbc = int64_t(d.B) * d.T * d.G * d.N;
-    const int64_t nn = int64_t(d.B) * d.T * d.H * d.N;
-    prep_k_kernel<T, float><<<grid_for(nx + nbc), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk,
+    prep_k_kernel<T, float><<<grid_rows(d), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk,
                                                                     w.ck);
-    prep_t_kernel<T, TS><<<grid_for(nn + nx), kThreads, 0, s>>>(d, w.W, xx, dyy, dt, A, bb, cc,
+    prep_t_kernel<T, TS><<<grid_rows(d), kThreads, size_t(d.H) * sizeof(float), s>>>(d, w.W, xx, dyy, dt, A, bb, cc,
                                                                 static_cast<TS *>(w.xb), static_cast<TS *>(w.xc),
                                                                 static_cast<TS *>(w.dyr), static_cast<TS *>(w.xrr));
     if (w.xf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(xx, w.xf, nx);
@@ -328,11 +340,13 @@ cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const 
     const int64_t nw = int64_t(d.B) * d.T * d.H;
     const int64_t BH = int64_t(d.B) * d.H;
     post_k_kernel<T, float><<<grid_for(nw * 32), kThreads, 0, s>>>(d, xx, dyy, dt, A, D, w.yk, w.yh,
-                                                                  static_cast<T *>(dx), w.xu, w.cc, w.rr);
+                                                                  static_cast<T *>(dx), w.xu, w.cc, w.rr, w.dd);
     r0_kernel<<<unsigned(BH), kThreads, 0, s>>>(BH, d.P * d.N, w.dh0, h0, w.R0);
-    prefix_kernel<<<grid_for(BH * 32), kThreads, 0, s>>>(d, dt, A, w.R0, w.xu, w.cc, w.rr, ddt, w.dA_part);
-    head_sums_kernel<T><<<unsigned(d.H), kThreads, 0, s>>>(d, w.dA_part, xx, dyy, dA, dD);
-    group_sums_kernel<T, TS><<<grid_for(int64_t(d.B) * d.T * d.G * d.N), kThreads, 0, s>>>(
+    prefix_kernel<<<grid_for(BH * 32), kThreads, 0, s>>>(d, dt, A, w.R0, w.xu, w.cc, w.rr, w.dd, ddt, w.dA_part,
+                                                         w.dD_part);
+    head_sums_kernel<<<unsigned((d.H + kThreads - 1) / kThreads), kThreads, 0, s>>>(d, w.dA_part, w.dD_part, dA,
+                                                                                       dD);
+    group_sums_kernel<T, TS><<<grid_rows(d), kThreads, 0, s>>>(
         d, w.W, dt, A, static_cast<const TS *>(w.yb), static_cast<const TS *>(w.yc), static_cast<T *>(dB),
         static_cast<T *>(dC));
     return cudaGetLastError();

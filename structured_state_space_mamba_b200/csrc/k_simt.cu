@@ -14,6 +14,7 @@
 //              + sum_{s <= t} exp(l_t - l_s) dt_s (C_t . B_s) x_s[p] + D_h x_t[p]
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.h"
 
 namespace ssd {
 
@@ -79,140 +80,186 @@ chunk_state_simt_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ B
 }
 
 // ---------------------------------------------------------------------------
-// chunk scan: one block per (64-row tile of the chunk, c, b*H + h).
+// chunk scan: one block per (64-row tile of the chunk, c, b, block of hpc heads
+// of one group).  The scores C_t . B_s do not depend on the head, so they are
+// computed once per block into shared memory (scores[s][t]); per head and per
+// 64-column slice of P, the state term and the masked, decayed product follow.
+// Every shared-memory operand is laid out [k][i] with rows of kLd floats, so
+// each thread's four values of a k step are one 16-byte load (one of the two
+// operands is the same for the 16 threads of a half-warp: a broadcast).
 // ---------------------------------------------------------------------------
+constexpr int kLd = kTile + 4;  // row stride (floats) of the [k][i] operand tiles
+
+struct ScanSmemSimt {
+    int scores, pt, xs, ak, bk, lt, ls, dts, total;  // float offsets
+};
+__host__ __device__ inline ScanSmemSimt simt_scan_smem(int Q) {
+    ScanSmemSimt m;
+    m.scores = 0;                     // [Q][kLd]   C_t . B_s as [s][t]
+    m.pt = m.scores + Q * kLd;        // [64][kLd]  masked, decayed scores of one source block, [s][t]
+    m.xs = m.pt + kTile * kLd;        // [64][kLd]  x rows of one source block, [s][p]
+    m.ak = m.xs + kTile * kLd;        // [kK][kLd]  C slice, [n][t]
+    m.bk = m.ak + kK * kLd;           // [kK][kLd]  B slice [n][s] or s_in slice [n][p]
+    m.lt = m.bk + kK * kLd;           // [64]       l of the tile's rows
+    m.ls = m.lt + kTile;              // [Q]        l of the sources
+    m.dts = m.ls + Q;                 // [Q]        dt of the sources
+    m.total = m.dts + Q;
+    return m;
+}
+
+__device__ __forceinline__ void fma44(float (&acc)[4][4], const float4 a, const float4 b) {
+    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+}
+
+// Stage a kK-column slice [k0, k0 + kK) of `nrows` rows (row r at src + r *
+// stride, columns < ncols) transposed into dst[k][r]; rows / columns outside
+// are zero.  Thread i takes row i / 4 and four consecutive columns.
+template <typename T>
+__device__ __forceinline__ void stage_slice(float *dst, const T *src, int64_t stride, int nrows, int k0,
+                                            int ncols) {
+    const int r = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 4;
+    const T *row = src + int64_t(r) * stride;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int n = k0 + kq + j;
+        dst[(kq + j) * kLd + r] = (r < nrows && n < ncols) ? to_f32(row[n]) : 0.f;
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-chunk_scan_simt_kernel(Dims d, const T *__restrict__ x, const float *__restrict__ dt,
+chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__restrict__ dt,
                        const T *__restrict__ Bm, const T *__restrict__ Cm,
                        const float *__restrict__ Dskip, const float *__restrict__ l,
                        const float *__restrict__ s_in, T *__restrict__ y) {
-    __shared__ float cs[kTile][kK + 1];     // C rows of this tile, one K slice
-    __shared__ float ks[kTile][kK + 1];     // B rows (scores) or s_in rows (state term)
-    __shared__ float gs[kTile][kTile + 1];  // masked scores [t][s]
-    __shared__ float vs[kTile][kTile + 1];  // x rows [s][p]
-    __shared__ float lt[kTile], ls[kTile], dts[kTile];
+    extern __shared__ float4 smem_f4[];
+    float *sm = reinterpret_cast<float *>(smem_f4);
+    const int Q = d.Q;
+    const ScanSmemSimt L = simt_scan_smem(Q);
+    float *scores = sm + L.scores, *pt = sm + L.pt, *xs = sm + L.xs, *ak = sm + L.ak, *bk = sm + L.bk;
+    float *lt = sm + L.lt, *ls = sm + L.ls, *dts = sm + L.dts;
     const int mt = blockIdx.x, c = blockIdx.y;
-    const int b = blockIdx.z / d.H, h = blockIdx.z % d.H;
-    const int g = h / d.r;
+    const int nhb = d.H / hpc;
+    const int b = blockIdx.z / nhb, hfirst = (blockIdx.z % nhb) * hpc;
+    const int g = hfirst / d.r;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int t0 = c * d.Q;        // first token of the chunk
+    const int t0 = c * Q;          // first token of the chunk
     const int r0 = mt * kTile;     // first row (within the chunk) of this tile
-    const int rows = min(kTile, d.Q - r0);
-    const float *lc = l + off_lq(d, b, h, c);
-    const float *sc = s_in + off_state(d, b, c, h);
-    const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
-    if (threadIdx.x < kTile) lt[threadIdx.x] = threadIdx.x < rows ? __ldg(lc + r0 + threadIdx.x) : 0.f;
-    __syncthreads();
+    const int rows = min(kTile, Q - r0);
+    const int s_len = r0 + rows;   // sources [0, s_len) of the chunk
+    const int64_t bc_stride = int64_t(d.G) * d.N;
+    const T *crow = Cm + off_bc(d, b, t0 + r0, g);  // C of the tile's first row
 
-    for (int p0 = 0; p0 < d.P; p0 += kTile) {
+    // ---- 1. scores[s][t] = C_t . B_s, t <- tx, s <- ty ----------------------
+    for (int s0 = 0; s0 < s_len; s0 += kTile) {
+        const int scols = min(kTile, s_len - s0);
         float acc[4][4] = {};
-        // ---- state term: exp(l_t) * C_t . s_in[p, :] -------------------------
         for (int k0 = 0; k0 < d.N; k0 += kK) {
-            for (int i = threadIdx.x; i < kTile * kK; i += kThreads) {
-                const int row = i / kK, kk = i % kK;
-                const int n = k0 + kk;
-                cs[row][kk] = (row < rows && n < d.N) ? to_f32(Cm[off_bc(d, b, t0 + r0 + row, g) + n]) : 0.f;
-                ks[row][kk] = (p0 + row < d.P && n < d.N) ? __ldg(sc + int64_t(p0 + row) * d.N + n) : 0.f;
-            }
+            stage_slice(ak, crow, bc_stride, rows, k0, d.N);
+            stage_slice(bk, Bm + off_bc(d, b, t0 + s0, g), bc_stride, scols, k0, d.N);
             __syncthreads();
 #pragma unroll
-            for (int kk = 0; kk < kK; ++kk) {
-                float cv[4], sv[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) cv[i] = cs[ty * 4 + i][kk];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) sv[j] = ks[tx * 4 + j][kk];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(cv[i], sv[j], acc[i][j]);
-            }
+            for (int kk = 0; kk < kK; ++kk)
+                fma44(acc, *reinterpret_cast<const float4 *>(ak + kk * kLd + tx * 4),
+                      *reinterpret_cast<const float4 *>(bk + kk * kLd + ty * 4));
             __syncthreads();
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float e = __expf(lt[ty * 4 + i]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] *= e;
+        for (int j = 0; j < 4; ++j)
+            if (ty * 4 + j < scols)
+                *reinterpret_cast<float4 *>(scores + (s0 + ty * 4 + j) * kLd + tx * 4) =
+                    make_float4(acc[0][j], acc[1][j], acc[2][j], acc[3][j]);
+    }
+
+    for (int hi = 0; hi < hpc; ++hi) {
+        const int h = hfirst + hi;
+        const float *lc = l + off_lq(d, b, h, c);
+        const float *sc = s_in + off_state(d, b, c, h);
+        const float Dh = Dskip ? __ldg(Dskip + h) : 0.f;
+        __syncthreads();  // the previous head's l / dt are no longer read
+        for (int i = threadIdx.x; i < s_len; i += kThreads) {
+            ls[i] = __ldg(lc + i);
+            dts[i] = __ldg(dt + off_dt(d, b, t0 + i) + h);
         }
-        // ---- intra-chunk term, 64 source tokens at a time --------------------
-        for (int s0 = 0; s0 < r0 + rows; s0 += kTile) {
-            const int srows = min(kTile, d.Q - s0);
-            if (threadIdx.x < kTile) {
-                const int s = threadIdx.x;
-                ls[s] = s < srows ? __ldg(lc + s0 + s) : 0.f;
-                dts[s] = s < srows ? __ldg(dt + off_dt(d, b, t0 + s0 + s) + h) : 0.f;
-            }
-            // scores G[t][s] = C_t . B_s
-            float sco[4][4] = {};
+        if (threadIdx.x < kTile) lt[threadIdx.x] = threadIdx.x < rows ? __ldg(lc + r0 + threadIdx.x) : 0.f;
+        __syncthreads();
+        for (int p0 = 0; p0 < d.P; p0 += kTile) {
+            const int pcols = min(kTile, d.P - p0);
+            float acc[4][4] = {};  // t <- ty, p <- tx
+            // ---- 2. state term: exp(l_t) C_t . s_in[p, :] -----------------------
             for (int k0 = 0; k0 < d.N; k0 += kK) {
-                for (int i = threadIdx.x; i < kTile * kK; i += kThreads) {
-                    const int row = i / kK, kk = i % kK;
-                    const int n = k0 + kk;
-                    cs[row][kk] = (row < rows && n < d.N) ? to_f32(Cm[off_bc(d, b, t0 + r0 + row, g) + n]) : 0.f;
-                    ks[row][kk] = (row < srows && n < d.N) ? to_f32(Bm[off_bc(d, b, t0 + s0 + row, g) + n]) : 0.f;
-                }
+                stage_slice(ak, crow, bc_stride, rows, k0, d.N);
+                stage_slice(bk, sc + int64_t(p0) * d.N, int64_t(d.N), pcols, k0, d.N);
                 __syncthreads();
 #pragma unroll
-                for (int kk = 0; kk < kK; ++kk) {
-                    float cv[4], bv[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) cv[i] = cs[ty * 4 + i][kk];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) bv[j] = ks[tx * 4 + j][kk];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) sco[i][j] = fmaf(cv[i], bv[j], sco[i][j]);
-                }
+                for (int kk = 0; kk < kK; ++kk)
+                    fma44(acc, *reinterpret_cast<const float4 *>(ak + kk * kLd + ty * 4),
+                          *reinterpret_cast<const float4 *>(bk + kk * kLd + tx * 4));
                 __syncthreads();
             }
-            // mask and decay: L[t][s] = exp(l_t - l_s) for s <= t, times dt_s
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float e = __expf(lt[ty * 4 + i]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] *= e;
+            }
+            // ---- 3. intra-chunk term, 64 source tokens at a time ------------------
+            for (int s0 = 0; s0 < s_len; s0 += kTile) {
+                const int scols = min(kTile, s_len - s0);
+                // masked, decayed scores: exp(l_t - l_s) dt_s (C_t . B_s) for s <= t
+                for (int e = threadIdx.x; e < kTile * (kTile / 4); e += kThreads) {
+                    const int s = e >> 4, tq = (e & 15) * 4;
+                    const float4 v = s < scols ? *reinterpret_cast<const float4 *>(scores + (s0 + s) * kLd + tq)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+                    float o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int t = tq + q;
+                        const bool keep = s < scols && s0 + s <= r0 + t && t < rows;
+                        o[q] = keep ? vv[q] * __expf(lt[t] - ls[s0 + s]) * dts[s0 + s] : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(pt + s * kLd + tq) = make_float4(o[0], o[1], o[2], o[3]);
+                }
+                for (int e = threadIdx.x; e < kTile * kTile; e += kThreads) {
+                    const int s = e >> 6, p = e & 63;
+                    xs[s * kLd + p] = (s < scols && p < pcols) ? to_f32(x[off_x(d, b, t0 + s0 + s, h) + p0 + p])
+                                                               : 0.f;
+                }
+                __syncthreads();
+#pragma unroll 8
+                for (int s = 0; s < kTile; ++s)
+                    fma44(acc, *reinterpret_cast<const float4 *>(pt + s * kLd + ty * 4),
+                          *reinterpret_cast<const float4 *>(xs + s * kLd + tx * 4));
+                __syncthreads();
+            }
+            // ---- 4. skip term and store ---------------------------------------
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = ty * 4 + i;
+                if (t >= rows) continue;
+                const int64_t base = off_x(d, b, t0 + r0 + t, h) + p0;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int s = tx * 4 + j;
-                    const bool keep = (s0 + s <= r0 + t) && (s < srows) && (t < rows);
-                    gs[t][s] = keep ? sco[i][j] * __expf(lt[t] - ls[s]) * dts[s] : 0.f;
+                    const int p = tx * 4 + j;
+                    if (p >= pcols) continue;
+                    y[base + p] = from_f32<T>(fmaf(Dh, to_f32(x[base + p]), acc[i][j]));
                 }
-            }
-            for (int i = threadIdx.x; i < kTile * kTile; i += kThreads) {
-                const int s = i / kTile, p = i % kTile;
-                vs[s][p] = (s < srows && p0 + p < d.P) ? to_f32(x[off_x(d, b, t0 + s0 + s, h) + p0 + p]) : 0.f;
-            }
-            __syncthreads();
-#pragma unroll 4
-            for (int s = 0; s < kTile; ++s) {
-                float gv[4], xv[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) gv[i] = gs[ty * 4 + i][s];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) xv[j] = vs[s][tx * 4 + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(gv[i], xv[j], acc[i][j]);
-            }
-            __syncthreads();
-        }
-        // ---- skip term and store ---------------------------------------------
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = ty * 4 + i;
-            if (t >= rows) continue;
-            const int64_t base = off_x(d, b, t0 + r0 + t, h);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int p = p0 + tx * 4 + j;
-                if (p >= d.P) continue;
-                const float xv = to_f32(x[base + p]);
-                y[base + p] = from_f32<T>(fmaf(Dh, xv, acc[i][j]));
             }
         }
     }
+}
+
+// heads per block of the CUDA-core scan: the largest divisor of H / G up to 8
+int simt_heads_per_block(const Dims &d) {
+    int best = 1;
+    for (int k = 1; k <= 8; ++k)
+        if (d.r % k == 0) best = k;
+    return best;
 }
 
 }  // namespace
@@ -233,15 +280,22 @@ cudaError_t launch_chunk_scan_simt(const Dims &d, bool bf16, const void *x, cons
                                    const void *Bm, const void *Cm, const float *D,
                                    const float *l, const float *s_in, void *y,
                                    cudaStream_t stream) {
-    dim3 grid((d.Q + kTile - 1) / kTile, d.nc, d.B * d.H);
-    if (bf16)
-        chunk_scan_simt_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-            d, static_cast<const __nv_bfloat16 *>(x), dt, static_cast<const __nv_bfloat16 *>(Bm),
+    const int hpc = simt_heads_per_block(d);
+    dim3 grid((d.Q + kTile - 1) / kTile, d.nc, d.B * (d.H / hpc));
+    const int smem = simt_scan_smem(d.Q).total * int(sizeof(float));
+    if (bf16) {
+        if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan_simt_kernel<__nv_bfloat16>), smem))
+            return cudaErrorInvalidValue;
+        chunk_scan_simt_kernel<__nv_bfloat16><<<grid, kThreads, smem, stream>>>(
+            d, hpc, static_cast<const __nv_bfloat16 *>(x), dt, static_cast<const __nv_bfloat16 *>(Bm),
             static_cast<const __nv_bfloat16 *>(Cm), D, l, s_in, static_cast<__nv_bfloat16 *>(y));
-    else
-        chunk_scan_simt_kernel<float><<<grid, kThreads, 0, stream>>>(
-            d, static_cast<const float *>(x), dt, static_cast<const float *>(Bm),
+    } else {
+        if (!smem_attr_once(reinterpret_cast<const void *>(chunk_scan_simt_kernel<float>), smem))
+            return cudaErrorInvalidValue;
+        chunk_scan_simt_kernel<float><<<grid, kThreads, smem, stream>>>(
+            d, hpc, static_cast<const float *>(x), dt, static_cast<const float *>(Bm),
             static_cast<const float *>(Cm), D, l, s_in, static_cast<float *>(y));
+    }
     return cudaGetLastError();
 }
 

@@ -94,8 +94,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
     uint8_t *sP = smem + L.p_off;
     float *sl = reinterpret_cast<float *>(smem + L.l_off);
     float *sdt = reinterpret_cast<float *>(smem + L.dt_off);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // ld, cb, x, mma
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // ld, cb, x, mma, drain
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 5);
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -115,7 +115,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
     if (device_failed(err)) return;  // an earlier wait expired: skip all work
     if (tid == 0) {
         s_abort = 0;
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_b);
@@ -130,7 +130,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
     const uint32_t lane_base = uint32_t(qd * 32) << 16;
     // phases: bars[0] and bars[1] complete once per unit, bars[2] and bars[3] once per head
     uint32_t jc = 0, hc = 0;
-    bool issued0 = false;
+    // thread 0: phase parity of the last C / B and x / s_in loads it issued (-1: none)
+    int ld0_par = -1, ld2_par = -1;
 
     for (int unit = items ? int(blockIdx.x) : 0; unit < nunits && s_abort == 0;
          unit += items ? int(gridDim.x) : 1, ++jc) {
@@ -159,7 +160,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
             constexpr int slabs = N >= 64 ? N / 64 : 1;
             const uint32_t bytes = uint32_t(kRows) * N * 2 + uint32_t(s_len) * N * 2;
             mbar_expect_tx(&bars[0], bytes);
-            issued0 = true;
+            ld0_par = int(jpar);
             for (int sl_i = 0; sl_i < slabs; ++sl_i) {
                 tma_load_3d(sC + sl_i * kRows * 128, &tm_c, &bars[0], sl_i * 64, g, trow0 + mt * kRows);
                 for (int i = 0; i <= mt; ++i)
@@ -191,6 +192,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
                 constexpr int slabs = N >= 64 ? N / 64 : 1;
                 const uint32_t bytes = uint32_t(s_len) * 128 + 64u * N * 2;
                 mbar_expect_tx(&bars[2], bytes);
+                ld2_par = int(par);
                 for (int i = 0; i <= mt; ++i)
                     tma_load_3d(sX + i * kRows * 128, &tm_x, &bars[2], 0, h, trow0 + i * kRows);
                 const int srow = ((b * d.nc + c) * d.H + h) * 64;
@@ -295,11 +297,15 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_cons
             __syncthreads();
         }
     }
-    // after an abandoned wait, give copies still in flight a bounded chance to
-    // land: the unit's C / B loads and its current head's x / s_in loads
+    // after an abandoned wait, give the work still in flight a bounded chance
+    // to finish before the tensor memory is released: the last C / B and x /
+    // s_in loads issued, and every MMA this thread issued (one commit tracks
+    // them all)
     if (tid == 0 && s_abort) {
-        if (issued0) mbar_wait(&bars[0], jc & 1, nullptr);
-        mbar_wait(&bars[2], hc & 1, nullptr);
+        if (ld0_par >= 0) mbar_wait(&bars[0], uint32_t(ld0_par), nullptr);
+        if (ld2_par >= 0) mbar_wait(&bars[2], uint32_t(ld2_par), nullptr);
+        mma_commit(&bars[4]);
+        mbar_wait(&bars[4], 0, nullptr);
     }
     tc_fence_before();
     __syncthreads();

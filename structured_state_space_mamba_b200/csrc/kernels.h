@@ -133,7 +133,7 @@ cudaError_t launch_tail(const Dims &d, bool bf16, int t_begin, const void *x, co
 struct BackwardBuffers {
     void *xb, *xc, *dyr, *xrr, *yb, *yc;
     float *xk, *bk, *ck, *yk, *yh;
-    float *dtr, *xf, *dyf, *bf, *cf, *dh0, *xu, *cc, *rr, *R0, *dA_part;
+    float *dtr, *xf, *dyf, *bf, *cf, *dh0, *xu, *cc, *rr, *dd, *R0, *dA_part, *dD_part;
     int W;           // dstate columns per transposed scan
     bool scan_bf16;  // transposed-scan buffers in bf16
 };

@@ -43,7 +43,50 @@ unsigned int *device_error_word() {
     return g_err_ptr[dev];
 }
 
+// Workspace memory of the entry points that allocate their own: a stream-
+// ordered pool per device, private to the library, that keeps what it has
+// reserved between calls (release threshold unlimited), so a repeated call
+// reuses its memory instead of mapping it again at every synchronisation
+// (the default pool returns it; for the backward's 3 GB on the 2.7B-shaped
+// layer that mapping cost about a third of the call).  ssd_workspace_trim
+// returns the unused part.  Falls back to the device's default pool.
+cudaMemPool_t g_pool[kMaxDevices];
+std::once_flag g_pool_once[kMaxDevices];
+
+cudaMemPool_t workspace_pool(int dev) {
+    std::call_once(g_pool_once[dev], [dev] {
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return;
+        }
+        uint64_t keep = ~uint64_t(0);
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+            cudaGetLastError();
+        g_pool[dev] = pool;
+    });
+    return g_pool[dev];
+}
+
+cudaError_t workspace_alloc(void **p, size_t bytes, cudaStream_t st) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return cudaErrorInvalidDevice;
+    }
+    cudaMemPool_t pool = workspace_pool(dev);
+    return pool ? cudaMallocFromPoolAsync(p, bytes, pool, st) : cudaMallocAsync(p, bytes, st);
+}
+
 constexpr size_t kAlign = 256;
+// the backward's per-row kernels keep one factor per head in shared memory
+constexpr int64_t kMaxBackwardHeads = 12288;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
@@ -431,7 +474,7 @@ ssd_status_t ssd_forward(const ssd_dims_t *dims, const void *x, const float *dt,
     if (s != SSD_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     void *ws = nullptr;
-    if (cudaMallocAsync(&ws, pl.ws.total_bytes, st) != cudaSuccess) {
+    if (workspace_alloc(&ws, pl.ws.total_bytes, st) != cudaSuccess) {
         cudaGetLastError();
         return SSD_ERR_WORKSPACE;
     }
@@ -481,7 +524,7 @@ ssd_status_t ssd_forward_block(const ssd_dims_t *dims, const void *x, const floa
     void *ws = workspace;
     if (ws) {
         if (workspace_bytes < need || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return SSD_ERR_WORKSPACE;
-    } else if (cudaMallocAsync(&ws, need, st) != cudaSuccess) {
+    } else if (workspace_alloc(&ws, need, st) != cudaSuccess) {
         cudaGetLastError();
         return SSD_ERR_WORKSPACE;
     }
@@ -564,6 +607,7 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
     ssd_status_t s = make_plan(dims, chunk_len, &pf);
     if (s != SSD_OK) return s;
     if (!x || !dt || !A || !Bm || !Cm || !dy || !dx || !ddt || !dA || !dB || !dC) return SSD_ERR_NULL_ARG;
+    if (dims->nheads > kMaxBackwardHeads) return SSD_ERR_UNSUPPORTED;
     {
         const void *ptrs[] = {x, dt, A, Bm, Cm, D, init_state, dy, dfinal_state, dx, ddt, dA, dB, dC, dD,
                               dinit_state};
@@ -620,14 +664,14 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
                  o_bf = copies ? take(nbc * 4) : 0, o_cf = copies ? take(nbc * 4) : 0;
     const size_t o_yk = take(nx * 4), o_yh = take(nx * 4), o_yb = take(nn * es), o_yc = take(nn * es);
     const size_t o_dh0 = dinit_state ? 0 : take(nst * 4);
-    const size_t o_xu = take(ntok * 4), o_cc = take(ntok * 4), o_rr = take(ntok * 4), o_R0 = take(nbh * 4),
-                 o_dAp = take(nbh * 4);
+    const size_t o_xu = take(ntok * 4), o_cc = take(ntok * 4), o_rr = take(ntok * 4), o_dd = take(ntok * 4),
+                 o_R0 = take(nbh * 4), o_dAp = take(nbh * 4), o_dDp = take(nbh * 4);
     const size_t o_ft = dfinal_state ? take(nst * 4) : 0, o_ht = init_state ? take(nst * 4) : 0;
     const size_t o_ws = off;
     off = align_up(off + (pk.ws.total_bytes > pt.ws.total_bytes ? pk.ws.total_bytes : pt.ws.total_bytes));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *buf = nullptr;
-    if (cudaMallocAsync(reinterpret_cast<void **>(&buf), off, st) != cudaSuccess) {
+    if (workspace_alloc(reinterpret_cast<void **>(&buf), off, st) != cudaSuccess) {
         cudaGetLastError();
         return SSD_ERR_WORKSPACE;
     }
@@ -640,7 +684,8 @@ ssd_status_t ssd_backward(const ssd_dims_t *dims, const void *x, const float *dt
     w.xf = copies ? F(o_xf) : nullptr; w.dyf = dy_copy ? F(o_dyf) : nullptr;
     w.bf = copies ? F(o_bf) : nullptr; w.cf = copies ? F(o_cf) : nullptr;
     w.dh0 = dinit_state ? dinit_state : F(o_dh0);
-    w.xu = F(o_xu); w.cc = F(o_cc); w.rr = F(o_rr); w.R0 = F(o_R0); w.dA_part = F(o_dAp);
+    w.xu = F(o_xu); w.cc = F(o_cc); w.rr = F(o_rr); w.dd = F(o_dd); w.R0 = F(o_R0); w.dA_part = F(o_dAp);
+    w.dD_part = F(o_dDp);
     w.W = W;
     w.scan_bf16 = scan_bf16;
     float *ft = dfinal_state ? F(o_ft) : nullptr, *ht = init_state ? F(o_ht) : nullptr;
@@ -710,6 +755,21 @@ ssd_status_t ssd_device_status(void *stream) {
         if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
             return SSD_ERR_CUDA;
         return SSD_ERR_DEVICE_TIMEOUT;
+    }
+    return SSD_OK;
+}
+
+ssd_status_t ssd_workspace_trim(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return SSD_ERR_CUDA;
+    }
+    cudaMemPool_t pool = workspace_pool(dev);
+    if (!pool) return SSD_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess || cudaMemPoolTrimTo(pool, 0) != cudaSuccess) {
+        cudaGetLastError();
+        return SSD_ERR_CUDA;
     }
     return SSD_OK;
 }

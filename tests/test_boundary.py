@@ -295,3 +295,20 @@ def test_varlen_argument_checks(lib):
     st = lib.ssd_forward_varlen(ctypes.byref(d), cu.ctypes.data_as(i64), 2, None, None, None, None, None, None,
                                 256, None, None, None, None, 0, None)
     assert st == 1  # SSD_ERR_NULL_ARG
+
+
+def test_backward_argument_checks(lib):
+    """ssd_backward validates before anything runs: missing required tensors
+    give SSD_ERR_NULL_ARG, more heads than its per-row kernels hold give
+    SSD_ERR_UNSUPPORTED (no pointer is touched on either path)."""
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: the checks return first
+
+    def call(d, ptr):
+        return lib.ssd_backward(ctypes.byref(d), ptr, ptr, ptr, ptr, ptr, None, 128, None, ptr, None, ptr, ptr,
+                                ptr, ptr, ptr, None, None, None)
+
+    d = binding.make_dims(1, 256, 4, 64, 64, 1, "bf16")
+    assert call(d, None) == 1  # SSD_ERR_NULL_ARG
+    many = binding.make_dims(1, 256, 12289, 64, 64, 1, "bf16")
+    assert call(many, fake) == 3  # SSD_ERR_UNSUPPORTED

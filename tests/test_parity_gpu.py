@@ -79,6 +79,8 @@ def test_tiny_f32_workload(oracle):
     dict(batch=2, seqlen=96, nheads=3, headdim=5, dstate=7, ngroups=1, chunk_len=32),
     dict(batch=1, seqlen=256, nheads=4, headdim=64, dstate=128, ngroups=2, chunk_len=128),
     dict(batch=1, seqlen=512, nheads=2, headdim=256, dstate=256, ngroups=2, chunk_len=256),
+    # eight heads per group share one block's scores; P and N not multiples of 16
+    dict(batch=2, seqlen=256, nheads=16, headdim=48, dstate=40, ngroups=2, chunk_len=128),
 ])
 @pytest.mark.parametrize("h0", [False, True])
 def test_f32_shapes(oracle, shape, h0):
