@@ -26,13 +26,27 @@ constexpr int kK = 16;
 
 // ---------------------------------------------------------------------------
 // chunk state: one block per (c, h, b); loops over 64 x 64 tiles of P x N.
+// K (the chunk's tokens) runs in slices of kK through two shared-memory
+// buffers: the next slice's global loads are in flight in registers while the
+// current one is multiplied (16-byte operand loads, one barrier per slice).
 // ---------------------------------------------------------------------------
+constexpr int kLd = kTile + 4;  // row stride (floats) of the [k][i] operand tiles
+
+__device__ __forceinline__ void fma44(float (&acc)[4][4], const float4 a, const float4 b) {
+    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_simt_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ Bm,
                         const float *__restrict__ w, float *__restrict__ states) {
-    __shared__ float xs[kK][kTile + 4];  // [token][p], weighted by w
-    __shared__ float bs[kK][kTile + 4];  // [token][n]
+    __shared__ __align__(16) float xs[2][kK][kLd];  // [token][p], weighted by w
+    __shared__ __align__(16) float bs[2][kK][kLd];  // [token][n]
+    constexpr int kPer = kK * kTile / kThreads;     // staged elements per thread and operand
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int g = h / d.r;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -42,29 +56,42 @@ chunk_state_simt_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ B
     for (int p0 = 0; p0 < d.P; p0 += kTile)
         for (int n0 = 0; n0 < d.N; n0 += kTile) {
             float acc[4][4] = {};
-            for (int k0 = 0; k0 < d.Q; k0 += kK) {
-                for (int i = threadIdx.x; i < kK * kTile; i += kThreads) {
+            float px[kPer], pb[kPer];
+            auto fetch = [&](int k0) {
+#pragma unroll
+                for (int q = 0; q < kPer; ++q) {
+                    const int i = threadIdx.x + q * kThreads;
                     const int kk = i / kTile, j = i % kTile;
                     const int t = t0 + k0 + kk;
                     const bool tin = (k0 + kk) < d.Q;
                     const float wt = tin ? __ldg(wc + k0 + kk) : 0.f;
-                    xs[kk][j] = (tin && p0 + j < d.P) ? wt * to_f32(x[off_x(d, b, t, h) + p0 + j]) : 0.f;
-                    bs[kk][j] = (tin && n0 + j < d.N) ? to_f32(Bm[off_bc(d, b, t, g) + n0 + j]) : 0.f;
+                    px[q] = (tin && p0 + j < d.P) ? wt * to_f32(x[off_x(d, b, t, h) + p0 + j]) : 0.f;
+                    pb[q] = (tin && n0 + j < d.N) ? to_f32(Bm[off_bc(d, b, t, g) + n0 + j]) : 0.f;
                 }
-                __syncthreads();
+            };
+            auto put = [&](int buf) {
 #pragma unroll
-                for (int kk = 0; kk < kK; ++kk) {
-                    float xv[4], bv[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty * 4 + i];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) bv[j] = bs[kk][tx * 4 + j];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xv[i], bv[j], acc[i][j]);
+                for (int q = 0; q < kPer; ++q) {
+                    const int i = threadIdx.x + q * kThreads;
+                    xs[buf][i / kTile][i % kTile] = px[q];
+                    bs[buf][i / kTile][i % kTile] = pb[q];
                 }
+            };
+            __syncthreads();  // the previous tile's last slice is no longer read
+            fetch(0);
+            put(0);
+            __syncthreads();
+            int buf = 0;
+            for (int k0 = 0; k0 < d.Q; k0 += kK) {
+                const bool more = k0 + kK < d.Q;
+                if (more) fetch(k0 + kK);
+#pragma unroll
+                for (int kk = 0; kk < kK; ++kk)
+                    fma44(acc, *reinterpret_cast<const float4 *>(&xs[buf][kk][ty * 4]),
+                          *reinterpret_cast<const float4 *>(&bs[buf][kk][tx * 4]));
+                if (more) put(buf ^ 1);
                 __syncthreads();
+                buf ^= 1;
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -88,8 +115,6 @@ chunk_state_simt_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ B
 // each thread's four values of a k step are one 16-byte load (one of the two
 // operands is the same for the 16 threads of a half-warp: a broadcast).
 // ---------------------------------------------------------------------------
-constexpr int kLd = kTile + 4;  // row stride (floats) of the [k][i] operand tiles
-
 struct ScanSmemSimt {
     int scores, pt, xs, ak, bk, lt, ls, dts, total;  // float offsets
 };
@@ -107,27 +132,26 @@ __host__ __device__ inline ScanSmemSimt simt_scan_smem(int Q) {
     return m;
 }
 
-__device__ __forceinline__ void fma44(float (&acc)[4][4], const float4 a, const float4 b) {
-    const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-}
-
-// Stage a kK-column slice [k0, k0 + kK) of `nrows` rows (row r at src + r *
-// stride, columns < ncols) transposed into dst[k][r]; rows / columns outside
-// are zero.  Thread i takes row i / 4 and four consecutive columns.
+// A kK-column slice [k0, k0 + kK) of `nrows` rows (row r at src + r * stride,
+// columns < ncols; zero outside), staged transposed into dst[k][r]: thread i
+// takes row i / 4 and four consecutive columns.  fetch_slice loads them into
+// registers (so the loads of the next slice are in flight during a multiply),
+// put_slice stores them.
 template <typename T>
-__device__ __forceinline__ void stage_slice(float *dst, const T *src, int64_t stride, int nrows, int k0,
+__device__ __forceinline__ void fetch_slice(float (&r)[4], const T *src, int64_t stride, int nrows, int k0,
                                             int ncols) {
-    const int r = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 4;
-    const T *row = src + int64_t(r) * stride;
+    const int row = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 4;
+    const T *p = src + int64_t(row) * stride;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int n = k0 + kq + j;
-        dst[(kq + j) * kLd + r] = (r < nrows && n < ncols) ? to_f32(row[n]) : 0.f;
+        r[j] = (row < nrows && n < ncols) ? to_f32(p[n]) : 0.f;
     }
+}
+__device__ __forceinline__ void put_slice(float *dst, const float (&r)[4]) {
+    const int row = threadIdx.x >> 2, kq = (threadIdx.x & 3) * 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[(kq + j) * kLd + row] = r[j];
 }
 
 template <typename T>
@@ -155,13 +179,21 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
     const T *crow = Cm + off_bc(d, b, t0 + r0, g);  // C of the tile's first row
 
     // ---- 1. scores[s][t] = C_t . B_s, t <- tx, s <- ty ----------------------
+    float ra[4], rb[4];  // the next slice, in flight
     for (int s0 = 0; s0 < s_len; s0 += kTile) {
         const int scols = min(kTile, s_len - s0);
+        const T *brow = Bm + off_bc(d, b, t0 + s0, g);
         float acc[4][4] = {};
+        fetch_slice(ra, crow, bc_stride, rows, 0, d.N);
+        fetch_slice(rb, brow, bc_stride, scols, 0, d.N);
         for (int k0 = 0; k0 < d.N; k0 += kK) {
-            stage_slice(ak, crow, bc_stride, rows, k0, d.N);
-            stage_slice(bk, Bm + off_bc(d, b, t0 + s0, g), bc_stride, scols, k0, d.N);
+            put_slice(ak, ra);
+            put_slice(bk, rb);
             __syncthreads();
+            if (k0 + kK < d.N) {
+                fetch_slice(ra, crow, bc_stride, rows, k0 + kK, d.N);
+                fetch_slice(rb, brow, bc_stride, scols, k0 + kK, d.N);
+            }
 #pragma unroll
             for (int kk = 0; kk < kK; ++kk)
                 fma44(acc, *reinterpret_cast<const float4 *>(ak + kk * kLd + tx * 4),
@@ -191,10 +223,17 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
             const int pcols = min(kTile, d.P - p0);
             float acc[4][4] = {};  // t <- ty, p <- tx
             // ---- 2. state term: exp(l_t) C_t . s_in[p, :] -----------------------
+            const float *srow = sc + int64_t(p0) * d.N;
+            fetch_slice(ra, crow, bc_stride, rows, 0, d.N);
+            fetch_slice(rb, srow, int64_t(d.N), pcols, 0, d.N);
             for (int k0 = 0; k0 < d.N; k0 += kK) {
-                stage_slice(ak, crow, bc_stride, rows, k0, d.N);
-                stage_slice(bk, sc + int64_t(p0) * d.N, int64_t(d.N), pcols, k0, d.N);
+                put_slice(ak, ra);
+                put_slice(bk, rb);
                 __syncthreads();
+                if (k0 + kK < d.N) {
+                    fetch_slice(ra, crow, bc_stride, rows, k0 + kK, d.N);
+                    fetch_slice(rb, srow, int64_t(d.N), pcols, k0 + kK, d.N);
+                }
 #pragma unroll
                 for (int kk = 0; kk < kK; ++kk)
                     fma44(acc, *reinterpret_cast<const float4 *>(ak + kk * kLd + ty * 4),
@@ -208,6 +247,21 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
                 for (int j = 0; j < 4; ++j) acc[i][j] *= e;
             }
             // ---- 3. intra-chunk term, 64 source tokens at a time ------------------
+            // this thread's x values of a source block: s = e / 64, p = e % 64 for
+            // e = threadIdx.x + kThreads q; the next block's are loaded during
+            // the current block's multiply
+            constexpr int kXPer = kTile * kTile / kThreads;
+            float rx[kXPer];
+            auto fetch_x = [&](int s0) {
+                const int scols = min(kTile, s_len - s0);
+#pragma unroll
+                for (int q = 0; q < kXPer; ++q) {
+                    const int e = threadIdx.x + q * kThreads;
+                    const int s = e >> 6, p = e & 63;
+                    rx[q] = (s < scols && p < pcols) ? to_f32(x[off_x(d, b, t0 + s0 + s, h) + p0 + p]) : 0.f;
+                }
+            };
+            fetch_x(0);
             for (int s0 = 0; s0 < s_len; s0 += kTile) {
                 const int scols = min(kTile, s_len - s0);
                 // masked, decayed scores: exp(l_t - l_s) dt_s (C_t . B_s) for s <= t
@@ -225,12 +279,13 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
                     }
                     *reinterpret_cast<float4 *>(pt + s * kLd + tq) = make_float4(o[0], o[1], o[2], o[3]);
                 }
-                for (int e = threadIdx.x; e < kTile * kTile; e += kThreads) {
-                    const int s = e >> 6, p = e & 63;
-                    xs[s * kLd + p] = (s < scols && p < pcols) ? to_f32(x[off_x(d, b, t0 + s0 + s, h) + p0 + p])
-                                                               : 0.f;
+#pragma unroll
+                for (int q = 0; q < kXPer; ++q) {
+                    const int e = threadIdx.x + q * kThreads;
+                    xs[(e >> 6) * kLd + (e & 63)] = rx[q];
                 }
                 __syncthreads();
+                if (s0 + kTile < s_len) fetch_x(s0 + kTile);
 #pragma unroll 8
                 for (int s = 0; s < kTile; ++s)
                     fma44(acc, *reinterpret_cast<const float4 *>(pt + s * kLd + ty * 4),
