@@ -57,24 +57,27 @@ chunk_state_simt_kernel(Dims d, const T *__restrict__ x, const T *__restrict__ B
         for (int n0 = 0; n0 < d.N; n0 += kTile) {
             float acc[4][4] = {};
             float px[kPer], pb[kPer];
+            // this thread stages column j of rows kb, kb + 4, ... of each slice
+            const int j = threadIdx.x % kTile, kb = threadIdx.x / kTile;
+            const bool pin = p0 + j < d.P, nin = n0 + j < d.N;
+            const T *xcol = x + off_x(d, b, t0, h) + p0 + j;
+            const T *bcol = Bm + off_bc(d, b, t0, g) + n0 + j;
+            const int64_t xstride = int64_t(d.H) * d.P, bstride = int64_t(d.G) * d.N;
             auto fetch = [&](int k0) {
 #pragma unroll
                 for (int q = 0; q < kPer; ++q) {
-                    const int i = threadIdx.x + q * kThreads;
-                    const int kk = i / kTile, j = i % kTile;
-                    const int t = t0 + k0 + kk;
-                    const bool tin = (k0 + kk) < d.Q;
-                    const float wt = tin ? __ldg(wc + k0 + kk) : 0.f;
-                    px[q] = (tin && p0 + j < d.P) ? wt * to_f32(x[off_x(d, b, t, h) + p0 + j]) : 0.f;
-                    pb[q] = (tin && n0 + j < d.N) ? to_f32(Bm[off_bc(d, b, t, g) + n0 + j]) : 0.f;
+                    const int kk = k0 + kb + q * (kThreads / kTile);
+                    const bool tin = kk < d.Q;
+                    const float wt = tin ? __ldg(wc + kk) : 0.f;
+                    px[q] = (tin && pin) ? wt * to_f32(xcol[kk * xstride]) : 0.f;
+                    pb[q] = (tin && nin) ? to_f32(bcol[kk * bstride]) : 0.f;
                 }
             };
             auto put = [&](int buf) {
 #pragma unroll
                 for (int q = 0; q < kPer; ++q) {
-                    const int i = threadIdx.x + q * kThreads;
-                    xs[buf][i / kTile][i % kTile] = px[q];
-                    bs[buf][i / kTile][i % kTile] = pb[q];
+                    xs[buf][kb + q * (kThreads / kTile)][j] = px[q];
+                    bs[buf][kb + q * (kThreads / kTile)][j] = pb[q];
                 }
             };
             __syncthreads();  // the previous tile's last slice is no longer read
@@ -120,8 +123,8 @@ struct ScanSmemSimt {
 };
 __host__ __device__ inline ScanSmemSimt simt_scan_smem(int Q) {
     ScanSmemSimt m;
-    m.scores = 0;                     // [Q][kLd]   C_t . B_s as [s][t]
-    m.pt = m.scores + Q * kLd;        // [64][kLd]  masked, decayed scores of one source block, [s][t]
+    m.scores = 0;                     // [Q][64]    C_t . B_s as [s][t] (whole-row float4 access: no padding)
+    m.pt = m.scores + Q * kTile;      // [64][kLd]  masked, decayed scores of one source block, [s][t]
     m.xs = m.pt + kTile * kLd;        // [64][kLd]  x rows of one source block, [s][p]
     m.ak = m.xs + kTile * kLd;        // [kK][kLd]  C slice, [n][t]
     m.bk = m.ak + kK * kLd;           // [kK][kLd]  B slice [n][s] or s_in slice [n][p]
@@ -155,7 +158,7 @@ __device__ __forceinline__ void put_slice(float *dst, const float (&r)[4]) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)  // two blocks per SM at chunk length 256 (109 KB each)
 chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__restrict__ dt,
                        const T *__restrict__ Bm, const T *__restrict__ Cm,
                        const float *__restrict__ Dskip, const float *__restrict__ l,
@@ -203,7 +206,7 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             if (ty * 4 + j < scols)
-                *reinterpret_cast<float4 *>(scores + (s0 + ty * 4 + j) * kLd + tx * 4) =
+                *reinterpret_cast<float4 *>(scores + (s0 + ty * 4 + j) * kTile + tx * 4) =
                     make_float4(acc[0][j], acc[1][j], acc[2][j], acc[3][j]);
     }
 
@@ -267,7 +270,7 @@ chunk_scan_simt_kernel(Dims d, int hpc, const T *__restrict__ x, const float *__
                 // masked, decayed scores: exp(l_t - l_s) dt_s (C_t . B_s) for s <= t
                 for (int e = threadIdx.x; e < kTile * (kTile / 4); e += kThreads) {
                     const int s = e >> 4, tq = (e & 15) * 4;
-                    const float4 v = s < scols ? *reinterpret_cast<const float4 *>(scores + (s0 + s) * kLd + tq)
+                    const float4 v = s < scols ? *reinterpret_cast<const float4 *>(scores + (s0 + s) * kTile + tq)
                                                : make_float4(0.f, 0.f, 0.f, 0.f);
                     const float vv[4] = {v.x, v.y, v.z, v.w};
                     float o[4];
