@@ -379,11 +379,15 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * ssd_forward_stage then runs that kernel, stage 2 nothing, and stage 3 the
  * block-factored scan of the tiles it listed.  `scan_engine` names the kernel
  * that computes y.  `chunk_len` is the chunk length the kernels run with: the
- * caller's, except that SSD_BF16 with chunk_len 64 runs the tensor-core
- * kernels with 128-token chunks (their tile height; two of the caller's chunks
- * per tile, the same recurrence), and so does SSD_BF16 with dstate 256 at
- * chunk_len 256 (the chunk-wide scan holds one 128-token tile of C at that
- * dstate); the arrays above then describe 128-token chunks (nc = T / 128).
+ * caller's, except on the tensor-core path (SSD_BF16, headdim 64), where the
+ * chunk length only sets the blocking of the same recurrence: chunk_len 64
+ * runs 128-token chunks (the kernels' tile height) when the single pass
+ * applies; the four-kernel sequence runs 256-token chunks at chunk_len 32 /
+ * 64 / 128 (half the chunk states to write and read back); dstate 256 runs
+ * 128-token chunks (the chunk-wide scan holds one 128-token tile of C at that
+ * dstate).  None of these is taken when it would lengthen the ragged tail
+ * (seqlen mod chunk length).  The arrays above then describe the chunks the
+ * kernels run (nc = T / chunk_len of this struct).
  */
 typedef enum {
     SSD_ENGINE_SIMT = 0,            /* chunk scan on the CUDA cores                     */

@@ -113,6 +113,14 @@ struct Plan {
     ssd_workspace_layout_t ws;
 };
 
+// The single-pass kernel applies: its support, and (batch, head pair) chains
+// for at least kMinChainNum / kMinChainDen of the SMs (fewer chains leave most
+// SMs idle, and the four-kernel sequence is faster there).
+bool single_pass_applies(const Dims &d) {
+    return ssd::tc_chunk_scan_supported(d) && ssd::tc_chunk_scan4_supported(d) && ssd::tc_chunk_fused_supported(d) &&
+           int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
+}
+
 ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     if (!dims || !plan) return SSD_ERR_NULL_ARG;
     const ssd_dims_t &a = *dims;
@@ -147,16 +155,30 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
         d2.nc = d.T / 128;
         if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2)) d = d2;
     }
-    // dstate 256 at chunk_len 256: the chunk-wide tensor-core scan holds one
-    // 128-token tile of C (C_0 in tensor memory) but not a second, so the chunks
-    // are 128 tokens (the same recurrence, blocked finer; the workspace arrays
-    // then describe 128-token chunks)
-    if (a.dtype == SSD_BF16 && d.N == 256 && d.Q == 256) {
+    // dstate 256: the chunk-wide tensor-core scan holds one 128-token tile of C
+    // (C_0 in tensor memory) but not a second, so the chunks are 128 tokens
+    // (the same recurrence, blocked differently; the workspace arrays then
+    // describe 128-token chunks), unless that lengthens the ragged tail
+    if (a.dtype == SSD_BF16 && d.N == 256 && d.Q != 128 && d.T % 128 <= d.T % chunk_len && d.T / 128 <= 65535) {
         Dims d2 = d;
         d2.Q = 128;
         d2.nc = d.T / 128;
         if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2) &&
             ssd::tc_chunk_scan5_supported(d2))
+            d = d2;
+    }
+    // chunk_len 32 / 64 / 128 on the four-kernel tensor-core path: 256-token
+    // chunks halve the chunk states that path writes and reads back (S and
+    // s_in), and its scans take 256-token chunks (on the dstate-128 sweep shape
+    // 0.127 -> 0.102 ms per call).  Not where the single pass applies (it keeps
+    // no chunk states), for dstate 256 (above), or when the tail kernel would
+    // get more tokens (T mod 256 > T mod chunk_len).
+    if (a.dtype == SSD_BF16 && d.Q < 256 && d.N != 256 && d.T % 256 <= d.T % chunk_len &&
+        !single_pass_applies(d)) {
+        Dims d2 = d;
+        d2.Q = 256;
+        d2.nc = d.T / 256;
+        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2) && !single_pass_applies(d2))
             d = d2;
     }
     // a length that is not a multiple of chunk_len: the chunked kernels take the
@@ -175,12 +197,9 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     // take every decay exactly
     plan->scan5 = plan->tc_scan && ssd::tc_chunk_scan5_supported(d);
     plan->tile_finish = plan->scan5 && !ssd::tc_chunk_scan4_supported(d);
-    // the single-pass kernel walks each (b, head pair) chain chunk by chunk: used
-    // when the chains fill at least kMinChainNum / kMinChainDen of the SMs (fewer
-    // chains leave most SMs idle, and the four-kernel sequence is faster there);
-    // the tiles it lists as steep go to the block-factored scan
-    plan->single = plan->tc_scan && ssd::tc_chunk_scan4_supported(d) && ssd::tc_chunk_fused_supported(d) &&
-                   int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
+    // the single-pass kernel walks each (b, head pair) chain chunk by chunk; the
+    // tiles it lists as steep go to the block-factored scan
+    plan->single = plan->bf16 && single_pass_applies(d);
     if (plan->single) plan->fused = false;
 
     ssd_workspace_layout_t &w = plan->ws;

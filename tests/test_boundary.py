@@ -65,16 +65,20 @@ def dims(**kw):
 def test_workspace_layout(lib):
     d = dims()
     lay = binding.workspace_layout(d, 128)
-    nc = 512 // 128
+    # the four-kernel tensor-core path runs 256-token chunks; the arrays
+    # describe the chunks the kernels run
+    q = lay.chunk_len
+    assert q == 256
+    nc = 512 // q
     assert lay.l_offset == 0
-    assert lay.w_offset >= 2 * 8 * nc * 128 * 4
+    assert lay.w_offset >= 2 * 8 * nc * q * 4
     assert lay.states_offset % 256 == 0 and lay.s_in_offset % 256 == 0
     state_elems = 2 * nc * 8 * 64 * 128
     ssz = 2 if lay.states_dtype == binding.SSD_BF16 else 4
     assert lay.s_in_offset >= lay.states_offset + state_elems * ssz
     sz = 2 if lay.s_in_dtype == binding.SSD_BF16 else 4
     assert lay.total_bytes >= lay.s_in_offset + state_elems * sz
-    # N = 128, chunk_len 128: chunk-wide scan + block-factored pass over steep tiles
+    # N = 128: chunk-wide scan + block-factored pass over steep tiles
     assert lay.launches == 5 and lay.fused_state == 0
     assert binding.workspace_bytes(d, 128) == lay.total_bytes
     # fp32 storage never uses the tensor-core kernels
@@ -126,14 +130,24 @@ def test_single_pass_layout_selection(lib):
 
 
 def test_chunk_len_64_on_the_tensor_cores(lib):
-    """bf16 chunk_len 64 takes the tensor-core kernels with 128-token chunks when
-    T is a multiple of 128; otherwise, and for fp32, it keeps chunk_len 64."""
-    for n in (16, 32, 64, 128, 256):
-        lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), 64)
-        assert lay.tensor_core == 1 and lay.chunk_len == 128, n
-        assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", n
+    """bf16 chunk_len 32 / 64 / 128 on the four-kernel tensor-core path runs
+    256-token chunks (dstate 256: 128-token chunks) when that does not lengthen
+    the ragged tail; where the single pass applies, chunk_len 64 runs 128-token
+    chunks; fp32 keeps the caller's chunk_len."""
+    for q in (32, 64, 128):
+        for n in (16, 32, 64, 128, 256):
+            lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
+            assert lay.tensor_core == 1 and lay.chunk_len == (128 if n == 256 else 256), (q, n)
+            assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (q, n)
+    # T mod 256 = 192 > T mod 64 = 0: the tail would grow, chunk_len 64 stays
     odd = binding.workspace_layout(binding.make_dims(2, 960, 8, 64, 128, 1, "bf16"), 64)
     assert odd.chunk_len == 64
+    # T mod 256 = 64 = T mod 128: 256-token chunks, the same 64-token tail
+    tail = binding.workspace_layout(binding.make_dims(2, 1088, 8, 64, 128, 1, "bf16"), 128)
+    assert tail.chunk_len == 256
+    # enough chains for the single pass: it keeps 128-token chunks
+    single = binding.workspace_layout(binding.make_dims(4, 4096, 80, 64, 128, 1, "bf16"), 64)
+    assert single.single_pass == 1 and single.chunk_len == 128
     f32 = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, 128, 1, "f32"), 64)
     assert f32.chunk_len == 64 and f32.tensor_core == 0
 

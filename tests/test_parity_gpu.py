@@ -116,12 +116,11 @@ def test_tensor_core_path_selected():
             assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
             assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (n, q)
             # dstate 32 / 64 take the block-factored scan, 256 the chunk-wide one
-            # on 128-token chunks
+            # on 128-token chunks; the others run 256-token chunks
             want = {32: "block_factored", 64: "block_factored", 256: "chunk_wide"}.get(n)
             if want:
                 assert binding.SCAN_ENGINES[lay.scan_engine] == want, (n, q)
-            if n == 256:
-                assert lay.chunk_len == 128, q
+            assert lay.chunk_len == (128 if n == 256 else 256), (n, q)
     lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 32, 64, 1, "bf16"), 128)
     assert lay.tensor_core == 0
 
@@ -270,15 +269,17 @@ def test_workspace_entry_point_and_intermediates(oracle):
                              init_state=a["init_state"], return_final_state=True)
     torch.cuda.synchronize()
     assert torch.equal(y, y0) and torch.equal(f, f0)
-    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, 128, D=inp.D, h0=inp.h0,
+    # the intermediates describe the chunks the kernels ran (lay.chunk_len)
+    q = lay.chunk_len
+    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, q, D=inp.D, h0=inp.h0,
                                   intermediates=True)
-    nc = 4
+    nc = 512 // q
 
     def view(off, count, dtype):
         return ws[off: off + count * torch.tensor([], dtype=dtype).element_size()].view(dtype)
 
-    l = view(lay.l_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
-    w = view(lay.w_offset, 4 * nc * 128, torch.float32).double().cpu().numpy().reshape(1, 4, nc, 128)
+    l = view(lay.l_offset, 4 * nc * q, torch.float32).double().cpu().numpy().reshape(1, 4, nc, q)
+    w = view(lay.w_offset, 4 * nc * q, torch.float32).double().cpu().numpy().reshape(1, 4, nc, q)
     al = view(lay.alpha_offset, 4 * nc, torch.float32).double().cpu().numpy().reshape(1, 4, nc)
     stdt = torch.bfloat16 if lay.states_dtype == binding.SSD_BF16 else torch.float32
     S = view(lay.states_offset, nc * 4 * 64 * 128, stdt).double().cpu().numpy()
@@ -320,7 +321,7 @@ def test_fused_state_intermediates(oracle):
     binding.forward(a["x"], a["dt"], a["A"], a["B"], a["C"], D=a["D"], chunk_len=128,
                     init_state=a["init_state"], return_final_state=True, workspace=ws)
     torch.cuda.synchronize()
-    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, 128, D=inp.D, h0=inp.h0,
+    _, _, it = oracle.ssd_chunked(inp.x, inp.dt, inp.A, inp.B, inp.C, lay.chunk_len, D=inp.D, h0=inp.h0,
                                   intermediates=True)
     n = it["s_in"].size
     s_in = ws[lay.s_in_offset: lay.s_in_offset + 2 * n].view(torch.bfloat16)
