@@ -356,7 +356,10 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  *   w      fp32 [B, H, nc, Q]  exp(l_last - l_s) * dt_s (chunk-state weights)
  *   dtq    fp32 [B, H, nc, Q]  dt regrouped per chunk and head
  *   beta   fp32 [B, H, nc, Q]  exp(l_{32k+31} - l_s) * dt_s, k = s / 32 (source
- *                              factors of the factored in-chunk decay)
+ *                              factors of the factored in-chunk decay); dtq
+ *                              and beta are written for every chunk when the
+ *                              block-factored scan is the scan engine, else
+ *                              only for chunks it finishes (steep tiles)
  *   alpha  fp32 [B, H, nc]     exp(l_last), the decay across a whole chunk
  *   states [B, nc, H, P, N]    per-chunk states S_c = sum_s w_s x_s B_s^T;
  *                              element type given by states_dtype

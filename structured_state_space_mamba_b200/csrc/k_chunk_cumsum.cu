@@ -14,7 +14,8 @@
 //             of the tile is 0, below 1e-30: such tiles are computed by the
 //             block-factored scan), then r.  The reference r is 0, or l[127]
 //             when -l[Q-1] reaches kScanSteep but neither tile's own decay
-//             range does
+//             range does; dtq and beta are then written only for chunks with a
+//             flagged tile (the block-factored scan reads no others)
 //   fused mode (the single-pass kernel of k_tc_chunk_fused.cu): the same gq
 //             layout with a reference that also keeps the chunk state exact --
 //             r = 0 or l[127] as above, otherwise r = l[Q-1] (then every
@@ -154,13 +155,7 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
         }
         return;
     }
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-        dtq_out[base + 32 * k + lane] = dts[k];
-        beta_out[base + 32 * k + lane] = __expf(bend[k] - lv[k]) * dts[k];
-        w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
-    }
-    if (lane == 0) alpha_out[off_alpha(d, b, h, c)] = __expf(last);
+    bool flagged = false;  // a tile of this (chunk, head) is left to the block-factored scan
     if (gq_out && E >= 4) {
         float *g = gq_out + ((int64_t(b) * d.H + h) * d.nc + c) * chunk_gq(Q);
         // reference r of the chunk-wide factors: 0, or l[127] when the decay over
@@ -176,7 +171,9 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
             if ((k & 3) == 3) {  // last 32 tokens of a 128-token tile
                 const bool any0 = __any_sync(0xffffffffu, zero);
                 const float lend = __shfl_sync(0xffffffffu, lv[k], 31);
-                if (lane == 0) g[Q + (k >> 2)] = (r - lend >= kScanSteep || any0) ? 1.f : 0.f;
+                const bool steep = r - lend >= kScanSteep || any0;
+                flagged |= steep;
+                if (lane == 0) g[Q + (k >> 2)] = steep ? 1.f : 0.f;
                 zero = false;
             }
         }
@@ -184,6 +181,19 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
         if (lane == 0 && E == 4) g[Q + 1] = 0.f;
         if (lane == 0) g[Q + 3] = 0.f;
     }
+    // dtq and beta feed the block-factored scan: every chunk when it is the
+    // scan, only the chunks with a flagged tile when it finishes the chunk-wide
+    // scan's list (the plans that take gq)
+    const bool factored = !gq_out || flagged;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        if (factored) {
+            dtq_out[base + 32 * k + lane] = dts[k];
+            beta_out[base + 32 * k + lane] = __expf(bend[k] - lv[k]) * dts[k];
+        }
+        w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
+    }
+    if (lane == 0) alpha_out[off_alpha(d, b, h, c)] = __expf(last);
 }
 
 }  // namespace
