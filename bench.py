@@ -110,6 +110,27 @@ def work_model(cfg, final_state=True, lay=None):
     gq_bytes = B * H * nc * (Q + 4) * 4
     h0_bytes = state_bytes if cfg.get("init_state") else 0
     fin_bytes = state_bytes if final_state else 0
+    if lay is not None and getattr(lay, "single_pass", 0) and lay.launches == 5:
+        # presolved single pass: cumsum (fused mode, plus w and alpha); the range
+        # states: x, B, w, alpha, h0 -> one partial state per CTA, chained along
+        # each chain (small); the single pass from those states, then the
+        # block-factored scan of the listed tiles
+        pre_bytes = min(B * (H // 2) * nc, 148) * 128 * N * 4  # one state per CTA of the single pass
+        per_kernel = {
+            "ssd_chunk_cumsum": dt_bytes + H * 4 + 2 * lq + gq_bytes + B * H * nc * 4,
+            "ssd_range_states": x_bytes + bc_bytes // 2 + lq + B * H * nc * 4 + h0_bytes + 3 * pre_bytes,
+            "ssd_chunk_fused": (2 * x_bytes + bc_bytes + lq + gq_bytes + H * 4 + h0_bytes + fin_bytes
+                                + pre_bytes),
+        }
+        per_kernel_comp = {
+            "ssd_chunk_cumsum": dt_bytes + H * 4,
+            "ssd_range_states": 0,
+            "ssd_chunk_fused": 2 * x_bytes + bc_bytes + H * 4 + h0_bytes + fin_bytes,
+        }
+        per_kernel_flops = {"ssd_range_states": 2 * B * nc * H * Q * N * P, "ssd_chunk_fused": flops}
+        return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
+                    per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops,
+                    stages=("ssd_chunk_cumsum", "ssd_range_states", None, "ssd_chunk_fused"))
     if lay is not None and getattr(lay, "single_pass", 0):
         # cumsum (fused mode): dt, A -> l and g (dtq and beta only for chunks with
         # a steep tile); the single-pass kernel: x, B, C, l, g, D, h0 -> y, final

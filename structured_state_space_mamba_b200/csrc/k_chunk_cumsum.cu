@@ -21,10 +21,10 @@
 //             r = 0 or l[127] as above, otherwise r = l[Q-1] (then every
 //             g_s <= dt_s); a tile is flagged only when a factor it needs,
 //             u_t = exp(l_t - r) or g_s, would reach e^kScanSteep (a zero dt
-//             is handled by the scan itself); w and alpha are not written, and
-//             dtq and beta only for chunks with a flagged tile (the
-//             block-factored scan reads them); the pairs' chain flags are
-//             reset to 0
+//             is handled by the scan itself); w and alpha are written only
+//             when w is given (the presolved single pass reads them), dtq and
+//             beta only for chunks with a flagged tile (the block-factored
+//             scan reads them); the pairs' chain flags are reset to 0
 // With a dt bias or softplus requested (the Mamba-2 block's dt preprocessing),
 // every use above takes dt_eff = softplus(dt + dt_bias) (or dt + dt_bias), and
 // dt_eff is also written in dt's layout for the scans that read dt directly.
@@ -152,6 +152,11 @@ chunk_cumsum_kernel(Dims d, const float *__restrict__ dt, const float *__restric
                 dtq_out[base + 32 * k + lane] = dts[k];
                 beta_out[base + 32 * k + lane] = __expf(bend[k] - lv[k]) * dts[k];
             }
+        }
+        if (w_out) {  // presolved ranges: their pass over x and B takes w and alpha
+#pragma unroll
+            for (int k = 0; k < E; ++k) w_out[base + 32 * k + lane] = __expf(last - lv[k]) * dts[k];
+            if (lane == 0) alpha_out[off_alpha(d, b, h, c)] = __expf(last);
         }
         return;
     }

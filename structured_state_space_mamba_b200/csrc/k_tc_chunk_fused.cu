@@ -57,6 +57,7 @@
 // warp 15 MMA issuer for Z and CS.
 #include <cmath>
 
+#include "chain_ranges.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -119,14 +120,12 @@ struct Range {
     int nseg;
 };
 __device__ __forceinline__ Range cta_range(const Dims &d) {
-    const long long chains = (long long)d.B * (d.H / 2);
-    const long long items = chains * d.nc;
-    const long long i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
+    const ChainRange c = chain_range((long long)d.B * (d.H / 2), d.nc, blockIdx.x, gridDim.x);
     Range r;
-    r.cf = int(i0 / d.nc);
-    r.cfc = int(i0 % d.nc);
-    r.cl = int((i1 - 1) / d.nc);
-    r.clc = int((i1 - 1) % d.nc) + 1;
+    r.cf = c.cf;
+    r.cfc = c.cfc;
+    r.cl = c.cl;
+    r.clc = c.clc;
     r.nseg = r.cf == r.cl ? 1 : r.cl - r.cf + 1;
     return r;
 }
@@ -233,7 +232,8 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                    Dims d, const __nv_bfloat16 *__restrict__ x, const float *__restrict__ gq,
                    const float *__restrict__ lcum, const float *__restrict__ Dskip,
                    const float *__restrict__ h0, float *__restrict__ fin, float *__restrict__ chain,
-                   unsigned int *__restrict__ flags, __nv_bfloat16 *__restrict__ s_in,
+                   unsigned int *__restrict__ flags, const float *__restrict__ presolved,
+                   __nv_bfloat16 *__restrict__ s_in,
                    int *__restrict__ nsteep, long long *__restrict__ steep_items, int max_steep,
                    unsigned int *err) {
     using L = FusedLayout<NS>;
@@ -543,6 +543,9 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 const float *src = nullptr;
                 if (T.c0 == 0) {
                     src = h0 ? h0 + row_off : nullptr;
+                } else if (presolved) {
+                    // the state entering this CTA's range, computed before the launch
+                    src = presolved + (int64_t(blockIdx.x) * 128 + m) * NS;
                 } else {
                     if (m == 0)
                         *state_ok = wait_flag(flags + int64_t(T.b) * np + T.p, unsigned(T.c0), err) ? 1 : 0;
@@ -600,7 +603,8 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         if (c + 1 == T.c1) {
                             // ticket end: the state leaves through the chain slot (or final_state)
                             const bool last = c + 1 == d.nc;
-                            float *dst = last ? (fin ? fin + row_off : nullptr) : chain + row_off;
+                            // presolved ranges: the next CTA's entering state is known already
+                            float *dst = last ? (fin ? fin + row_off : nullptr) : (presolved ? nullptr : chain + row_off);
                             if (dst) {
 #pragma unroll 1
                                 for (int seg = 0; seg < NS / 32; ++seg) {
@@ -616,7 +620,7 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                                 }
                             }
                             tc_fence_before();
-                            if (!last) {
+                            if (!last && !presolved) {
                                 __threadfence();
                                 named_barrier(kBarState, 128);
                                 if (m == 0) st_release(flags + int64_t(T.b) * np + T.p, unsigned(T.c1));
@@ -788,18 +792,20 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
 template <int NS>
 cudaError_t launch_fused(const Dims &d, const CUtensorMap *maps, const __nv_bfloat16 *x, const float *gq,
                          const float *l, const float *D, const float *h0, float *fin, float *chain,
-                         unsigned int *flags, __nv_bfloat16 *s_in, int *nsteep, long long *items,
-                         int max_items, unsigned int *err, cudaStream_t stream) {
+                         unsigned int *flags, const float *presolved, int presolved_grid, __nv_bfloat16 *s_in,
+                         int *nsteep, long long *items, int max_items, unsigned int *err, cudaStream_t stream) {
     using L = FusedLayout<NS>;
     if (!smem_attr_once(reinterpret_cast<const void *>(chunk_fused_kernel<NS>), int(L::kTotal)))
         return cudaErrorInvalidValue;
-    // one CTA per SM (shared memory), at most one per chain
+    // hand-off mode: one CTA per SM (shared memory), at most one per chain, so
+    // every range holds at most one hand-off and all CTAs are resident at once;
+    // presolved mode: the given grid (no CTA waits on another)
     const long long chains = (long long)d.B * (d.H / 2);
     const int sms = device_sm_count();
-    const int grid = chains < sms ? int(chains) : sms;
+    const int grid = presolved ? presolved_grid : (chains < sms ? int(chains) : sms);
     chunk_fused_kernel<NS><<<grid, kThreads, L::kTotal, stream>>>(maps[0], maps[1], maps[2], maps[3], d, x, gq,
-                                                                  l, D, h0, fin, chain, flags, s_in, nsteep,
-                                                                  items, max_items, err);
+                                                                  l, D, h0, fin, chain, flags, presolved, s_in,
+                                                                  nsteep, items, max_items, err);
     return cudaGetLastError();
 }
 
@@ -816,8 +822,10 @@ size_t chunk_fused_flag_bytes(const Dims &d) { return size_t(d.B) * (d.H / 2) * 
 
 cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
                                const float *D, const float *l, const float *h0, void *y, float *fin,
-                               float *chain, unsigned int *flags, void *s_in_bf16, int *nsteep,
-                               long long *items, int max_items, unsigned int *err, cudaStream_t stream) {
+                               float *chain, unsigned int *flags, const float *presolved, int presolved_grid,
+                               void *s_in_bf16, int *nsteep, long long *items, int max_items, unsigned int *err,
+                               cudaStream_t stream) {
+    if (presolved && presolved_grid <= 0) return cudaErrorInvalidValue;
     const uint64_t bcdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
     const uint64_t bcstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
     const uint32_t bcbox[3] = {64, 1, uint32_t(kRows)};
@@ -834,10 +842,10 @@ cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, co
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
     __nv_bfloat16 *sb = static_cast<__nv_bfloat16 *>(s_in_bf16);
     switch (d.N) {
-        case 64: return launch_fused<64>(d, maps, xb, gq, l, D, h0, fin, chain, flags, sb, nsteep, items,
-                                         max_items, err, stream);
-        case 128: return launch_fused<128>(d, maps, xb, gq, l, D, h0, fin, chain, flags, sb, nsteep, items,
-                                           max_items, err, stream);
+        case 64: return launch_fused<64>(d, maps, xb, gq, l, D, h0, fin, chain, flags, presolved, presolved_grid,
+                                         sb, nsteep, items, max_items, err, stream);
+        case 128: return launch_fused<128>(d, maps, xb, gq, l, D, h0, fin, chain, flags, presolved, presolved_grid,
+                                           sb, nsteep, items, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -26,6 +26,15 @@
 //
 // Roles (10 warps): warp 0 TMA producer, warp 1 MMA issuer, warps 2..5 scale x
 // rows by w in shared memory, warps 6..9 state update + stores.
+//
+// Range mode (seg_out != nullptr) serves the presolved single pass: the grid
+// splits the (chain = head-pair unit, chunk) items exactly as the single pass
+// does (chain_ranges.cuh), and each CTA runs only its range's LAST segment, if
+// that ends inside its chain: from h0 when the segment starts a chain, from
+// zero otherwise, with no s_in written; its end state goes to seg_out[CTA].
+// range_states_kernel (below) then chains those partial states along each
+// chain into the state entering every range.
+#include "chain_ranges.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -64,6 +73,28 @@ constexpr uint32_t kStgWarpBytes = 2 * 32 * 64;
 __host__ __device__ constexpr uint32_t stg_off(int ns) { return uint32_t(num_stages(ns)) * stage_bytes(ns) + 1024; }
 size_t fused_smem_bytes(int ns) { return 1024 + stg_off(ns) + 4 * kStgWarpBytes; }
 
+// Work item k of this CTA: unit u over chunks [c0, c1).  Normal mode: units
+// blockIdx.x + k gridDim.x over all chunks.  Range mode: at most one item, the
+// last segment of the CTA's single-pass range when it ends inside its chain.
+struct UnitWork {
+    int u, c0, c1;
+};
+__device__ __forceinline__ bool unit_work(int k, const Dims &d, int units, bool range_mode, UnitWork &w) {
+    if (!range_mode) {
+        const int u = int(blockIdx.x) + k * int(gridDim.x);
+        w.u = u;
+        w.c0 = 0;
+        w.c1 = d.nc;
+        return u < units;
+    }
+    if (k > 0) return false;
+    const ChainRange r = chain_range(units, d.nc, blockIdx.x, gridDim.x);
+    w.u = r.cl;
+    w.c0 = r.cf == r.cl ? r.cfc : 0;
+    w.c1 = r.clc;
+    return w.c1 < d.nc;
+}
+
 __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *v, int n) {
     uint4 *o = reinterpret_cast<uint4 *>(dst);
     for (int q = 0; q < n / 8; ++q)
@@ -77,7 +108,8 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_s, Dims d, int nh, int units,
                    const float *__restrict__ w,
                    const float *__restrict__ alpha, const float *__restrict__ h0,
-                   __nv_bfloat16 *__restrict__ s_in, float *__restrict__ fin, unsigned int *err) {
+                   __nv_bfloat16 *__restrict__ s_in, float *__restrict__ fin, float *__restrict__ seg_out,
+                   unsigned int *err) {
     constexpr int kAcc = acc_cols(NS);
     constexpr int kStages = num_stages(NS);
     constexpr int kCols = alloc_cols(NS);
@@ -94,6 +126,7 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nhp = d.H / nh;
     const int ksteps = d.Q / kKS;
+    const bool range_mode = seg_out != nullptr;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -121,10 +154,12 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            UnitWork W;
+            for (int wk = 0; ok && unit_work(wk, d, units, range_mode, W); ++wk) {
+                const int u = W.u;
                 const int hp = u % nhp, b = u / nhp;
                 const int hh = hp * nh, g = hh / d.r;
-                for (int c = 0; c < d.nc && ok; ++c) {
+                for (int c = W.c0; c < W.c1 && ok; ++c) {
                     const int trow = b * d.T + c * d.Q;
                     for (int ks = 0; ks < ksteps; ++ks) {
                         const int s = it % kStages;
@@ -159,8 +194,9 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             constexpr uint32_t idesc = idesc_bf16_f32(128, kAcc, 1, 1);
             uint32_t it = 0, ci = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                for (int c = 0; c < d.nc && ok; ++c, ++ci) {
+            UnitWork W;
+            for (int wk = 0; ok && unit_work(wk, d, units, range_mode, W); ++wk) {
+                for (int c = W.c0; c < W.c1 && ok; ++c, ++ci) {
                     const int a = ci & 1;
                     if (!mbar_wait(&acce[a], ((ci >> 1) & 1) ^ 1, err)) { ok = false; break; }
                     tc_fence_after();
@@ -196,8 +232,9 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         const int st = tid - 64;  // 0..127
         uint32_t it = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            for (int c = 0; c < d.nc && ok; ++c) {
+        UnitWork W;
+        for (int wk = 0; ok && unit_work(wk, d, units, range_mode, W); ++wk) {
+            for (int c = W.c0; c < W.c1 && ok; ++c) {
                 for (int ks = 0; ks < ksteps; ++ks) {
                     const int s = it % kStages;
                     if (!mbar_wait(&full[s], (it / kStages) & 1, err)) { ok = false; break; }
@@ -247,7 +284,9 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         uint8_t *stg = smem + stg_off(NS) + qd * kStgWarpBytes;
         uint32_t ci = 0, nst = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        UnitWork W;
+        for (int wk = 0; ok && unit_work(wk, d, units, range_mode, W); ++wk) {
+            const int u = W.u;
             const int hp = u % nhp, b = u / nhp;
             const int h = hp * nh + (valid ? j : 0);
             const int64_t row = (int64_t(b) * d.H + h) * d.P + p;  // row of [B, H, P, N]
@@ -275,13 +314,13 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     store_bf16_row(s_in + off_state(d, b, cc, h) + int64_t(p) * NS + n0, v, kSeg);
                 }
             };
-            // R = h0 (or 0); s_in[0] = R
+            // R = h0 (or 0: range mode inside a chain); s_in[0] = R
 #pragma unroll 1
             for (int n0 = 0; n0 < NS; n0 += kSeg) {
                 float v[32];
 #pragma unroll
                 for (int e = 0; e < kSeg; ++e) v[e] = 0.f;
-                if (h0 && valid) {
+                if (h0 && valid && W.c0 == 0) {
                     const float4 *src = reinterpret_cast<const float4 *>(h0 + row * NS + n0);
 #pragma unroll
                     for (int q = 0; q < kSeg / 4; ++q) {
@@ -292,15 +331,15 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 #pragma unroll
                 for (int q = 0; q < kSeg / 16; ++q)
                     tmem_st16(tR + n0 + 16 * q, reinterpret_cast<const uint32_t *>(v + 16 * q));
-                emit(v, 0, n0);
+                if (!range_mode) emit(v, 0, n0);
             }
             tmem_wait_st();
-            for (int c = 0; c < d.nc; ++c, ++ci) {
+            for (int c = W.c0; c < W.c1; ++c, ++ci) {
                 const int a = ci & 1;
                 if (!mbar_wait(&accf[a], (ci >> 1) & 1, err)) { ok = false; break; }
                 tc_fence_after();
                 const float al = valid ? __ldg(alpha + off_alpha(d, b, h, c)) : 0.f;
-                const bool last = c + 1 == d.nc;
+                const bool last = c + 1 == W.c1;
 #pragma unroll 1
                 for (int n0 = 0; n0 < NS; n0 += kSeg) {
                     uint32_t r[32], sc[32];
@@ -320,7 +359,14 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 #pragma unroll
                         for (int q = 0; q < kSeg / 16; ++q)
                             tmem_st16(tR + n0 + 16 * q, reinterpret_cast<const uint32_t *>(v + 16 * q));
-                        emit(v, c + 1, n0);
+                        if (!range_mode) emit(v, c + 1, n0);
+                    } else if (range_mode) {
+                        if (valid) {
+                            float4 *o = reinterpret_cast<float4 *>(seg_out + (int64_t(blockIdx.x) * 128 + m) * NS + n0);
+#pragma unroll
+                            for (int q = 0; q < kSeg / 4; ++q)
+                                o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        }
                     } else if (fin && valid) {
                         float4 *o = reinterpret_cast<float4 *>(fin + row * NS + n0);
 #pragma unroll
@@ -343,16 +389,56 @@ state_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
 template <int NS>
 cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &tb,
                       const CUtensorMap &ts, int nh, const float *w, const float *alpha,
-                      const float *h0, __nv_bfloat16 *s_in, float *fin, unsigned int *err,
-                      cudaStream_t stream) {
+                      const float *h0, __nv_bfloat16 *s_in, float *fin, float *seg_out, int range_grid,
+                      unsigned int *err, cudaStream_t stream) {
     const size_t smem = fused_smem_bytes(NS);
     if (!smem_attr_once(reinterpret_cast<const void *>(state_fused_kernel<NS>), int(smem)))
         return cudaErrorInvalidValue;
     const int units = d.B * (d.H / nh);
-    const int grid = units < device_sm_count() ? units : device_sm_count();
+    const int grid = seg_out ? range_grid : (units < device_sm_count() ? units : device_sm_count());
     state_fused_kernel<NS><<<grid, kThreads, smem, stream>>>(tx, tb, ts, d, nh, units, w, alpha,
-                                                             h0, s_in, fin, err);
+                                                             h0, s_in, fin, seg_out, err);
     return cudaGetLastError();
+}
+
+// One thread per element e of a head pair's state (row m = (head of the pair,
+// p), column n) and per chain: walks the CTAs whose single-pass range starts
+// inside the chain, in order.  CTA k - 1's last segment [cp, ck) ends where CTA
+// k's range starts; its partial end state (seg[k - 1]) started from h0 when cp
+// is 0, from zero otherwise, so the state entering CTA k is
+//     start[k] = seg[k - 1]                                   (cp == 0)
+//     start[k] = (prod_{c in [cp, ck)} alpha_c) start[k - 1] + seg[k - 1]
+__global__ void __launch_bounds__(256)
+range_states_kernel(Dims d, int G, const float *__restrict__ alpha, const float *__restrict__ seg,
+                    float *__restrict__ start) {
+    const int64_t per = int64_t(128) * d.N;
+    const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (e >= per) return;
+    const int np = d.H / 2;
+    const int chain = blockIdx.y;
+    const int b = chain / np, h = 2 * (chain % np) + int(e / d.N) / 64;
+    const long long items = (long long)d.B * np * d.nc;
+    const long long first = (long long)chain * d.nc, end = first + d.nc;
+    // first CTA whose range begins strictly inside the chain
+    int k = int(first * G / items);
+    while (k < G && chain_range_begin(items, k, G) <= first) ++k;
+    float s = 0.f;
+    int cp = 0;
+    for (; k < G; ++k) {
+        const long long i0 = chain_range_begin(items, k, G);
+        if (i0 >= end) break;
+        const int ck = int(i0 - first);
+        const float part = seg[(int64_t(k) - 1) * per + e];
+        if (cp == 0) {
+            s = part;
+        } else {
+            float dec = 1.f;
+            for (int c = cp; c < ck; ++c) dec *= __ldg(alpha + off_alpha(d, b, h, c));
+            s = fmaf(dec, s, part);
+        }
+        start[int64_t(k) * per + e] = s;
+        cp = ck;
+    }
 }
 
 int fused_heads_per_unit(const Dims &d) { return d.r % 2 == 0 ? 2 : 1; }
@@ -392,12 +478,43 @@ cudaError_t launch_state_fused(const Dims &d, const void *x, const void *Bm, con
     const int nh = fused_heads_per_unit(d);
     __nv_bfloat16 *s = static_cast<__nv_bfloat16 *>(s_in_bf16);
     switch (d.N) {
-        case 16: return launch_ns<16>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
-        case 32: return launch_ns<32>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
-        case 64: return launch_ns<64>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
-        case 128: return launch_ns<128>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, err, stream);
+        case 16: return launch_ns<16>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, nullptr, 0, err, stream);
+        case 32: return launch_ns<32>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, nullptr, 0, err, stream);
+        case 64: return launch_ns<64>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, nullptr, 0, err, stream);
+        case 128: return launch_ns<128>(d, tx, tb, ts, nh, w, alpha, h0, s, fin, nullptr, 0, err, stream);
     }
     return cudaErrorInvalidValue;
+}
+
+bool presolved_ranges_supported(const Dims &d) {
+    return d.P == 64 && (d.N == 64 || d.N == 128) && (d.Q == 128 || d.Q == 256) && d.r % 2 == 0 &&
+           fused_smem_bytes(d.N) <= 227 * 1024;
+}
+
+size_t presolved_state_bytes(int G, const Dims &d) { return size_t(G) * 128 * d.N * sizeof(float); }
+
+cudaError_t launch_presolve_ranges(const Dims &d, int G, const void *x, const void *Bm, const float *w,
+                                   const float *alpha, const float *h0, float *seg, float *start,
+                                   unsigned int *err, cudaStream_t stream) {
+    if (G <= 0 || !presolved_ranges_supported(d)) return cudaErrorInvalidValue;
+    const uint64_t xdims[3] = {uint64_t(d.P), uint64_t(d.H), uint64_t(d.B) * d.T};
+    const uint64_t xstr[2] = {uint64_t(d.P) * 2, uint64_t(d.H) * d.P * 2};
+    const uint32_t xbox[3] = {64, 1, uint32_t(kKS)};
+    const uint64_t bdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
+    const uint64_t bstr[2] = {uint64_t(d.N) * 2, uint64_t(d.G) * d.N * 2};
+    const uint32_t bbox[3] = {64, 1, uint32_t(kKS)};
+    CUtensorMap tx, tb, ts{};
+    if (!make_tmap_bf16(&tx, 3, x, xdims, xstr, xbox, 128) ||
+        !make_tmap_bf16(&tb, 3, Bm, bdims, bstr, bbox, brow_bytes(d.N)))
+        return cudaErrorInvalidValue;
+    cudaError_t e = d.N == 64
+        ? launch_ns<64>(d, tx, tb, ts, 2, w, alpha, h0, nullptr, nullptr, seg, G, err, stream)
+        : launch_ns<128>(d, tx, tb, ts, 2, w, alpha, h0, nullptr, nullptr, seg, G, err, stream);
+    if (e != cudaSuccess) return e;
+    const int64_t per = int64_t(128) * d.N;
+    const dim3 grid(unsigned((per + 255) / 256), unsigned(d.B * (d.H / 2)));
+    range_states_kernel<<<grid, 256, 0, stream>>>(d, G, alpha, seg, start);
+    return cudaGetLastError();
 }
 
 }  // namespace ssd

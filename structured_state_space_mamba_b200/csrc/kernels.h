@@ -56,6 +56,16 @@ bool tc_chunk_state_supported(const Dims &d);
 // chunk_state + state_passing as one kernel (units of (b, head pair) walked over
 // all chunks); `sms` is the SM count the launch will fill
 bool tc_state_fused_supported(const Dims &d, int sms);
+// The states entering the ranges of a presolved single pass with G CTAs:
+// the fused state kernel in range mode (each CTA's last segment from zero, or
+// from h0 at a chain start, into seg [G][128][N] fp32), then those partial
+// states chained along every chain into start [G][128][N] (rows = head of the
+// pair x P).  Needs w and alpha from the cumsum.
+bool presolved_ranges_supported(const Dims &d);
+size_t presolved_state_bytes(int G, const Dims &d);
+cudaError_t launch_presolve_ranges(const Dims &d, int G, const void *x, const void *Bm, const float *w,
+                                   const float *alpha, const float *h0, float *seg, float *start,
+                                   unsigned int *err, cudaStream_t stream);
 bool tc_chunk_scan_supported(const Dims &d);
 // `err` is a device word: bit 0 is set when a bounded wait inside a kernel
 // expired (the kernel then skips its remaining work and exits cleanly).
@@ -103,10 +113,15 @@ cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq,
 bool tc_chunk_fused_supported(const Dims &d);
 size_t chunk_fused_chain_bytes(const Dims &d);
 size_t chunk_fused_flag_bytes(const Dims &d);
+// presolved != nullptr: the grid is presolved_grid CTAs (any number), and CTA
+// k's range starts from the fp32 state presolved[k] ([128 rows (head of the
+// pair, p)][N], computed by the two passes below) instead of waiting for the
+// CTA before it; no state is handed on.
 cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
                                const float *D, const float *l, const float *h0, void *y, float *fin,
-                               float *chain, unsigned int *flags, void *s_in_bf16, int *nsteep,
-                               long long *items, int max_items, unsigned int *err, cudaStream_t stream);
+                               float *chain, unsigned int *flags, const float *presolved, int presolved_grid,
+                               void *s_in_bf16, int *nsteep, long long *items, int max_items, unsigned int *err,
+                               cudaStream_t stream);
 
 // The last T mod chunk_len tokens of every (b, h) as the recurrence, from
 // h_in (the full chunks' final state, or the initial state; nullptr = zeros),

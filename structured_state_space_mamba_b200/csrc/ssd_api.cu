@@ -103,6 +103,8 @@ struct Plan {
     bool fused;     // chunk_state + state_passing in one kernel (no states buffer)
     bool scan5;     // chunk-wide scan, steep tiles finished by the block-factored scan
     bool single;    // the single-pass kernel (chunk state + state passing + scan)
+    bool presolved; // single pass whose ranges start from states computed by two passes before it
+    int G = 0;      // presolved: CTAs of the single pass (and of its range-state pass)
     bool tile_finish;  // scan5's steep tiles go to the per-tile scan (no block-factored plan)
     int t_full = 0;       // tokens in full chunks; the tail [t_full, T) runs in the tail kernel
     size_t mid_offset = 0;  // tail: fp32 state after the full chunks [B,H,P,N]
@@ -110,16 +112,34 @@ struct Plan {
     size_t gq_offset;     // scan5 / single: per-token column factors [B,H,nc,chunk_gq(Q)]
     size_t chain_offset;  // single: per-(b, h) fp32 state slots [B,H,P,N]
     size_t flag_offset;   // single: per-(b, head pair) chain flags [B, H/2]
+    size_t seg_offset;    // presolved: partial end states of the ranges [G][128][N] fp32
+    size_t start_offset;  // presolved: states entering the ranges [G][128][N] fp32
     ssd_workspace_layout_t ws;
 };
 
-// The single-pass kernel applies: its support, and (batch, head pair) chains
-// for at least kMinChainNum / kMinChainDen of the SMs (fewer chains leave most
-// SMs idle, and the four-kernel sequence is faster there).
-bool single_pass_applies(const Dims &d) {
-    return ssd::tc_chunk_scan_supported(d) && ssd::tc_chunk_scan4_supported(d) && ssd::tc_chunk_fused_supported(d) &&
-           int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
+// The single-pass kernel applies in one of two forms.
+//  * Hand-off: (batch, head pair) chains for at least kMinChainNum /
+//    kMinChainDen of the SMs; a CTA takes at most one chain's worth of chunks
+//    and hands a state to the next CTA at most once.
+//  * Presolved (fewer chains): the ranges of a full grid start from states that
+//    two passes compute first (one more pass over x and B).  Measured on B200:
+//    it pays off when the ranges are long (16 chunks or more each: the long
+//    grouped layer, 0.383 -> 0.350 ms) or when the alternative is the
+//    block-factored scan (dstate 64: the sweep shape 0.108 -> 0.098 ms); with
+//    short ranges at dstate 128 the per-range pipeline refill and the extra
+//    pass lose to the four-kernel sequence (0.101 against 0.120 ms).
+bool single_pass_supported(const Dims &d) {
+    return ssd::tc_chunk_scan_supported(d) && ssd::tc_chunk_scan4_supported(d) && ssd::tc_chunk_fused_supported(d);
 }
+bool handoff_applies(const Dims &d) {
+    return single_pass_supported(d) && int64_t(d.B) * (d.H / 2) * kMinChainDen >= int64_t(kB200Sms) * kMinChainNum;
+}
+bool presolved_applies(const Dims &d) {
+    const long long chains = (long long)d.B * (d.H / 2);
+    return single_pass_supported(d) && !handoff_applies(d) && ssd::presolved_ranges_supported(d) &&
+           (d.N == 64 || chains * d.nc >= 16ll * kB200Sms);
+}
+bool single_pass_applies(const Dims &d) { return handoff_applies(d) || presolved_applies(d); }
 
 ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     if (!dims || !plan) return SSD_ERR_NULL_ARG;
@@ -167,18 +187,18 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
             ssd::tc_chunk_scan5_supported(d2))
             d = d2;
     }
-    // chunk_len 32 / 64 / 128 on the four-kernel tensor-core path: 256-token
-    // chunks halve the chunk states that path writes and reads back (S and
-    // s_in), and its scans take 256-token chunks (on the dstate-128 sweep shape
-    // 0.127 -> 0.102 ms per call).  Not where the single pass applies (it keeps
-    // no chunk states), for dstate 256 (above), or when the tail kernel would
-    // get more tokens (T mod 256 > T mod chunk_len).
-    if (a.dtype == SSD_BF16 && d.Q < 256 && d.N != 256 && d.T % 256 <= d.T % chunk_len &&
-        !single_pass_applies(d)) {
+    // chunk_len 32 / 64 / 128 on the four-kernel tensor-core path or the
+    // presolved single pass: 256-token chunks halve the chunk states the
+    // four-kernel path writes and reads back (S and s_in; on the dstate-128
+    // sweep shape 0.127 -> 0.102 ms per call) and the presolved ranges' chunk
+    // count.  Not where the hand-off single pass applies (it keeps its
+    // length), for dstate 256 (above), or when the tail kernel would get more
+    // tokens (T mod 256 > T mod chunk_len).
+    if (a.dtype == SSD_BF16 && d.Q < 256 && d.N != 256 && d.T % 256 <= d.T % chunk_len && !handoff_applies(d)) {
         Dims d2 = d;
         d2.Q = 256;
         d2.nc = d.T / 256;
-        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2) && !single_pass_applies(d2))
+        if (ssd::tc_chunk_state_supported(d2) && ssd::tc_chunk_scan_supported(d2) && !handoff_applies(d2))
             d = d2;
     }
     // a length that is not a multiple of chunk_len: the chunked kernels take the
@@ -200,6 +220,11 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     // the single-pass kernel walks each (b, head pair) chain chunk by chunk; the
     // tiles it lists as steep go to the block-factored scan
     plan->single = plan->bf16 && single_pass_applies(d);
+    plan->presolved = plan->single && presolved_applies(d);
+    if (plan->presolved) {
+        const long long items = (long long)d.B * (d.H / 2) * d.nc;
+        plan->G = int(items < kB200Sms ? items : kB200Sms);
+    }
     if (plan->single) plan->fused = false;
 
     ssd_workspace_layout_t &w = plan->ws;
@@ -228,11 +253,17 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     if (plan->single) off = align_up(off + ssd::chunk_fused_chain_bytes(d));
     plan->flag_offset = off;
     if (plan->single) off = align_up(off + ssd::chunk_fused_flag_bytes(d));
+    plan->seg_offset = off;
+    if (plan->presolved) off = align_up(off + ssd::presolved_state_bytes(plan->G, d));
+    plan->start_offset = off;
+    if (plan->presolved) off = align_up(off + ssd::presolved_state_bytes(plan->G, d));
     plan->mid_offset = off;
     if (plan->t_full < d.T) off = align_up(off + size_t(d.B) * d.H * d.P * d.N * sizeof(float));
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
-    w.launches = d.nc == 0 ? 0 : plan->single ? 3 : (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
+    w.launches = d.nc == 0 ? 0
+                 : plan->presolved ? 5
+                 : plan->single ? 3 : (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
     if (plan->t_full < d.T) w.launches += 1;
     w.fused_state = plan->fused ? 1 : 0;
     w.single_pass = plan->single ? 1 : 0;
@@ -323,6 +354,8 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
     float *gq = (pl.scan5 || pl.single) ? reinterpret_cast<float *>(ws + pl.gq_offset) : nullptr;
     float *chain = pl.single ? reinterpret_cast<float *>(ws + pl.chain_offset) : nullptr;
     unsigned int *flags = pl.single ? reinterpret_cast<unsigned int *>(ws + pl.flag_offset) : nullptr;
+    float *seg = pl.presolved ? reinterpret_cast<float *>(ws + pl.seg_offset) : nullptr;
+    float *start = pl.presolved ? reinterpret_cast<float *>(ws + pl.start_offset) : nullptr;
     for (int stage = 0; stage < 4; ++stage) {
         if (only_stage >= 0 && stage != only_stage) continue;
         cudaError_t e = cudaSuccess;
@@ -334,21 +367,33 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
         }
         if (pl.single) {
             // cumsum (fused mode), the single-pass kernel, the block-factored scan
-            // over the tiles it listed as steep
+            // over the tiles it listed as steep.  Presolved: the cumsum also
+            // writes w and alpha, stage 1 computes the state entering every
+            // range of the single pass (two launches), and stage 3 runs the
+            // single pass from those states, then the block-factored scan.
+            const int max_steep = ssd::chunk_scan5_max_steep(d);
             switch (stage) {
                 case SSD_STAGE_CHUNK_CUMSUM:
-                    e = ssd::launch_chunk_cumsum(d, dt, A, l, w, dtq, beta, alpha, gq, nsteep, flags,
-                                                 nb->dt_bias, nb->softplus, nullptr, stream);
+                    e = ssd::launch_chunk_cumsum(d, dt, A, l, pl.presolved ? w : nullptr, dtq, beta, alpha, gq,
+                                                 nsteep, flags, nb->dt_bias, nb->softplus, nullptr, stream);
                     break;
                 case SSD_STAGE_CHUNK_STATE:
-                    e = ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags, s_in,
-                                                nsteep, steep_items, ssd::chunk_scan5_max_steep(d), err, stream);
+                    e = pl.presolved
+                            ? ssd::launch_presolve_ranges(d, pl.G, x, Bm, w, alpha, init_state, seg, start, err,
+                                                          stream)
+                            : ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags,
+                                                      nullptr, 0, s_in, nsteep, steep_items, max_steep, err,
+                                                      stream);
                     break;
                 case SSD_STAGE_STATE_PASSING:
                     break;
                 case SSD_STAGE_CHUNK_SCAN:
-                    e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, steep_items, nsteep,
-                                                   ssd::chunk_scan5_max_steep(d), err, stream);
+                    if (pl.presolved)
+                        e = ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags, start,
+                                                    pl.G, s_in, nsteep, steep_items, max_steep, err, stream);
+                    if (e == cudaSuccess)
+                        e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, steep_items, nsteep,
+                                                       max_steep, err, stream);
                     if (e == cudaSuccess) e = finish_scan();
                     break;
             }
@@ -793,6 +838,6 @@ ssd_status_t ssd_workspace_trim(void) {
     return SSD_OK;
 }
 
-const char *ssd_version(void) { return "ssd-b200 0.2.1 sm_100a"; }
+const char *ssd_version(void) { return "ssd-b200 0.3.0 sm_100a"; }
 
 }  // extern "C"

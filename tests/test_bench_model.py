@@ -15,14 +15,14 @@ def layout(cfg):
     return binding.workspace_layout(d, cfg["chunk_len"])
 
 
-def test_scan_bytes_of_the_long_context_layer_by_hand():
-    """Four-kernel sequence (few (batch, head pair) chains): the chunk-wide scan
-    reads x, B, C, l, g and the bf16 s_in, and writes y."""
-    cfg = dict(WORKLOADS["long_g8"])
+def test_scan_bytes_of_the_sweep_layer_by_hand():
+    """Four-kernel sequence (few (batch, head pair) chains with short ranges):
+    the chunk-wide scan reads x, B, C, l, g and the bf16 s_in, and writes y."""
+    cfg = dict(WORKLOADS["sweep_N128_Q256"])
     lay = layout(cfg)
     assert lay.single_pass == 0
-    wm = bench.work_model(cfg, True, lay)
-    B, T, H, P, N, G, Q = 1, 65536, 32, 64, 128, 8, 256
+    wm = bench.work_model(cfg, False, lay)
+    B, T, H, P, N, G, Q = 2, 8192, 32, 64, 128, 1, 256
     nc = T // Q
     x = B * T * H * P * 2
     bc = 2 * B * T * G * N * 2
@@ -30,8 +30,24 @@ def test_scan_bytes_of_the_long_context_layer_by_hand():
     s_in = B * nc * H * P * N * 2
     assert wm["per_kernel_bytes"]["ssd_chunk_scan"] == 2 * x + bc + l_g + s_in + H * 4
     assert wm["stages"] == ("ssd_chunk_cumsum", "ssd_chunk_state", "ssd_state_passing", "ssd_chunk_scan")
+
+
+def test_presolved_bytes_of_the_long_context_layer_by_hand():
+    """The long grouped layer runs the presolved single pass: the range states
+    read x, B (once per head pair), w and alpha; the single pass moves the
+    compulsory bytes plus l and g and the ranges' entering states."""
+    cfg = dict(WORKLOADS["long_g8"])
+    lay = layout(cfg)
+    assert lay.single_pass == 1 and lay.launches == 5
+    wm = bench.work_model(cfg, True, lay)
+    B, T, H, P, N, G, Q = 1, 65536, 32, 64, 128, 8, 256
+    nc = T // Q
+    x = B * T * H * P * 2
+    bc = 2 * B * T * G * N * 2
     comp = 2 * x + bc + B * T * H * 4 + 2 * H * 4 + 2 * B * H * P * N * 4  # h0 and final
     assert wm["bytes"] == comp
+    assert wm["stages"] == ("ssd_chunk_cumsum", "ssd_range_states", None, "ssd_chunk_fused")
+    assert wm["per_kernel_comp"]["ssd_chunk_fused"] == 2 * x + bc + H * 4 + 2 * B * H * P * N * 4
 
 
 def test_single_pass_bytes_of_the_2p7b_layer_by_hand():
@@ -97,9 +113,9 @@ def test_traffic_figure_only_for_the_captured_kernel_and_build():
 def test_kernel_roofline_counts_compulsory_bytes_only():
     """A scan's roofline bytes are the compulsory bytes it moves itself (x in,
     y out, B, C and D in); the chunk states it reads are not among them."""
-    cfg = dict(WORKLOADS["long_g8"])
+    cfg = dict(WORKLOADS["sweep_N128_Q256"])
     wm = bench.work_model(cfg, True, layout(cfg))
-    B, T, H, P, N, G = 1, 65536, 32, 64, 128, 8
+    B, T, H, P, N, G = 2, 8192, 32, 64, 128, 1
     x = B * T * H * P * 2
     bc = 2 * B * T * G * N * 2
     assert wm["per_kernel_comp"]["ssd_chunk_scan"] == 2 * x + bc + H * 4

@@ -112,11 +112,23 @@ def test_single_pass_layout_selection(lib):
         assert lay.single_pass == 1 and lay.launches == 3, (b, h, q, n)
         assert lay.fused_state == 0 and lay.states_offset == lay.s_in_offset
         assert binding.SCAN_ENGINES[lay.scan_engine] == "single_pass"
+    # 16 chains of 256 chunks: the presolved single pass (the range states, then
+    # the single pass from them: five launches, no chunk-state region)
     few = binding.workspace_layout(binding.make_dims(batch=1, seqlen=65536, nheads=32, headdim=64,
                                                      dstate=128, ngroups=8, dtype="bf16"), 256)
-    assert few.single_pass == 0 and few.launches == 5
-    assert binding.SCAN_ENGINES[few.scan_engine] == "chunk_wide"
-    assert few.s_in_offset > few.states_offset
+    assert few.single_pass == 1 and few.launches == 5
+    assert binding.SCAN_ENGINES[few.scan_engine] == "single_pass"
+    assert few.s_in_offset == few.states_offset
+    # 32 chains of 32 chunks at dstate 128: short ranges keep the four-kernel sequence
+    short = binding.workspace_layout(binding.make_dims(batch=2, seqlen=8192, nheads=32, headdim=64,
+                                                       dstate=128, ngroups=1, dtype="bf16"), 256)
+    assert short.single_pass == 0 and short.launches == 5
+    assert binding.SCAN_ENGINES[short.scan_engine] == "chunk_wide"
+    assert short.s_in_offset > short.states_offset
+    # the same at dstate 64: presolved (the alternative is the block-factored scan)
+    n64 = binding.workspace_layout(binding.make_dims(batch=2, seqlen=8192, nheads=32, headdim=64,
+                                                     dstate=64, ngroups=1, dtype="bf16"), 256)
+    assert n64.single_pass == 1 and n64.launches == 5
     # an odd number of heads per group, dstate 32 or 256: not taken
     for kw, q in ((dict(nheads=81, ngroups=1), 256), (dict(nheads=80, ngroups=1, dstate=32), 256),
                   (dict(nheads=80, ngroups=1, dstate=256), 256)):

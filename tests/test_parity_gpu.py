@@ -115,9 +115,10 @@ def test_tensor_core_path_selected():
             lay = binding.workspace_layout(binding.make_dims(2, 1024, 8, 64, n, 1, "bf16"), q)
             assert lay.tensor_core == 1 and lay.s_in_dtype == binding.SSD_BF16, (n, q)
             assert binding.SCAN_ENGINES[lay.scan_engine] != "simt", (n, q)
-            # dstate 32 / 64 take the block-factored scan, 256 the chunk-wide one
-            # on 128-token chunks; the others run 256-token chunks
-            want = {32: "block_factored", 64: "block_factored", 256: "chunk_wide"}.get(n)
+            # dstate 32 takes the block-factored scan, 64 the presolved single
+            # pass, 256 the chunk-wide scan on 128-token chunks; the others run
+            # 256-token chunks
+            want = {32: "block_factored", 64: "single_pass", 256: "chunk_wide"}.get(n)
             if want:
                 assert binding.SCAN_ENGINES[lay.scan_engine] == want, (n, q)
             assert lay.chunk_len == (128 if n == 256 else 256), (n, q)
@@ -178,6 +179,42 @@ def test_dstate_256_steep_list(oracle):
     rng = np.random.default_rng(29)
     inp.dt = rng.uniform(0.3, 0.5, size=inp.dt.shape).astype(np.float32)
     inp.A = np.array([-4.0, -0.05, -8.0, -16.0, -3.0, -5.0, -6.0, -7.0], dtype=np.float32)
+    y, f = run_gpu(inp)
+    yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
+    for h in range(8):
+        assert rel(y[:, :, h], yr[:, :, h]) <= TOL["bf16"], (h, rel(y[:, :, h], yr[:, :, h]))
+        assert rel(f[:, h], fr[:, h]) <= TOL["bf16"], (h, rel(f[:, h], fr[:, h]))
+
+
+@pytest.mark.parametrize("shape", [
+    # 4 chains of 8 chunks over 32 CTAs: every range inside one chain
+    dict(batch=1, seqlen=2048, nheads=8, headdim=64, dstate=64, ngroups=2, chunk_len=256),
+    # 9 chains, 128-token chunks and a ragged tail (the tail kernel continues from the final state)
+    dict(batch=3, seqlen=1000, nheads=6, headdim=64, dstate=64, ngroups=3, chunk_len=128),
+    # 32 chains over 148 CTAs: ranges of about 3.5 chunks, most spanning two chains
+    dict(batch=2, seqlen=4096, nheads=32, headdim=64, dstate=64, ngroups=1, chunk_len=256),
+])
+@pytest.mark.parametrize("h0", [False, True])
+def test_presolved_single_pass(oracle, shape, h0):
+    """The presolved single pass: each CTA's range starts from the state that the
+    range-state passes computed (the partial states of the ranges before it,
+    chained along the chain), not from a hand-off."""
+    d = binding.make_dims(**{k: shape[k] for k in ("batch", "seqlen", "nheads", "headdim", "dstate",
+                                                     "ngroups")}, dtype="bf16")
+    lay = binding.workspace_layout(d, shape["chunk_len"])
+    assert lay.single_pass == 1 and lay.launches == 5 + (1 if shape["seqlen"] % lay.chunk_len else 0)
+    inp = make_inputs(**shape, dtype="bf16", seed=31, init_state=h0)
+    check_full(inp, oracle)
+
+
+def test_presolved_single_pass_steep_tiles(oracle):
+    """Steep heads on the presolved path: the chunks of flagged tiles get their
+    s_in written and the block-factored scan finishes those tiles; the range
+    states stay exact (their factors never exceed 1)."""
+    inp = make_inputs(2, 2048, 8, 64, 64, 2, 256, dtype="bf16", seed=37, init_state=True, h0_std=1.0)
+    rng = np.random.default_rng(37)
+    inp.dt = rng.uniform(0.3, 0.5, size=inp.dt.shape).astype(np.float32)
+    inp.A = np.array([-4.0, -0.05, -16.0, -0.5, -1.0, -0.01, -2.0, -8.0], dtype=np.float32)
     y, f = run_gpu(inp)
     yr, fr = oracle.ssd_recurrent(inp.x, inp.dt, inp.A, inp.B, inp.C, D=inp.D, h0=inp.h0)
     for h in range(8):
