@@ -401,43 +401,64 @@ cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &t
     return cudaGetLastError();
 }
 
-// One thread per element e of a head pair's state (row m = (head of the pair,
-// p), column n) and per chain: walks the CTAs whose single-pass range starts
-// inside the chain, in order.  CTA k - 1's last segment [cp, ck) ends where CTA
-// k's range starts; its partial end state (seg[k - 1]) started from h0 when cp
-// is 0, from zero otherwise, so the state entering CTA k is
+// One block per (slice of a head pair's state, chain); one thread per element
+// e of that state (row m = (head of the pair, p), column n).  The CTAs whose
+// single-pass range begins strictly inside the chain are k0 .. k0 + M - 1, in
+// order; CTA k - 1's last segment [cp, ck) ends where CTA k's range starts, and
+// its partial end state seg[k - 1] started from h0 when cp is 0, from zero
+// otherwise, so the state entering CTA k is
 //     start[k] = seg[k - 1]                                   (cp == 0)
 //     start[k] = (prod_{c in [cp, ck)} alpha_c) start[k - 1] + seg[k - 1]
+// The products (one per listed CTA and head) are formed once per block in
+// shared memory; each thread then walks the list with one load per step.
+constexpr int kMaxRangesPerChain = 160;  // >= the grid (148) + 1
 __global__ void __launch_bounds__(256)
 range_states_kernel(Dims d, int G, const float *__restrict__ alpha, const float *__restrict__ seg,
                     float *__restrict__ start) {
+    __shared__ float dec[kMaxRangesPerChain][2];
+    __shared__ int s_k0, s_m;
     const int64_t per = int64_t(128) * d.N;
-    const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (e >= per) return;
     const int np = d.H / 2;
     const int chain = blockIdx.y;
-    const int b = chain / np, h = 2 * (chain % np) + int(e / d.N) / 64;
+    const int b = chain / np, hp = chain % np;
     const long long items = (long long)d.B * np * d.nc;
     const long long first = (long long)chain * d.nc, end = first + d.nc;
-    // first CTA whose range begins strictly inside the chain
-    int k = int(first * G / items);
-    while (k < G && chain_range_begin(items, k, G) <= first) ++k;
+    if (threadIdx.x == 0) {
+        // first CTA whose range begins strictly inside the chain, and how many do
+        int k = int(first * G / items);
+        while (k < G && chain_range_begin(items, k, G) <= first) ++k;
+        int m = 0;
+        while (k + m < G && chain_range_begin(items, k + m, G) < end) ++m;
+        s_k0 = k;
+        s_m = m;
+    }
+    __syncthreads();
+    const int k0 = s_k0, M = s_m;
+    // decay over the segment ending where listed CTA i starts (unused for i = 0):
+    // one warp per (i, head), the segment's chunks spread over the lanes
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int t = warp; t < 2 * M; t += blockDim.x >> 5) {
+        const int i = t >> 1, jh = t & 1;
+        const int ck = int(chain_range_begin(items, k0 + i, G) - first);
+        const int cp = i == 0 ? ck : int(chain_range_begin(items, k0 + i - 1, G) - first);
+        float pr = 1.f;
+        for (int c = cp + lane; c < ck; c += 32) pr *= __ldg(alpha + off_alpha(d, b, 2 * hp + jh, c));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pr *= __shfl_xor_sync(0xffffffffu, pr, o);
+        if (lane == 0) dec[i][jh] = pr;
+    }
+    __syncthreads();
+    const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (e >= per) return;
+    const int jh = int(e / d.N) / 64;
     float s = 0.f;
-    int cp = 0;
-    for (; k < G; ++k) {
-        const long long i0 = chain_range_begin(items, k, G);
-        if (i0 >= end) break;
-        const int ck = int(i0 - first);
+#pragma unroll 4
+    for (int i = 0; i < M; ++i) {
+        const int k = k0 + i;
         const float part = seg[(int64_t(k) - 1) * per + e];
-        if (cp == 0) {
-            s = part;
-        } else {
-            float dec = 1.f;
-            for (int c = cp; c < ck; ++c) dec *= __ldg(alpha + off_alpha(d, b, h, c));
-            s = fmaf(dec, s, part);
-        }
+        // the first listed CTA follows one whose last segment started the chain
+        s = i == 0 ? part : fmaf(dec[i][jh], s, part);
         start[int64_t(k) * per + e] = s;
-        cp = ck;
     }
 }
 
@@ -496,7 +517,7 @@ size_t presolved_state_bytes(int G, const Dims &d) { return size_t(G) * 128 * d.
 cudaError_t launch_presolve_ranges(const Dims &d, int G, const void *x, const void *Bm, const float *w,
                                    const float *alpha, const float *h0, float *seg, float *start,
                                    unsigned int *err, cudaStream_t stream) {
-    if (G <= 0 || !presolved_ranges_supported(d)) return cudaErrorInvalidValue;
+    if (G <= 0 || G >= kMaxRangesPerChain || !presolved_ranges_supported(d)) return cudaErrorInvalidValue;
     const uint64_t xdims[3] = {uint64_t(d.P), uint64_t(d.H), uint64_t(d.B) * d.T};
     const uint64_t xstr[2] = {uint64_t(d.P) * 2, uint64_t(d.H) * d.P * 2};
     const uint32_t xbox[3] = {64, 1, uint32_t(kKS)};
