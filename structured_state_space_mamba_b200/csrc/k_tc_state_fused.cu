@@ -401,8 +401,8 @@ cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &t
     return cudaGetLastError();
 }
 
-// One block per (slice of a head pair's state, chain); one thread per element
-// e of that state (row m = (head of the pair, p), column n).  The CTAs whose
+// One block per (slice of a head pair's state, chain); four consecutive
+// elements e of that state per thread (row m = (head of the pair, p), column n).  The CTAs whose
 // single-pass range begins strictly inside the chain are k0 .. k0 + M - 1, in
 // order; CTA k - 1's last segment [cp, ck) ends where CTA k's range starts, and
 // its partial end state seg[k - 1] started from h0 when cp is 0, from zero
@@ -410,7 +410,8 @@ cudaError_t launch_ns(const Dims &d, const CUtensorMap &tx, const CUtensorMap &t
 //     start[k] = seg[k - 1]                                   (cp == 0)
 //     start[k] = (prod_{c in [cp, ck)} alpha_c) start[k - 1] + seg[k - 1]
 // The products (one per listed CTA and head) are formed once per block in
-// shared memory; each thread then walks the list with one load per step.
+// shared memory; each thread (four elements) then walks the list with one
+// 16-byte load and store per step.
 constexpr int kMaxRangesPerChain = 160;  // >= the grid (148) + 1
 __global__ void __launch_bounds__(256)
 range_states_kernel(Dims d, int G, const float *__restrict__ alpha, const float *__restrict__ seg,
@@ -448,17 +449,23 @@ range_states_kernel(Dims d, int G, const float *__restrict__ alpha, const float 
         if (lane == 0) dec[i][jh] = pr;
     }
     __syncthreads();
-    const int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    // four consecutive elements per thread (one row: N is a multiple of 4)
+    const int64_t e = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
     if (e >= per) return;
     const int jh = int(e / d.N) / 64;
-    float s = 0.f;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int i = 0; i < M; ++i) {
         const int k = k0 + i;
-        const float part = seg[(int64_t(k) - 1) * per + e];
+        const float4 part = *reinterpret_cast<const float4 *>(seg + (int64_t(k) - 1) * per + e);
         // the first listed CTA follows one whose last segment started the chain
-        s = i == 0 ? part : fmaf(dec[i][jh], s, part);
-        start[int64_t(k) * per + e] = s;
+        if (i == 0) {
+            s = part;
+        } else {
+            const float dk = dec[i][jh];
+            s = make_float4(fmaf(dk, s.x, part.x), fmaf(dk, s.y, part.y), fmaf(dk, s.z, part.z), fmaf(dk, s.w, part.w));
+        }
+        *reinterpret_cast<float4 *>(start + int64_t(k) * per + e) = s;
     }
 }
 
@@ -533,7 +540,7 @@ cudaError_t launch_presolve_ranges(const Dims &d, int G, const void *x, const vo
         : launch_ns<128>(d, tx, tb, ts, 2, w, alpha, h0, nullptr, nullptr, seg, G, err, stream);
     if (e != cudaSuccess) return e;
     const int64_t per = int64_t(128) * d.N;
-    const dim3 grid(unsigned((per + 255) / 256), unsigned(d.B * (d.H / 2)));
+    const dim3 grid(unsigned((per / 4 + 255) / 256), unsigned(d.B * (d.H / 2)));
     range_states_kernel<<<grid, 256, 0, stream>>>(d, G, alpha, seg, start);
     return cudaGetLastError();
 }
