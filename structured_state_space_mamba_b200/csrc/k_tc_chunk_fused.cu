@@ -44,7 +44,7 @@
 //   Z   X''_k^T B_k    -> ACC += (M = 128: both heads' P rows, N = dstate)
 //   PX  P X''_k        -> Y buffer (N = 128: both heads)
 //   CS  C_k S'^T       -> Y buffer += (S' read back from ACC, written into the
-//                         tile's B region once Z has read it)
+//                         tile's B region once Z and C B^T have both read it)
 // Tensor memory (512 columns): Y buffers [0,128) and [128,256) alternating per
 // tile, ACC [256, 256 + N), score buffer [384,512).  The Y buffers are released
 // by the epilogue two tiles ahead of their next use, so a slow epilogue does not
@@ -584,8 +584,14 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                 const float *gqh = gq + ((int64_t(T.b) * d.H + h) * d.nc + c) * ngq;
                 const float r = __ldg(gqh + Q + 2);
                 for (int k = 0; k < ntile; ++k, ++kt) {
-                    // Z has read B_k: S'_k into the tile's B region for C_k S'_k^T
-                    if (!mbar_wait(z_done, kt & 1, err)) { ok = false; break; }
+                    // Z and C B^T (the other issuer's) have read B_k: S'_k into the
+                    // tile's B region for C_k S'_k^T.  The two products come from
+                    // different issuing threads, so Z's completion alone does not
+                    // order the overwrite after C B^T's reads.
+                    if (!mbar_wait(z_done, kt & 1, err) || !mbar_wait(&cbm_done[kt & 1], (kt >> 1) & 1, err)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     {
                         uint8_t *bq = cb_at(kt) + L::kCB;

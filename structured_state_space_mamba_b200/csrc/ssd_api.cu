@@ -845,6 +845,6 @@ ssd_status_t ssd_workspace_trim(void) {
     return SSD_OK;
 }
 
-const char *ssd_version(void) { return "ssd-b200 0.3.0 sm_100a"; }
+const char *ssd_version(void) { return "ssd-b200 0.3.1 sm_100a"; }
 
 }  // extern "C"
