@@ -25,6 +25,32 @@ from __future__ import annotations
 import torch
 
 
+def slice_summary(local_scan, x, dt, A, B, C, chunk_len=256):
+    """Step 1 for one slice: (alpha [B, H], S [B, H, P, N]).
+
+    S is the state the slice leaves when it starts from zero; alpha is the
+    slice's total decay, read off a scan of x = 0 from an all-ones state (the
+    states keep the local scan's dtype: fp32 from the library, fp64 from a
+    reference scan).
+    """
+    bsz, _, H, P = x.shape
+    N = B.shape[3]
+    _, S = local_scan(x, dt, A, B, C, None, chunk_len, None)
+    ones = torch.ones((bsz, H, P, N), dtype=S.dtype, device=x.device)
+    _, decayed = local_scan(torch.zeros_like(x), dt, A, B, C, None, chunk_len, ones)
+    return decayed[:, :, 0, 0].contiguous(), S
+
+
+def entering_state(alphas, states, rank, h0=None):
+    """Step 3: the state entering slice `rank` from the summaries of the slices
+    before it (lists indexed by rank) and the whole sequence's initial state."""
+    S0 = states[0]
+    s_in = h0.to(S0.dtype).clone() if h0 is not None else torch.zeros_like(S0)
+    for q in range(rank):
+        s_in = alphas[q][:, :, None, None] * s_in + states[q]
+    return s_in
+
+
 def forward_sequence_split(local_scan, x, dt, A, B, C, D=None, chunk_len=256, h0=None, group=None):
     """Sequence-parallel forward scan of this rank's slice.
 
@@ -40,13 +66,8 @@ def forward_sequence_split(local_scan, x, dt, A, B, C, D=None, chunk_len=256, h0
     rank = dist.get_rank(group)
     bsz, _, H, P = x.shape
     N = B.shape[3]
-    # 1. the state the slice alone leaves, and its total decay (states keep the
-    #    local scan's dtype: fp32 from the library, fp64 from a reference scan)
-    _, S = local_scan(x, dt, A, B, C, None, chunk_len, None)
-    zeros_state = torch.zeros((bsz, H, P, N), dtype=S.dtype, device=x.device)
-    ones = torch.ones_like(zeros_state)
-    _, decayed = local_scan(torch.zeros_like(x), dt, A, B, C, None, chunk_len, ones)
-    alpha = decayed[:, :, 0, 0].contiguous()  # [B, H]
+    # 1. the state the slice alone leaves, and its total decay
+    alpha, S = slice_summary(local_scan, x, dt, A, B, C, chunk_len)
     # 2. one all-gather of (alpha, S)
     payload = torch.cat([alpha.reshape(-1), S.reshape(-1)])
     gathered = [torch.empty_like(payload) for _ in range(world)]
@@ -55,8 +76,6 @@ def forward_sequence_split(local_scan, x, dt, A, B, C, D=None, chunk_len=256, h0
     alphas = [g[:na].reshape(bsz, H) for g in gathered]
     states = [g[na:].reshape(bsz, H, P, N) for g in gathered]
     # 3. the state entering this rank: the recurrence over the ranks before it
-    s_in = h0.to(S.dtype).clone() if h0 is not None else zeros_state.clone()
-    for q in range(rank):
-        s_in = alphas[q][:, :, None, None] * s_in + states[q]
+    s_in = entering_state(alphas, states, rank, h0)
     # 4. the slice from its true incoming state
     return local_scan(x, dt, A, B, C, D, chunk_len, s_in)
