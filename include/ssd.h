@@ -325,10 +325,11 @@ SSD_API ssd_status_t ssd_forward_varlen(const ssd_dims_t *dims, const int64_t *c
  *   ddt_t = x_t . (G_t B_t) + A_h exp(dt_t A_h) (G_t : h_{t-1}),
  *   dA_h = sum dt_t exp(dt_t A_h) (G_t : h_{t-1}),   dinit = exp(dt_0 A_h) G_0.
  * Computed with four scans of the library's own chunked forward (G backwards
- * in time and h forwards, in fp32; each transposed for dB and dC, on the bf16
- * tensor-core plans when the inputs are bf16 with headdim 64 and dstate a
- * multiple of 64, in fp32 otherwise) plus element-wise and prefix-sum kernels
- * (k_backward.cu gives the identities).
+ * in time and h forwards, in fp32 with 64-token chunks whatever chunk_len is;
+ * each transposed for dB and dC, with chunk_len, on the bf16 tensor-core plans
+ * when the inputs are bf16 with headdim 64 and dstate a multiple of 64, in
+ * fp32 otherwise) plus element-wise and prefix-sum kernels (k_backward.cu
+ * gives the identities).
  *
  *   inputs as for ssd_forward; dy [B,T,H,P] dtype; dfinal_state [B,H,P,N] fp32
  *   or NULL (zero)

@@ -28,6 +28,50 @@ constexpr int kThreads = 256;
 template <typename T>
 __device__ __forceinline__ float ld(const T *p, int64_t i) { return to_f32<T>(p[i]); }
 
+// kVec consecutive elements at a 16-byte aligned address, widened to fp32 on
+// load and rounded to the element type on store (the same conversions as the
+// scalar ld / from_f32, so either path gives the same values)
+constexpr int kVec = 8;
+__device__ __forceinline__ void ld8(const float *p, float (&v)[kVec]) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&v)[kVec]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+    const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&a);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) v[i] = __bfloat162float(e[i]);
+}
+__device__ __forceinline__ void ld2(const float *p, float (&v)[2]) {
+    const float2 a = *reinterpret_cast<const float2 *>(p);
+    v[0] = a.x; v[1] = a.y;
+}
+__device__ __forceinline__ void ld2(const __nv_bfloat16 *p, float (&v)[2]) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(p);
+    v[0] = __low2float(a); v[1] = __high2float(a);
+}
+__device__ __forceinline__ void st2(float *p, const float (&v)[2]) {
+    *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+}
+__device__ __forceinline__ void st2(__nv_bfloat16 *p, const float (&v)[2]) {
+    __nv_bfloat162 a;
+    a.x = __float2bfloat16_rn(v[0]);
+    a.y = __float2bfloat16_rn(v[1]);
+    *reinterpret_cast<__nv_bfloat162 *>(p) = a;
+}
+__device__ __forceinline__ void st8(float *p, const float (&v)[kVec]) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void st8(__nv_bfloat16 *p, const float (&v)[kVec]) {
+    uint4 a;
+    __nv_bfloat16 *e = reinterpret_cast<__nv_bfloat16 *>(&a);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) e[i] = __float2bfloat16_rn(v[i]);
+    *reinterpret_cast<uint4 *>(p) = a;
+}
+
 // The row kernels below take one (b, t) row per block, blocks striding over
 // the B*T rows; inside a row the indices are 32-bit (a row holds H*N or H*P
 // elements).
@@ -38,25 +82,45 @@ template <typename T, typename TS>
 __global__ void __launch_bounds__(kThreads)
 prep_k_kernel(Dims d, const T *__restrict__ dy, const float *__restrict__ dt, const float *__restrict__ A,
               const T *__restrict__ Bm, const T *__restrict__ Cm, TS *__restrict__ xr, float *__restrict__ dtr,
-              TS *__restrict__ Br, TS *__restrict__ Cr) {
+              TS *__restrict__ Br, TS *__restrict__ Cr, bool vec) {
     for (int64_t row = blockIdx.x; row < int64_t(d.B) * d.T; row += gridDim.x) {
         const int b = int(row / d.T), t = int(row % d.T);
         const int tau = d.T - 1 - t;
         const int64_t sdt = off_dt(d, b, t), ddt_ = off_dt(d, b, tau);
         const int64_t sx = off_x(d, b, t, 0), dx_ = off_x(d, b, tau, 0);
         const int HP = d.H * d.P;
-        for (int k = threadIdx.x; k < HP; k += blockDim.x) {
-            const int h = k / d.P;
-            const float dtt = __ldg(dt + sdt + h);
-            xr[dx_ + k] = from_f32<TS>(__expf(dtt * __ldg(A + h)) * ld(dy, sx + k) / dtt);
-        }
-        for (int h = threadIdx.x; h < d.H; h += blockDim.x) dtr[ddt_ + h] = __ldg(dt + sdt + h);
         const int GN = d.G * d.N;
         const int64_t sbc = off_bc(d, b, t, 0), dbc = off_bc(d, b, tau, 0);
-        for (int k = threadIdx.x; k < GN; k += blockDim.x) {
-            Br[dbc + k] = from_f32<TS>(ld(Cm, sbc + k));
-            Cr[dbc + k] = from_f32<TS>(ld(Bm, sbc + k));
+        if (vec) {  // headdim and dstate multiples of kVec: whole vectors of one head / group
+            for (int k = threadIdx.x * kVec; k < HP; k += blockDim.x * kVec) {
+                const int h = k / d.P;
+                const float dtt = __ldg(dt + sdt + h);
+                const float f = __expf(dtt * __ldg(A + h));
+                float v[kVec];
+                ld8(dy + sx + k, v);
+#pragma unroll
+                for (int e = 0; e < kVec; ++e) v[e] = f * v[e] / dtt;
+                st8(xr + dx_ + k, v);
+            }
+            for (int k = threadIdx.x * kVec; k < GN; k += blockDim.x * kVec) {
+                float v[kVec];
+                ld8(Cm + sbc + k, v);
+                st8(Br + dbc + k, v);
+                ld8(Bm + sbc + k, v);
+                st8(Cr + dbc + k, v);
+            }
+        } else {
+            for (int k = threadIdx.x; k < HP; k += blockDim.x) {
+                const int h = k / d.P;
+                const float dtt = __ldg(dt + sdt + h);
+                xr[dx_ + k] = from_f32<TS>(__expf(dtt * __ldg(A + h)) * ld(dy, sx + k) / dtt);
+            }
+            for (int k = threadIdx.x; k < GN; k += blockDim.x) {
+                Br[dbc + k] = from_f32<TS>(ld(Cm, sbc + k));
+                Cr[dbc + k] = from_f32<TS>(ld(Bm, sbc + k));
+            }
         }
+        for (int h = threadIdx.x; h < d.H; h += blockDim.x) dtr[ddt_ + h] = __ldg(dt + sdt + h);
     }
 }
 
@@ -76,7 +140,7 @@ template <typename T, typename TS>
 __global__ void __launch_bounds__(kThreads)
 prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy, const float *__restrict__ dt,
               const float *__restrict__ A, const T *__restrict__ Bm, const T *__restrict__ Cm,
-              TS *__restrict__ xb, TS *__restrict__ xc, TS *__restrict__ dyr, TS *__restrict__ xrr) {
+              TS *__restrict__ xb, TS *__restrict__ xc, TS *__restrict__ dyr, TS *__restrict__ xrr, bool vec) {
     // xb and xc are split along dstate into slices of W columns, slice-major:
     // slice s holds [B, T, H, W] (each slice is one transposed scan's x)
     extern __shared__ float f_h[];  // a_t / dt_t of this row, per head
@@ -93,6 +157,32 @@ prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy, 
         }
         __syncthreads();
         const int HN = d.H * d.N;
+        const int HP = d.H * d.P;
+        const int64_t sx = off_x(d, b, t, 0), dx_ = off_x(d, b, tau, 0);
+        if (vec) {  // headdim, dstate and W multiples of kVec: a vector stays in one head and slice
+            for (int k = threadIdx.x * kVec; k < HN; k += blockDim.x * kVec) {
+                const int h = k / d.N, n = k - h * d.N;
+                const int g = h / d.r;
+                const int sl = n / W, nn = n - sl * W;
+                const int64_t o = sl * slice + int64_t(h) * W + nn;
+                const float f = f_h[h];
+                float v[kVec];
+                ld8(Cm + sbc + g * d.N + n, v);
+#pragma unroll
+                for (int e = 0; e < kVec; ++e) v[e] *= f;
+                st8(xb + o + rowr, v);
+                ld8(Bm + sbc + g * d.N + n, v);
+                st8(xc + o + rowf, v);
+            }
+            for (int k = threadIdx.x * kVec; k < HP; k += blockDim.x * kVec) {
+                float v[kVec];
+                ld8(dy + sx + k, v);
+                st8(dyr + dx_ + k, v);
+                ld8(x + sx + k, v);
+                st8(xrr + dx_ + k, v);
+            }
+            continue;
+        }
         for (int k = threadIdx.x; k < HN; k += blockDim.x) {
             const int h = k / d.N, n = k - h * d.N;
             const int g = h / d.r;
@@ -101,8 +191,6 @@ prep_t_kernel(Dims d, int W, const T *__restrict__ x, const T *__restrict__ dy, 
             xb[o + rowr] = from_f32<TS>(f_h[h] * ld(Cm, sbc + g * d.N + n));
             xc[o + rowf] = from_f32<TS>(ld(Bm, sbc + g * d.N + n));
         }
-        const int HP = d.H * d.P;
-        const int64_t sx = off_x(d, b, t, 0), dx_ = off_x(d, b, tau, 0);
         for (int k = threadIdx.x; k < HP; k += blockDim.x) {
             dyr[dx_ + k] = from_f32<TS>(ld(dy, sx + k));
             xrr[dx_ + k] = from_f32<TS>(ld(x, sx + k));
@@ -134,7 +222,8 @@ __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restri
                               const float *__restrict__ dt, const float *__restrict__ A,
                               const float *__restrict__ D, const TS *__restrict__ yk,
                               const TS *__restrict__ yh, T *__restrict__ dx, float *__restrict__ xu,
-                              float *__restrict__ cc, float *__restrict__ rr, float *__restrict__ dd) {
+                              float *__restrict__ cc, float *__restrict__ rr, float *__restrict__ dd,
+                              bool pairs) {
     const int lane = threadIdx.x & 31;
     const int64_t nw = int64_t(d.B) * d.T * d.H;
     for (int64_t w = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5; w < nw;
@@ -149,13 +238,34 @@ __global__ void post_k_kernel(Dims d, const T *__restrict__ x, const T *__restri
         const int64_t row = off_x(d, b, t, h);
         const int64_t rowr = off_x(d, b, d.T - 1 - t, h);
         float sx = 0.f, sr = 0.f, sd = 0.f;
-        for (int p = lane; p < d.P; p += 32) {
-            const float u = ld(yk, rowr + p) * inv_a;
-            const float dyp = ld(dy, row + p), xp = ld(x, row + p);
-            dx[row + p] = from_f32<T>(dtt * u + Dh * dyp);
-            sx = fmaf(xp, u, sx);
-            sr = fmaf(dyp, ld(yh, row + p), sr);
-            sd = fmaf(dyp, xp, sd);
+        if (pairs) {
+            // two adjacent elements per lane (headdim even: 8- and 4-byte aligned pairs)
+            for (int p = 2 * lane; p < d.P; p += 64) {
+                float uk[2], dyv[2], xv[2], yv[2];
+                ld2(yk + rowr + p, uk);
+                ld2(dy + row + p, dyv);
+                ld2(x + row + p, xv);
+                ld2(yh + row + p, yv);
+                float o[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float u = uk[e] * inv_a;
+                    o[e] = dtt * u + Dh * dyv[e];
+                    sx = fmaf(xv[e], u, sx);
+                    sr = fmaf(dyv[e], yv[e], sr);
+                    sd = fmaf(dyv[e], xv[e], sd);
+                }
+                st2(dx + row + p, o);
+            }
+        } else {
+            for (int p = lane; p < d.P; p += 32) {
+                const float u = ld(yk, rowr + p) * inv_a;
+                const float dyp = ld(dy, row + p), xp = ld(x, row + p);
+                dx[row + p] = from_f32<T>(dtt * u + Dh * dyp);
+                sx = fmaf(xp, u, sx);
+                sr = fmaf(dyp, ld(yh, row + p), sr);
+                sd = fmaf(dyp, xp, sd);
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -260,9 +370,11 @@ constexpr int kParts = 4;
 template <typename T, typename TS>
 __global__ void __launch_bounds__(kThreads)
 group_sums_kernel(Dims d, int W, const float *__restrict__ dt, const float *__restrict__ A,
-                  const TS *__restrict__ yb, const TS *__restrict__ yc, T *__restrict__ dB, T *__restrict__ dC) {
+                  const TS *__restrict__ yb, const TS *__restrict__ yc, T *__restrict__ dB, T *__restrict__ dC,
+                  bool vec) {
     constexpr int kCols = kThreads / kParts;  // outputs per pass
     __shared__ float red_b[kParts][kCols], red_c[kParts][kCols];
+    __shared__ float4 red8_b[kThreads][2], red8_c[kThreads][2];
     const int64_t slice = int64_t(d.B) * d.T * d.H * W;
     const int col = threadIdx.x % kCols, part = threadIdx.x / kCols;
     for (int64_t row = blockIdx.x; row < int64_t(d.B) * d.T; row += gridDim.x) {
@@ -271,6 +383,59 @@ group_sums_kernel(Dims d, int W, const float *__restrict__ dt, const float *__re
         const int64_t sdt = off_dt(d, b, t), obc = off_bc(d, b, t, 0);
         const int64_t rowr = off_dt(d, b, tau) * W, rowf = off_dt(d, b, t) * W;
         const int GN = d.G * d.N;
+        if (vec) {
+            // kVec consecutive outputs (one group, one slice) per thread; the
+            // row's GN / kVec vectors take `cols` threads, the heads of a group
+            // are split over `parts` = kThreads / cols of them (partial sums
+            // combined in shared memory, in part order)
+            const int nv = GN / kVec;
+            const int cols = nv < kThreads ? nv : kThreads;
+            const int parts = kThreads / cols;
+            const int vcol = threadIdx.x % cols, vpart = threadIdx.x / cols;
+            for (int v0 = 0; v0 < nv; v0 += cols) {
+                const int v = v0 + vcol;
+                const bool act = vpart < parts && v < nv;
+                float sb[kVec] = {}, sc[kVec] = {};
+                if (act) {
+                    const int k = v * kVec;
+                    const int g = k / d.N, n = k - g * d.N;
+                    const int sl = n / W, nn = n - sl * W;
+                    const int64_t o = sl * slice + nn;
+                    for (int j = vpart; j < d.r; j += parts) {
+                        const int h = g * d.r + j;
+                        const float dtt = __ldg(dt + sdt + h);
+                        const float f = dtt * __expf(-dtt * __ldg(A + h));
+                        float vb[kVec], vc[kVec];
+                        ld8(yb + o + rowr + int64_t(h) * W, vb);
+                        ld8(yc + o + rowf + int64_t(h) * W, vc);
+#pragma unroll
+                        for (int e = 0; e < kVec; ++e) {
+                            sb[e] = fmaf(f, vb[e], sb[e]);
+                            sc[e] += vc[e];
+                        }
+                    }
+                }
+                red8_b[threadIdx.x][0] = make_float4(sb[0], sb[1], sb[2], sb[3]);
+                red8_b[threadIdx.x][1] = make_float4(sb[4], sb[5], sb[6], sb[7]);
+                red8_c[threadIdx.x][0] = make_float4(sc[0], sc[1], sc[2], sc[3]);
+                red8_c[threadIdx.x][1] = make_float4(sc[4], sc[5], sc[6], sc[7]);
+                __syncthreads();
+                if (vpart == 0 && v < nv) {
+                    float tb[kVec] = {}, tc[kVec] = {};
+                    for (int q = 0; q < parts; ++q)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const float4 b4 = red8_b[q * cols + vcol][hh], c4 = red8_c[q * cols + vcol][hh];
+                            tb[4 * hh] += b4.x; tb[4 * hh + 1] += b4.y; tb[4 * hh + 2] += b4.z; tb[4 * hh + 3] += b4.w;
+                            tc[4 * hh] += c4.x; tc[4 * hh + 1] += c4.y; tc[4 * hh + 2] += c4.z; tc[4 * hh + 3] += c4.w;
+                        }
+                    st8(dB + obc + int64_t(v) * kVec, tb);
+                    st8(dC + obc + int64_t(v) * kVec, tc);
+                }
+                __syncthreads();
+            }
+            continue;
+        }
         for (int k0 = 0; k0 < GN; k0 += kCols) {
             const int k = k0 + col;
             float sb = 0.f, sc = 0.f;
@@ -320,11 +485,14 @@ cudaError_t backward_prep_t(const Dims &d, const void *x, const void *dy, const 
     const T *xx = static_cast<const T *>(x), *dyy = static_cast<const T *>(dy);
     const T *bb = static_cast<const T *>(Bm), *cc = static_cast<const T *>(Cm);
     const int64_t nx = int64_t(d.B) * d.T * d.H * d.P, nbc = int64_t(d.B) * d.T * d.G * d.N;
+    // whole 16-byte vectors where every row, head and slice starts on one
+    const bool vec = d.P % kVec == 0 && d.N % kVec == 0 && w.W % kVec == 0;
     prep_k_kernel<T, float><<<grid_rows(d), kThreads, 0, s>>>(d, dyy, dt, A, bb, cc, w.xk, w.dtr, w.bk,
-                                                                    w.ck);
+                                                                    w.ck, vec);
     prep_t_kernel<T, TS><<<grid_rows(d), kThreads, size_t(d.H) * sizeof(float), s>>>(d, w.W, xx, dyy, dt, A, bb, cc,
                                                                 static_cast<TS *>(w.xb), static_cast<TS *>(w.xc),
-                                                                static_cast<TS *>(w.dyr), static_cast<TS *>(w.xrr));
+                                                                static_cast<TS *>(w.dyr), static_cast<TS *>(w.xrr),
+                                                                vec);
     if (w.xf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(xx, w.xf, nx);
     if (w.dyf) to_f32_kernel<T><<<grid_for(nx), kThreads, 0, s>>>(dyy, w.dyf, nx);
     if (w.bf) to_f32_kernel<T><<<grid_for(nbc), kThreads, 0, s>>>(bb, w.bf, nbc);
@@ -340,7 +508,8 @@ cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const 
     const int64_t nw = int64_t(d.B) * d.T * d.H;
     const int64_t BH = int64_t(d.B) * d.H;
     post_k_kernel<T, float><<<grid_for(nw * 32), kThreads, 0, s>>>(d, xx, dyy, dt, A, D, w.yk, w.yh,
-                                                                  static_cast<T *>(dx), w.xu, w.cc, w.rr, w.dd);
+                                                                  static_cast<T *>(dx), w.xu, w.cc, w.rr, w.dd,
+                                                                  d.P % 2 == 0);
     r0_kernel<<<unsigned(BH), kThreads, 0, s>>>(BH, d.P * d.N, w.dh0, h0, w.R0);
     prefix_kernel<<<grid_for(BH * 32), kThreads, 0, s>>>(d, dt, A, w.R0, w.xu, w.cc, w.rr, w.dd, ddt, w.dA_part,
                                                          w.dD_part);
@@ -348,7 +517,7 @@ cudaError_t backward_post_t(const Dims &d, const void *x, const void *dy, const 
                                                                                        dD);
     group_sums_kernel<T, TS><<<grid_rows(d), kThreads, 0, s>>>(
         d, w.W, dt, A, static_cast<const TS *>(w.yb), static_cast<const TS *>(w.yc), static_cast<T *>(dB),
-        static_cast<T *>(dC));
+        static_cast<T *>(dC), d.N % kVec == 0 && w.W % kVec == 0);
     return cudaGetLastError();
 }
 

@@ -33,6 +33,14 @@ SHAPES = [
     # bf16 inputs whose scans cannot take the tensor-core plans (headdim 32): fp32 scans
     dict(batch=1, seqlen=160, nheads=4, headdim=32, dstate=32, ngroups=2, chunk_len=64, dtype="bf16"),
     dict(batch=1, seqlen=192, nheads=6, headdim=32, dstate=48, ngroups=3, chunk_len=64, dtype="f32"),
+    # headdim and dstate off the 8-element vectors of the element-wise kernels
+    # (fp32 only: bf16 takes multiples of 8): odd (every element on its own)
+    # and even (pairs)
+    dict(batch=2, seqlen=128, nheads=3, headdim=5, dstate=7, ngroups=1, chunk_len=32, dtype="f32"),
+    dict(batch=1, seqlen=192, nheads=4, headdim=12, dstate=24, ngroups=2, chunk_len=64, dtype="f32"),
+    # a ragged length whose tail the 64-token scans cannot take (dstate 48):
+    # the scans of K and h keep the caller's chunk length
+    dict(batch=1, seqlen=96, nheads=2, headdim=16, dstate=48, ngroups=1, chunk_len=32, dtype="f32"),
 ]
 
 
