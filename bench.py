@@ -622,17 +622,33 @@ BACKWARD_METRIC = "SSD backward tokens/sec on 1 B200 (gradients of every input) 
 
 
 def backward_launches(inp):
-    """Kernels one ssd_backward call launches: the input preparation, the
-    transposed states, four fp32 scans (each its plan's launches) and the five
-    kernels that finish the gradients."""
+    """Kernels one ssd_backward call launches, following the choices it makes:
+    the input preparation (2 kernels, plus fp32 copies of x, B and C for bf16
+    inputs and of dy when the transposed scans run in fp32), the transposed
+    dfinal and h0, the scans of K and h (fp32, 64-token chunks unless that plan
+    is refused, then the caller's length), the transposed scans (per 64-wide
+    dstate slice on the bf16 tensor-core plans where they apply, else one fp32
+    scan each) and the five kernels that finish the gradients."""
     from structured_state_space_mamba_b200 import binding
     B_, T, H, P = inp.x.shape
     G, N = inp.B.shape[2], inp.B.shape[3]
-    fwd = binding.workspace_layout(binding.make_dims(B_, T, H, P, N, G, "f32"), inp.chunk_len).launches
-    tr = binding.workspace_layout(binding.make_dims(B_, T, H, N, P, H, "f32"), inp.chunk_len).launches
-    prep = 2 + (4 if inp.dtype == "bf16" else 0)
+    bf16 = inp.dtype == "bf16"
+    f32 = binding.make_dims(B_, T, H, P, N, G, "f32")
+    try:
+        scan = binding.workspace_layout(f32, 64).launches
+    except binding.SSDError:
+        scan = binding.workspace_layout(f32, inp.chunk_len).launches
+    scan_bf16 = False
+    if bf16 and P == 64 and N % 64 == 0:
+        lay = binding.workspace_layout(binding.make_dims(B_, T, H, 64, P, H, "bf16"), inp.chunk_len)
+        scan_bf16 = binding.SCAN_ENGINES.get(lay.scan_engine) != "simt"
+    if scan_bf16:
+        transposed = 2 * (N // 64) * lay.launches
+    else:
+        transposed = 2 * binding.workspace_layout(binding.make_dims(B_, T, H, N, P, H, "f32"), inp.chunk_len).launches
+    prep = 2 + (3 if bf16 else 0) + (1 if bf16 and not scan_bf16 else 0)
     states = 1 + (1 if inp.h0 is not None else 0)  # dfinal (always given here) and h0
-    return prep + states + 2 * fwd + 2 * tr + 5
+    return prep + states + 2 * scan + transposed + 5
 
 
 def run_backward(args, cfg, rank, world, local_rank):

@@ -134,3 +134,14 @@ def test_both_arms_build_the_same_config_block():
     assert a == b
     # without a GPU the helper falls back to the nominal L2 size
     assert bench.device_l2_bytes() > 0
+
+
+def test_backward_launch_count_by_hand():
+    """The launches one ssd_backward call makes on the 2.7B-shaped layer (bf16,
+    no initial state): prep_k, prep_t and three fp32 copies (x, B, C); the
+    transposed dfinal; the scans of K and h (4 launches each); the transposed
+    scans, two 64-wide dstate slices each on the bf16 tensor-core plan (4
+    launches each); and the five finishing kernels -- 35, the count of the
+    ncu launch list of that layer (175 launches over 5 calls)."""
+    from structured_state_space_mamba_b200.inputs import make_workload
+    assert bench.backward_launches(make_workload("mamba2_2p7b")) == 5 + 1 + 2 * 4 + 2 * 2 * 4 + 5
