@@ -209,7 +209,7 @@ def test_presolved_single_pass(oracle, shape, h0):
 
 def test_presolved_single_pass_steep_tiles(oracle):
     """Steep heads on the presolved path: the chunks of flagged tiles get their
-    s_in written and the single pass computes those tiles at its end; the range
+    s_in written and the block-factored scan finishes those tiles; the range
     states stay exact (their factors never exceed 1)."""
     inp = make_inputs(2, 2048, 8, 64, 64, 2, 256, dtype="bf16", seed=37, init_state=True, h0_std=1.0)
     rng = np.random.default_rng(37)
@@ -405,8 +405,7 @@ def test_single_pass_no_skip_no_final(oracle):
 
 @pytest.mark.parametrize("shape", [SINGLE_SHAPES[0], SINGLE_SHAPES[3], SINGLE_SHAPES[5]])
 def test_single_pass_steep_and_zero_dt(oracle, shape):
-    """Per head: a decay steep enough that tiles are listed (the single pass
-    computes them at its end from the chunk equations on the CUDA cores),
+    """Per head: a decay steep enough that tiles go to the block-factored scan,
     a decay range across the chunk (reference moved to the middle), zero dt on
     a run of tokens, and a gentle decay, all in one launch."""
     assert single_pass(shape)
