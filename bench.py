@@ -52,10 +52,10 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 # build it was taken from, so a rebuilt kernel reports traffic None until it is
 # captured again.
 NCU_TRAFFIC = {
-    # profiles/full_chunk_fused_mamba2_2p7b.md: 187.99 MB read + 137.50 MB written
-    ("mamba2_2p7b", "ssd_chunk_fused", "ssd-b200 0.3.2 sm_100a"): 325_497_856,
-    # profiles/sol_kernels_long_g8.md (presolved single pass): 564.63 MB read + 236.60 MB written
-    ("long_g8", "ssd_chunk_fused", "ssd-b200 0.3.2 sm_100a"): 801_234_688,
+    # profiles/full_chunk_fused_mamba2_2p7b.md: 187.87 MB read + 139.70 MB written
+    ("mamba2_2p7b", "ssd_chunk_fused", "ssd-b200 0.3.1 sm_100a"): 327_571_456,
+    # profiles/sol_kernels_long_g8.md (presolved single pass): 564.46 MB read + 236.48 MB written
+    ("long_g8", "ssd_chunk_fused", "ssd-b200 0.3.1 sm_100a"): 800_936_704,
 }
 
 
