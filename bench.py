@@ -112,12 +112,11 @@ def work_model(cfg, final_state=True, lay=None):
     gq_bytes = B * H * nc * (Q + 4) * 4
     h0_bytes = state_bytes if cfg.get("init_state") else 0
     fin_bytes = state_bytes if final_state else 0
-    tail = 1 if lay is not None and T % lay.chunk_len else 0  # the ragged tail's launch
-    if lay is not None and getattr(lay, "single_pass", 0) and lay.launches - tail == 4:
+    if lay is not None and getattr(lay, "single_pass", 0) and lay.launches == 5:
         # presolved single pass: cumsum (fused mode, plus w and alpha); the range
         # states: x, B, w, alpha, h0 -> one partial state per CTA, chained along
-        # each chain (small); the single pass from those states (it computes
-        # the tiles it lists as steep itself)
+        # each chain (small); the single pass from those states, then the
+        # block-factored scan of the listed tiles
         pre_bytes = min(B * (H // 2) * nc, 148) * 128 * N * 4  # one state per CTA of the single pass
         per_kernel = {
             "ssd_chunk_cumsum": dt_bytes + H * 4 + 2 * lq + gq_bytes + B * H * nc * 4,
@@ -138,19 +137,21 @@ def work_model(cfg, final_state=True, lay=None):
         # cumsum (fused mode): dt, A -> l and g (dtq and beta only for chunks with
         # a steep tile); the single-pass kernel: x, B, C, l, g, D, h0 -> y, final
         # (its per-(b, h) state slots stay in L2: B*H*P*N*4 bytes, each written
-        # and read once per chunk; the tiles it lists as steep it computes itself)
+        # and read once per chunk); the block-factored scan: only listed tiles
         per_kernel = {
             "ssd_chunk_cumsum": dt_bytes + H * 4 + lq + gq_bytes,
             "ssd_chunk_fused": (2 * x_bytes + bc_bytes + lq + gq_bytes + H * 4 + h0_bytes + fin_bytes),
+            "ssd_chunk_scan_steep": 0,
         }
         per_kernel_comp = {
             "ssd_chunk_cumsum": dt_bytes + H * 4,
             "ssd_chunk_fused": 2 * x_bytes + bc_bytes + H * 4 + h0_bytes + fin_bytes,
+            "ssd_chunk_scan_steep": 0,
         }
         per_kernel_flops = {"ssd_chunk_fused": flops}
         return dict(flops=flops, bytes=comp, per_kernel_bytes=per_kernel,
                     per_kernel_comp=per_kernel_comp, per_kernel_flops=per_kernel_flops,
-                    stages=("ssd_chunk_cumsum", "ssd_chunk_fused", None, None))
+                    stages=("ssd_chunk_cumsum", "ssd_chunk_fused", None, "ssd_chunk_scan_steep"))
     per_kernel = {
         # dt, A -> l, w, dtq, beta, alpha (and g for the chunk-wide scan)
         "ssd_chunk_cumsum": dt_bytes + H * 4 + 4 * lq + B * H * nc * 4 + (gq_bytes if chunkwide else 0),
@@ -496,7 +497,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
     # A GPU-side sleep before each step lets the host enqueue all four stages
     # (and the events between them) first, so no host launch gap lands inside
     # an event pair.  Stage names follow the call's layout (the single-pass
-    # layout runs stages 1-3 of the four-kernel sequence as one kernel).
+    # layout runs stages 1-3 of the four-kernel sequence as one kernel, plus the
+    # block-factored scan of the listed steep tiles).
     names = work_model(cfg, final_state=want_final, lay=lay)["stages"]
     nst = len(names)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]

@@ -377,17 +377,17 @@ SSD_API size_t ssd_workspace_bytes(const ssd_dims_t *dims, int chunk_len);
  * kernel (bf16, headdim 64, dstate 64 or 128, chunk_len 128 / 256 (64 as 128),
  * an even number of heads per group), in one of two forms:
  *  - hand-off (at least 40% as many (batch, head pair) chains as the GPU has
- *    SMs; launches == 2): each chunk's state is carried to the next through an
+ *    SMs; launches == 3): each chunk's state is carried to the next through an
  *    fp32 slot per (batch, head) in the workspace, so neither the per-chunk
  *    states nor the incoming states reach memory (w, alpha and states are not
- *    written, s_in only for chunks with a steep tile, which the kernel
- *    computes at its end on the CUDA cores).  Stage 1 of ssd_forward_stage
- *    runs that kernel, stages 2 and 3 nothing (but the ragged tail);
+ *    written, s_in only for chunks with a tile the block-factored scan
+ *    finishes).  Stage 1 of ssd_forward_stage runs that kernel, stage 2
+ *    nothing, stage 3 the block-factored scan of the tiles it listed;
  *  - presolved (fewer chains, with ranges of at least 16 chunks per CTA or
- *    dstate 64; launches == 4): stage 1 computes the state entering each CTA's
+ *    dstate 64; launches == 5): stage 1 computes the state entering each CTA's
  *    range (a pass over x and B in range mode, then a pass chaining those
  *    states along each chain; w and alpha are written), stage 2 nothing,
- *    stage 3 the single pass from those states.
+ *    stage 3 the single pass from those states and the block-factored scan.
  * `scan_engine` names the kernel
  * that computes y.  `chunk_len` is the chunk length the kernels run with: the
  * caller's, except on the tensor-core path (SSD_BF16, headdim 64), where the

@@ -32,11 +32,9 @@
 // and y written once; no chunk state reaches HBM.
 //
 // Tiles the cumsum kernel flagged as steep (a factor would pass e^72) are not
-// stored by the tile pipeline: the state path stays exact (r keeps every
-// g_s <= 1 there), the kernel writes s_in_c in bf16 for the flagged chunk and
-// lists the tile in the CTA's own slice of the steep-tile list, and once the
-// pipeline is done the CTA computes those tiles' y on the CUDA cores from the
-// chunk equations (every exponent there is <= 0).
+// stored here: the state path stays exact (r keeps every g_s <= 1 there), the
+// kernel writes s_in_c in bf16 for the listed chunk, and the block-factored
+// scan (k_tc_chunk_scan4.cu, list mode) computes those tiles' y afterwards.
 //
 // Per tile (128 tokens of one chunk of one chain), on the tensor cores, from
 // two issuing threads: PX(k) then CB(k+1) from one, Z(k) then CS(k) from the
@@ -227,95 +225,6 @@ __device__ __noinline__ bool wait_flag(const unsigned int *f, unsigned int want,
     return false;
 }
 
-// One tile the cumsum flagged as steep (rows r0 = 128 k .. r0 + 127 of chunk c,
-// head h), from the chunk equations on the CUDA cores:
-//   y_t = exp(l_t) C_t . s_in_c[p, :] + sum_{s <= t in the chunk} exp(l_t - l_s) dt_s (C_t . B_s) x_s[p]
-//         + D_h x_t[p]
-// (l chunk-local and inclusive, so every exponent is <= 0).  A rare path: the
-// tensor-core form's factors u_t, g_s would pass e^72 there.  All threads of
-// the CTA: thread (t = tid / 4, columns p0 = 16 (tid % 4) .. p0 + 15); the
-// sources go through shared memory 64 at a time.
-template <int NS>
-__device__ __noinline__ void steep_tile(uint8_t *smem, const Dims d, int b, int c, int k, int h,
-                                        const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Bm,
-                                        const __nv_bfloat16 *__restrict__ Cm, const float *__restrict__ dtq,
-                                        const float *__restrict__ lcum, const float *__restrict__ Dskip,
-                                        const __nv_bfloat16 *__restrict__ s_in, __nv_bfloat16 *__restrict__ y) {
-    constexpr int kSrc = 64;     // sources per block
-    constexpr int kLdS = kSrc + 1;
-    float *sS = reinterpret_cast<float *>(smem);                                      // [128][kLdS] weights
-    __nv_bfloat16 *sC = reinterpret_cast<__nv_bfloat16 *>(sS + kRows * kLdS);          // [128][NS] C of the rows
-    __nv_bfloat16 *sB = sC + kRows * NS;                                              // [kSrc][NS] B of the sources
-    __nv_bfloat16 *sX = sB + kSrc * NS;                                               // [kSrc][64] x of the sources
-    __nv_bfloat16 *sI = sX + kSrc * 64;                                               // [64][NS] s_in_c
-    float *sl = reinterpret_cast<float *>(sI + 64 * NS);                              // [Q] l of the chunk
-    float *sd = sl + d.Q;                                                             // [Q] dt of the chunk
-    const int tid = threadIdx.x, nt = blockDim.x;
-    const int g = h / d.r, Q = d.Q;
-    const int tok0 = c * Q, r0 = k * kRows;
-    const int64_t lq = off_lq(d, b, h, c);
-    __syncthreads();  // the previous tile's shared memory is no longer read
-    for (int i = tid; i < Q; i += nt) {
-        sl[i] = lcum[lq + i];
-        sd[i] = dtq[lq + i];
-    }
-    for (int e = tid; e < kRows * NS; e += nt) sC[e] = Cm[off_bc(d, b, tok0 + r0 + e / NS, g) + e % NS];
-    const __nv_bfloat16 *si = s_in + off_state(d, b, c, h);
-    for (int e = tid; e < 64 * NS; e += nt) sI[e] = si[e];
-    __syncthreads();
-    const int t = tid >> 2, p0 = (tid & 3) * 16;
-    float acc[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    // the incoming state: exp(l_t) C_t . s_in_c[p, :]
-#pragma unroll 1
-    for (int n = 0; n < NS; ++n) {
-        const float cv = __bfloat162float(sC[t * NS + n]);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] = fmaf(cv, __bfloat162float(sI[(p0 + j) * NS + n]), acc[j]);
-    }
-    {
-        const float e = __expf(sl[r0 + t]);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] *= e;
-    }
-    // the chunk's sources s <= t, kSrc at a time
-#pragma unroll 1
-    for (int s0 = 0; s0 < r0 + kRows; s0 += kSrc) {
-        __syncthreads();  // the previous block's sources and weights are no longer read
-        for (int e = tid; e < kSrc * NS; e += nt) sB[e] = Bm[off_bc(d, b, tok0 + s0 + e / NS, g) + e % NS];
-        for (int e = tid; e < kSrc * 64; e += nt) sX[e] = x[off_x(d, b, tok0 + s0 + e / 64, h) + e % 64];
-        __syncthreads();
-        // w[t][s] = exp(l_t - l_s) dt_s (C_t . B_s) for s <= t, else 0: 16 sources per thread
-        const float lt = sl[r0 + t];
-#pragma unroll 1
-        for (int js = 0; js < 16; ++js) {
-            const int s = (tid & 3) * 16 + js, sa = s0 + s;
-            float w = 0.f;
-            if (sa <= r0 + t) {
-                float dot = 0.f;
-#pragma unroll 8
-                for (int n = 0; n < NS; ++n)
-                    dot = fmaf(__bfloat162float(sC[t * NS + n]), __bfloat162float(sB[s * NS + n]), dot);
-                w = __expf(lt - sl[sa]) * sd[sa] * dot;
-            }
-            sS[t * kLdS + s] = w;
-        }
-        __syncthreads();
-#pragma unroll 1
-        for (int s = 0; s < kSrc; ++s) {
-            const float w = sS[t * kLdS + s];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = fmaf(w, __bfloat162float(sX[s * 64 + p0 + j]), acc[j]);
-        }
-    }
-    // the skip term, and y
-    const float Dh = Dskip ? Dskip[h] : 0.f;
-    const int64_t yo = off_x(d, b, tok0 + r0 + t, h) + p0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) y[yo + j] = __float2bfloat16_rn(fmaf(Dh, __bfloat162float(x[yo + j]), acc[j]));
-}
-
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_b,
@@ -324,9 +233,9 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                    const float *__restrict__ lcum, const float *__restrict__ Dskip,
                    const float *__restrict__ h0, float *__restrict__ fin, float *__restrict__ chain,
                    unsigned int *__restrict__ flags, const float *__restrict__ presolved,
-                   __nv_bfloat16 *__restrict__ s_in, long long *__restrict__ steep_items,
-                   const __nv_bfloat16 *__restrict__ Bm, const __nv_bfloat16 *__restrict__ Cm,
-                   const float *__restrict__ dtq, __nv_bfloat16 *__restrict__ y, unsigned int *err) {
+                   __nv_bfloat16 *__restrict__ s_in,
+                   int *__restrict__ nsteep, long long *__restrict__ steep_items, int max_steep,
+                   unsigned int *err) {
     using L = FusedLayout<NS>;
     constexpr int kCBS = L::kCBStages, kXS = L::kXStages;
     if (device_failed(err)) return;  // an earlier wait expired: skip all work
@@ -341,7 +250,6 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     uint64_t *acc_ready = px_done + 2, *z_done = acc_ready + 1, *sp_ready = z_done + 1, *done = sp_ready + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(done + 1);
     volatile int *state_ok = reinterpret_cast<volatile int *>(done + 2);
-    int *steep_count = reinterpret_cast<int *>(done + 3);  // tiles this CTA listed
     auto cb_at = [&](uint32_t kt) { return smem + (kt % kCBS) * L::kCBSlot; };
     auto x_at = [&](uint32_t kt) { return smem + L::kXOff + (kt % kXS) * L::kX; };
 
@@ -349,9 +257,6 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     const int Q = d.Q, ntile = Q / kRows, ngq = chunk_gq(Q);
     const int np = d.H / 2;
     const Range R = cta_range(d);
-    // this CTA's slice of the steep-tile list: two heads per tile of its items
-    const long long list_base =
-        2ll * ntile * chain_range_begin((long long)d.B * np * d.nc, int(blockIdx.x), int(gridDim.x));
 
     if (tid == 0) {
         for (int i = 0; i < kCBS; ++i) {
@@ -374,7 +279,6 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
         mbar_init(z_done, 1);
         mbar_init(sp_ready, 128);
         mbar_init(done, 2);  // both MMA issuers
-        *steep_count = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_c);
         tma_prefetch_desc(&tm_b);
@@ -867,8 +771,9 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
                         for (int jh = 0; jh < 2; ++jh) {
                             if (stp[jh]) {
                                 if (qd == 0) {
-                                    const int idx = atomicAdd(steep_count, 1);
-                                    steep_items[list_base + idx] = ((long long)T.b << 40) | ((long long)c << 24) |
+                                    const int idx = atomicAdd(nsteep, 1);
+                                    if (idx < max_steep)
+                                        steep_items[idx] = ((long long)T.b << 40) | ((long long)c << 24) |
                                                            ((long long)k << 16) | (2 * T.p + jh);
                                 }
                                 continue;
@@ -888,21 +793,13 @@ chunk_fused_kernel(const __grid_constant__ CUtensorMap tm_c, const __grid_consta
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 512);
-    // the tiles listed as steep, from the chunk equations (the rings are free now)
-    const int nfix = *steep_count;
-    for (int i = 0; i < nfix; ++i) {
-        const long long v = steep_items[list_base + i];
-        steep_tile<NS>(smem, d, int(v >> 40), int((v >> 24) & 0xFFFF), int((v >> 16) & 0xFF), int(v & 0xFFFF),
-                       x, Bm, Cm, dtq, lcum, Dskip, s_in, y);
-    }
 }
 
 template <int NS>
 cudaError_t launch_fused(const Dims &d, const CUtensorMap *maps, const __nv_bfloat16 *x, const float *gq,
                          const float *l, const float *D, const float *h0, float *fin, float *chain,
                          unsigned int *flags, const float *presolved, int presolved_grid, __nv_bfloat16 *s_in,
-                         long long *items, const __nv_bfloat16 *Bm, const __nv_bfloat16 *Cm, const float *dtq,
-                         __nv_bfloat16 *y, unsigned int *err, cudaStream_t stream) {
+                         int *nsteep, long long *items, int max_items, unsigned int *err, cudaStream_t stream) {
     using L = FusedLayout<NS>;
     if (!smem_attr_once(reinterpret_cast<const void *>(chunk_fused_kernel<NS>), int(L::kTotal)))
         return cudaErrorInvalidValue;
@@ -914,7 +811,7 @@ cudaError_t launch_fused(const Dims &d, const CUtensorMap *maps, const __nv_bflo
     const int grid = presolved ? presolved_grid : (chains < sms ? int(chains) : sms);
     chunk_fused_kernel<NS><<<grid, kThreads, L::kTotal, stream>>>(maps[0], maps[1], maps[2], maps[3], d, x, gq,
                                                                   l, D, h0, fin, chain, flags, presolved, s_in,
-                                                                  items, Bm, Cm, dtq, y, err);
+                                                                  nsteep, items, max_items, err);
     return cudaGetLastError();
 }
 
@@ -932,7 +829,7 @@ size_t chunk_fused_flag_bytes(const Dims &d) { return size_t(d.B) * (d.H / 2) * 
 cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
                                const float *D, const float *l, const float *h0, void *y, float *fin,
                                float *chain, unsigned int *flags, const float *presolved, int presolved_grid,
-                               void *s_in_bf16, long long *items, const float *dtq, unsigned int *err,
+                               void *s_in_bf16, int *nsteep, long long *items, int max_items, unsigned int *err,
                                cudaStream_t stream) {
     if (presolved && presolved_grid <= 0) return cudaErrorInvalidValue;
     const uint64_t bcdims[3] = {uint64_t(d.N), uint64_t(d.G), uint64_t(d.B) * d.T};
@@ -949,14 +846,12 @@ cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, co
         !make_tmap_bf16(&maps[3], 3, y, xdims, xstr, ybox, 128))
         return cudaErrorInvalidValue;
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-    const __nv_bfloat16 *bb = static_cast<const __nv_bfloat16 *>(Bm), *cb = static_cast<const __nv_bfloat16 *>(Cm);
     __nv_bfloat16 *sb = static_cast<__nv_bfloat16 *>(s_in_bf16);
-    __nv_bfloat16 *yb = static_cast<__nv_bfloat16 *>(y);
     switch (d.N) {
         case 64: return launch_fused<64>(d, maps, xb, gq, l, D, h0, fin, chain, flags, presolved, presolved_grid,
-                                         sb, items, bb, cb, dtq, yb, err, stream);
+                                         sb, nsteep, items, max_items, err, stream);
         case 128: return launch_fused<128>(d, maps, xb, gq, l, D, h0, fin, chain, flags, presolved, presolved_grid,
-                                           sb, items, bb, cb, dtq, yb, err, stream);
+                                           sb, nsteep, items, max_items, err, stream);
     }
     return cudaErrorInvalidValue;
 }

@@ -108,10 +108,8 @@ cudaError_t launch_chunk_scan_tc5(const Dims &d, const void *x, const float *gq,
 // N in {64, 128}, chunk_len 128 / 256, an even number of heads per group):
 // chunk state, state passing through per-(b, h) fp32 slots `chain` [B,H,P,N]
 // with flags [B, H/2], and chunk scan.  Tiles flagged steep by the cumsum are
-// listed in the CTA's slice of `items` (room for every (tile, head)), with s_in
-// (bf16 [B,nc,H,P,N]) written for their chunks, and computed at the end of the
-// kernel on the CUDA cores from x, B, C, l, dtq (dt of the flagged chunks) and
-// s_in.
+// appended to (nsteep, items) for the block-factored scan, with s_in (bf16
+// [B,nc,H,P,N]) written for their chunks.
 bool tc_chunk_fused_supported(const Dims &d);
 size_t chunk_fused_chain_bytes(const Dims &d);
 size_t chunk_fused_flag_bytes(const Dims &d);
@@ -122,7 +120,7 @@ size_t chunk_fused_flag_bytes(const Dims &d);
 cudaError_t launch_chunk_fused(const Dims &d, const void *x, const float *gq, const void *Bm, const void *Cm,
                                const float *D, const float *l, const float *h0, void *y, float *fin,
                                float *chain, unsigned int *flags, const float *presolved, int presolved_grid,
-                               void *s_in_bf16, long long *items, const float *dtq, unsigned int *err,
+                               void *s_in_bf16, int *nsteep, long long *items, int max_items, unsigned int *err,
                                cudaStream_t stream);
 
 // The last T mod chunk_len tokens of every (b, h) as the recurrence, from

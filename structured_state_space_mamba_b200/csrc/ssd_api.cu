@@ -274,8 +274,8 @@ ssd_status_t make_plan(const ssd_dims_t *dims, int chunk_len, Plan *plan) {
     w.total_bytes = off;
     w.tensor_core = (plan->tc_state || plan->tc_scan) ? 1 : 0;
     w.launches = d.nc == 0 ? 0
-                 : plan->presolved ? 4
-                 : plan->single ? 2 : (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
+                 : plan->presolved ? 5
+                 : plan->single ? 3 : (plan->fused ? 3 : 4) + (plan->scan5 ? 1 : 0);
     if (plan->t_full < d.T) w.launches += 1;
     w.fused_state = plan->fused ? 1 : 0;
     w.single_pass = plan->single ? 1 : 0;
@@ -378,11 +378,12 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
             continue;
         }
         if (pl.single) {
-            // cumsum (fused mode), then the single-pass kernel (which computes
-            // the tiles it lists as steep itself).  Presolved: the cumsum also
+            // cumsum (fused mode), the single-pass kernel, the block-factored scan
+            // over the tiles it listed as steep.  Presolved: the cumsum also
             // writes w and alpha, stage 1 computes the state entering every
             // range of the single pass (two launches), and stage 3 runs the
-            // single pass from those states.
+            // single pass from those states, then the block-factored scan.
+            const int max_steep = ssd::chunk_scan5_max_steep(d);
             switch (stage) {
                 case SSD_STAGE_CHUNK_CUMSUM:
                     e = ssd::launch_chunk_cumsum(d, dt, A, l, pl.presolved ? w : nullptr, dtq, beta, alpha, gq,
@@ -393,14 +394,18 @@ ssd_status_t run(const Plan &pl, const void *x, const float *dt, const float *A,
                             ? ssd::launch_presolve_ranges(d, pl.G, x, Bm, w, alpha, init_state, seg, start, err,
                                                           stream)
                             : ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags,
-                                                      nullptr, 0, s_in, steep_items, dtq, err, stream);
+                                                      nullptr, 0, s_in, nsteep, steep_items, max_steep, err,
+                                                      stream);
                     break;
                 case SSD_STAGE_STATE_PASSING:
                     break;
                 case SSD_STAGE_CHUNK_SCAN:
                     if (pl.presolved)
                         e = ssd::launch_chunk_fused(d, x, gq, Bm, Cm, D, l, init_state, y, fin, chain, flags, start,
-                                                    pl.G, s_in, steep_items, dtq, err, stream);
+                                                    pl.G, s_in, nsteep, steep_items, max_steep, err, stream);
+                    if (e == cudaSuccess)
+                        e = ssd::launch_chunk_scan_tc4(d, x, dtq, beta, Bm, Cm, D, l, s_in, y, steep_items, nsteep,
+                                                       max_steep, err, stream);
                     if (e == cudaSuccess) e = finish_scan();
                     break;
             }
@@ -847,6 +852,6 @@ ssd_status_t ssd_workspace_trim(void) {
     return SSD_OK;
 }
 
-const char *ssd_version(void) { return "ssd-b200 0.3.2 sm_100a"; }
+const char *ssd_version(void) { return "ssd-b200 0.3.1 sm_100a"; }
 
 }  // extern "C"
