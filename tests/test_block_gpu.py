@@ -130,3 +130,37 @@ def test_block_full_size_layers(oracle, name):
     assert rel(out, ref) <= tol, rel(out, ref)
     assert rel(fin, fref) <= tol
     assert rel(rstd, rref) <= tol
+
+
+def test_many_steep_tiles_stay_fast():
+    """The 2.7B-shaped block with softplus(dt + bias) step sizes large enough
+    that almost every 128-token tile of the single pass is steep (a factor of
+    the tensor-core form would pass e^72): those tiles go to the tensor-core
+    block-factored scan in list mode, so the call stays well under a
+    millisecond.  A CUDA-core fix-up of the listed tiles inside the single
+    pass took 44 ms per call here; the bound of 5 ms catches such a path."""
+    inp = make_workload("mamba2_2p7b")
+    tt = torch.bfloat16
+    t = lambda a, ty=torch.float32: torch.from_numpy(np.ascontiguousarray(a)).to(DEV).to(ty)  # noqa: E731
+    x, dt, A, B, C, D = t(inp.x, tt), t(inp.dt), t(inp.A), t(inp.B, tt), t(inp.C, tt), t(inp.D)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    z = torch.randn(x.shape, generator=g).to(DEV).to(tt)
+    H, P = x.shape[2], x.shape[3]
+    w = (1.0 + 0.1 * torch.randn(H * P, generator=g)).to(DEV)
+    bias = (0.1 * torch.randn(H, generator=g)).to(DEV)
+    y = torch.empty_like(x)
+    call = lambda: binding.forward_block(x, dt, A, B, C, D=D, chunk_len=inp.chunk_len, dt_bias=bias,  # noqa: E731
+                                         dt_softplus=True, z=z, norm_weight=w, out=y)
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    assert torch.isfinite(y.float()).all()
+    ms = e0.elapsed_time(e1) / 5
+    assert ms < 5.0, ms
