@@ -112,7 +112,8 @@ def work_model(cfg, final_state=True, lay=None):
     gq_bytes = B * H * nc * (Q + 4) * 4
     h0_bytes = state_bytes if cfg.get("init_state") else 0
     fin_bytes = state_bytes if final_state else 0
-    if lay is not None and getattr(lay, "single_pass", 0) and lay.launches == 5:
+    tail = 1 if lay is not None and T % lay.chunk_len else 0  # the ragged tail's own launch
+    if lay is not None and getattr(lay, "single_pass", 0) and lay.launches - tail == 5:
         # presolved single pass: cumsum (fused mode, plus w and alpha); the range
         # states: x, B, w, alpha, h0 -> one partial state per CTA, chained along
         # each chain (small); the single pass from those states, then the

@@ -145,3 +145,14 @@ def test_backward_launch_count_by_hand():
     ncu launch list of that layer (175 launches over 5 calls)."""
     from structured_state_space_mamba_b200.inputs import make_workload
     assert bench.backward_launches(make_workload("mamba2_2p7b")) == 5 + 1 + 2 * 4 + 2 * 2 * 4 + 5
+
+
+def test_presolved_layout_recognised_with_a_ragged_tail():
+    """A presolved single-pass layout keeps its accounting when the length
+    leaves a ragged tail (one more launch, the tail kernel)."""
+    cfg = dict(WORKLOADS["long_g8"])
+    cfg["seqlen"] = cfg["seqlen"] - 100
+    lay = layout(cfg)
+    assert lay.single_pass == 1 and lay.launches == 6
+    wm = bench.work_model(cfg, True, lay)
+    assert wm["stages"] == ("ssd_chunk_cumsum", "ssd_range_states", None, "ssd_chunk_fused")
