@@ -61,7 +61,12 @@ struct Vec<float> {
     }
 };
 
-__device__ __forceinline__ float silu_gate(float y, float z) { return y * (z / (1.f + __expf(-z))); }
+// y * silu(z) = y * z / (1 + e^-z).  The kernel is bound by its instruction
+// issue, not by HBM (ncu on the 2.7B-shaped block: issue slots 76 % busy, DRAM
+// 37 %), and an IEEE division costs several times the rest of the gate, so it
+// takes the approximate division (2 ulp; for z below about -88, e^-z is inf
+// and the quotient 0, the limit of silu).
+__device__ __forceinline__ float silu_gate(float y, float z) { return y * __fdividef(z, 1.f + __expf(-z)); }
 
 // block-wide sum over NT threads (every thread gets the result)
 template <int NT = kThreads>
